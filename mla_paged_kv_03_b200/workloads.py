@@ -1,0 +1,267 @@
+"""Seeded synthetic inputs for MLA decode over a paged latent KV cache.
+
+This module only draws random numbers and lays them out (shapes, block tables,
+length mixes, index sets, the byte layout of the FP8 cache).  It holds none of
+the attention arithmetic and imports neither the CUDA binding nor the oracle,
+so both sides of a parity check take their inputs from here.
+
+Workloads (shapes and distributions as specified for this library):
+
+* ``tiny``      dense bf16, b=2, s_q=1, h_q=16, lengths {37, 200}
+* ``compute``   dense bf16, b=64, s_q=1, h_q=128, L ~ U[4096, 8192], q,k ~ 0.5 N(0,1)
+* ``memory``    dense bf16, b=128, s_q=2 (causal pair), h_q=16,
+                L log-uniform in [1024, 16384], q,k ~ N(0,1)
+* ``fused``     s_q=1, h_q=64, d_v=576, L ~ U[2048, 32768], b in {1, 32},
+                q_raw ~ N(0,1), RMSNorm gain ~ N(1, 0.1), eps 1e-6, RoPE base 1e4
+* ``sparse``    b=32, s_q=1, h_q=128, 65536-token cache per sequence, topk=2048
+                indices drawn without replacement, round(5%) of slots = -1,
+                656-byte FP8 rows.
+
+The cache of the fused workload is specified as "already rotated at its own
+positions".  A rotation of an isotropic Gaussian pair is again an isotropic
+Gaussian pair, so drawing the RoPE dims N(0,1) directly gives exactly the
+distribution of rotated N(0,1) dims; no rotation is applied here.
+
+The FP8 rows are prepared the way a cache writer would: x ~ N(0,1), one fp32
+scale = absmax/448 per 128-value tile, codes = torch's float8_e4m3fn cast of
+x/scale; RoPE dims stored as bf16.  Byte order per row:
+``[512 x e4m3][4 x fp32 little-endian][64 x bf16]``.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+from typing import Optional
+
+import torch
+
+D_QK = 576
+D_NOPE = 512
+D_ROPE = 64
+PAGE = 64
+ROW656 = 656
+
+
+def _gen(seed: int, device) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    return g
+
+
+@dataclass
+class DenseCase:
+    q: torch.Tensor            # [b, s_q, h_q, 576] bf16
+    kcache: torch.Tensor       # [num_blocks, 64, 1, 576] bf16
+    block_table: torch.Tensor  # [b, max_pages] int32 (-1 = unused)
+    cache_seqlens: torch.Tensor  # [b] int32
+    s_q: int
+    h_q: int
+    d_v: int
+    causal: bool
+    softmax_scale: float
+    name: str = ""
+
+    @property
+    def batch(self):
+        return int(self.q.shape[0])
+
+
+@dataclass
+class FusedCase:
+    q_raw: torch.Tensor        # [b, 1, h_q, 576] bf16
+    gain: torch.Tensor         # [576] fp32
+    eps: float
+    rope_base: float
+    kcache: torch.Tensor
+    block_table: torch.Tensor
+    cache_seqlens: torch.Tensor
+    h_q: int
+    softmax_scale: float
+    positions: Optional[torch.Tensor] = None
+    name: str = ""
+    d_v: int = D_QK
+
+    @property
+    def batch(self):
+        return int(self.q_raw.shape[0])
+
+
+@dataclass
+class SparseCase:
+    q: torch.Tensor            # [b, s_q, h_q, 576] bf16
+    kcache: torch.Tensor       # [num_blocks, 64, 656] uint8
+    indices: torch.Tensor      # [b, s_q, topk] int32, physical slot or -1
+    h_q: int
+    s_q: int
+    d_v: int
+    softmax_scale: float
+    topk: int
+    seqlen: int
+    block_table: torch.Tensor = field(default=None)  # logical -> physical (for checks)
+    name: str = ""
+
+    @property
+    def batch(self):
+        return int(self.q.shape[0])
+
+
+def default_scale() -> float:
+    return 1.0 / math.sqrt(D_QK)
+
+
+def paged_block_table(seqlens, gen, spare_blocks=0, device="cpu"):
+    """Random permutation of the sum(ceil(L/64)) (+spare) physical blocks dealt
+    out to the sequences in order; unused table entries are -1."""
+    seqlens = [int(x) for x in seqlens]
+    pages = [(L + PAGE - 1) // PAGE for L in seqlens]
+    total = sum(pages) + int(spare_blocks)
+    max_pages = max(1, max(pages) if pages else 1)
+    perm = torch.randperm(max(total, 1), generator=gen, device=gen.device).to(torch.int32)
+    bt = torch.full((len(seqlens), max_pages), -1, dtype=torch.int32, device=gen.device)
+    pos = 0
+    for b, p in enumerate(pages):
+        if p:
+            bt[b, :p] = perm[pos:pos + p]
+        pos += p
+    return bt.to(device), max(total, 1)
+
+
+def _randn_bf16(shape, gen, std=1.0, device="cpu", chunk_rows=None):
+    """N(0, std^2) drawn in fp32 and rounded to bf16, optionally in row chunks
+    to bound temporary memory for very large caches."""
+    out = torch.empty(shape, dtype=torch.bfloat16, device=gen.device)
+    flat = out.view(shape[0], -1)
+    rows = shape[0]
+    step = chunk_rows or rows
+    for r0 in range(0, rows, step):
+        r1 = min(rows, r0 + step)
+        x = torch.randn((r1 - r0, flat.shape[1]), generator=gen, device=gen.device,
+                        dtype=torch.float32)
+        if std != 1.0:
+            x.mul_(std)
+        flat[r0:r1] = x.to(torch.bfloat16)
+    return out.to(device)
+
+
+def make_dense(seqlens, s_q, h_q, *, seed=0, q_std=1.0, k_std=1.0, d_v=D_NOPE, causal=True,
+               spare_blocks=0, device="cpu", name="", gen_device=None):
+    """Dense paged case with the given per-sequence lengths."""
+    gd = gen_device or device
+    g = _gen(seed, gd)
+    b = len(seqlens)
+    bt, nb = paged_block_table(seqlens, g, spare_blocks)
+    kcache = _randn_bf16((nb, PAGE, 1, D_QK), g, std=k_std, chunk_rows=4096)
+    q = _randn_bf16((b, s_q, h_q, D_QK), g, std=q_std)
+    sl = torch.tensor([int(x) for x in seqlens], dtype=torch.int32)
+    return DenseCase(q=q.to(device), kcache=kcache.to(device), block_table=bt.to(device),
+                     cache_seqlens=sl.to(device), s_q=s_q, h_q=h_q, d_v=d_v, causal=causal,
+                     softmax_scale=default_scale(), name=name)
+
+
+# ----------------------------------------------------------- length mixes
+
+def lengths_uniform(b, lo, hi, seed):
+    g = _gen(seed + 7919, "cpu")
+    return torch.randint(lo, hi + 1, (b,), generator=g).tolist()
+
+
+def lengths_loguniform(b, lo, hi, seed):
+    g = _gen(seed + 7919, "cpu")
+    u = torch.rand((b,), generator=g, dtype=torch.float64)
+    return [int(round(math.exp(math.log(lo) + float(x) * (math.log(hi) - math.log(lo)))))
+            for x in u]
+
+
+# -------------------------------------------------------- named workloads
+
+def tiny(seed=0, device="cpu"):
+    return make_dense([37, 200], 1, 16, seed=seed, spare_blocks=3, device=device, name="tiny")
+
+
+def compute_bound(seed=0, device="cpu", batch=64, lo=4096, hi=8192):
+    sl = lengths_uniform(batch, lo, hi, seed)
+    return make_dense(sl, 1, 128, seed=seed, q_std=0.5, k_std=0.5, device=device,
+                      name="compute", gen_device=device)
+
+
+def memory_bound(seed=0, device="cpu", batch=128, lo=1024, hi=16384):
+    sl = lengths_loguniform(batch, lo, hi, seed)
+    return make_dense(sl, 2, 16, seed=seed, device=device, name="memory", gen_device=device)
+
+
+def fused(seed=0, device="cpu", batch=32, lo=2048, hi=32768, h_q=64, seqlens=None):
+    sl = seqlens if seqlens is not None else lengths_uniform(batch, lo, hi, seed)
+    g = _gen(seed, device)
+    bt, nb = paged_block_table(sl, g)
+    kcache = _randn_bf16((nb, PAGE, 1, D_QK), g, chunk_rows=4096)
+    q_raw = _randn_bf16((len(sl), 1, h_q, D_QK), g)
+    gain = (1.0 + 0.1 * torch.randn((D_QK,), generator=g, device=g.device,
+                                    dtype=torch.float32))
+    return FusedCase(q_raw=q_raw.to(device), gain=gain.to(device), eps=1e-6, rope_base=10000.0,
+                     kcache=kcache.to(device), block_table=bt.to(device),
+                     cache_seqlens=torch.tensor(sl, dtype=torch.int32).to(device), h_q=h_q,
+                     softmax_scale=default_scale(), name=f"fused_b{len(sl)}")
+
+
+def quantize_rows656(x_nope: torch.Tensor, rope_bf16: torch.Tensor) -> torch.Tensor:
+    """Cache-writer layout of the 656-byte row from fp32 nope values [n, 512]
+    and bf16 rope dims [n, 64]: per 128-value tile scale = absmax/448 (1 if the
+    tile is all zero), codes = float8_e4m3fn cast of x/scale."""
+    n = x_nope.shape[0]
+    tiles = x_nope.view(n, 4, 128)
+    amax = tiles.abs().amax(dim=2, keepdim=True)
+    scale = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
+    codes = (tiles / scale).to(torch.float8_e4m3fn).view(torch.uint8).view(n, 512)
+    out = torch.empty((n, ROW656), dtype=torch.uint8, device=x_nope.device)
+    out[:, :512] = codes
+    out[:, 512:528] = scale.view(n, 4).contiguous().view(torch.uint8).view(n, 16)
+    out[:, 528:] = rope_bf16.contiguous().view(torch.uint8).view(n, 128)
+    return out
+
+
+def sparse(seed=0, device="cpu", batch=32, h_q=128, s_q=1, seqlen=65536, topk=2048,
+           invalid_frac=0.05, seqlens=None):
+    """Sparse FP8 case.  Each sequence owns ceil(seqlen/64) physical blocks of
+    a shuffled pool; each query's topk logical tokens are drawn without
+    replacement from [0, L) and mapped through that block table to physical
+    slots; round(invalid_frac * topk) random slots are set to -1."""
+    gd = device
+    g = _gen(seed, gd)
+    sl = seqlens if seqlens is not None else [seqlen] * batch
+    bt, nb = paged_block_table(sl, g)
+    n_rows = nb * PAGE
+    cache = torch.empty((n_rows, ROW656), dtype=torch.uint8, device=g.device)
+    step = 1 << 16
+    for r0 in range(0, n_rows, step):
+        r1 = min(n_rows, r0 + step)
+        x = torch.randn((r1 - r0, D_NOPE), generator=g, device=g.device, dtype=torch.float32)
+        rope = torch.randn((r1 - r0, D_ROPE), generator=g, device=g.device,
+                           dtype=torch.float32).to(torch.bfloat16)
+        cache[r0:r1] = quantize_rows656(x, rope)
+    q = _randn_bf16((len(sl), s_q, h_q, D_QK), g)
+    n_bad = int(round(invalid_frac * topk))
+    idx = torch.empty((len(sl), s_q, topk), dtype=torch.int32, device=g.device)
+    for b, L in enumerate(sl):
+        for i in range(s_q):
+            k = min(topk, L)
+            logical = torch.randperm(L, generator=g, device=g.device)[:k].to(torch.int64)
+            phys = bt[b].to(torch.int64)[logical // PAGE] * PAGE + logical % PAGE
+            row = torch.full((topk,), -1, dtype=torch.int64, device=g.device)
+            row[:k] = phys
+            if n_bad:
+                bad = torch.randperm(topk, generator=g, device=g.device)[:n_bad]
+                row[bad] = -1
+            idx[b, i] = row.to(torch.int32)
+    return SparseCase(q=q.to(device), kcache=cache.view(nb, PAGE, ROW656).to(device),
+                      indices=idx.to(device), h_q=h_q, s_q=s_q, d_v=D_NOPE,
+                      softmax_scale=default_scale(), topk=topk, seqlen=max(sl),
+                      block_table=bt.to(device), name="sparse")
+
+
+WORKLOADS = {
+    "tiny": tiny,
+    "compute": compute_bound,
+    "memory": memory_bound,
+    "fused": fused,
+    "sparse": sparse,
+}
