@@ -35,6 +35,8 @@ def lib():
         L.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
         L.oracle_e4m3_encode.restype = ctypes.c_uint8
         L.oracle_e4m3_encode.argtypes = [ctypes.c_double]
+        L.oracle_round_bf16.restype = ctypes.c_double
+        L.oracle_round_bf16.argtypes = [ctypes.c_double]
         L.oracle_rmsnorm.restype = None
         L.oracle_rmsnorm.argtypes = [f64p, f64p, ctypes.c_int, ctypes.c_double, f64p]
         L.oracle_rope64.restype = None
@@ -106,6 +108,13 @@ def e4m3_encode(x):
     a = np.asarray(x, dtype=np.float64)
     f = lib().oracle_e4m3_encode
     return np.array([f(float(v)) for v in a.ravel()], dtype=np.uint8).reshape(a.shape)
+
+
+def round_bf16(x):
+    """oracle_round_bf16 (ties to even) over an array -> float64."""
+    a = np.asarray(x, dtype=np.float64)
+    f = lib().oracle_round_bf16
+    return np.array([f(float(v)) for v in a.ravel()], dtype=np.float64).reshape(a.shape)
 
 
 def decode_row656(row):

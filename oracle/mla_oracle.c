@@ -38,6 +38,9 @@
  *  - Row byte order of the 656-byte cache: [512 x e4m3][4 x fp32][64 x bf16].
  *  - RoPE pairs are interleaved (2k, 2k+1), theta_k = pos * base^(-2k/64);
  *    conjugate RoPE rotates by -theta_k.
+ *  - Fused path: the normalised, rotated query enters the attention in bf16
+ *    (the tensor-core operand precision); the pages leave this precision
+ *    open, and fixing it makes the FP8 code decisions comparable.
  *  - FP8 output: scale = absmax/448 (scale := 1 when absmax == 0), code =
  *    E4M3 round-to-nearest-even with saturation to +-448 of (o / scale),
  *    where the ratio is rounded to fp32 before encoding (the kernel takes
@@ -125,6 +128,18 @@ uint8_t oracle_e4m3_encode(double x) {
       return sign | (uint8_t)((be << 3) | (int)m);
     }
   }
+}
+
+/* Round to the nearest bf16 value (8 significant bits, ties to even); bf16
+ * shares fp32's exponent range, and the values rounded here are normal. */
+double oracle_round_bf16(double v) {
+  int e;
+  double m, r;
+  if (v == 0.0 || !isfinite(v)) return v;
+  m = frexp(fabs(v), &e); /* |v| = m * 2^e, m in [0.5, 1) */
+  r = rne(ldexp(m, 8));   /* 8 significant bits */
+  r = ldexp(r, e - 8);
+  return v < 0 ? -r : r;
 }
 
 /* ---------------------------------------------------------------- RMSNorm */
@@ -362,6 +377,7 @@ int oracle_fused_decode(const uint16_t* q_raw, const double* gain, double eps, d
     oracle_rmsnorm(x, gain, ORACLE_D, eps, y);
     oracle_rope64(y + ORACLE_NOPE, pos, rope_base, +1, x + ORACLE_NOPE);
     for (d = 0; d < ORACLE_NOPE; ++d) x[d] = y[d];
+    for (d = 0; d < ORACLE_D; ++d) x[d] = oracle_round_bf16(x[d]);
     ctx.kcache = kcache;
     ctx.block_table = block_table;
     ctx.max_pages = max_pages;

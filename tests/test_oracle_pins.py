@@ -116,6 +116,18 @@ def test_e4m3_encode_matches_torch_rne():
     assert (ref == ours).all(), np.nonzero(ref != ours)[0][:10]
 
 
+def test_round_bf16_matches_torch():
+    g = torch.Generator().manual_seed(2)
+    x = torch.randn(50000, generator=g, dtype=torch.float64) * 3.0
+    # exact midpoints between neighbouring bf16 values exercise the ties
+    b = x[:2000].to(torch.bfloat16).to(torch.float64)
+    mid = b + (torch.nextafter(b.to(torch.bfloat16), torch.tensor(1e9, dtype=torch.bfloat16))
+               .to(torch.float64) - b) / 2
+    x = torch.cat([x, mid])
+    ref = x.to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(oracle.round_bf16(x.numpy()), ref)
+
+
 def test_e4m3_saturates():
     assert oracle.e4m3_encode(np.array([1e6, -1e6, 470.0, 448.0])).tolist() == \
         [0x7E, 0xFE, 0x7E, 0x7E]
@@ -307,7 +319,7 @@ def fused_library_reference(case):
         z = (y[:, 512::2] + 1j * y[:, 513::2]) * np.exp(1j * pos * theta_k)
         y[:, 512::2], y[:, 513::2] = z.real, z.imag
         K = contiguous_k(case, bi)
-        q = torch.tensor(y)
+        q = torch.tensor(y).to(torch.bfloat16).to(torch.float64)  # attention input in bf16
         o = F.scaled_dot_product_attention(q[None], K[None], K[None],
                                            scale=case.softmax_scale)[0].numpy()
         lses[bi] = torch.logsumexp((q @ K.T) * case.softmax_scale, dim=-1).numpy()
@@ -349,13 +361,13 @@ def test_fused_reduces_to_dense_without_norm_and_rotation():
                                               want_pre_cast=True)
     x = case.q_raw.to(torch.float64)
     rms = torch.sqrt((x * x).mean(-1, keepdim=True))
-    scale_eff = case.softmax_scale / rms  # per (b, h)
+    qn = (x / rms).to(torch.bfloat16)  # normalised query, in the attention's bf16
     for b in range(2):
         for h in range(2):
-            dcase = W.DenseCase(q=case.q_raw[b:b + 1, :, h:h + 1].contiguous(),
+            dcase = W.DenseCase(q=qn[b:b + 1, :, h:h + 1].contiguous(),
                                 kcache=case.kcache, block_table=case.block_table[b:b + 1],
                                 cache_seqlens=case.cache_seqlens[b:b + 1], s_q=1, h_q=1, d_v=576,
-                                causal=False, softmax_scale=float(scale_eff[b, 0, h, 0]))
+                                causal=False, softmax_scale=case.softmax_scale)
             o, l = oracle.dense_decode(dcase.q, dcase.kcache, dcase.block_table,
                                        dcase.cache_seqlens, 576, dcase.softmax_scale,
                                        causal=False)
