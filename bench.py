@@ -1,0 +1,485 @@
+"""Benchmark of MLA decoding over a paged latent KV cache on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the whole decode path over one batch of synthetic input:
+the split-KV planner, the decode kernel (page fetch, QK, online softmax, PV,
+finalize) and the split-combine kernel (for the fused workload also the
+RMSNorm/RoPE prologue and the conjugate-RoPE/FP8 epilogue; for the sparse
+workload the FP8 gather/dequant).  Inputs are resident in HBM before the timed
+region; every workload's KV cache is larger than the 126 MB L2, so no L2 flush
+is inserted between steps.
+
+Rank 0 prints ONE JSON line.  Multi-GPU runs are independent replicas (the
+decode path has no exchange step): each rank decodes its own batch and
+`value` aggregates all ranks' work over the slowest rank's time.
+"""
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from mla_paged_kv_03_b200 import workloads as W  # noqa: E402
+
+METRIC = "MLA decode TFLOPS & KV-read GB/s on 1 B200, % of roofline"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+WORKLOAD_INFO = {
+    "compute": ("Compute-bound dense decode, bf16: batch 64, s_q 1, h_q 128, d_qk 576, d_v 512, "
+                "L ~ U[4096, 8192], block 64, shuffled blocks, q,k ~ 0.5 N(0,1)", "tensor"),
+    "memory": ("Memory-bound dense decode, bf16: batch 128, s_q 2 (causal pair), h_q 16, d_qk 576, "
+               "d_v 512, L log-uniform [1024, 16384], block 64, shuffled blocks", "hbm"),
+    "fused": ("Fused RMSNorm-RoPE-attn-conjRoPE-FP8 decode: batch 32, s_q 1, h_q 64, d 576, d_v 576, "
+              "L ~ U[2048, 32768], block 64", "hbm"),
+    "fused_b1": ("Fused RMSNorm-RoPE-attn-conjRoPE-FP8 decode: batch 1, s_q 1, h_q 64, d 576, "
+                 "d_v 576, L ~ U[2048, 32768], block 64", "hbm"),
+    "sparse": ("Token-level sparse decode, FP8 656-byte cache: batch 32, s_q 1, h_q 128, d_v 512, "
+               "65536-token cache per sequence, topk 2048, 5% -1 slots", "tensor"),
+    "tiny": ("Tiny dense decode, bf16: batch 2, s_q 1, h_q 16, lengths {37, 200}", "tensor"),
+}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+# ------------------------------------------------------------ work counting
+
+def dense_work(case):
+    """Algorithmic FLOPs and bytes: 2*|T|*(576 + d_v) per query row over its
+    visible tokens; bytes = the latent rows read once per sequence (all rows
+    share one KV head) + q + O + LSE + block table + lengths."""
+    sl = case.cache_seqlens.cpu().tolist()
+    flops = 0
+    kv_tokens = 0
+    for L in sl:
+        for i in range(case.s_q):
+            vis = max(0, min(L, L - case.s_q + 1 + i)) if case.causal else L
+            flops += 2 * vis * (576 + case.d_v) * case.h_q
+        kv_tokens += L
+    kv_bytes = kv_tokens * 576 * 2
+    io = case.q.numel() * 2 + case.batch * case.s_q * case.h_q * (case.d_v * 2 + 4) + \
+        case.block_table.numel() * 4 + case.batch * 4
+    return flops, kv_bytes, kv_bytes + io
+
+
+def fused_work(case):
+    sl = case.cache_seqlens.cpu().tolist()
+    flops = sum(2 * L * (576 + 576) * case.h_q for L in sl)
+    kv_bytes = sum(sl) * 576 * 2
+    io = case.q_raw.numel() * 2 + 576 * 4 + case.batch * case.h_q * (576 + 4 + 4) + \
+        case.block_table.numel() * 4 + case.batch * 4
+    return flops, kv_bytes, kv_bytes + io
+
+
+def sparse_work(case):
+    valid = int((case.indices >= 0).sum())  # (b, s_q) pairs x valid slots
+    flops = 2 * valid * (576 + case.d_v) * case.h_q
+    kv_bytes = valid * 656
+    io = case.q.numel() * 2 + case.indices.numel() * 4 + \
+        case.batch * case.s_q * case.h_q * (case.d_v * 2 + 4)
+    return flops, kv_bytes, kv_bytes + io
+
+
+# ----------------------------------------------------------------- GPU arm
+
+class GpuStep:
+    """One decode step through the library's public API, inputs resident."""
+
+    def __init__(self, name, seed, dev):
+        from mla_paged_kv_03_b200 import binding as B
+        self.B = B
+        self.name = name
+        self.dev = dev
+        if name in ("compute", "memory", "tiny"):
+            self.case = W.WORKLOADS[name](seed=seed, device=dev)
+            self.kind = "dense"
+            self.work = dense_work(self.case)
+            c = self.case
+            self.R = c.s_q * c.h_q
+        elif name in ("fused", "fused_b1"):
+            self.case = W.fused(seed=seed, device=dev, batch=32 if name == "fused" else 1)
+            self.kind = "fused"
+            self.work = fused_work(self.case)
+            self.R = self.case.h_q
+        elif name == "sparse":
+            self.case = W.sparse(seed=seed, device=dev)
+            self.kind = "sparse"
+            self.work = sparse_work(self.case)
+            self.R = self.case.h_q
+        else:
+            raise ValueError(name)
+        c = self.case
+        self.parts = B.mla_num_sm_parts(self.R, 1, dev)
+        b = c.batch
+        if self.kind == "dense":
+            self.out = torch.empty((b, c.s_q, c.h_q, c.d_v), dtype=torch.bfloat16, device=dev)
+            self.lse = torch.empty((b, c.s_q, c.h_q), dtype=torch.float32, device=dev)
+            self.ws = torch.empty((B.mla_workspace_size(b, self.R, c.d_v, self.parts),),
+                                  dtype=torch.uint8, device=dev)
+        elif self.kind == "fused":
+            self.out = torch.empty((b, 1, c.h_q, 576), dtype=torch.uint8, device=dev)
+            self.scale = torch.empty((b, 1, c.h_q), dtype=torch.float32, device=dev)
+            self.lse = torch.empty((b, 1, c.h_q), dtype=torch.float32, device=dev)
+            self.ws = torch.empty((B.mla_workspace_size(b, self.R, 576, self.parts),),
+                                  dtype=torch.uint8, device=dev)
+        else:
+            self.out = torch.empty((b, c.s_q, c.h_q, c.d_v), dtype=torch.bfloat16, device=dev)
+            self.lse = torch.empty((b, c.s_q, c.h_q), dtype=torch.float32, device=dev)
+            self.ws = torch.empty((B.mla_sparse_workspace_size(b, c.s_q, c.h_q, c.topk, c.d_v,
+                                                               self.parts),),
+                                  dtype=torch.uint8, device=dev)
+        if self.kind != "sparse":
+            self.meta = torch.empty((self.parts, 8), dtype=torch.int32, device=dev)
+            self.ns = torch.empty((b + 1,), dtype=torch.int32, device=dev)
+
+    def launches_per_step(self):
+        return 3  # planner + decode + combine
+
+    def step(self, q=None):
+        B, c = self.B, self.case
+        if self.kind == "dense":
+            m, n, _ = B.mla_get_metadata(c.cache_seqlens, self.R, 1, self.parts)
+            B.mla_decode_fwd(c.q if q is None else q, c.kcache, c.block_table, c.cache_seqlens,
+                             c.d_v, m, n, self.parts, causal=c.causal,
+                             softmax_scale=c.softmax_scale, out=self.out, lse=self.lse,
+                             workspace=self.ws)
+        elif self.kind == "fused":
+            m, n, _ = B.mla_get_metadata(c.cache_seqlens, self.R, 1, self.parts)
+            B.mla_fused_norm_rope_attn_rope_cast(
+                c.q_raw if q is None else q, c.gain, c.eps, c.rope_base, c.kcache,
+                c.block_table, c.cache_seqlens, m, n, self.parts,
+                softmax_scale=c.softmax_scale, out=self.out, out_scale=self.scale, lse=self.lse,
+                workspace=self.ws)
+        else:
+            B.mla_sparse_decode(c.q if q is None else q, c.kcache, c.indices, c.d_v,
+                                c.softmax_scale, self.parts, out=self.out, lse=self.lse,
+                                workspace=self.ws)
+
+    def query(self):
+        return self.case.q_raw if self.kind == "fused" else self.case.q
+
+
+def sample_clocks_start(dev_index):
+    path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{os.getpid()}.csv")
+    try:
+        os.makedirs(os.path.dirname(path), exist_ok=True)
+        f = open(path, "w")
+        p = subprocess.Popen(
+            ["nvidia-smi", f"--id={dev_index}",
+             "--query-gpu=clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap",
+             "--format=csv,noheader,nounits", "-lms", "200"], stdout=f, stderr=subprocess.DEVNULL)
+        return p, f, path
+    except Exception:
+        return None, None, None
+
+
+def sample_clocks_stop(handle):
+    p, f, path = handle
+    if p is None:
+        return None
+    p.terminate()
+    try:
+        p.wait(timeout=5)
+    except Exception:
+        p.kill()
+    f.close()
+    sm, mx, reasons = [], [], set()
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    for line in open(path):
+        parts = [x.strip() for x in line.split(",")]
+        if len(parts) < 8:
+            continue
+        try:
+            sm.append(float(parts[0]))
+            mx.append(float(parts[1]))
+        except ValueError:
+            continue
+        for nm, v in zip(names, parts[4:8]):
+            if v.lower() == "active":
+                reasons.add(nm)
+    if not sm:
+        return None
+    return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+            "samples": len(sm)}
+
+
+def run_gpu_arm(args, rank, world):
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    gs = GpuStep(args.workload, seed=args.seed + rank, dev=dev)
+    flops, kv_bytes, total_bytes = gs.work
+    st = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        gs.step()
+    torch.cuda.synchronize(dev)
+    status = gs.B.device_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status:#x} after warm-up")
+
+    if world > 1:
+        torch.distributed.barrier()
+    clk = sample_clocks_start(dev.index)
+    torch.cuda.synchronize(dev)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    ev0.record(st)
+    for _ in range(args.steps):
+        gs.step()
+    ev1.record(st)
+    torch.cuda.synchronize(dev)
+    ms_total = ev0.elapsed_time(ev1)
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sample_clocks_stop(clk)
+
+    # end to end through the same API with host buffers: H2D of the step's
+    # query from pinned memory, the step, D2H of the outputs
+    q_dev = gs.query()
+    q_host = q_dev.cpu().pin_memory()
+    q_buf = torch.empty_like(q_dev)
+    out_host = torch.empty(gs.out.shape, dtype=gs.out.dtype).pin_memory()
+    lse_host = torch.empty(gs.lse.shape, dtype=gs.lse.dtype).pin_memory()
+    e2e_steps = max(3, min(args.steps, 50))
+    for _ in range(2):
+        q_buf.copy_(q_host, non_blocking=True)
+        gs.step(q_buf)
+        out_host.copy_(gs.out, non_blocking=True)
+        lse_host.copy_(gs.lse, non_blocking=True)
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(e2e_steps):
+        q_buf.copy_(q_host, non_blocking=True)
+        gs.step(q_buf)
+        out_host.copy_(gs.out, non_blocking=True)
+        lse_host.copy_(gs.lse, non_blocking=True)
+    e1.record(st)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    status = gs.B.device_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status:#x} after timing")
+
+    ms_step = ms_total / args.steps
+    t = torch.tensor([ms_step, e2e_ms], dtype=torch.float64, device=dev)
+    w = torch.tensor([flops, kv_bytes], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        torch.distributed.all_reduce(w, op=torch.distributed.ReduceOp.SUM)
+    ms_step, e2e_ms = float(t[0]), float(t[1])
+    flops_all, kv_all = float(w[0]), float(w[1])
+    if rank != 0:
+        return None
+
+    peaks, peak_src = load_peaks()
+    desc, bound = WORKLOAD_INFO[args.workload]
+    tflops = flops_all / (ms_step * 1e-3) / 1e12
+    gbs = kv_all / (ms_step * 1e-3) / 1e9
+    # dominant kernel: the decode call (decode + combine kernels), one per step
+    per_launch_s = ms_step * 1e-3
+    if bound == "tensor":
+        achieved = flops / per_launch_s / 1e12
+        peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+        roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
+                "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                "peak_source": f"{peak_src} bf16 sustained (burst {peaks['bf16_tflops']})",
+                "frac_of_burst": round(achieved / peaks["bf16_tflops"], 4), "traffic": None}
+    else:
+        achieved = total_bytes / per_launch_s / 1e9
+        peak = peaks["hbm_gbs"]
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "peak_source": f"{peak_src} hbm copy",
+                "traffic": None}
+    line = {
+        "metric": METRIC,
+        "value": round(tflops, 3),
+        "unit": "TFLOPS",
+        "kv_read_gbs": round(gbs, 1),
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if args.workload != "sparse" else "bf16 (fp8 cache dequantised)",
+        "data": "synthetic",
+        "config": {"workload": desc, "name": args.workload,
+                   "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas x{world}"},
+        "e2e": {"value": round(flops_all / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOPS",
+                "h2d_bytes_per_step": int(q_dev.numel() * q_dev.element_size()),
+                "d2h_bytes_per_step": int(gs.out.numel() * gs.out.element_size() +
+                                          gs.lse.numel() * 4),
+                "ms_per_step": round(e2e_ms, 5)},
+        "gpu_launches": gs.launches_per_step() * args.steps,
+        "roofline": roof,
+        "clocks": clocks,
+    }
+    if args.cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_baseline(args.workload, seed=args.seed, budget_s=args.cpu_budget,
+                                            case=gs.case)
+    return line
+
+
+# ------------------------------------------------------ CPU oracle (baseline)
+
+def oracle_rows_timed(name, case, rows):
+    import oracle
+    if name in ("compute", "memory", "tiny"):
+        c = case
+        t0 = time.perf_counter()
+        oracle.dense_decode(c.q.cpu(), c.kcache_cpu, c.block_table.cpu(), c.cache_seqlens.cpu(),
+                            c.d_v, c.softmax_scale, causal=c.causal, rows=rows)
+        return time.perf_counter() - t0
+    if name in ("fused", "fused_b1"):
+        c = case
+        t0 = time.perf_counter()
+        oracle.fused_decode(c.q_raw.cpu(), c.gain.cpu(), c.eps, c.rope_base, c.kcache_cpu,
+                            c.block_table.cpu(), c.cache_seqlens.cpu(), c.softmax_scale,
+                            rows=rows)
+        return time.perf_counter() - t0
+    c = case
+    t0 = time.perf_counter()
+    oracle.sparse_decode(c.q.cpu(), c.kcache_cpu, c.indices.cpu(), c.d_v, c.softmax_scale,
+                         rows=rows)
+    return time.perf_counter() - t0
+
+
+def row_flops(name, case, rows):
+    """Algorithmic FLOPs of the sampled rows (same counting as the GPU arm)."""
+    f = 0
+    if name in ("compute", "memory", "tiny"):
+        sl = case.cache_seqlens.cpu().tolist()
+        for r in rows:
+            b = r // (case.s_q * case.h_q)
+            i = (r // case.h_q) % case.s_q
+            L = sl[b]
+            vis = max(0, min(L, L - case.s_q + 1 + i)) if case.causal else L
+            f += 2 * vis * (576 + case.d_v)
+    elif name in ("fused", "fused_b1"):
+        sl = case.cache_seqlens.cpu().tolist()
+        for r in rows:
+            f += 2 * sl[r // case.h_q] * 1152
+    else:
+        valid = (case.indices.cpu() >= 0).sum(-1).reshape(-1).tolist()
+        for r in rows:
+            f += 2 * valid[r // case.h_q] * (576 + case.d_v)
+    return f
+
+
+def cpu_baseline(name, seed=0, budget_s=15.0, case=None):
+    """Time the oracle as it stands on a bounded row sample of the workload."""
+    import numpy as np
+    import oracle
+    if case is None:
+        case = (W.WORKLOADS[name](seed=seed) if name in ("compute", "memory", "tiny")
+                else W.fused(seed=seed, batch=32 if name == "fused" else 1) if name.startswith("fused")
+                else W.sparse(seed=seed))
+    case.kcache_cpu = case.kcache.cpu()
+    total_rows = case.batch * (case.s_q if hasattr(case, "s_q") else 1) * case.h_q
+    rng = np.random.default_rng(seed)
+    n = 8
+    elapsed = oracle_rows_timed(name, case, np.sort(rng.choice(total_rows, n, replace=False)))
+    per_row = max(elapsed / n, 1e-6)
+    n = int(min(total_rows, max(8, budget_s / per_row)))
+    rows = np.sort(rng.choice(total_rows, n, replace=False))
+    elapsed = oracle_rows_timed(name, case, rows)
+    f = row_flops(name, case, rows)
+    return {"value": f / elapsed / 1e12, "unit": "TFLOPS", "cores": oracle.num_threads(),
+            "kind": "oracle", "seconds": round(elapsed, 2),
+            "sample": f"{n} of {total_rows} query rows (uniform random), fp64 C oracle, OpenMP"}
+
+
+def run_reference_arm(args, rank, world):
+    """The oracle timed on the host cores, each step a bounded row sample."""
+    if rank != 0:
+        return None
+    desc, _ = WORKLOAD_INFO[args.workload]
+    name = args.workload
+    case = (W.WORKLOADS[name](seed=args.seed) if name in ("compute", "memory", "tiny")
+            else W.fused(seed=args.seed, batch=32 if name == "fused" else 1)
+            if name.startswith("fused") else W.sparse(seed=args.seed))
+    per_step = max(1.0, args.cpu_budget / max(1, args.steps + args.warmup))
+    import numpy as np
+    import oracle
+    case.kcache_cpu = case.kcache.cpu()
+    total_rows = case.batch * (case.s_q if hasattr(case, "s_q") else 1) * case.h_q
+    rng = np.random.default_rng(args.seed)
+    t8 = oracle_rows_timed(name, case, np.sort(rng.choice(total_rows, 8, replace=False))) / 8
+    n = int(min(total_rows, max(4, per_step / max(t8, 1e-6))))
+    times, fl = [], []
+    for s in range(args.warmup + args.steps):
+        rows = np.sort(rng.choice(total_rows, n, replace=False))
+        dt = oracle_rows_timed(name, case, rows)
+        if s >= args.warmup:
+            times.append(dt)
+            fl.append(row_flops(name, case, rows))
+    sec = sum(times)
+    value = sum(fl) / sec / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec / len(times) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference",
+        "config": {"workload": desc, "name": name},
+        "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": oracle.num_threads(),
+                         "kind": "oracle",
+                         "sample": f"{n} of {total_rows} query rows per step, fp64 C oracle"},
+        "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    return line
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="compute", choices=sorted(WORKLOAD_INFO))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--cpu-baseline", dest="cpu_baseline", type=int, default=1)
+    ap.add_argument("--cpu-budget", dest="cpu_budget", type=float, default=15.0)
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group(
+            "nccl" if args.impl == "ours" else "gloo",
+            timeout=datetime.timedelta(seconds=300))
+    try:
+        if args.impl == "reference":
+            line = run_reference_arm(args, rank, world)
+        else:
+            line = run_gpu_arm(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,189 @@
+/*
+ * mla.h -- C ABI of libmla_b200: Multi-head Latent Attention (MLA) decoding
+ * over a paged latent KV cache on NVIDIA B200 (sm_100a).
+ *
+ * The method (sources by page title and section):
+ *   - every query head attends to ONE shared latent KV head of 576 dims
+ *     (512 "nope" dims followed by 64 decoupled-RoPE dims); V is the first
+ *     d_v dims of the same latent row
+ *       [FlashMLA (AI Wiki), "How does MLA differ from MHA and GQA?"]
+ *   - the cache is paged in 64-token blocks reached through a block table,
+ *     sequences have variable lengths
+ *       [FlashMLA (AI Wiki), "What is FlashMLA?"]
+ *   - the call pair get_mla_metadata(cache_seqlens, s_q*h_q/h_kv, h_kv) ->
+ *     (tile_scheduler_metadata, num_splits), then per layer
+ *     flash_mla_with_kvcache(q, kcache, block_table, cache_seqlens, dv,
+ *     metadata, num_splits, causal) -> (o, lse)
+ *       [FlashMLA Ampere port README, "Usage"]
+ *   - outputs come with their log-sum-exp; token-level sparse decoding takes
+ *     indices (b, s_q, topk) of physical slots (block*64 + offset), -1 =
+ *     invalid, and ignores the block table
+ *       [FlashMLA (AI Wiki), "Interfaces"]
+ *   - the fused kernel applies Q RMSNorm, Q-RoPE, attention, conjugate O-RoPE
+ *     and the FP8 cast in one pass
+ *       [FlashMLA fused norm-RoPE-attention-RoPE-cast kernel card,
+ *        "Arithmetic intensity"; deepseek-ai/FlashMLA README, "News"]
+ *   - the 656-byte FP8 cache row: 512 E4M3 values with one fp32 scale per 128,
+ *     then the 64 RoPE dims in bf16
+ *       [FlashMLA (AI Wiki), "The FP8 and FP4 KV cache"]
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller, unless an
+ *     argument says "host".  The library allocates no device memory; scratch
+ *     space is the caller's `workspace` (size from the *_size queries).
+ *   - Layouts are dense, row-major, innermost dimension last:
+ *       q            [batch, s_q, h_q, 576]        bf16 (16-byte aligned)
+ *       kcache       [num_blocks, 64, 1, 576]      bf16 (16-byte aligned)
+ *       block_table  [batch, max_pages]            int32
+ *       cache_seqlens[batch]                       int32
+ *       out          [batch, s_q, h_q, d_v]        bf16
+ *       lse          [batch, s_q, h_q]             fp32, natural log
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  All GPU work is enqueued asynchronously on it.
+ *   - Every function returns MLA_OK (0) or a negative status.  Arguments are
+ *     validated before anything is launched, so a failed call has enqueued
+ *     no work.  mla_last_error() returns a message for the calling thread's
+ *     most recent failure.
+ *   - An empty row (no visible token) produces O = 0 and LSE = -inf.
+ *   - Cache slots that are not visible to a row must still hold finite
+ *     values: masked tokens are multiplied by a zero probability.
+ */
+#ifndef MLA_B200_H_
+#define MLA_B200_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MLA_API __attribute__((visibility("default")))
+#else
+#define MLA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MLA_OK 0
+#define MLA_ERR_INVALID_ARG (-1) /* null/misaligned pointer, bad size or shape */
+#define MLA_ERR_UNSUPPORTED (-2) /* valid request outside what is built (h_kv != 1, ...) */
+#define MLA_ERR_CUDA (-3)        /* a CUDA runtime call failed; see mla_last_error() */
+#define MLA_ERR_TIMEOUT (-4)     /* a kernel gave up on a bounded wait (mla_device_status) */
+
+/* Message describing the calling thread's most recent failure ("" if none). */
+MLA_API const char* mla_last_error(void);
+
+/* Number of streaming multiprocessors of `device` (host out-pointer). */
+MLA_API int mla_num_sms(int device, int* num_sms);
+
+/* Scheduler partition count for `device`: num_SMs / ceil(heads_per_kv / 64)
+ * / h_kv.  heads_per_kv = s_q * h_q / h_kv is the number of query rows that
+ * share one KV head (the second argument of get_mla_metadata in the port
+ * README's "Usage").  Result in *num_sm_parts (host). */
+MLA_API int mla_num_sm_parts(int device, int heads_per_kv, int h_kv, int* num_sm_parts);
+
+/* Byte sizes of the two scheduler outputs for `batch` sequences and
+ * `num_sm_parts` partitions: metadata int32[num_sm_parts][8] and num_splits
+ * int32[batch + 1] (host out-pointers). */
+MLA_API int mla_metadata_size(int batch, int num_sm_parts, size_t* metadata_bytes,
+                      size_t* num_splits_bytes);
+
+/* Split-KV tile scheduler (the metadata call of the port README's "Usage").
+ * Deals the 128-token tiles of all sequences to `num_sm_parts` partitions of
+ * about equal cost (tiles + a fixed per-segment overhead); each partition
+ * covers one contiguous run of (sequence, tile) pairs.
+ *   cache_seqlens  int32[batch], device
+ *   metadata       int32[num_sm_parts][8], device, written:
+ *                  {begin_seq, begin_tile, end_seq, end_tile (exclusive),
+ *                   split index of begin_seq's segment, 0, 0, 0}
+ *   num_splits     int32[batch + 1], device, written: prefix sums of the
+ *                  number of partitions holding tiles of each sequence
+ * Runs as one small kernel on `stream`; compute it once per decode step and
+ * reuse it for every layer.  heads_per_kv and h_kv are validated only. */
+MLA_API int mla_get_metadata(const int32_t* cache_seqlens, int batch, int heads_per_kv, int h_kv,
+                     int num_sm_parts, int32_t* metadata, int32_t* num_splits, void* stream);
+
+/* The same planner on the host (all three arrays are host pointers); the
+ * result is bit-identical to mla_get_metadata's. */
+MLA_API int mla_get_metadata_host(const int32_t* cache_seqlens, int batch, int heads_per_kv, int h_kv,
+                          int num_sm_parts, int32_t* metadata, int32_t* num_splits);
+
+/* Workspace bytes for mla_decode_fwd / mla_fused_norm_rope_attn_rope_cast:
+ * fp32 partial outputs and LSEs of up to batch + num_sm_parts splits of
+ * `rows_per_kv` (= s_q*h_q) rows of d_v values. */
+MLA_API int mla_workspace_size(int batch, int rows_per_kv, int d_v, int num_sm_parts, size_t* bytes);
+
+/* Dense paged MLA decode, bf16 in, bf16 out + fp32 LSE
+ * (flash_mla_with_kvcache of the port README's "Usage").
+ *   q, kcache, block_table, cache_seqlens, out, lse: see the layouts above.
+ *   max_pages       second dimension of block_table
+ *   num_blocks      first dimension of kcache (block ids must be < num_blocks)
+ *   h_kv            must be 1 (MLA: one latent KV head)
+ *   d_v             512 (V = K[:, :512]) or 576
+ *   softmax_scale   multiplies q.k before the softmax (typically 1/sqrt(576))
+ *   causal          nonzero: query i of s_q sees L - s_q + 1 + i tokens
+ *                   (bottom-right alignment); zero: every query sees L tokens
+ *   metadata, num_splits, num_sm_parts: from mla_get_metadata for the same
+ *                   cache_seqlens and heads_per_kv = s_q*h_q
+ *   workspace       device scratch of >= mla_workspace_size() bytes,
+ *                   16-byte aligned; contents need no initialisation
+ * Launches the decode kernel and the split-combine kernel on `stream`. */
+MLA_API int mla_decode_fwd(const void* q, const void* kcache, const int32_t* block_table, int max_pages,
+                   int num_blocks, const int32_t* cache_seqlens, int batch, int s_q, int h_q,
+                   int h_kv, int d_v, float softmax_scale, int causal, const int32_t* metadata,
+                   const int32_t* num_splits, int num_sm_parts, void* workspace,
+                   size_t workspace_bytes, void* out, float* lse, void* stream);
+
+/* Fused Q RMSNorm -> Q-RoPE -> attention -> conjugate O-RoPE -> FP8 cast,
+ * s_q = 1, d_v = 576 (V is the whole latent row).
+ *   q_raw           [batch, 1, h_q, 576] bf16, before normalisation
+ *   norm_gain       fp32[576], shared by all heads; eps added to mean(x^2)
+ *   rope_base       RoPE base (e.g. 10000); pairs (2k, 2k+1) of dims
+ *                   512..575 rotate by theta_k = pos * base^(-2k/64)
+ *   positions       int32[batch] query positions, or NULL for L - 1
+ *   kcache ...      as in mla_decode_fwd; the cache's RoPE dims are expected
+ *                   to be rotated at their own positions already
+ *   out_e4m3        [batch, 1, h_q, 576] E4M3 codes (OCP FP8), RNE, saturating
+ *   out_scale       fp32[batch, 1, h_q]: absmax(O_row) / 448 (1 for a zero row);
+ *                   O ~= code * scale
+ *   lse             fp32[batch, 1, h_q]
+ *   metadata, num_splits from mla_get_metadata with heads_per_kv = h_q. */
+MLA_API int mla_fused_norm_rope_attn_rope_cast(
+    const void* q_raw, const float* norm_gain, float eps, float rope_base,
+    const int32_t* positions, const void* kcache, const int32_t* block_table, int max_pages,
+    int num_blocks, const int32_t* cache_seqlens, int batch, int h_q, float softmax_scale,
+    const int32_t* metadata, const int32_t* num_splits, int num_sm_parts, void* workspace,
+    size_t workspace_bytes, uint8_t* out_e4m3, float* out_scale, float* lse, void* stream);
+
+/* Workspace bytes for mla_sparse_decode (scheduler tables + split partials). */
+MLA_API int mla_sparse_workspace_size(int batch, int s_q, int h_q, int topk, int d_v, int num_sm_parts,
+                              size_t* bytes);
+
+/* Token-level sparse decode over the 656-byte FP8 latent cache.
+ *   q             [batch, s_q, h_q, 576] bf16
+ *   kcache_fp8    [num_slots, 656] bytes per row: 512 E4M3 codes, 4 fp32
+ *                 scales (one per 128 codes, little-endian), 64 bf16 RoPE dims
+ *   num_slots     rows of kcache_fp8 (num_blocks * 64)
+ *   indices       int32[batch, s_q, topk]: physical slots; -1 (or any value
+ *                 outside [0, num_slots)) marks an unused entry
+ *   d_v           512
+ *   out, lse      [batch, s_q, h_q, d_v] bf16 and [batch, s_q, h_q] fp32
+ *   num_sm_parts  from mla_num_sm_parts(device, h_q, 1)
+ * The scheduling tables are generated inside this call (into workspace). */
+MLA_API int mla_sparse_decode(const void* q, const uint8_t* kcache_fp8, int64_t num_slots,
+                      const int32_t* indices, int topk, int batch, int s_q, int h_q, int d_v,
+                      float softmax_scale, int num_sm_parts, void* workspace,
+                      size_t workspace_bytes, void* out, float* lse, void* stream);
+
+/* Reads the device status word that kernels set when a bounded wait expires
+ * or an out-of-range block id / index is met: 0 = ok, else (code << 16) |
+ * site, code 1 = timeout, 2 = bad index.  Synchronises the device; reset != 0
+ * clears the word afterwards.  Returns MLA_ERR_TIMEOUT if the word holds a
+ * timeout, else MLA_OK. */
+MLA_API int mla_device_status(int* status, int reset);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_B200_H_ */

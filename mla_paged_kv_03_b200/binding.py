@@ -1,0 +1,258 @@
+"""ctypes binding of libmla_b200 (the C ABI in include/mla.h).
+
+Argument marshalling only: every step of the decode path runs in the
+library's CUDA kernels.  torch supplies device memory (outputs, workspace) and
+the current CUDA stream.  There is no fallback: if the shared library is
+missing or was built for another GPU, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmla_b200.so")
+
+MLA_OK = 0
+MLA_ERR_INVALID_ARG = -1
+MLA_ERR_UNSUPPORTED = -2
+MLA_ERR_CUDA = -3
+MLA_ERR_TIMEOUT = -4
+
+D_QK = 576
+EXPORTED = [
+    "mla_last_error", "mla_num_sms", "mla_num_sm_parts", "mla_metadata_size",
+    "mla_get_metadata", "mla_get_metadata_host", "mla_workspace_size", "mla_decode_fwd",
+    "mla_fused_norm_rope_attn_rope_cast", "mla_sparse_workspace_size", "mla_sparse_decode",
+    "mla_device_status",
+]
+
+
+class MLAError(RuntimeError):
+    def __init__(self, code, msg):
+        super().__init__(f"libmla_b200 error {code}: {msg}")
+        self.code = code
+
+
+_lib = None
+
+
+def lib():
+    """Load libmla_b200.so (raises if it is not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m mla_paged_kv_03_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, i64, f32, sz = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float,
+                                 ctypes.c_size_t)
+        szp = ctypes.POINTER(ctypes.c_size_t)
+        ip = ctypes.POINTER(ctypes.c_int)
+        L.mla_last_error.restype = ctypes.c_char_p
+        L.mla_last_error.argtypes = []
+        L.mla_num_sms.argtypes = [i32, ip]
+        L.mla_num_sm_parts.argtypes = [i32, i32, i32, ip]
+        L.mla_metadata_size.argtypes = [i32, i32, szp, szp]
+        L.mla_get_metadata.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp]
+        L.mla_get_metadata_host.argtypes = [vp, i32, i32, i32, i32, vp, vp]
+        L.mla_workspace_size.argtypes = [i32, i32, i32, i32, szp]
+        L.mla_decode_fwd.argtypes = [vp, vp, vp, i32, i32, vp, i32, i32, i32, i32, i32, f32, i32,
+                                     vp, vp, i32, vp, sz, vp, vp, vp]
+        L.mla_fused_norm_rope_attn_rope_cast.argtypes = [
+            vp, vp, f32, f32, vp, vp, vp, i32, i32, vp, i32, i32, f32, vp, vp, i32, vp, sz, vp,
+            vp, vp, vp]
+        L.mla_sparse_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32, szp]
+        L.mla_sparse_decode.argtypes = [vp, vp, i64, vp, i32, i32, i32, i32, i32, f32, i32, vp,
+                                        sz, vp, vp, vp]
+        L.mla_device_status.argtypes = [ip, i32]
+        for name in EXPORTED:
+            if name != "mla_last_error":
+                getattr(L, name).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _check(rc):
+    if rc != MLA_OK:
+        raise MLAError(rc, lib().mla_last_error().decode())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _require(cond, msg):
+    if not cond:
+        raise ValueError(msg)
+
+
+# ---------------------------------------------------------------- scheduler
+
+def mla_num_sm_parts(heads_per_kv: int, h_kv: int = 1, device=None) -> int:
+    dev = torch.cuda.current_device() if device is None else torch.device(device).index or 0
+    out = ctypes.c_int(0)
+    _check(lib().mla_num_sm_parts(dev, int(heads_per_kv), int(h_kv), ctypes.byref(out)))
+    return out.value
+
+
+def mla_get_metadata_host(cache_seqlens, heads_per_kv: int, num_sm_parts: int, h_kv: int = 1):
+    """Host planner: returns (metadata int32[num_sm_parts, 8], num_splits
+    int32[batch + 1]) as CPU tensors."""
+    sl = torch.as_tensor(cache_seqlens, dtype=torch.int32).contiguous().cpu()
+    b = sl.numel()
+    meta = torch.zeros((num_sm_parts, 8), dtype=torch.int32)
+    ns = torch.zeros((b + 1,), dtype=torch.int32)
+    _check(lib().mla_get_metadata_host(_ptr(sl), b, int(heads_per_kv), int(h_kv),
+                                       int(num_sm_parts), _ptr(meta), _ptr(ns)))
+    return meta, ns
+
+
+def mla_get_metadata(cache_seqlens: torch.Tensor, heads_per_kv: int, h_kv: int = 1,
+                     num_sm_parts: Optional[int] = None):
+    """Device planner on the current stream: (metadata, num_splits, num_sm_parts)."""
+    _require(cache_seqlens.is_cuda and cache_seqlens.dtype == torch.int32,
+             "cache_seqlens must be a CUDA int32 tensor")
+    sl = cache_seqlens.contiguous()
+    if num_sm_parts is None:
+        num_sm_parts = mla_num_sm_parts(heads_per_kv, h_kv, sl.device)
+    b = sl.numel()
+    meta = torch.empty((num_sm_parts, 8), dtype=torch.int32, device=sl.device)
+    ns = torch.empty((b + 1,), dtype=torch.int32, device=sl.device)
+    _check(lib().mla_get_metadata(_ptr(sl), b, int(heads_per_kv), int(h_kv), int(num_sm_parts),
+                                  _ptr(meta), _ptr(ns), _stream(sl.device)))
+    return meta, ns, num_sm_parts
+
+
+def mla_workspace_size(batch, rows_per_kv, d_v, num_sm_parts) -> int:
+    out = ctypes.c_size_t(0)
+    _check(lib().mla_workspace_size(int(batch), int(rows_per_kv), int(d_v), int(num_sm_parts),
+                                    ctypes.byref(out)))
+    return out.value
+
+
+def mla_sparse_workspace_size(batch, s_q, h_q, topk, d_v, num_sm_parts) -> int:
+    out = ctypes.c_size_t(0)
+    _check(lib().mla_sparse_workspace_size(int(batch), int(s_q), int(h_q), int(topk), int(d_v),
+                                           int(num_sm_parts), ctypes.byref(out)))
+    return out.value
+
+
+def _workspace(nbytes, device, workspace):
+    if workspace is not None:
+        _require(workspace.numel() * workspace.element_size() >= nbytes, "workspace too small")
+        return workspace
+    return torch.empty((max(nbytes, 256),), dtype=torch.uint8, device=device)
+
+
+# ------------------------------------------------------------------ decode
+
+def mla_decode_fwd(q: torch.Tensor, kcache: torch.Tensor, block_table: torch.Tensor,
+                   cache_seqlens: torch.Tensor, d_v: int, metadata: torch.Tensor,
+                   num_splits: torch.Tensor, num_sm_parts: int, causal: bool = True,
+                   softmax_scale: Optional[float] = None, out=None, lse=None, workspace=None):
+    """Dense paged decode.  q [b, s_q, h_q, 576] bf16, kcache [NB, 64, 1, 576]
+    bf16, block_table [b, max_pages] int32, cache_seqlens [b] int32.
+    Returns (out [b, s_q, h_q, d_v] bf16, lse [b, s_q, h_q] fp32)."""
+    _require(q.dim() == 4 and q.shape[-1] == D_QK and q.dtype == torch.bfloat16,
+             "q must be [b, s_q, h_q, 576] bf16")
+    _require(kcache.dim() == 4 and kcache.shape[1] == 64 and kcache.shape[-1] == D_QK and
+             kcache.dtype == torch.bfloat16, "kcache must be [NB, 64, h_kv, 576] bf16")
+    b, s_q, h_q, _ = q.shape
+    h_kv = kcache.shape[2]
+    q = q.contiguous()
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(D_QK)
+    if out is None:
+        out = torch.empty((b, s_q, h_q, d_v), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((b, s_q, h_q), dtype=torch.float32, device=q.device)
+    ws_bytes = mla_workspace_size(b, s_q * h_q, d_v, num_sm_parts)
+    ws = _workspace(ws_bytes, q.device, workspace)
+    bt = block_table.contiguous()
+    _check(lib().mla_decode_fwd(
+        _ptr(q), _ptr(kcache), _ptr(bt), bt.shape[1], kcache.shape[0], _ptr(cache_seqlens), b,
+        s_q, h_q, h_kv, int(d_v), float(softmax_scale), int(bool(causal)), _ptr(metadata),
+        _ptr(num_splits), int(num_sm_parts), _ptr(ws), ws.numel(), _ptr(out), _ptr(lse),
+        _stream(q.device)))
+    return out, lse
+
+
+def mla_fused_norm_rope_attn_rope_cast(q_raw, norm_gain, eps, rope_base, kcache, block_table,
+                                       cache_seqlens, metadata, num_splits, num_sm_parts,
+                                       softmax_scale=None, positions=None, out=None,
+                                       out_scale=None, lse=None, workspace=None):
+    """Fused RMSNorm -> Q-RoPE -> attention -> conjugate O-RoPE -> E4M3 cast.
+    Returns (codes uint8 [b, 1, h_q, 576], scale fp32 [b, 1, h_q], lse)."""
+    _require(q_raw.dim() == 4 and q_raw.shape[1] == 1 and q_raw.shape[-1] == D_QK and
+             q_raw.dtype == torch.bfloat16, "q_raw must be [b, 1, h_q, 576] bf16")
+    b, _, h_q, _ = q_raw.shape
+    q_raw = q_raw.contiguous()
+    gain = norm_gain.to(torch.float32).contiguous()
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(D_QK)
+    dev = q_raw.device
+    if out is None:
+        out = torch.empty((b, 1, h_q, D_QK), dtype=torch.uint8, device=dev)
+    if out_scale is None:
+        out_scale = torch.empty((b, 1, h_q), dtype=torch.float32, device=dev)
+    if lse is None:
+        lse = torch.empty((b, 1, h_q), dtype=torch.float32, device=dev)
+    ws = _workspace(mla_workspace_size(b, h_q, D_QK, num_sm_parts), dev, workspace)
+    bt = block_table.contiguous()
+    pos = None if positions is None else positions.to(torch.int32).contiguous()
+    _check(lib().mla_fused_norm_rope_attn_rope_cast(
+        _ptr(q_raw), _ptr(gain), float(eps), float(rope_base), _ptr(pos), _ptr(kcache), _ptr(bt),
+        bt.shape[1], kcache.shape[0], _ptr(cache_seqlens), b, h_q, float(softmax_scale),
+        _ptr(metadata), _ptr(num_splits), int(num_sm_parts), _ptr(ws), ws.numel(), _ptr(out),
+        _ptr(out_scale), _ptr(lse), _stream(dev)))
+    return out, out_scale, lse
+
+
+def mla_sparse_decode(q, kcache_fp8, indices, d_v=512, softmax_scale=None, num_sm_parts=None,
+                      out=None, lse=None, workspace=None):
+    """Token-level sparse decode over the 656-byte FP8 cache.
+    q [b, s_q, h_q, 576] bf16; kcache_fp8 [..., 656] uint8; indices
+    [b, s_q, topk] int32 physical slots (-1 = unused).  Returns (out, lse)."""
+    _require(q.dim() == 4 and q.shape[-1] == D_QK and q.dtype == torch.bfloat16,
+             "q must be [b, s_q, h_q, 576] bf16")
+    _require(kcache_fp8.dtype == torch.uint8 and kcache_fp8.shape[-1] == 656,
+             "kcache_fp8 must be uint8 [..., 656]")
+    b, s_q, h_q, _ = q.shape
+    q = q.contiguous()
+    idx = indices.to(torch.int32).contiguous()
+    topk = idx.shape[-1]
+    num_slots = kcache_fp8.numel() // 656
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(D_QK)
+    if num_sm_parts is None:
+        num_sm_parts = mla_num_sm_parts(h_q, 1, q.device)
+    dev = q.device
+    if out is None:
+        out = torch.empty((b, s_q, h_q, d_v), dtype=torch.bfloat16, device=dev)
+    if lse is None:
+        lse = torch.empty((b, s_q, h_q), dtype=torch.float32, device=dev)
+    ws = _workspace(mla_sparse_workspace_size(b, s_q, h_q, topk, d_v, num_sm_parts), dev,
+                    workspace)
+    _check(lib().mla_sparse_decode(
+        _ptr(q), _ptr(kcache_fp8), num_slots, _ptr(idx), topk, b, s_q, h_q, int(d_v),
+        float(softmax_scale), int(num_sm_parts), _ptr(ws), ws.numel(), _ptr(out), _ptr(lse),
+        _stream(dev)))
+    return out, lse
+
+
+def device_status(reset: bool = True) -> int:
+    """Device status word (0 = ok); synchronises the device."""
+    v = ctypes.c_int(0)
+    rc = lib().mla_device_status(ctypes.byref(v), int(bool(reset)))
+    if rc not in (MLA_OK, MLA_ERR_TIMEOUT):
+        _check(rc)
+    return v.value

@@ -1,0 +1,833 @@
+// decode_kernel.cuh -- persistent, warp-specialised sm_100a MLA decode kernel.
+//
+// What it computes, per query row r of a sequence b (one shared latent KV head
+// of 576 dims, V = first d_v dims of the same row):
+//   O[r] = softmax(scale * Q[r] K^T) V ,  LSE[r] = log sum exp(scale * Q[r] K^T)
+// [FlashMLA (AI Wiki), "How does MLA differ from MHA and GQA?", "How is
+//  FlashMLA designed?", "Interfaces"]
+//
+// Orientation.  All query rows (s_q * h_q, up to 64 per CTA) share one KV
+// head, so the tensor-core tile puts TOKENS on the M axis and query rows on N:
+//   S^T[128 tok, 64 rows]  = K_tile[128 tok, 576] . Q[64 rows, 576]^T   (QK)
+//   O^T[128 d,   64 rows] += V^T[128 d, 128 tok] . P^T[64 rows, 128 tok]^T (PV)
+// so M = 128 is always full even for 16 or 32 query rows.  S^T and O^T live in
+// TMEM (fp32); the K tile in shared memory serves as the K-major A operand of
+// QK and, read through an MN-major descriptor, as V^T for PV.
+//
+// Memory pipeline.  The cache is read in 128-token tiles (two 64-token pages
+// found through the block table) split into 64-dim, 128-byte-wide chunks that
+// TMA writes in the 128B-swizzled layout.  A ring of 32 KB "pair slots" (two
+// chunks each) is consumed in a fixed order QK(0), QK(1), PV(0), QK(2), PV(1),
+// ..., so the softmax of tile k overlaps QK of tile k+1.  V chunks are fetched
+// a second time for PV (an L2 hit) instead of holding a whole 144 KB tile.
+//
+// Roles (warps):  0 = loader (TMA),  1 = MMA issuer + TMEM owner,
+//   2..5 = softmax warpgroup (one thread per token lane of the tile; also the
+//   epilogue and, for the fused variant, the Q RMSNorm + RoPE prologue),
+//   6..9 = FP8 gather/dequant warpgroup (sparse variant only).
+//
+// Softmax uses a lazily updated per-row reference max m: scores are
+// exponentiated against m until some score exceeds m by more than 8 (log2
+// units); only then is m raised and O, l rescaled.  The result is exact
+// either way because O and l are formed against the same m (the "skip scale"
+// idea of [FlashMLA (AI Wiki), "The Ascend kernel deep-dive"]).
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cstdint>
+
+#include "mla_common.h"
+#include "ptx.cuh"
+
+namespace mla {
+
+enum Mode : int { kDense = 0, kFused = 1, kSparse = 2 };
+
+struct DecodeParams {
+  int batch;       // sequences (dense/fused) or (sequence, query) pairs (sparse)
+  int s_q, h_q;    // query tokens per sequence and heads
+  int R;           // rows sharing one KV head: s_q*h_q (dense/fused), h_q (sparse)
+  int d_v;         // 512 or 576
+  int n_groups;    // ceil(R / 64)
+  int num_parts;   // scheduler parts; grid = num_parts * n_groups
+  int num_blocks;  // cache blocks (dense/fused)
+  int max_pages;
+  int causal;
+  int always_partial;  // write split partials even for unsplit sequences (fused)
+  float scale_log2;    // softmax_scale * log2(e)
+  const int32_t* block_table;
+  const int32_t* seqlens;     // per sequence (dense/fused)
+  const int32_t* metadata;    // [num_parts][8]
+  const int32_t* num_splits;  // [batch + 1] prefix sums
+  __nv_bfloat16* out;         // [batch*R, d_v] bf16 (unsplit rows)
+  float* lse;                 // [batch*R]
+  float* ws_o;                // [total_splits, R, d_v] fp32 partial O (normalised)
+  float* ws_lse;              // [total_splits, R]
+  // fused prologue
+  const __nv_bfloat16* q_raw;  // [batch, 1, h_q, 576]
+  const float* gain;           // [576]
+  float eps;
+  float rope_base;
+  const int32_t* positions;  // nullable: position = L - 1
+  double inv_freq[kRope / 2];  // base^(-2k/64), computed on the host in fp64
+  // sparse
+  const uint8_t* cache656;  // [num_slots, 656]
+  const int32_t* indices;   // [batch(pairs), topk]
+  int topk;
+  long long num_slots;
+};
+
+namespace cfg {
+constexpr int kQBytes = kNumChunks * kRowsPerCta * 128;  // 73728
+constexpr int kSubChunk = kTileT * 128;                  // 16384: [128 tok][64 d] bf16
+constexpr int kPairBytes = 2 * kSubChunk;                // 32768
+constexpr int kNPair = 3;                                // ring depth (pair slots)
+constexpr int kNP = 2;                                   // P buffer regions
+constexpr int kPBytes = kTileT * 128;                    // [128 tok][64 rows] bf16
+constexpr int kQOff = 0;
+constexpr int kRingOff = kQOff + kQBytes;
+constexpr int kPOff = kRingOff + kNPair * kPairBytes;
+constexpr int kBarOff = kPOff + kNP * kPBytes;
+constexpr int kMiscBytes = 4096;
+constexpr int kSmemBytes = kBarOff + kMiscBytes + 1024;  // + alignment slack
+constexpr int kTmemCols = 512;
+constexpr int kSCol = 0;     // S^T buffers at cols [0,64) and [64,128)
+constexpr int kOCol = 128;   // O^T chunk c at cols 128 + 64c (c < 5)
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+}  // namespace cfg
+
+// Softmax warpgroups (32 query-row columns each) and the named barrier that
+// spans all of them (ids 1..6 are per-group).
+constexpr int kSoftmaxGroups = 2;
+constexpr int kBarAllSoftmax = 7;
+constexpr int kGatherThreads = 64;  // sparse: each gather thread fills two token rows
+
+template <int kMode>
+struct Threads {
+  // loader + MMA warps, softmax groups, and for sparse two gather warps
+  static constexpr int value = 64 + 128 * kSoftmaxGroups + (kMode == kSparse ? kGatherThreads : 0);
+};
+
+// Shared-memory control block (at kBarOff).
+struct __align__(8) Ctrl {
+  uint64_t slot_full[cfg::kNPair];
+  uint64_t slot_empty[cfg::kNPair];
+  uint64_t q_full, q_empty;
+  uint64_t s_full[2], s_empty[2];
+  uint64_t p_full[cfg::kNP], p_empty[cfg::kNP];
+  uint64_t o_free;
+  uint64_t drain;
+  uint64_t rope_full;
+  uint32_t tmem_base;
+  uint32_t pad;
+  float red[8][32];     // cross-warp reduction scratch [group*4 + warp][column]
+  float m[64];          // per-column reference max (log2 domain)
+  float alpha[64];      // per-column rescale factor, then 1/l in the epilogue
+  int lim[64];          // per-column visible-token limit of the current unit
+  float rope_cs[32][2]; // cos/sin of the current unit's query position
+};
+static_assert(sizeof(Ctrl) <= cfg::kMiscBytes, "control block too large");
+
+struct Unit {
+  int b, lo, hi, split, nsplit, L;
+};
+
+// Iterates the (sequence, tile-range) segments of one scheduler part.
+struct UnitIter {
+  int b, b_first, b_end, t_begin, t_end, s_begin;
+  __device__ void init(const int32_t* m) {
+    b = b_first = m[0];
+    t_begin = m[1];
+    b_end = m[2];
+    t_end = m[3];
+    s_begin = m[4];
+  }
+  template <int kMode>
+  __device__ bool next(const DecodeParams& P, Unit& u) {
+    while (b <= b_end) {
+      const int bb = b++;
+      const int L = (kMode == kSparse) ? P.topk : P.seqlens[bb];
+      const int lo = (bb == b_first) ? t_begin : 0;
+      const int hi = (bb == b_end) ? t_end : tiles_of(L);
+      if (lo >= hi) continue;
+      u.b = bb;
+      u.lo = lo;
+      u.hi = hi;
+      u.split = (bb == b_first) ? s_begin : 0;
+      u.nsplit = P.num_splits[bb + 1] - P.num_splits[bb];
+      u.L = L;
+      return true;
+    }
+    return false;
+  }
+};
+
+// Warpgroup-uniform bounded wait: every thread of the 128-thread group waits,
+// then the group agrees (barrier AND-reduction) so that all threads take the
+// same path even if one of them timed out.
+__device__ __forceinline__ bool wg_wait(uint64_t* bar, uint32_t parity, int site, int bar_id,
+                                        int nthreads = 128) {
+  const bool mine = ptx::mbar_wait(bar, parity, site);
+  uint32_t all;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.b32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(all)
+      : "r"(mine ? 1 : 0), "r"(bar_id), "r"(nthreads));
+  return all != 0;
+}
+
+// cos/sin of theta = pos * inv_freq: the angle is formed and reduced modulo
+// 2*pi in fp64 (|theta| < 2^31 keeps the reduced angle accurate to ~1e-9), the
+// reduced angle in [-pi, pi] is then evaluated in fp32.
+__device__ __forceinline__ void rope_sincos(double pos, double inv_freq, float* sn, float* cs) {
+  const double kTwoPi = 6.283185307179586476925286766559;
+  const double theta = pos * inv_freq;
+  const double r = fma(-rint(theta * (1.0 / kTwoPi)), kTwoPi, theta);
+  __sincosf(static_cast<float>(r), sn, cs);
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ int clamp_block(int blk, int num_blocks) {
+  if (blk < 0 || blk >= num_blocks) {
+    ptx::set_error(MLA_DEVERR_BAD_INDEX, 0x51);
+    return 0;
+  }
+  return blk;
+}
+
+// --------------------------------------------------------------------------
+// Sparse gather: dequantise one token's chunks of a pair slot into the
+// swizzled bf16 layout.  Row layout: [512 e4m3][4 fp32 scales][64 bf16].
+// [FlashMLA (AI Wiki), "The FP8 and FP4 KV cache"]
+__device__ __forceinline__ void sparse_fill_pair(uint8_t* slot, int t, const uint8_t* row,
+                                                 bool valid, int pair) {
+  const int sw = t & 7;
+  uint8_t* rowbase = slot + t * 128;
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const int c = 2 * pair + j;
+    if (c >= kNumChunks) break;
+    uint8_t* dst = rowbase + j * cfg::kSubChunk;
+    if (!valid) {
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        *reinterpret_cast<uint4*>(dst + ((u ^ sw) << 4)) = make_uint4(0, 0, 0, 0);
+      continue;
+    }
+    if (c == kNumChunks - 1) {
+      // RoPE dims: bf16 copy
+      const uint4* src = reinterpret_cast<const uint4*>(row + kNope + 16);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) *reinterpret_cast<uint4*>(dst + ((u ^ sw) << 4)) = __ldg(src + u);
+    } else {
+      const float sc = __ldg(reinterpret_cast<const float*>(row + kNope) + (c >> 1));
+      const uint4* src = reinterpret_cast<const uint4*>(row + c * 64);
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const uint4 w = __ldg(src + v);  // 16 codes -> two 16-byte output units
+        const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+        uint32_t o[8];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint16_t lo16 = static_cast<uint16_t>(words[q] & 0xFFFF);
+          const uint16_t hi16 = static_cast<uint16_t>(words[q] >> 16);
+          uint32_t h0, h1;
+          asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h0) : "h"(lo16));
+          asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h1) : "h"(hi16));
+          const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&h0));
+          const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&h1));
+          o[2 * q] = ptx::pack_bf16x2(f0.x * sc, f0.y * sc);
+          o[2 * q + 1] = ptx::pack_bf16x2(f1.x * sc, f1.y * sc);
+        }
+        const int u0 = 2 * v, u1 = 2 * v + 1;
+        *reinterpret_cast<uint4*>(dst + ((u0 ^ sw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+        *reinterpret_cast<uint4*>(dst + ((u1 ^ sw) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+      }
+    }
+  }
+}
+
+// --------------------------------------------------------------------------
+template <int kMode>
+__global__ void __launch_bounds__(Threads<kMode>::value, 1)
+    mla_decode_kernel(const __grid_constant__ CUtensorMap tm_q,
+                      const __grid_constant__ CUtensorMap tm_kv, const DecodeParams P) {
+  using namespace cfg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sQ = smem + kQOff;
+  uint8_t* sRing = smem + kRingOff;
+  uint8_t* sP = smem + kPOff;
+  Ctrl& C = *reinterpret_cast<Ctrl*>(smem + kBarOff);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int part = blockIdx.x / P.n_groups;
+  const int grp = blockIdx.x % P.n_groups;
+  const int nv_pairs = (P.d_v + 127) / 128;  // PV pair slots per tile
+
+  // P^T buffers: two alternating bf16 buffers, or (fused variant) one buffer
+  // holding P as a bf16 hi/lo pair so that PV sees P to ~16 bits.
+  constexpr bool kPSplit = (kMode == kFused);
+  constexpr int NPm = kPSplit ? 1 : kNP;
+
+  const int32_t* meta = P.metadata + part * kMetaInts;
+  if (meta[0] > meta[2]) return;  // empty part: nothing to do (uniform exit)
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kNPair; ++i) {
+      ptx::mbar_init(&C.slot_full[i], kMode == kSparse ? kGatherThreads : 1);
+      ptx::mbar_init(&C.slot_empty[i], 1);
+    }
+    ptx::mbar_init(&C.q_full, kMode == kFused ? 128 * kSoftmaxGroups : 1);
+    ptx::mbar_init(&C.q_empty, 1);
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(&C.s_full[i], 1);
+      ptx::mbar_init(&C.s_empty[i], 128 * kSoftmaxGroups);
+    }
+    for (int i = 0; i < kNP; ++i) {
+      ptx::mbar_init(&C.p_full[i], 128 * kSoftmaxGroups);
+      ptx::mbar_init(&C.p_empty[i], 1);
+    }
+    ptx::mbar_init(&C.o_free, 128 * kSoftmaxGroups);
+    ptx::mbar_init(&C.drain, 1);
+    ptx::mbar_init(&C.rope_full, 32);
+    ptx::fence_mbar_init();
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(&C.tmem_base, kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    if (kMode != kFused) ptx::prefetch_tmap(&tm_q);
+    if (kMode != kSparse) ptx::prefetch_tmap(&tm_kv);
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = C.tmem_base;
+
+  UnitIter it;
+  it.init(meta);
+
+  if (warp == 0) {
+    // ============================== loader ==============================
+    // Lane 0 issues the TMA loads.  For the fused variant the whole warp also
+    // computes, per unit, the cos/sin table of the query position:
+    // theta_k = pos * base^(-2k/64), pos = positions[b] or L - 1.  A unit's
+    // table may be overwritten once the previous unit's QK finished
+    // (q_empty), which implies the prologue that read it is done.
+    uint32_t ring_it = 0;
+    int u_idx = 0;
+    Unit u;
+    bool ok = true;
+    auto load_pair = [&](const Unit& un, int tile, int pair) -> bool {
+      const int slot = ring_it % kNPair;
+      const uint32_t round = ring_it / kNPair;
+      ++ring_it;
+      if (!ptx::mbar_wait(&C.slot_empty[slot], (round & 1) ^ 1, 0x01)) return false;
+      const int c0 = 2 * pair;
+      const int nch = (c0 + 1 < kNumChunks) ? 2 : 1;
+      ptx::mbar_arrive_expect_tx(&C.slot_full[slot], nch * kSubChunk);
+      const int tok0 = tile * kTileT;
+      int npg = (un.L + kPage - 1) / kPage;
+      if (npg > P.max_pages) {
+        ptx::set_error(MLA_DEVERR_BAD_INDEX, 0x05);
+        npg = P.max_pages;
+      }
+      const int p0 = tok0 / kPage;
+      int blk0 = p0 < npg ? P.block_table[(size_t)un.b * P.max_pages + p0] : 0;
+      int blk1 = (p0 + 1 < npg) ? P.block_table[(size_t)un.b * P.max_pages + p0 + 1] : blk0;
+      blk0 = clamp_block(blk0, P.num_blocks);
+      blk1 = clamp_block(blk1, P.num_blocks);
+      uint8_t* dst = sRing + slot * kPairBytes;
+      for (int j = 0; j < nch; ++j) {
+        const int x = (c0 + j) * kChunkD;
+        ptx::tma_load_2d(dst + j * kSubChunk, &tm_kv, &C.slot_full[slot], x, blk0 * kPage);
+        ptx::tma_load_2d(dst + j * kSubChunk + kSubChunk / 2, &tm_kv, &C.slot_full[slot], x,
+                         blk1 * kPage);
+      }
+      return true;
+    };
+    while (ok && it.template next<kMode>(P, u)) {
+      if (kMode == kFused) {
+        ok = ptx::mbar_wait(&C.q_empty, (u_idx & 1) ^ 1, 0x06);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        const double pos =
+            P.positions ? static_cast<double>(P.positions[u.b]) : static_cast<double>(u.L - 1);
+        float sn, cs;
+        rope_sincos(pos, P.inv_freq[lane], &sn, &cs);
+        C.rope_cs[lane][0] = cs;
+        C.rope_cs[lane][1] = sn;
+        ptx::mbar_arrive(&C.rope_full);
+      }
+      if (lane == 0) {
+        if (kMode != kFused) {
+          // Q rows [64*grp, 64*grp+64) of this sequence (or query pair)
+          ok = ptx::mbar_wait(&C.q_empty, (u_idx & 1) ^ 1, 0x02);
+          if (ok) {
+            ptx::mbar_arrive_expect_tx(&C.q_full, kQBytes);
+            const int row0 = u.b * P.R + grp * kRowsPerCta;
+            for (int c = 0; c < kNumChunks; ++c)
+              ptx::tma_load_2d(sQ + c * (kRowsPerCta * 128), &tm_q, &C.q_full, c * kChunkD, row0);
+          }
+        }
+        if (kMode != kSparse && ok) {
+          const int n = u.hi - u.lo;
+          for (int k = 0; k < n && ok; ++k) {
+            for (int pr = 0; pr < 5 && ok; ++pr) ok = load_pair(u, u.lo + k, pr);
+            if (k >= 1)
+              for (int pr = 0; pr < nv_pairs && ok; ++pr) ok = load_pair(u, u.lo + k - 1, pr);
+          }
+          for (int pr = 0; pr < nv_pairs && ok; ++pr) ok = load_pair(u, u.hi - 1, pr);
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      ++u_idx;
+    }
+    if (lane == 0) {
+      // Never leave a TMA write in flight: wait (bounded) for the last load
+      // issued into each slot.  In the normal path these phases completed
+      // long ago and the waits return at once.
+      for (int i = 0; i < kNPair && i < static_cast<int>(ring_it); ++i) {
+        const uint32_t last = ring_it - 1 - i;
+        ptx::mbar_wait(&C.slot_full[last % kNPair], (last / kNPair) & 1, 0x03);
+      }
+      if (kMode != kFused && u_idx > 0) ptx::mbar_wait(&C.q_full, (u_idx - 1) & 1, 0x04);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ============================== MMA issuer ==============================
+    if (lane == 0) {
+      const uint32_t idesc_qk = ptx::idesc_bf16_f32(128, kRowsPerCta, 0, 0);
+      const uint32_t idesc_pv = ptx::idesc_bf16_f32(128, kRowsPerCta, 1, 1);
+      const uint32_t q_addr = ptx::smem_u32(sQ);
+      const uint32_t ring_addr = ptx::smem_u32(sRing);
+      const uint32_t p_addr = ptx::smem_u32(sP);
+      uint32_t ring_it = 0, gt = 0;
+      int u_idx = 0;
+      Unit u;
+      bool ok = true;
+      auto wait_slot = [&](uint32_t& addr) -> int {
+        const int slot = ring_it % kNPair;
+        const uint32_t round = ring_it / kNPair;
+        ++ring_it;
+        if (!ptx::mbar_wait(&C.slot_full[slot], round & 1, 0x11)) return -1;
+        ptx::tc_fence_after();
+        addr = ring_addr + slot * kPairBytes;
+        return slot;
+      };
+      auto do_qk = [&](uint32_t g) -> bool {
+        const int sb = g & 1;
+        if (!ptx::mbar_wait(&C.s_empty[sb], ((g >> 1) & 1) ^ 1, 0x12)) return false;
+        ptx::tc_fence_after();
+        const uint32_t d_tmem = tmem + kSCol + sb * kRowsPerCta;
+        for (int pr = 0; pr < 5; ++pr) {
+          uint32_t a0;
+          const int slot = wait_slot(a0);
+          if (slot < 0) return false;
+          for (int j = 0; j < 2; ++j) {
+            const int c = 2 * pr + j;
+            if (c >= kNumChunks) break;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t ad = ptx::smem_desc(a0 + j * kSubChunk + kk * 32, 16, 1024,
+                                                 ptx::kLayoutSW128);
+              const uint64_t bd = ptx::smem_desc(q_addr + c * (kRowsPerCta * 128) + kk * 32, 16,
+                                                 1024, ptx::kLayoutSW128);
+              ptx::umma_f16_ss(d_tmem, ad, bd, idesc_qk, (c | kk) ? 1u : 0u);
+            }
+          }
+          ptx::umma_commit(&C.slot_empty[slot]);
+        }
+        ptx::umma_commit(&C.s_full[sb]);
+        return true;
+      };
+      auto do_pv = [&](uint32_t g, bool first_of_unit) -> bool {
+        const int pb = g % NPm;
+        if (!ptx::mbar_wait(&C.p_full[pb], (g / NPm) & 1, 0x13)) return false;
+        ptx::tc_fence_after();
+        const uint32_t pbuf = p_addr + pb * kPBytes;
+        for (int pr = 0; pr < nv_pairs; ++pr) {
+          uint32_t a0;
+          const int slot = wait_slot(a0);
+          if (slot < 0) return false;
+          const uint32_t d_tmem = tmem + kOCol + pr * kRowsPerCta;
+#pragma unroll
+          for (int kk = 0; kk < kTileT / 16; ++kk) {
+            const uint64_t ad =
+                ptx::smem_desc(a0 + kk * 2048, kSubChunk, 1024, ptx::kLayoutSW128);
+            const uint64_t bd = ptx::smem_desc(pbuf + kk * 2048, 16, 1024, ptx::kLayoutSW128);
+            ptx::umma_f16_ss(d_tmem, ad, bd, idesc_pv, (first_of_unit && kk == 0) ? 0u : 1u);
+            if (kPSplit) {  // + V^T . P_lo^T
+              const uint64_t bl =
+                  ptx::smem_desc(pbuf + kPBytes + kk * 2048, 16, 1024, ptx::kLayoutSW128);
+              ptx::umma_f16_ss(d_tmem, ad, bl, idesc_pv, 1u);
+            }
+          }
+          ptx::umma_commit(&C.slot_empty[slot]);
+        }
+        ptx::umma_commit(&C.p_empty[pb]);
+        return true;
+      };
+      while (ok && it.template next<kMode>(P, u)) {
+        if (!ptx::mbar_wait(&C.q_full, u_idx & 1, 0x14)) break;
+        ptx::tc_fence_after();
+        const int n = u.hi - u.lo;
+        const uint32_t g0 = gt;
+        for (int k = 0; k < n && ok; ++k) {
+          ok = do_qk(g0 + k);
+          if (ok && k == n - 1) ptx::umma_commit(&C.q_empty);
+          if (ok && k >= 1) {
+            if (k == 1 && !ptx::mbar_wait(&C.o_free, (u_idx & 1) ^ 1, 0x15)) { ok = false; break; }
+            ok = do_pv(g0 + k - 1, k == 1);
+          }
+        }
+        if (ok) {
+          if (n == 1 && !ptx::mbar_wait(&C.o_free, (u_idx & 1) ^ 1, 0x16)) { ok = false; break; }
+          ok = do_pv(g0 + n - 1, n == 1);
+        }
+        gt += n;
+        ++u_idx;
+      }
+      // Drain the tensor pipe before TMEM is released.
+      ptx::umma_commit(&C.drain);
+      ptx::mbar_wait(&C.drain, 0, 0x17);
+    }
+    __syncwarp();
+  } else if (warp >= 2 && warp < 2 + 4 * kSoftmaxGroups) {
+    // ============================== softmax / epilogue ==============================
+    // Two warpgroups; group sg owns query-row columns [32*sg, 32*sg + 32).
+    const int sg = (warp - 2) >> 2;
+    const int cb = 32 * sg;               // first column of this group
+    const int wq = warp & 3;              // TMEM lane quarter of this warp
+    const int t = wq * 32 + lane;         // token lane within the tile (0..127)
+    const int wt = (threadIdx.x - 64) & 127;  // thread index within the warpgroup
+    const int bar_sync = 1 + 3 * sg, bar_or = 2 + 3 * sg, bar_and = 3 + 3 * sg;
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    uint32_t gt = 0;
+    int u_idx = 0;
+    Unit u;
+    bool ok = true;
+    while (ok && it.template next<kMode>(P, u)) {
+      const int n = u.hi - u.lo;
+      // ---- per-unit column limits (visible tokens of each query row)
+      if (wt < 32) {
+        const int rg = grp * kRowsPerCta + cb + wt;
+        int lim = 0;
+        if (rg < P.R) {
+          if (kMode == kSparse || !P.causal) {
+            lim = u.L;
+          } else {
+            lim = u.L - P.s_q + 1 + rg / P.h_q;
+            lim = lim < 0 ? 0 : lim;
+          }
+        }
+        C.lim[cb + wt] = lim;
+        C.m[cb + wt] = -INFINITY;
+      }
+      // ---- fused prologue: RMSNorm + Q-RoPE into the swizzled Q tile
+      if (kMode == kFused) {
+        // Q buffer free (previous unit's QK done) and this unit's RoPE table
+        // written by the loader warp.
+        if (!wg_wait(&C.q_empty, (u_idx & 1) ^ 1, 0x21, kBarAllSoftmax, 128 * kSoftmaxGroups) ||
+            !wg_wait(&C.rope_full, u_idx & 1, 0x26, kBarAllSoftmax, 128 * kSoftmaxGroups)) {
+          ok = false;
+          break;
+        }
+        const int wl = (threadIdx.x - 64) >> 5;  // warp within both groups (0..7)
+        for (int r = wl; r < kRowsPerCta; r += 4 * kSoftmaxGroups) {
+          const int rg = grp * kRowsPerCta + r;
+          const bool valid = rg < P.R;
+          const __nv_bfloat16* src = P.q_raw + ((size_t)u.b * P.R + (valid ? rg : 0)) * kD;
+          float x[3][8];
+          float ss = 0.f;
+    #pragma unroll
+          for (int j = 0; j < 3; ++j) {
+            const int uu = lane + 32 * j;
+            if (uu < kD / 8) {
+              const uint4 w = *reinterpret_cast<const uint4*>(src + uu * 8);
+              const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
+    #pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(h[e]);
+                x[j][2 * e] = f.x;
+                x[j][2 * e + 1] = f.y;
+                ss += f.x * f.x + f.y * f.y;
+              }
+            }
+          }
+    #pragma unroll
+          for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+          const float inv = valid ? 1.0f / sqrtf(ss / static_cast<float>(kD) + P.eps) : 0.f;
+    #pragma unroll
+          for (int j = 0; j < 3; ++j) {
+            const int uu = lane + 32 * j;
+            if (uu < kD / 8) {
+              float y[8];
+    #pragma unroll
+              for (int e = 0; e < 8; ++e) y[e] = x[j][e] * inv * __ldg(P.gain + uu * 8 + e);
+              if (uu >= kNope / 8) {
+    #pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const int k = (uu * 8 - kNope) / 2 + e;
+                  const float c = C.rope_cs[k][0], sn = C.rope_cs[k][1];
+                  const float a = y[2 * e], bq = y[2 * e + 1];
+                  y[2 * e] = a * c - bq * sn;
+                  y[2 * e + 1] = a * sn + bq * c;
+                }
+              }
+              uint4 o;
+              o.x = ptx::pack_bf16x2(y[0], y[1]);
+              o.y = ptx::pack_bf16x2(y[2], y[3]);
+              o.z = ptx::pack_bf16x2(y[4], y[5]);
+              o.w = ptx::pack_bf16x2(y[6], y[7]);
+              const int c = uu >> 3, unit = uu & 7;
+              *reinterpret_cast<uint4*>(sQ + c * (kRowsPerCta * 128) + r * 128 +
+                                        ((unit ^ (r & 7)) << 4)) = o;
+            }
+          }
+        }
+        ptx::fence_proxy_async_smem();
+        ptx::mbar_arrive(&C.q_full);
+      }
+      ptx::named_bar_sync(bar_sync, 128);  // C.lim, C.m of this group visible
+
+      int min_lim = 1 << 30;
+      for (int c = 0; c < 32; ++c) {
+        const int rg = grp * kRowsPerCta + cb + c;
+        if (rg < P.R && C.lim[cb + c] < min_lim) min_lim = C.lim[cb + c];
+      }
+      float lsum[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) lsum[c] = 0.f;
+
+      for (int k = 0; k < n && ok; ++k) {
+        const uint32_t g = gt + k;
+        const int sb = g & 1;
+        if (!wg_wait(&C.s_full[sb], (g >> 1) & 1, 0x22, bar_and)) { ok = false; break; }
+        ptx::tc_fence_after();
+        float x[32];
+        ptx::tmem_ld32(lane_addr + kSCol + sb * kRowsPerCta + cb, x);
+        ptx::tmem_ld_wait();
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(&C.s_empty[sb]);
+
+        const int tile_tok0 = (u.lo + k) * kTileT;
+        const int T = tile_tok0 + t;
+        bool tok_valid = true;
+        if (kMode == kSparse) {
+          const int idx = (T < P.topk) ? __ldg(P.indices + (size_t)u.b * P.topk + T) : -1;
+          tok_valid = idx >= 0 && static_cast<long long>(idx) < P.num_slots;
+        }
+        const bool need_mask = (tile_tok0 + kTileT > min_lim) || !tok_valid;
+        int need = 0;
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          float v = x[c] * P.scale_log2;
+          if (need_mask && (!tok_valid || T >= C.lim[cb + c])) v = -INFINITY;
+          x[c] = v;
+          need |= (v > C.m[cb + c] + kRescaleThreshold);
+        }
+        uint32_t any_need;
+        asm volatile(
+            "{\n\t.reg .pred p, q;\n\t"
+            "setp.ne.b32 p, %1, 0;\n\t"
+            "bar.red.or.pred q, %2, 128, p;\n\t"
+            "selp.u32 %0, 1, 0, q;\n\t}"
+            : "=r"(any_need)
+            : "r"(need), "r"(bar_or));
+        if (any_need) {
+          // Raise the reference max to this tile's exact column max.
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            float v = x[c];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+            if (lane == 0) C.red[4 * sg + wq][c] = v;
+          }
+          ptx::named_bar_sync(bar_sync, 128);
+          if (wt < 32) {
+            const float tm = fmaxf(fmaxf(C.red[4 * sg][wt], C.red[4 * sg + 1][wt]),
+                                   fmaxf(C.red[4 * sg + 2][wt], C.red[4 * sg + 3][wt]));
+            const float mo = C.m[cb + wt];
+            const float mn = fmaxf(mo, tm);
+            C.alpha[cb + wt] = (mn == -INFINITY) ? 1.f : ex2(mo - mn);
+            C.m[cb + wt] = mn;
+          }
+          ptx::named_bar_sync(bar_sync, 128);
+#pragma unroll
+          for (int c = 0; c < 32; ++c) lsum[c] *= C.alpha[cb + c];
+          if (k > 0) {
+            // O holds the sum through PV(g-1): wait for it, rescale this lane.
+            const uint32_t gp = g - 1;
+            if (!wg_wait(&C.p_empty[gp % NPm], (gp / NPm) & 1, 0x23, bar_and)) { ok = false; break; }
+            ptx::tc_fence_after();
+            for (int pr = 0; pr < nv_pairs; ++pr) {
+              float o[32];
+              const uint32_t a = lane_addr + kOCol + pr * kRowsPerCta + cb;
+              ptx::tmem_ld32(a, o);
+              ptx::tmem_ld_wait();
+#pragma unroll
+              for (int c = 0; c < 32; ++c) o[c] *= C.alpha[cb + c];
+              ptx::tmem_st32(a, o);
+            }
+            ptx::tmem_st_wait();
+          }
+        }
+        // P buffer free once PV(g - NPm) completed
+        const int pb = g % NPm;
+        if (!wg_wait(&C.p_empty[pb], ((g / NPm) & 1) ^ 1, 0x24, bar_and)) { ok = false; break; }
+        // probabilities: bf16 (or a bf16 hi/lo pair) for the PV operand, fp32
+        // for the row sums l
+        uint8_t* prow = sP + pb * kPBytes + t * 128;
+#pragma unroll
+        for (int uu = 0; uu < 4; ++uu) {
+          uint32_t pk[4], pl[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c = 8 * uu + 2 * e;
+            // fresh shared-memory reads (not registers kept from the check above)
+            const volatile float* mv = &C.m[cb + c];
+            const float m0 = mv[0], m1 = mv[1];
+            const float p0 = (x[c] == -INFINITY) ? 0.f : ex2(x[c] - m0);
+            const float p1 = (x[c + 1] == -INFINITY) ? 0.f : ex2(x[c + 1] - m1);
+            pk[e] = ptx::pack_bf16x2(p0, p1);
+            if (kPSplit)
+              pl[e] = ptx::pack_bf16x2(p0 - __uint_as_float(pk[e] << 16),
+                                       p1 - __uint_as_float(pk[e] & 0xFFFF0000u));
+            lsum[c] += p0;
+            lsum[c + 1] += p1;
+          }
+          const int unit = 4 * sg + uu;  // 16-byte unit = rows 8*unit .. 8*unit+7
+          *reinterpret_cast<uint4*>(prow + ((unit ^ (t & 7)) << 4)) =
+              make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          if (kPSplit)
+            *reinterpret_cast<uint4*>(prow + kPBytes + ((unit ^ (t & 7)) << 4)) =
+                make_uint4(pl[0], pl[1], pl[2], pl[3]);
+        }
+        ptx::fence_proxy_async_smem();
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(&C.p_full[pb]);
+      }
+      if (!ok) break;
+
+      // ---- epilogue: l = column sums over the 128 token lanes
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        float v = lsum[c];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == 0) C.red[4 * sg + wq][c] = v;
+      }
+      ptx::named_bar_sync(bar_sync, 128);
+      const bool partial = P.always_partial || u.nsplit > 1;
+      const int ws_row0 = (P.num_splits[u.b] + u.split) * P.R;
+      const int rows_here = min(kRowsPerCta, P.R - grp * kRowsPerCta);
+      if (wt < 32) {
+        const float l = (C.red[4 * sg][wt] + C.red[4 * sg + 1][wt]) +
+                        (C.red[4 * sg + 2][wt] + C.red[4 * sg + 3][wt]);
+        C.alpha[cb + wt] = l > 0.f ? 1.0f / l : 0.f;  // reused as 1/l
+        if (cb + wt < rows_here) {
+          const int rg = grp * kRowsPerCta + cb + wt;
+          const float lv =
+              l > 0.f ? (C.m[cb + wt] + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+          if (partial)
+            P.ws_lse[ws_row0 + rg] = lv;
+          else
+            P.lse[(size_t)u.b * P.R + rg] = lv;
+        }
+      }
+      ptx::named_bar_sync(bar_sync, 128);
+      const uint32_t glast = gt + n - 1;
+      if (!wg_wait(&C.p_empty[glast % NPm], (glast / NPm) & 1, 0x25, bar_and)) { ok = false; break; }
+      ptx::tc_fence_after();
+      const int ncols = min(32, rows_here - cb);  // valid columns of this group
+      const size_t row_first = partial ? (size_t)ws_row0 + grp * kRowsPerCta + cb
+                                       : (size_t)u.b * P.R + grp * kRowsPerCta + cb;
+      for (int pr = 0; pr < nv_pairs; ++pr) {
+        const int d = pr * 128 + t;
+        float o[32];
+        ptx::tmem_ld32(lane_addr + kOCol + pr * kRowsPerCta + cb, o);
+        ptx::tmem_ld_wait();
+        if (d < P.d_v && ncols > 0) {
+          if (partial) {
+            float* dst = P.ws_o + row_first * P.d_v + d;
+#pragma unroll
+            for (int c = 0; c < 32; ++c)
+              if (c < ncols) dst[(size_t)c * P.d_v] = o[c] * C.alpha[cb + c];
+          } else {
+            __nv_bfloat16* dst = P.out + row_first * P.d_v + d;
+#pragma unroll
+            for (int c = 0; c < 32; ++c)
+              if (c < ncols) dst[(size_t)c * P.d_v] = __float2bfloat16_rn(o[c] * C.alpha[cb + c]);
+          }
+        }
+      }
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(&C.o_free);
+      ptx::named_bar_sync(bar_sync, 128);  // C.alpha / C.red / C.lim reusable
+      gt += n;
+      ++u_idx;
+    }
+  } else if (kMode == kSparse && warp >= 2 + 4 * kSoftmaxGroups) {
+    // ============================== FP8 gather / dequant ==============================
+    const int t0 = threadIdx.x - (64 + 128 * kSoftmaxGroups);  // token lanes t0, t0 + 64
+    uint32_t ring_it = 0;
+    Unit u;
+    bool ok = true;
+    auto fill = [&](const Unit& un, int tile, int pair) -> bool {
+      const int slot = ring_it % kNPair;
+      const uint32_t round = ring_it / kNPair;
+      ++ring_it;
+      if (!ptx::mbar_wait(&C.slot_empty[slot], (round & 1) ^ 1, 0x31)) return false;
+#pragma unroll 1
+      for (int h = 0; h < kTileT / kGatherThreads; ++h) {
+        const int t = t0 + h * kGatherThreads;
+        const int j = tile * kTileT + t;
+        const int idx = (j < P.topk) ? __ldg(P.indices + (size_t)un.b * P.topk + j) : -1;
+        bool valid = idx >= 0;
+        if (valid && static_cast<long long>(idx) >= P.num_slots) {
+          ptx::set_error(MLA_DEVERR_BAD_INDEX, 0x32);
+          valid = false;
+        }
+        const uint8_t* row = P.cache656 + (valid ? (size_t)idx * kRow656 : 0);
+        sparse_fill_pair(sRing + slot * kPairBytes, t, row, valid, pair);
+      }
+      ptx::fence_proxy_async_smem();
+      ptx::mbar_arrive(&C.slot_full[slot]);
+      return true;
+    };
+    while (ok && it.template next<kMode>(P, u)) {
+      const int n = u.hi - u.lo;
+      for (int k = 0; k < n && ok; ++k) {
+        for (int pr = 0; pr < 5 && ok; ++pr) ok = fill(u, u.lo + k, pr);
+        if (k >= 1)
+          for (int pr = 0; pr < nv_pairs && ok; ++pr) ok = fill(u, u.lo + k - 1, pr);
+      }
+      for (int pr = 0; pr < nv_pairs && ok; ++pr) ok = fill(u, u.hi - 1, pr);
+    }
+  }
+
+  // ---- teardown: every role has finished issuing; wait for the MMA pipe to
+  // drain before releasing TMEM.
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace mla

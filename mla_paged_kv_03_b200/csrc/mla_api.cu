@@ -1,0 +1,471 @@
+// mla_api.cu -- the C ABI of libmla_b200 (declared in include/mla.h):
+// argument validation, TMA descriptor encoding and kernel launches.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/mla.h"
+#include "combine_kernel.cuh"
+#include "decode_kernel.cuh"
+#include "mla_common.h"
+
+namespace {
+
+thread_local std::string g_err;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return code;
+}
+
+#define MLA_CHECK_ARG(cond, ...)                              \
+  do {                                                        \
+    if (!(cond)) return fail(MLA_ERR_INVALID_ARG, __VA_ARGS__); \
+  } while (0)
+
+#define MLA_CUDA(call)                                                                  \
+  do {                                                                                  \
+    cudaError_t e_ = (call);                                                            \
+    if (e_ != cudaSuccess)                                                              \
+      return fail(MLA_ERR_CUDA, "%s failed: %s", #call, cudaGetErrorString(e_));        \
+  } while (0)
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// ---------------------------------------------------------------- TMA maps
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 view [rows, 576] with a {64 cols, 64 rows} box, 128-byte swizzle.
+int make_latent_map(CUtensorMap* map, const void* base, long long rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(mla::kD), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(mla::kD) * 2};
+  cuuint32_t box[2] = {64, 64};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return MLA_OK;
+}
+
+template <int kMode>
+int prepare_kernel() {
+  static int done = 0;
+  static int rc = MLA_OK;
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!done) {
+    cudaError_t e = cudaFuncSetAttribute(mla::mla_decode_kernel<kMode>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         mla::cfg::kSmemBytes);
+    rc = (e == cudaSuccess) ? MLA_OK
+                            : fail(MLA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    done = 1;
+  }
+  return rc;
+}
+
+struct WsLayout {
+  size_t o_off, lse_off, meta_off, splits_off, lens_off, total;
+};
+
+WsLayout dense_ws_layout(int batch, int R, int d_v, int parts) {
+  WsLayout w{};
+  const size_t splits = static_cast<size_t>(batch) + parts;
+  w.o_off = 0;
+  w.lse_off = align_up(splits * R * d_v * sizeof(float), 256);
+  w.total = w.lse_off + align_up(splits * R * sizeof(float), 256);
+  return w;
+}
+
+WsLayout sparse_ws_layout(int pairs, int R, int d_v, int parts) {
+  WsLayout w = dense_ws_layout(pairs, R, d_v, parts);
+  w.meta_off = w.total;
+  w.splits_off = w.meta_off + align_up(static_cast<size_t>(parts) * mla::kMetaInts * 4, 256);
+  w.lens_off = w.splits_off + align_up((static_cast<size_t>(pairs) + 1) * 4, 256);
+  w.total = w.lens_off + align_up(static_cast<size_t>(pairs) * 4, 256);
+  return w;
+}
+
+int launch_combine(const mla::CombineParams& cp, bool fused, cudaStream_t st) {
+  const long long rows = static_cast<long long>(cp.batch) * cp.R;
+  if (rows == 0) return MLA_OK;
+  const int threads = 256;
+  const long long blocks = (rows * 32 + threads - 1) / threads;
+  if (fused)
+    mla::mla_combine_kernel<true><<<static_cast<unsigned>(blocks), threads, 0, st>>>(cp);
+  else
+    mla::mla_combine_kernel<false><<<static_cast<unsigned>(blocks), threads, 0, st>>>(cp);
+  MLA_CUDA(cudaGetLastError());
+  return MLA_OK;
+}
+
+template <int kMode>
+int launch_decode(const CUtensorMap& tq, const CUtensorMap& tkv, const mla::DecodeParams& p,
+                  cudaStream_t st) {
+  int rc = prepare_kernel<kMode>();
+  if (rc != MLA_OK) return rc;
+  const unsigned grid = static_cast<unsigned>(p.num_parts * p.n_groups);
+  mla::mla_decode_kernel<kMode>
+      <<<grid, mla::Threads<kMode>::value, mla::cfg::kSmemBytes, st>>>(tq, tkv, p);
+  MLA_CUDA(cudaGetLastError());
+  return MLA_OK;
+}
+
+int check_common_dense(const void* q, const void* kcache, const int32_t* block_table,
+                       int max_pages, int num_blocks, const int32_t* cache_seqlens, int batch,
+                       int h_q, float softmax_scale, const int32_t* metadata,
+                       const int32_t* num_splits, int num_sm_parts, void* workspace) {
+  MLA_CHECK_ARG(batch >= 0, "batch must be >= 0 (got %d)", batch);
+  MLA_CHECK_ARG(h_q >= 1, "h_q must be >= 1 (got %d)", h_q);
+  MLA_CHECK_ARG(num_sm_parts >= 1, "num_sm_parts must be >= 1 (got %d)", num_sm_parts);
+  MLA_CHECK_ARG(max_pages >= 1, "max_pages must be >= 1 (got %d)", max_pages);
+  MLA_CHECK_ARG(num_blocks >= 1, "num_blocks must be >= 1 (got %d)", num_blocks);
+  MLA_CHECK_ARG(static_cast<long long>(num_blocks) * mla::kPage < (1LL << 31),
+                "num_blocks * 64 must fit in int32");
+  MLA_CHECK_ARG(std::isfinite(softmax_scale) && softmax_scale > 0.f,
+                "softmax_scale must be finite and > 0");
+  MLA_CHECK_ARG(q && kcache && block_table && cache_seqlens && metadata && num_splits && workspace,
+                "null device pointer argument");
+  MLA_CHECK_ARG(aligned(q, 16) && aligned(kcache, 16), "q and kcache must be 16-byte aligned");
+  MLA_CHECK_ARG(aligned(workspace, 16), "workspace must be 16-byte aligned");
+  MLA_CHECK_ARG(aligned(block_table, 4) && aligned(cache_seqlens, 4) && aligned(metadata, 4) &&
+                    aligned(num_splits, 4),
+                "int32 arrays must be 4-byte aligned");
+  return MLA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* mla_last_error(void) { return g_err.c_str(); }
+
+int mla_num_sms(int device, int* num_sms) {
+  MLA_CHECK_ARG(num_sms, "num_sms is null");
+  int v = 0;
+  MLA_CUDA(cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, device));
+  *num_sms = v;
+  return MLA_OK;
+}
+
+int mla_num_sm_parts(int device, int heads_per_kv, int h_kv, int* num_sm_parts) {
+  MLA_CHECK_ARG(num_sm_parts, "num_sm_parts is null");
+  MLA_CHECK_ARG(heads_per_kv >= 1, "heads_per_kv must be >= 1");
+  if (h_kv != 1) return fail(MLA_ERR_UNSUPPORTED, "h_kv must be 1 (got %d)", h_kv);
+  int sms = 0;
+  int rc = mla_num_sms(device, &sms);
+  if (rc != MLA_OK) return rc;
+  const int groups = mla::ceil_div(heads_per_kv, mla::kRowsPerCta);
+  int parts = sms / groups / h_kv;
+  *num_sm_parts = parts < 1 ? 1 : parts;
+  return MLA_OK;
+}
+
+int mla_metadata_size(int batch, int num_sm_parts, size_t* metadata_bytes,
+                      size_t* num_splits_bytes) {
+  MLA_CHECK_ARG(batch >= 0 && num_sm_parts >= 1, "batch >= 0 and num_sm_parts >= 1 required");
+  MLA_CHECK_ARG(metadata_bytes && num_splits_bytes, "null out-pointer");
+  *metadata_bytes = static_cast<size_t>(num_sm_parts) * mla::kMetaInts * sizeof(int32_t);
+  *num_splits_bytes = (static_cast<size_t>(batch) + 1) * sizeof(int32_t);
+  return MLA_OK;
+}
+
+int mla_get_metadata(const int32_t* cache_seqlens, int batch, int heads_per_kv, int h_kv,
+                     int num_sm_parts, int32_t* metadata, int32_t* num_splits, void* stream) {
+  MLA_CHECK_ARG(batch >= 0 && num_sm_parts >= 1, "batch >= 0 and num_sm_parts >= 1 required");
+  MLA_CHECK_ARG(heads_per_kv >= 1, "heads_per_kv must be >= 1");
+  if (h_kv != 1) return fail(MLA_ERR_UNSUPPORTED, "h_kv must be 1 (got %d)", h_kv);
+  MLA_CHECK_ARG(metadata && num_splits && (cache_seqlens || batch == 0), "null device pointer");
+  mla::mla_plan_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(cache_seqlens, batch,
+                                                                         num_sm_parts, metadata,
+                                                                         num_splits);
+  MLA_CUDA(cudaGetLastError());
+  return MLA_OK;
+}
+
+int mla_get_metadata_host(const int32_t* cache_seqlens, int batch, int heads_per_kv, int h_kv,
+                          int num_sm_parts, int32_t* metadata, int32_t* num_splits) {
+  MLA_CHECK_ARG(batch >= 0 && num_sm_parts >= 1, "batch >= 0 and num_sm_parts >= 1 required");
+  MLA_CHECK_ARG(heads_per_kv >= 1, "heads_per_kv must be >= 1");
+  if (h_kv != 1) return fail(MLA_ERR_UNSUPPORTED, "h_kv must be 1 (got %d)", h_kv);
+  MLA_CHECK_ARG(metadata && num_splits && (cache_seqlens || batch == 0), "null host pointer");
+  for (int b = 0; b < batch; ++b)
+    MLA_CHECK_ARG(cache_seqlens[b] >= 0, "cache_seqlens[%d] = %d is negative", b, cache_seqlens[b]);
+  mla::plan_splits(cache_seqlens, batch, num_sm_parts, metadata, num_splits);
+  return MLA_OK;
+}
+
+int mla_workspace_size(int batch, int rows_per_kv, int d_v, int num_sm_parts, size_t* bytes) {
+  MLA_CHECK_ARG(bytes, "bytes is null");
+  MLA_CHECK_ARG(batch >= 0 && rows_per_kv >= 1 && num_sm_parts >= 1, "bad sizes");
+  MLA_CHECK_ARG(d_v == 512 || d_v == 576, "d_v must be 512 or 576 (got %d)", d_v);
+  *bytes = dense_ws_layout(batch, rows_per_kv, d_v, num_sm_parts).total;
+  return MLA_OK;
+}
+
+int mla_decode_fwd(const void* q, const void* kcache, const int32_t* block_table, int max_pages,
+                   int num_blocks, const int32_t* cache_seqlens, int batch, int s_q, int h_q,
+                   int h_kv, int d_v, float softmax_scale, int causal, const int32_t* metadata,
+                   const int32_t* num_splits, int num_sm_parts, void* workspace,
+                   size_t workspace_bytes, void* out, float* lse, void* stream) {
+  if (h_kv != 1) return fail(MLA_ERR_UNSUPPORTED, "h_kv must be 1 (got %d)", h_kv);
+  MLA_CHECK_ARG(s_q >= 1, "s_q must be >= 1 (got %d)", s_q);
+  MLA_CHECK_ARG(d_v == 512 || d_v == 576, "d_v must be 512 or 576 (got %d)", d_v);
+  int rc = check_common_dense(q, kcache, block_table, max_pages, num_blocks, cache_seqlens, batch,
+                              h_q, softmax_scale, metadata, num_splits, num_sm_parts, workspace);
+  if (rc != MLA_OK) return rc;
+  MLA_CHECK_ARG(out && lse, "null output pointer");
+  MLA_CHECK_ARG(aligned(out, 8) && aligned(lse, 4), "out must be 8-byte aligned, lse 4-byte");
+  const int R = s_q * h_q;
+  const WsLayout w = dense_ws_layout(batch, R, d_v, num_sm_parts);
+  MLA_CHECK_ARG(workspace_bytes >= w.total, "workspace too small: %zu < %zu", workspace_bytes,
+                w.total);
+  if (batch == 0) return MLA_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  CUtensorMap tq, tkv;
+  if ((rc = make_latent_map(&tq, q, static_cast<long long>(batch) * R)) != MLA_OK) return rc;
+  if ((rc = make_latent_map(&tkv, kcache, static_cast<long long>(num_blocks) * mla::kPage)) !=
+      MLA_OK)
+    return rc;
+
+  mla::DecodeParams p{};
+  p.batch = batch;
+  p.s_q = s_q;
+  p.h_q = h_q;
+  p.R = R;
+  p.d_v = d_v;
+  p.n_groups = mla::ceil_div(R, mla::kRowsPerCta);
+  p.num_parts = num_sm_parts;
+  p.num_blocks = num_blocks;
+  p.max_pages = max_pages;
+  p.causal = causal ? 1 : 0;
+  p.always_partial = 0;
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  p.block_table = block_table;
+  p.seqlens = cache_seqlens;
+  p.metadata = metadata;
+  p.num_splits = num_splits;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.ws_o = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.o_off);
+  p.ws_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.lse_off);
+  if ((rc = launch_decode<mla::kDense>(tq, tkv, p, st)) != MLA_OK) return rc;
+
+  mla::CombineParams cp{};
+  cp.batch = batch;
+  cp.R = R;
+  cp.d_v = d_v;
+  cp.h_q = h_q;
+  cp.num_splits = num_splits;
+  cp.ws_o = p.ws_o;
+  cp.ws_lse = p.ws_lse;
+  cp.out = p.out;
+  cp.lse = lse;
+  return launch_combine(cp, false, st);
+}
+
+int mla_fused_norm_rope_attn_rope_cast(
+    const void* q_raw, const float* norm_gain, float eps, float rope_base,
+    const int32_t* positions, const void* kcache, const int32_t* block_table, int max_pages,
+    int num_blocks, const int32_t* cache_seqlens, int batch, int h_q, float softmax_scale,
+    const int32_t* metadata, const int32_t* num_splits, int num_sm_parts, void* workspace,
+    size_t workspace_bytes, uint8_t* out_e4m3, float* out_scale, float* lse, void* stream) {
+  int rc = check_common_dense(q_raw, kcache, block_table, max_pages, num_blocks, cache_seqlens,
+                              batch, h_q, softmax_scale, metadata, num_splits, num_sm_parts,
+                              workspace);
+  if (rc != MLA_OK) return rc;
+  MLA_CHECK_ARG(norm_gain && out_e4m3 && out_scale && lse, "null pointer argument");
+  MLA_CHECK_ARG(aligned(norm_gain, 16), "norm_gain must be 16-byte aligned");
+  MLA_CHECK_ARG(aligned(out_e4m3, 4) && aligned(out_scale, 4) && aligned(lse, 4),
+                "outputs must be 4-byte aligned");
+  MLA_CHECK_ARG(std::isfinite(eps) && eps >= 0.f, "eps must be finite and >= 0");
+  MLA_CHECK_ARG(std::isfinite(rope_base) && rope_base > 0.f, "rope_base must be > 0");
+  const int R = h_q;
+  const int d_v = mla::kD;
+  const WsLayout w = dense_ws_layout(batch, R, d_v, num_sm_parts);
+  MLA_CHECK_ARG(workspace_bytes >= w.total, "workspace too small: %zu < %zu", workspace_bytes,
+                w.total);
+  if (batch == 0) return MLA_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  CUtensorMap tkv;
+  if ((rc = make_latent_map(&tkv, kcache, static_cast<long long>(num_blocks) * mla::kPage)) !=
+      MLA_OK)
+    return rc;
+
+  mla::DecodeParams p{};
+  p.batch = batch;
+  p.s_q = 1;
+  p.h_q = h_q;
+  p.R = R;
+  p.d_v = d_v;
+  p.n_groups = mla::ceil_div(R, mla::kRowsPerCta);
+  p.num_parts = num_sm_parts;
+  p.num_blocks = num_blocks;
+  p.max_pages = max_pages;
+  p.causal = 0;
+  p.always_partial = 1;
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  p.block_table = block_table;
+  p.seqlens = cache_seqlens;
+  p.metadata = metadata;
+  p.num_splits = num_splits;
+  p.ws_o = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.o_off);
+  p.ws_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.lse_off);
+  p.q_raw = static_cast<const __nv_bfloat16*>(q_raw);
+  p.gain = norm_gain;
+  p.eps = eps;
+  p.rope_base = rope_base;
+  p.positions = positions;
+  for (int k = 0; k < mla::kRope / 2; ++k)
+    p.inv_freq[k] = std::pow(static_cast<double>(rope_base), -2.0 * k / mla::kRope);
+  if ((rc = launch_decode<mla::kFused>(tkv, tkv, p, st)) != MLA_OK) return rc;
+
+  mla::CombineParams cp{};
+  cp.batch = batch;
+  cp.R = R;
+  cp.d_v = d_v;
+  cp.h_q = h_q;
+  cp.num_splits = num_splits;
+  cp.ws_o = p.ws_o;
+  cp.ws_lse = p.ws_lse;
+  cp.lse = lse;
+  cp.out_fp8 = out_e4m3;
+  cp.out_scale = out_scale;
+  cp.seqlens = cache_seqlens;
+  cp.positions = positions;
+  for (int k = 0; k < mla::kRope / 2; ++k) cp.inv_freq[k] = p.inv_freq[k];
+  return launch_combine(cp, true, st);
+}
+
+int mla_sparse_workspace_size(int batch, int s_q, int h_q, int topk, int d_v, int num_sm_parts,
+                              size_t* bytes) {
+  MLA_CHECK_ARG(bytes, "bytes is null");
+  MLA_CHECK_ARG(batch >= 0 && s_q >= 1 && h_q >= 1 && topk >= 1 && num_sm_parts >= 1,
+                "bad sizes");
+  MLA_CHECK_ARG(d_v == 512, "sparse decode supports d_v = 512 (got %d)", d_v);
+  *bytes = sparse_ws_layout(batch * s_q, h_q, d_v, num_sm_parts).total;
+  return MLA_OK;
+}
+
+int mla_sparse_decode(const void* q, const uint8_t* kcache_fp8, int64_t num_slots,
+                      const int32_t* indices, int topk, int batch, int s_q, int h_q, int d_v,
+                      float softmax_scale, int num_sm_parts, void* workspace,
+                      size_t workspace_bytes, void* out, float* lse, void* stream) {
+  MLA_CHECK_ARG(batch >= 0 && s_q >= 1 && h_q >= 1, "bad sizes");
+  MLA_CHECK_ARG(topk >= 1, "topk must be >= 1 (got %d)", topk);
+  MLA_CHECK_ARG(num_slots >= 1 && num_slots < (1LL << 31), "num_slots must be in [1, 2^31)");
+  MLA_CHECK_ARG(d_v == 512, "sparse decode supports d_v = 512 (got %d)", d_v);
+  MLA_CHECK_ARG(num_sm_parts >= 1, "num_sm_parts must be >= 1");
+  MLA_CHECK_ARG(std::isfinite(softmax_scale) && softmax_scale > 0.f,
+                "softmax_scale must be finite and > 0");
+  MLA_CHECK_ARG(q && kcache_fp8 && indices && workspace && out && lse, "null device pointer");
+  MLA_CHECK_ARG(aligned(q, 16) && aligned(kcache_fp8, 16), "q and kcache_fp8 must be 16-byte aligned");
+  MLA_CHECK_ARG(aligned(workspace, 256), "workspace must be 256-byte aligned");
+  MLA_CHECK_ARG(aligned(out, 8) && aligned(lse, 4) && aligned(indices, 4), "misaligned output");
+  const int pairs = batch * s_q;
+  const WsLayout w = sparse_ws_layout(pairs, h_q, d_v, num_sm_parts);
+  MLA_CHECK_ARG(workspace_bytes >= w.total, "workspace too small: %zu < %zu", workspace_bytes,
+                w.total);
+  if (batch == 0) return MLA_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int32_t* meta = reinterpret_cast<int32_t*>(ws + w.meta_off);
+  int32_t* splits = reinterpret_cast<int32_t*>(ws + w.splits_off);
+  int32_t* lens = reinterpret_cast<int32_t*>(ws + w.lens_off);
+  mla::mla_plan_uniform_kernel<<<1, 256, 0, st>>>(topk, pairs, num_sm_parts, lens, meta, splits);
+  MLA_CUDA(cudaGetLastError());
+
+  CUtensorMap tq;
+  int rc = make_latent_map(&tq, q, static_cast<long long>(pairs) * h_q);
+  if (rc != MLA_OK) return rc;
+
+  mla::DecodeParams p{};
+  p.batch = pairs;
+  p.s_q = 1;
+  p.h_q = h_q;
+  p.R = h_q;
+  p.d_v = d_v;
+  p.n_groups = mla::ceil_div(h_q, mla::kRowsPerCta);
+  p.num_parts = num_sm_parts;
+  p.num_blocks = 1;
+  p.max_pages = 1;
+  p.causal = 0;
+  p.always_partial = 0;
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  p.metadata = meta;
+  p.num_splits = splits;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.ws_o = reinterpret_cast<float*>(ws + w.o_off);
+  p.ws_lse = reinterpret_cast<float*>(ws + w.lse_off);
+  p.cache656 = kcache_fp8;
+  p.indices = indices;
+  p.topk = topk;
+  p.num_slots = num_slots;
+  if ((rc = launch_decode<mla::kSparse>(tq, tq, p, st)) != MLA_OK) return rc;
+
+  mla::CombineParams cp{};
+  cp.batch = pairs;
+  cp.R = h_q;
+  cp.d_v = d_v;
+  cp.h_q = h_q;
+  cp.num_splits = splits;
+  cp.ws_o = p.ws_o;
+  cp.ws_lse = p.ws_lse;
+  cp.out = p.out;
+  cp.lse = lse;
+  return launch_combine(cp, false, st);
+}
+
+int mla_device_status(int* status, int reset) {
+  MLA_CHECK_ARG(status, "status is null");
+  MLA_CUDA(cudaDeviceSynchronize());
+  int v = 0;
+  MLA_CUDA(cudaMemcpyFromSymbol(&v, mla::ptx::g_status, sizeof(int)));
+  *status = v;
+  if (reset) {
+    const int z = 0;
+    MLA_CUDA(cudaMemcpyToSymbol(mla::ptx::g_status, &z, sizeof(int)));
+  }
+  if ((v >> 16) == mla::MLA_DEVERR_TIMEOUT)
+    return fail(MLA_ERR_TIMEOUT, "a kernel wait timed out (site 0x%x)", v & 0xFFFF);
+  return MLA_OK;
+}
+
+}  // extern "C"

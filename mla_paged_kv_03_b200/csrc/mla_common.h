@@ -1,0 +1,125 @@
+// mla_common.h -- constants, device status codes and the split-KV planner
+// shared by the host entry points and the device kernels of libmla_b200.
+#pragma once
+#include <cstdint>
+
+#ifdef __CUDACC__
+#define MLA_HD __host__ __device__
+#else
+#define MLA_HD
+#endif
+
+namespace mla {
+
+// Latent geometry of MLA: one shared KV head of 576 dims, 512 "nope" dims
+// followed by 64 decoupled-RoPE dims; V is a prefix of the latent row.
+// [FlashMLA (AI Wiki), "How does MLA differ from MHA and GQA?"]
+constexpr int kD = 576;
+constexpr int kNope = 512;
+constexpr int kRope = 64;
+constexpr int kPage = 64;        // paged cache block size [FlashMLA (AI Wiki), "What is FlashMLA?"]
+constexpr int kRow656 = 656;     // FP8 cache row [FlashMLA (AI Wiki), "The FP8 and FP4 KV cache"]
+
+// Kernel tiling: 128-token tiles (two pages), at most 64 query rows per CTA,
+// 64-dim (128-byte) column chunks in the SW128 layout.
+constexpr int kTileT = 128;
+constexpr int kRowsPerCta = 64;
+constexpr int kChunkD = 64;
+constexpr int kNumChunks = kD / kChunkD;  // 9
+
+// Planner cost of one work segment beyond its tiles (Q load, pipeline fill,
+// epilogue), in tile units.
+constexpr int kSegmentOverheadTiles = 2;
+
+// Metadata row per SM part: {begin_b, begin_tile, end_b, end_tile,
+// first_split, 0, 0, 0}; end_tile is exclusive within batch end_b.
+constexpr int kMetaInts = 8;
+
+// Device status codes (upper 16 bits of the status word).
+constexpr int MLA_DEVERR_TIMEOUT = 1;
+constexpr int MLA_DEVERR_BAD_INDEX = 2;
+
+constexpr unsigned long long kWaitBudgetNs = 2000000000ull;  // 2 s per wait
+
+MLA_HD inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// Tiles (of 128 tokens) a sequence of length L contributes.  An empty
+// sequence still owns one (fully masked) tile so that some CTA writes its
+// O = 0, LSE = -inf result.
+MLA_HD inline int tiles_of(int L) { return L > 0 ? ceil_div(L, kTileT) : 1; }
+
+// Greedy dealing of tiles to parts with a cost cap `target` per part; a
+// segment costs its tiles plus kSegmentOverheadTiles.  Returns the number of
+// parts used; writes the plan when metadata != nullptr.
+MLA_HD inline int deal_tiles(const int32_t* seqlens, int batch, long long target, int max_parts,
+                             int32_t* metadata, int32_t* num_splits) {
+  int p = 0;
+  long long used = 0;
+  bool part_open = false;
+  if (num_splits) num_splits[0] = 0;
+  for (int b = 0; b < batch; ++b) {
+    const int n = tiles_of(seqlens[b]);
+    int t = 0;
+    int splits = 0;
+    while (t < n) {
+      if (part_open && used + kSegmentOverheadTiles + 1 > target) {
+        ++p;
+        used = 0;
+        part_open = false;
+      }
+      const long long avail = target - used - kSegmentOverheadTiles;
+      int take = static_cast<int>(avail < 1 ? 1 : (avail < n - t ? avail : n - t));
+      if (p >= max_parts - 1) take = n - t;  // the last part takes the rest
+      if (metadata && p < max_parts) {
+        int32_t* m = metadata + p * kMetaInts;
+        if (!part_open) {
+          m[0] = b;
+          m[1] = t;
+          m[4] = splits;
+        }
+        m[2] = b;
+        m[3] = t + take;
+      }
+      part_open = true;
+      used += take + kSegmentOverheadTiles;
+      t += take;
+      ++splits;
+    }
+    if (num_splits) num_splits[b + 1] = num_splits[b] + splits;
+  }
+  return part_open ? p + 1 : p;
+}
+
+// Split-KV planner.  Finds the smallest per-part cost cap for which the
+// greedy dealing (sequences in order, tiles of 128 tokens, a segment costing
+// its tiles plus kSegmentOverheadTiles) fits in `num_parts` parts, then
+// writes metadata[num_parts][8] and the prefix sums num_splits[batch + 1]
+// (num_splits[b+1] - num_splits[b] = number of parts holding tiles of
+// sequence b).  Each part covers one contiguous run of (sequence, tile)
+// pairs; unused parts are marked empty (begin_seq > end_seq).  Runs
+// identically on host and device.
+MLA_HD inline void plan_splits(const int32_t* seqlens, int batch, int num_parts,
+                               int32_t* metadata, int32_t* num_splits) {
+  for (int p = 0; p < num_parts; ++p) {
+    int32_t* m = metadata + p * kMetaInts;
+    m[0] = batch;  // empty part: begins after every sequence
+    m[1] = 0;
+    m[2] = batch - 1;
+    m[3] = 0;
+    m[4] = m[5] = m[6] = m[7] = 0;
+  }
+  long long total = 0;
+  for (int b = 0; b < batch; ++b) total += tiles_of(seqlens[b]) + kSegmentOverheadTiles;
+  long long lo = kSegmentOverheadTiles + 1;
+  long long hi = total > lo ? total : lo;
+  while (lo < hi) {
+    const long long mid = lo + (hi - lo) / 2;
+    if (deal_tiles(seqlens, batch, mid, num_parts + 1, nullptr, nullptr) <= num_parts)
+      hi = mid;
+    else
+      lo = mid + 1;
+  }
+  deal_tiles(seqlens, batch, lo, num_parts, metadata, num_splits);
+}
+
+}  // namespace mla

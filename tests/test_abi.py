@@ -1,0 +1,91 @@
+"""The C-ABI library loads on a machine without a GPU, exports every symbol
+that include/mla.h declares, and rejects bad arguments before launching."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from mla_paged_kv_03_b200 import binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "mla.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(mla_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declarations_are_exported():
+    names = declared_functions()
+    assert len(names) >= 10
+    L = B.lib()
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(B.EXPORTED)
+
+
+def test_no_other_global_symbols_leak():
+    out = os.popen(f"nm -D --defined-only {B.LIB_PATH}").read().split("\n")
+    funcs = [l.split()[-1] for l in out if " T " in l]
+    assert set(funcs) == set(declared_functions()), set(funcs) ^ set(declared_functions())
+
+
+def call_decode(**over):
+    args = dict(q=16, kc=16, bt=16, max_pages=4, num_blocks=8, sl=16, batch=2, s_q=1, h_q=16,
+                h_kv=1, d_v=512, scale=0.04, causal=1, meta=16, ns=16, parts=4, ws=16,
+                ws_bytes=1 << 30, out=16, lse=16)
+    args.update(over)
+    a = args
+    return B.lib().mla_decode_fwd(a["q"], a["kc"], a["bt"], a["max_pages"], a["num_blocks"], a["sl"],
+                                  a["batch"], a["s_q"], a["h_q"], a["h_kv"], a["d_v"], a["scale"],
+                                  a["causal"], a["meta"], a["ns"], a["parts"], a["ws"],
+                                  a["ws_bytes"], a["out"], a["lse"], None)
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(h_kv=2), B.MLA_ERR_UNSUPPORTED),
+    (dict(d_v=256), B.MLA_ERR_INVALID_ARG),
+    (dict(q=None), B.MLA_ERR_INVALID_ARG),
+    (dict(q=18), B.MLA_ERR_INVALID_ARG),       # misaligned (not 16-byte)
+    (dict(kc=24), B.MLA_ERR_INVALID_ARG),
+    (dict(scale=0.0), B.MLA_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), B.MLA_ERR_INVALID_ARG),
+    (dict(parts=0), B.MLA_ERR_INVALID_ARG),
+    (dict(s_q=0), B.MLA_ERR_INVALID_ARG),
+    (dict(ws_bytes=10), B.MLA_ERR_INVALID_ARG),
+    (dict(max_pages=0), B.MLA_ERR_INVALID_ARG),
+    (dict(num_blocks=1 << 26), B.MLA_ERR_INVALID_ARG),
+])
+def test_decode_rejects_before_launch(over, code):
+    assert call_decode(**over) == code
+    assert B.lib().mla_last_error().decode() != ""
+
+
+def test_decode_empty_batch_is_a_no_op():
+    assert call_decode(batch=0) == B.MLA_OK
+
+
+def test_sparse_and_fused_validation():
+    L = B.lib()
+    rc = L.mla_sparse_decode(16, 16, 100, 16, 2048, 2, 1, 128, 576, 0.04, 74, 256, 1 << 30, 16, 16,
+                             None)
+    assert rc == B.MLA_ERR_INVALID_ARG  # d_v must be 512
+    rc = L.mla_sparse_decode(16, 16, 0, 16, 2048, 2, 1, 128, 512, 0.04, 74, 256, 1 << 30, 16, 16,
+                             None)
+    assert rc == B.MLA_ERR_INVALID_ARG  # num_slots
+    rc = L.mla_fused_norm_rope_attn_rope_cast(16, 16, -1.0, 1e4, None, 16, 16, 4, 8, 16, 2, 64,
+                                              0.04, 16, 16, 4, 16, 1 << 30, 16, 16, 16, None)
+    assert rc == B.MLA_ERR_INVALID_ARG  # eps < 0
+
+
+def test_size_queries():
+    m = ctypes.c_size_t()
+    s = ctypes.c_size_t()
+    assert B.lib().mla_metadata_size(10, 74, ctypes.byref(m), ctypes.byref(s)) == 0
+    assert m.value == 74 * 8 * 4 and s.value == 11 * 4
+    n = B.mla_workspace_size(64, 128, 512, 74)
+    assert n >= (64 + 74) * 128 * 512 * 4
+    assert B.mla_sparse_workspace_size(32, 1, 128, 2048, 512, 74) > n // 2
