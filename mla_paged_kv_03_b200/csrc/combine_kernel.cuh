@@ -41,124 +41,166 @@ __device__ __forceinline__ uint32_t cvt_e4m3x4(float a, float b, float c, float 
   return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
 }
 
-// One warp per row; lane l owns float4 groups l, l+32, ... of the row.
+// One CTA per row; thread i owns the float4 group i of the row (d_v / 4 = 128
+// or 144 threads).  The split weights are formed once in shared memory.
+constexpr int kCombineMaxSplits = 1024;  // splits of one sequence (<= SM parts)
+constexpr int kCombineThreads = 160;
+
 template <bool kFusedOut>
-__global__ void __launch_bounds__(256) mla_combine_kernel(const CombineParams P) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (warp >= P.batch * P.R) return;
-  const int b = warp / P.R;
-  const int r = warp % P.R;
+__global__ void __launch_bounds__(kCombineThreads) mla_combine_kernel(const CombineParams P) {
+  __shared__ float s_w[kCombineMaxSplits];
+  __shared__ float s_red[kCombineThreads / 32];
+  __shared__ float s_lse;
+  const int row_id = blockIdx.x;
+  const int b = row_id / P.R;
+  const int r = row_id % P.R;
   const int base = P.num_splits[b];
   const int n = P.num_splits[b + 1] - base;
   if (!kFusedOut && n <= 1) return;  // written directly by the decode kernel
+  const int tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
+  constexpr int kWarps = kCombineThreads / 32;
 
+  // max over the split LSEs
   float m = -INFINITY;
-  for (int i = 0; i < n; ++i) m = fmaxf(m, P.ws_lse[(size_t)(base + i) * P.R + r]);
+  for (int i = tid; i < n; i += kCombineThreads) {
+    const float li = P.ws_lse[(size_t)(base + i) * P.R + r];
+    s_w[i] = li;
+    m = fmaxf(m, li);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (lane == 0) s_red[warp] = m;
+  __syncthreads();
+  m = s_red[0];
+#pragma unroll
+  for (int w = 1; w < kWarps; ++w) m = fmaxf(m, s_red[w]);
+  __syncthreads();
   float sum = 0.f;
   if (m != -INFINITY)
-    for (int i = 0; i < n; ++i) sum += expf(P.ws_lse[(size_t)(base + i) * P.R + r] - m);
-  const float lse = (m == -INFINITY) ? -INFINITY : m + logf(sum);
+    for (int i = tid; i < n; i += kCombineThreads) sum += expf(s_w[i] - m);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if (lane == 0) s_red[warp] = sum;
+  __syncthreads();
+  if (tid == 0) {
+    float t = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) t += s_red[w];
+    s_lse = (m == -INFINITY) ? -INFINITY : m + logf(t);
+  }
+  __syncthreads();
+  const float lse = s_lse;
+  for (int i = tid; i < n; i += kCombineThreads)
+    s_w[i] = (lse == -INFINITY || s_w[i] == -INFINITY) ? 0.f : expf(s_w[i] - lse);
+  __syncthreads();
 
-  constexpr int kMaxG = 5;  // float4 groups per lane (576 / 4 / 32 -> 5)
   const int ngroups = P.d_v / 4;
-  float4 acc[kMaxG];
-#pragma unroll
-  for (int j = 0; j < kMaxG; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (m != -INFINITY) {
-    for (int i = 0; i < n; ++i) {
-      const float li = P.ws_lse[(size_t)(base + i) * P.R + r];
-      if (li == -INFINITY) continue;
-      const float w = expf(li - lse);
-      const float4* src =
-          reinterpret_cast<const float4*>(P.ws_o + ((size_t)(base + i) * P.R + r) * P.d_v);
-#pragma unroll
-      for (int j = 0; j < kMaxG; ++j) {
-        const int g = lane + 32 * j;
-        if (g < ngroups) {
-          const float4 v = src[g];
-          acc[j].x += w * v.x;
-          acc[j].y += w * v.y;
-          acc[j].z += w * v.z;
-          acc[j].w += w * v.w;
-        }
-      }
+  const int g = tid;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (g < ngroups) {
+    const float4* src = reinterpret_cast<const float4*>(P.ws_o + ((size_t)base * P.R + r) * P.d_v) + g;
+    const size_t stride = (size_t)P.R * P.d_v / 4;  // float4s between consecutive splits
+    int i = 0;
+    for (; i + 4 <= n; i += 4) {
+      const float4 v0 = src[(i + 0) * stride], v1 = src[(i + 1) * stride];
+      const float4 v2 = src[(i + 2) * stride], v3 = src[(i + 3) * stride];
+      const float w0 = s_w[i], w1 = s_w[i + 1], w2 = s_w[i + 2], w3 = s_w[i + 3];
+      acc.x += w0 * v0.x + w1 * v1.x + w2 * v2.x + w3 * v3.x;
+      acc.y += w0 * v0.y + w1 * v1.y + w2 * v2.y + w3 * v3.y;
+      acc.z += w0 * v0.z + w1 * v1.z + w2 * v2.z + w3 * v3.z;
+      acc.w += w0 * v0.w + w1 * v1.w + w2 * v2.w + w3 * v3.w;
+    }
+    for (; i < n; ++i) {
+      const float4 v = src[i * stride];
+      const float w = s_w[i];
+      acc.x += w * v.x;
+      acc.y += w * v.y;
+      acc.z += w * v.z;
+      acc.w += w * v.w;
     }
   }
 
   const size_t row = (size_t)b * P.R + r;
   if (!kFusedOut) {
-#pragma unroll
-    for (int j = 0; j < kMaxG; ++j) {
-      const int g = lane + 32 * j;
-      if (g < ngroups) {
-        __nv_bfloat162 lo = __floats2bfloat162_rn(acc[j].x, acc[j].y);
-        __nv_bfloat162 hi = __floats2bfloat162_rn(acc[j].z, acc[j].w);
-        uint2 pk;
-        pk.x = *reinterpret_cast<uint32_t*>(&lo);
-        pk.y = *reinterpret_cast<uint32_t*>(&hi);
-        *reinterpret_cast<uint2*>(P.out + row * P.d_v + 4 * g) = pk;
-      }
+    if (g < ngroups) {
+      __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+      __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+      uint2 pk;
+      pk.x = *reinterpret_cast<uint32_t*>(&lo);
+      pk.y = *reinterpret_cast<uint32_t*>(&hi);
+      *reinterpret_cast<uint2*>(P.out + row * P.d_v + 4 * g) = pk;
     }
-    if (lane == 0) P.lse[row] = lse;
+    if (tid == 0) P.lse[row] = lse;
     return;
   }
 
   // ---- fused epilogue: conjugate RoPE on dims 512..575, absmax, E4M3 cast
-  const int L = P.seqlens[b];
-  const double pos = P.positions ? static_cast<double>(P.positions[b]) : static_cast<double>(L - 1);
-  float amax = 0.f;
+  if (g < ngroups && 4 * g >= kNope) {
+    const int L = P.seqlens[b];
+    const double pos =
+        P.positions ? static_cast<double>(P.positions[b]) : static_cast<double>(L - 1);
+    const int k0 = (4 * g - kNope) / 2;  // pair index of (x, y); (z, w) is k0 + 1
 #pragma unroll
-  for (int j = 0; j < kMaxG; ++j) {
-    const int g = lane + 32 * j;
-    if (g < ngroups && 4 * g >= kNope) {
-      const int k0 = (4 * g - kNope) / 2;  // pair index of (x, y); (z, w) is k0 + 1
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        float s, c;
-        rope_sincos(pos, P.inv_freq[k0 + e], &s, &c);
-        float& a = e ? acc[j].z : acc[j].x;
-        float& bb = e ? acc[j].w : acc[j].y;
-        const float na = a * c + bb * s;   // rotate by -theta
-        const float nb = -a * s + bb * c;
-        a = na;
-        bb = nb;
-      }
+    for (int e = 0; e < 2; ++e) {
+      float sn, c;
+      rope_sincos(pos, P.inv_freq[k0 + e], &sn, &c);
+      float& a = e ? acc.z : acc.x;
+      float& bb = e ? acc.w : acc.y;
+      const float na = a * c + bb * sn;  // rotate by -theta
+      const float nb = -a * sn + bb * c;
+      a = na;
+      bb = nb;
     }
-    if (g < ngroups)
-      amax = fmaxf(amax, fmaxf(fmaxf(fabsf(acc[j].x), fabsf(acc[j].y)),
-                               fmaxf(fabsf(acc[j].z), fabsf(acc[j].w))));
   }
+  float amax = 0.f;
+  if (g < ngroups)
+    amax = fmaxf(fmaxf(fabsf(acc.x), fabsf(acc.y)), fmaxf(fabsf(acc.z), fabsf(acc.w)));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  const float scale = amax > 0.f ? amax / 448.0f : 1.0f;
+  __syncthreads();
+  if (lane == 0) s_red[warp] = amax;
+  __syncthreads();
+  amax = s_red[0];
 #pragma unroll
-  for (int j = 0; j < kMaxG; ++j) {
-    const int g = lane + 32 * j;
-    if (g < ngroups) {
-      const uint32_t codes = cvt_e4m3x4(acc[j].x / scale, acc[j].y / scale, acc[j].z / scale,
-                                        acc[j].w / scale);
-      *reinterpret_cast<uint32_t*>(P.out_fp8 + row * kD + 4 * g) = codes;
-    }
+  for (int w = 1; w < kWarps; ++w) amax = fmaxf(amax, s_red[w]);
+  const float scale = amax > 0.f ? amax / 448.0f : 1.0f;
+  if (g < ngroups) {
+    const uint32_t codes =
+        cvt_e4m3x4(acc.x / scale, acc.y / scale, acc.z / scale, acc.w / scale);
+    *reinterpret_cast<uint32_t*>(P.out_fp8 + row * kD + 4 * g) = codes;
   }
-  if (lane == 0) {
+  if (tid == 0) {
     P.out_scale[row] = scale;
     P.lse[row] = lse;
   }
 }
 
-// Device-side planner launch: one thread runs the same planner the host uses.
-__global__ void mla_plan_kernel(const int32_t* seqlens, int batch, int num_parts,
-                                int32_t* metadata, int32_t* num_splits) {
-  if (blockIdx.x == 0 && threadIdx.x == 0) plan_splits(seqlens, batch, num_parts, metadata, num_splits);
+// Device-side planner: the block stages tiles_of(seqlens) in shared memory
+// (or, for very large batches, in the caller's scratch), then one thread runs
+// the same planner the host uses.
+constexpr int kPlanSmemBatch = 8192;
+
+__global__ void __launch_bounds__(256) mla_plan_kernel(const int32_t* seqlens, int batch,
+                                                       int num_parts, int32_t* tiles_scratch,
+                                                       int32_t* metadata, int32_t* num_splits) {
+  __shared__ int32_t s_tiles[kPlanSmemBatch];
+  int32_t* tiles = batch <= kPlanSmemBatch ? s_tiles : tiles_scratch;
+  for (int i = threadIdx.x; i < batch; i += blockDim.x) tiles[i] = tiles_of(seqlens[i]);
+  __syncthreads();
+  if (threadIdx.x == 0) plan_splits_tiles(tiles, batch, num_parts, metadata, num_splits);
 }
 
 // Planner over `batch` items of equal length `len` (sparse decode).
-__global__ void mla_plan_uniform_kernel(int len, int batch, int num_parts, int32_t* lens_scratch,
-                                        int32_t* metadata, int32_t* num_splits) {
-  for (int i = threadIdx.x; i < batch; i += blockDim.x) lens_scratch[i] = len;
+__global__ void __launch_bounds__(256) mla_plan_uniform_kernel(int len, int batch, int num_parts,
+                                                               int32_t* tiles_scratch,
+                                                               int32_t* metadata,
+                                                               int32_t* num_splits) {
+  __shared__ int32_t s_tiles[kPlanSmemBatch];
+  int32_t* tiles = batch <= kPlanSmemBatch ? s_tiles : tiles_scratch;
+  for (int i = threadIdx.x; i < batch; i += blockDim.x) tiles[i] = tiles_of(len);
   __syncthreads();
-  if (threadIdx.x == 0) plan_splits(lens_scratch, batch, num_parts, metadata, num_splits);
+  if (threadIdx.x == 0) plan_splits_tiles(tiles, batch, num_parts, metadata, num_splits);
 }
 
 }  // namespace mla

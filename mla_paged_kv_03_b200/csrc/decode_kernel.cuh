@@ -57,6 +57,7 @@ struct DecodeParams {
   int always_partial;  // write split partials even for unsplit sequences (fused)
   float scale_log2;    // softmax_scale * log2(e)
   const int32_t* block_table;
+  const uint8_t* kcache;      // cache base (L2 prefetch of whole pages)
   const int32_t* seqlens;     // per sequence (dense/fused)
   const int32_t* metadata;    // [num_parts][8]
   const int32_t* num_splits;  // [batch + 1] prefix sums
@@ -95,6 +96,7 @@ constexpr int kTmemCols = 512;
 constexpr int kSCol = 0;     // S^T buffers at cols [0,64) and [64,128)
 constexpr int kOCol = 128;   // O^T chunk c at cols 128 + 64c (c < 5)
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr int kPrefetchTiles = 2;  // pages of tile k + kPrefetchTiles are pulled into L2
 }  // namespace cfg
 
 // Softmax warpgroups (32 query-row columns each) and the named barrier that
@@ -125,7 +127,7 @@ struct __align__(8) Ctrl {
   float m[64];          // per-column reference max (log2 domain)
   float alpha[64];      // per-column rescale factor, then 1/l in the epilogue
   int lim[64];          // per-column visible-token limit of the current unit
-  float rope_cs[32][2]; // cos/sin of the current unit's query position
+  double rope_cs[32][2];  // cos/sin of the current unit's query position (fp64)
 };
 static_assert(sizeof(Ctrl) <= cfg::kMiscBytes, "control block too large");
 
@@ -180,9 +182,15 @@ __device__ __forceinline__ bool wg_wait(uint64_t* bar, uint32_t parity, int site
   return all != 0;
 }
 
-// cos/sin of theta = pos * inv_freq: the angle is formed and reduced modulo
-// 2*pi in fp64 (|theta| < 2^31 keeps the reduced angle accurate to ~1e-9), the
-// reduced angle in [-pi, pi] is then evaluated in fp32.
+// cos/sin of theta = pos * inv_freq in fp64 (the fused prologue rounds the
+// rotated query to bf16; computing it in fp64 makes that rounding decision
+// agree with an fp64 reference except at exact ties).
+__device__ __forceinline__ void rope_sincos64(double pos, double inv_freq, double* sn, double* cs) {
+  sincos(pos * inv_freq, sn, cs);
+}
+
+// fp32 cos/sin for the output rotation: the angle is formed and reduced
+// modulo 2*pi in fp64, the reduced angle in [-pi, pi] is evaluated in fp32.
 __device__ __forceinline__ void rope_sincos(double pos, double inv_freq, float* sn, float* cs) {
   const double kTwoPi = 6.283185307179586476925286766559;
   const double theta = pos * inv_freq;
@@ -359,6 +367,16 @@ __global__ void __launch_bounds__(Threads<kMode>::value, 1)
       }
       return true;
     };
+    // Pull both pages of a tile into L2 ahead of the TMA loads (a page is one
+    // contiguous 64 x 1152-byte block).
+    auto prefetch_tile = [&](const Unit& un, int tile) {
+      const int npg = min((un.L + kPage - 1) / kPage, P.max_pages);
+      for (int pg = 2 * tile; pg < 2 * tile + 2 && pg < npg; ++pg) {
+        const int blk = P.block_table[(size_t)un.b * P.max_pages + pg];
+        if (blk >= 0 && blk < P.num_blocks)
+          ptx::prefetch_l2_bulk(P.kcache + (size_t)blk * (kPage * kD * 2), kPage * kD * 2);
+      }
+    };
     while (ok && it.template next<kMode>(P, u)) {
       if (kMode == kFused) {
         ok = ptx::mbar_wait(&C.q_empty, (u_idx & 1) ^ 1, 0x06);
@@ -366,8 +384,8 @@ __global__ void __launch_bounds__(Threads<kMode>::value, 1)
         if (!ok) break;
         const double pos =
             P.positions ? static_cast<double>(P.positions[u.b]) : static_cast<double>(u.L - 1);
-        float sn, cs;
-        rope_sincos(pos, P.inv_freq[lane], &sn, &cs);
+        double sn, cs;
+        rope_sincos64(pos, P.inv_freq[lane], &sn, &cs);
         C.rope_cs[lane][0] = cs;
         C.rope_cs[lane][1] = sn;
         ptx::mbar_arrive(&C.rope_full);
@@ -385,7 +403,9 @@ __global__ void __launch_bounds__(Threads<kMode>::value, 1)
         }
         if (kMode != kSparse && ok) {
           const int n = u.hi - u.lo;
+          for (int k = 0; k < kPrefetchTiles && k < n; ++k) prefetch_tile(u, u.lo + k);
           for (int k = 0; k < n && ok; ++k) {
+            if (k + kPrefetchTiles < n) prefetch_tile(u, u.lo + k + kPrefetchTiles);
             for (int pr = 0; pr < 5 && ok; ++pr) ok = load_pair(u, u.lo + k, pr);
             if (k >= 1)
               for (int pr = 0; pr < nv_pairs && ok; ++pr) ok = load_pair(u, u.lo + k - 1, pr);
@@ -546,53 +566,59 @@ __global__ void __launch_bounds__(Threads<kMode>::value, 1)
           ok = false;
           break;
         }
+        // RMSNorm and RoPE in fp64; one bf16 rounding at the end.
         const int wl = (threadIdx.x - 64) >> 5;  // warp within both groups (0..7)
         for (int r = wl; r < kRowsPerCta; r += 4 * kSoftmaxGroups) {
           const int rg = grp * kRowsPerCta + r;
           const bool valid = rg < P.R;
           const __nv_bfloat16* src = P.q_raw + ((size_t)u.b * P.R + (valid ? rg : 0)) * kD;
-          float x[3][8];
-          float ss = 0.f;
-    #pragma unroll
+          double ss = 0.0;
+#pragma unroll
           for (int j = 0; j < 3; ++j) {
             const int uu = lane + 32 * j;
             if (uu < kD / 8) {
               const uint4 w = *reinterpret_cast<const uint4*>(src + uu * 8);
               const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
-    #pragma unroll
+#pragma unroll
               for (int e = 0; e < 4; ++e) {
                 const float2 f = __bfloat1622float2(h[e]);
-                x[j][2 * e] = f.x;
-                x[j][2 * e + 1] = f.y;
-                ss += f.x * f.x + f.y * f.y;
+                ss = fma(static_cast<double>(f.x), static_cast<double>(f.x), ss);
+                ss = fma(static_cast<double>(f.y), static_cast<double>(f.y), ss);
               }
             }
           }
-    #pragma unroll
+#pragma unroll
           for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-          const float inv = valid ? 1.0f / sqrtf(ss / static_cast<float>(kD) + P.eps) : 0.f;
-    #pragma unroll
+          const double inv = valid ? 1.0 / sqrt(ss / static_cast<double>(kD) + P.eps) : 0.0;
+#pragma unroll 1
           for (int j = 0; j < 3; ++j) {
             const int uu = lane + 32 * j;
             if (uu < kD / 8) {
-              float y[8];
-    #pragma unroll
-              for (int e = 0; e < 8; ++e) y[e] = x[j][e] * inv * __ldg(P.gain + uu * 8 + e);
+              const uint4 w = *reinterpret_cast<const uint4*>(src + uu * 8);
+              const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
+              double y[8];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(h[e]);
+                y[2 * e] = static_cast<double>(f.x) * inv * static_cast<double>(__ldg(P.gain + uu * 8 + 2 * e));
+                y[2 * e + 1] =
+                    static_cast<double>(f.y) * inv * static_cast<double>(__ldg(P.gain + uu * 8 + 2 * e + 1));
+              }
               if (uu >= kNope / 8) {
-    #pragma unroll
+#pragma unroll
                 for (int e = 0; e < 4; ++e) {
                   const int k = (uu * 8 - kNope) / 2 + e;
-                  const float c = C.rope_cs[k][0], sn = C.rope_cs[k][1];
-                  const float a = y[2 * e], bq = y[2 * e + 1];
+                  const double c = C.rope_cs[k][0], sn = C.rope_cs[k][1];
+                  const double a = y[2 * e], bq = y[2 * e + 1];
                   y[2 * e] = a * c - bq * sn;
                   y[2 * e + 1] = a * sn + bq * c;
                 }
               }
               uint4 o;
-              o.x = ptx::pack_bf16x2(y[0], y[1]);
-              o.y = ptx::pack_bf16x2(y[2], y[3]);
-              o.z = ptx::pack_bf16x2(y[4], y[5]);
-              o.w = ptx::pack_bf16x2(y[6], y[7]);
+              o.x = ptx::pack_bf16x2_f64(y[0], y[1]);
+              o.y = ptx::pack_bf16x2_f64(y[2], y[3]);
+              o.z = ptx::pack_bf16x2_f64(y[4], y[5]);
+              o.w = ptx::pack_bf16x2_f64(y[6], y[7]);
               const int c = uu >> 3, unit = uu & 7;
               *reinterpret_cast<uint4*>(sQ + c * (kRowsPerCta * 128) + r * 128 +
                                         ((unit ^ (r & 7)) << 4)) = o;

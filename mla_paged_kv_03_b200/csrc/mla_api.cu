@@ -9,6 +9,7 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <vector>
 
 #include "../../include/mla.h"
 #include "combine_kernel.cuh"
@@ -123,12 +124,10 @@ WsLayout sparse_ws_layout(int pairs, int R, int d_v, int parts) {
 int launch_combine(const mla::CombineParams& cp, bool fused, cudaStream_t st) {
   const long long rows = static_cast<long long>(cp.batch) * cp.R;
   if (rows == 0) return MLA_OK;
-  const int threads = 256;
-  const long long blocks = (rows * 32 + threads - 1) / threads;
   if (fused)
-    mla::mla_combine_kernel<true><<<static_cast<unsigned>(blocks), threads, 0, st>>>(cp);
+    mla::mla_combine_kernel<true><<<static_cast<unsigned>(rows), mla::kCombineThreads, 0, st>>>(cp);
   else
-    mla::mla_combine_kernel<false><<<static_cast<unsigned>(blocks), threads, 0, st>>>(cp);
+    mla::mla_combine_kernel<false><<<static_cast<unsigned>(rows), mla::kCombineThreads, 0, st>>>(cp);
   MLA_CUDA(cudaGetLastError());
   return MLA_OK;
 }
@@ -151,7 +150,8 @@ int check_common_dense(const void* q, const void* kcache, const int32_t* block_t
                        const int32_t* num_splits, int num_sm_parts, void* workspace) {
   MLA_CHECK_ARG(batch >= 0, "batch must be >= 0 (got %d)", batch);
   MLA_CHECK_ARG(h_q >= 1, "h_q must be >= 1 (got %d)", h_q);
-  MLA_CHECK_ARG(num_sm_parts >= 1, "num_sm_parts must be >= 1 (got %d)", num_sm_parts);
+  MLA_CHECK_ARG(num_sm_parts >= 1 && num_sm_parts <= mla::kCombineMaxSplits,
+                "num_sm_parts must be in [1, %d] (got %d)", mla::kCombineMaxSplits, num_sm_parts);
   MLA_CHECK_ARG(max_pages >= 1, "max_pages must be >= 1 (got %d)", max_pages);
   MLA_CHECK_ARG(num_blocks >= 1, "num_blocks must be >= 1 (got %d)", num_blocks);
   MLA_CHECK_ARG(static_cast<long long>(num_blocks) * mla::kPage < (1LL << 31),
@@ -210,9 +210,11 @@ int mla_get_metadata(const int32_t* cache_seqlens, int batch, int heads_per_kv, 
   MLA_CHECK_ARG(heads_per_kv >= 1, "heads_per_kv must be >= 1");
   if (h_kv != 1) return fail(MLA_ERR_UNSUPPORTED, "h_kv must be 1 (got %d)", h_kv);
   MLA_CHECK_ARG(metadata && num_splits && (cache_seqlens || batch == 0), "null device pointer");
-  mla::mla_plan_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(cache_seqlens, batch,
-                                                                         num_sm_parts, metadata,
-                                                                         num_splits);
+  // For batches beyond the kernel's shared-memory staging, num_splits[1..]
+  // doubles as the tile-count scratch: each entry is read before the planner
+  // overwrites it with the prefix sum.
+  mla::mla_plan_kernel<<<1, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      cache_seqlens, batch, num_sm_parts, num_splits + 1, metadata, num_splits);
   MLA_CUDA(cudaGetLastError());
   return MLA_OK;
 }
@@ -225,7 +227,9 @@ int mla_get_metadata_host(const int32_t* cache_seqlens, int batch, int heads_per
   MLA_CHECK_ARG(metadata && num_splits && (cache_seqlens || batch == 0), "null host pointer");
   for (int b = 0; b < batch; ++b)
     MLA_CHECK_ARG(cache_seqlens[b] >= 0, "cache_seqlens[%d] = %d is negative", b, cache_seqlens[b]);
-  mla::plan_splits(cache_seqlens, batch, num_sm_parts, metadata, num_splits);
+  std::vector<int32_t> tiles(static_cast<size_t>(batch));
+  for (int b = 0; b < batch; ++b) tiles[b] = mla::tiles_of(cache_seqlens[b]);
+  mla::plan_splits_tiles(tiles.data(), batch, num_sm_parts, metadata, num_splits);
   return MLA_OK;
 }
 
@@ -277,6 +281,7 @@ int mla_decode_fwd(const void* q, const void* kcache, const int32_t* block_table
   p.always_partial = 0;
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
   p.block_table = block_table;
+  p.kcache = static_cast<const uint8_t*>(kcache);
   p.seqlens = cache_seqlens;
   p.metadata = metadata;
   p.num_splits = num_splits;
@@ -342,6 +347,7 @@ int mla_fused_norm_rope_attn_rope_cast(
   p.always_partial = 1;
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
   p.block_table = block_table;
+  p.kcache = static_cast<const uint8_t*>(kcache);
   p.seqlens = cache_seqlens;
   p.metadata = metadata;
   p.num_splits = num_splits;
@@ -391,7 +397,8 @@ int mla_sparse_decode(const void* q, const uint8_t* kcache_fp8, int64_t num_slot
   MLA_CHECK_ARG(topk >= 1, "topk must be >= 1 (got %d)", topk);
   MLA_CHECK_ARG(num_slots >= 1 && num_slots < (1LL << 31), "num_slots must be in [1, 2^31)");
   MLA_CHECK_ARG(d_v == 512, "sparse decode supports d_v = 512 (got %d)", d_v);
-  MLA_CHECK_ARG(num_sm_parts >= 1, "num_sm_parts must be >= 1");
+  MLA_CHECK_ARG(num_sm_parts >= 1 && num_sm_parts <= mla::kCombineMaxSplits,
+                "num_sm_parts must be in [1, %d]", mla::kCombineMaxSplits);
   MLA_CHECK_ARG(std::isfinite(softmax_scale) && softmax_scale > 0.f,
                 "softmax_scale must be finite and > 0");
   MLA_CHECK_ARG(q && kcache_fp8 && indices && workspace && out && lse, "null device pointer");

@@ -49,16 +49,17 @@ MLA_HD inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
 MLA_HD inline int tiles_of(int L) { return L > 0 ? ceil_div(L, kTileT) : 1; }
 
 // Greedy dealing of tiles to parts with a cost cap `target` per part; a
-// segment costs its tiles plus kSegmentOverheadTiles.  Returns the number of
-// parts used; writes the plan when metadata != nullptr.
-MLA_HD inline int deal_tiles(const int32_t* seqlens, int batch, long long target, int max_parts,
+// segment costs its tiles plus kSegmentOverheadTiles.  `tiles[b]` is
+// tiles_of(seqlens[b]).  Returns the number of parts used (stops counting at
+// max_parts + 1); writes the plan when metadata != nullptr.
+MLA_HD inline int deal_tiles(const int32_t* tiles, int batch, long long target, int max_parts,
                              int32_t* metadata, int32_t* num_splits) {
   int p = 0;
   long long used = 0;
   bool part_open = false;
   if (num_splits) num_splits[0] = 0;
   for (int b = 0; b < batch; ++b) {
-    const int n = tiles_of(seqlens[b]);
+    const int n = tiles[b];
     int t = 0;
     int splits = 0;
     while (t < n) {
@@ -66,11 +67,12 @@ MLA_HD inline int deal_tiles(const int32_t* seqlens, int batch, long long target
         ++p;
         used = 0;
         part_open = false;
+        if (!metadata && p >= max_parts) return max_parts + 1;  // does not fit
       }
       const long long avail = target - used - kSegmentOverheadTiles;
       int take = static_cast<int>(avail < 1 ? 1 : (avail < n - t ? avail : n - t));
-      if (p >= max_parts - 1) take = n - t;  // the last part takes the rest
-      if (metadata && p < max_parts) {
+      if (metadata && p >= max_parts - 1) take = n - t;  // the last part takes the rest
+      if (metadata) {
         int32_t* m = metadata + p * kMetaInts;
         if (!part_open) {
           m[0] = b;
@@ -96,10 +98,12 @@ MLA_HD inline int deal_tiles(const int32_t* seqlens, int batch, long long target
 // writes metadata[num_parts][8] and the prefix sums num_splits[batch + 1]
 // (num_splits[b+1] - num_splits[b] = number of parts holding tiles of
 // sequence b).  Each part covers one contiguous run of (sequence, tile)
-// pairs; unused parts are marked empty (begin_seq > end_seq).  Runs
-// identically on host and device.
-MLA_HD inline void plan_splits(const int32_t* seqlens, int batch, int num_parts,
-                               int32_t* metadata, int32_t* num_splits) {
+// pairs; unused parts are marked empty (begin_seq > end_seq).  The search
+// starts at the lower bound ceil(total / num_parts), which usually fits after
+// a few steps, and falls back to bisection.  `tiles` holds tiles_of() of every
+// sequence.  Runs identically on host and device.
+MLA_HD inline void plan_splits_tiles(const int32_t* tiles, int batch, int num_parts,
+                                     int32_t* metadata, int32_t* num_splits) {
   for (int p = 0; p < num_parts; ++p) {
     int32_t* m = metadata + p * kMetaInts;
     m[0] = batch;  // empty part: begins after every sequence
@@ -109,17 +113,26 @@ MLA_HD inline void plan_splits(const int32_t* seqlens, int batch, int num_parts,
     m[4] = m[5] = m[6] = m[7] = 0;
   }
   long long total = 0;
-  for (int b = 0; b < batch; ++b) total += tiles_of(seqlens[b]) + kSegmentOverheadTiles;
-  long long lo = kSegmentOverheadTiles + 1;
-  long long hi = total > lo ? total : lo;
+  for (int b = 0; b < batch; ++b) total += tiles[b] + kSegmentOverheadTiles;
+  long long lo = (total + num_parts - 1) / num_parts;
+  if (lo < kSegmentOverheadTiles + 1) lo = kSegmentOverheadTiles + 1;
+  long long hi = total > lo ? total : lo;  // one part holding everything always fits
+  // linear probe from the lower bound, then bisection on what remains
+  for (int probe = 0; probe < 4 && lo < hi; ++probe) {
+    if (deal_tiles(tiles, batch, lo, num_parts, nullptr, nullptr) <= num_parts) {
+      hi = lo;
+      break;
+    }
+    ++lo;
+  }
   while (lo < hi) {
     const long long mid = lo + (hi - lo) / 2;
-    if (deal_tiles(seqlens, batch, mid, num_parts + 1, nullptr, nullptr) <= num_parts)
+    if (deal_tiles(tiles, batch, mid, num_parts, nullptr, nullptr) <= num_parts)
       hi = mid;
     else
       lo = mid + 1;
   }
-  deal_tiles(seqlens, batch, lo, num_parts, metadata, num_splits);
+  deal_tiles(tiles, batch, lo, num_parts, metadata, num_splits);
 }
 
 }  // namespace mla

@@ -7,6 +7,7 @@
 #pragma once
 #include <cstdint>
 #include <cuda.h>
+#include <cuda_bf16.h>
 
 #include "mla_common.h"
 
@@ -106,6 +107,11 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
       : "memory");
+}
+
+// Prefetch `bytes` (multiple of 16, 16-byte aligned) of global memory into L2.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* gptr, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(gptr), "r"(bytes) : "memory");
 }
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
@@ -231,6 +237,14 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %2, %1;" : "=r"(r) : "f"(lo), "f"(hi));
   return r;
+}
+
+// fp64 -> bf16 with one rounding (round to nearest even), packed as a pair.
+__device__ __forceinline__ uint32_t pack_bf16x2_f64(double lo, double hi) {
+  const __nv_bfloat16 l = __double2bfloat16(lo);
+  const __nv_bfloat16 h = __double2bfloat16(hi);
+  return static_cast<uint32_t>(__bfloat16_as_ushort(l)) |
+         (static_cast<uint32_t>(__bfloat16_as_ushort(h)) << 16);
 }
 
 }  // namespace ptx

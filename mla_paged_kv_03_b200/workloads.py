@@ -149,7 +149,7 @@ def make_dense(seqlens, s_q, h_q, *, seed=0, q_std=1.0, k_std=1.0, d_v=D_NOPE, c
     gd = gen_device or device
     g = _gen(seed, gd)
     b = len(seqlens)
-    bt, nb = paged_block_table(seqlens, g, spare_blocks)
+    bt, nb = paged_block_table(seqlens, g, spare_blocks, device=g.device)
     kcache = _randn_bf16((nb, PAGE, 1, D_QK), g, std=k_std, chunk_rows=4096)
     q = _randn_bf16((b, s_q, h_q, D_QK), g, std=q_std)
     sl = torch.tensor([int(x) for x in seqlens], dtype=torch.int32)
@@ -192,7 +192,7 @@ def memory_bound(seed=0, device="cpu", batch=128, lo=1024, hi=16384):
 def fused(seed=0, device="cpu", batch=32, lo=2048, hi=32768, h_q=64, seqlens=None):
     sl = seqlens if seqlens is not None else lengths_uniform(batch, lo, hi, seed)
     g = _gen(seed, device)
-    bt, nb = paged_block_table(sl, g)
+    bt, nb = paged_block_table(sl, g, device=g.device)
     kcache = _randn_bf16((nb, PAGE, 1, D_QK), g, chunk_rows=4096)
     q_raw = _randn_bf16((len(sl), 1, h_q, D_QK), g)
     gain = (1.0 + 0.1 * torch.randn((D_QK,), generator=g, device=g.device,
@@ -228,7 +228,7 @@ def sparse(seed=0, device="cpu", batch=32, h_q=128, s_q=1, seqlen=65536, topk=20
     gd = device
     g = _gen(seed, gd)
     sl = seqlens if seqlens is not None else [seqlen] * batch
-    bt, nb = paged_block_table(sl, g)
+    bt, nb = paged_block_table(sl, g, device=g.device)
     n_rows = nb * PAGE
     cache = torch.empty((n_rows, ROW656), dtype=torch.uint8, device=g.device)
     step = 1 << 16

@@ -50,6 +50,11 @@ def assert_fp8_close(codes, scale, ref_codes, ref_scale, min_equal=0.999):
     eq = (c == ref_codes).mean()
     assert eq >= min_equal, f"only {eq:.5f} of E4M3 codes equal the oracle's"
     nb = e4m3_neighbours(c, ref_codes)
-    assert nb.all(), f"{(~nb).sum()} codes more than one step from the oracle's"
+    if not nb.all():
+        bad = np.argwhere(~nb)[:5]
+        det = [(tuple(int(v) for v in i), hex(int(c[tuple(i)])), hex(int(ref_codes[tuple(i)])))
+               for i in bad]
+        raise AssertionError(f"{(~nb).sum()} codes more than one step from the oracle's: "
+                             f"(index, gpu, oracle) {det}")
     rel = np.abs(s - ref_scale) / np.maximum(np.abs(ref_scale), 1e-30)
     assert (rel <= 1e-3).all(), f"scale rel err {rel.max():.3e}"
