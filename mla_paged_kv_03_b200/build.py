@@ -39,11 +39,13 @@ def _stale():
     return any(os.path.getmtime(d) > t for d in DEPS)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not _stale():
+def build(force: bool = False, verbose: bool = False, out: str = None, defines=()) -> str:
+    """Compile libmla_b200.so (or `out`, with extra -D `defines`)."""
+    target = out or LIB
+    if not force and not defines and out is None and not _stale():
         return LIB
-    cmd = [NVCC] + FLAGS + ["-I", os.path.join(ROOT, "include"), "-o", LIB] + SOURCES + \
-        ["-lcudart"]
+    cmd = [NVCC] + FLAGS + [f"-D{d}" for d in defines] + \
+        ["-I", os.path.join(ROOT, "include"), "-o", target] + SOURCES + ["-lcudart"]
     r = subprocess.run(cmd, capture_output=True, text=True)
     log = r.stdout + r.stderr
     if r.returncode != 0:
@@ -52,15 +54,16 @@ def build(force: bool = False, verbose: bool = False) -> str:
     spills = [l for l in log.splitlines()
               if (m := re.search(r"(\d+) bytes spill stores", l)) and int(m.group(1)) > SPILL_LIMIT]
     if spills:
-        if os.path.exists(LIB):
-            os.remove(LIB)
+        if os.path.exists(target):
+            os.remove(target)
         sys.stderr.write(log)
         raise RuntimeError("register spill in libmla_b200 kernels:\n" + "\n".join(spills))
     if verbose:
         sys.stderr.write(log)
-    with open(os.path.join(HERE, "ptxas_report.txt"), "w") as f:
-        f.write(log)
-    return LIB
+    if out is None:
+        with open(os.path.join(HERE, "ptxas_report.txt"), "w") as f:
+            f.write(log)
+    return target
 
 
 if __name__ == "__main__":

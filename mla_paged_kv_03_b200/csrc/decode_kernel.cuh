@@ -83,8 +83,14 @@ namespace cfg {
 constexpr int kQBytes = kNumChunks * kRowsPerCta * 128;  // 73728
 constexpr int kSubChunk = kTileT * 128;                  // 16384: [128 tok][64 d] bf16
 constexpr int kPairBytes = 2 * kSubChunk;                // 32768
-constexpr int kNPair = 3;                                // ring depth (pair slots)
-constexpr int kNP = 2;                                   // P buffer regions
+#ifndef MLA_RING_PAIRS
+#define MLA_RING_PAIRS 3
+#endif
+#ifndef MLA_P_BUFFERS
+#define MLA_P_BUFFERS 2
+#endif
+constexpr int kNPair = MLA_RING_PAIRS;                   // ring depth (pair slots)
+constexpr int kNP = MLA_P_BUFFERS;                       // P buffer regions
 constexpr int kPBytes = kTileT * 128;                    // [128 tok][64 rows] bf16
 constexpr int kQOff = 0;
 constexpr int kRingOff = kQOff + kQBytes;
@@ -96,7 +102,10 @@ constexpr int kTmemCols = 512;
 constexpr int kSCol = 0;     // S^T buffers at cols [0,64) and [64,128)
 constexpr int kOCol = 128;   // O^T chunk c at cols 128 + 64c (c < 5)
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-constexpr int kPrefetchTiles = 2;  // pages of tile k + kPrefetchTiles are pulled into L2
+#ifndef MLA_PREFETCH_TILES
+#define MLA_PREFETCH_TILES 0
+#endif
+constexpr int kPrefetchTiles = MLA_PREFETCH_TILES;  // pages of tile k + this are pulled into L2
 }  // namespace cfg
 
 // Softmax warpgroups (32 query-row columns each) and the named barrier that
@@ -288,6 +297,7 @@ __global__ void __launch_bounds__(Threads<kMode>::value, 1)
   // holding P as a bf16 hi/lo pair so that PV sees P to ~16 bits.
   constexpr bool kPSplit = (kMode == kFused);
   constexpr int NPm = kPSplit ? 1 : kNP;
+  static_assert(!kPSplit || kNP >= 2, "the hi/lo P pair needs two P buffer regions");
 
   const int32_t* meta = P.metadata + part * kMetaInts;
   if (meta[0] > meta[2]) return;  // empty part: nothing to do (uniform exit)
@@ -448,25 +458,31 @@ __global__ void __launch_bounds__(Threads<kMode>::value, 1)
         addr = ring_addr + slot * kPairBytes;
         return slot;
       };
+      // Descriptor words of each operand's base; inner loops only add offsets.
+      const ptx::DescWords dq = ptx::desc_words(q_addr, 16, 1024, ptx::kLayoutSW128);
+      const ptx::DescWords dring = ptx::desc_words(ring_addr, 16, 1024, ptx::kLayoutSW128);
+      const ptx::DescWords dv = ptx::desc_words(ring_addr, kSubChunk, 1024, ptx::kLayoutSW128);
+      const ptx::DescWords dp = ptx::desc_words(p_addr, 16, 1024, ptx::kLayoutSW128);
       auto do_qk = [&](uint32_t g) -> bool {
         const int sb = g & 1;
         if (!ptx::mbar_wait(&C.s_empty[sb], ((g >> 1) & 1) ^ 1, 0x12)) return false;
         ptx::tc_fence_after();
         const uint32_t d_tmem = tmem + kSCol + sb * kRowsPerCta;
+#pragma unroll
         for (int pr = 0; pr < 5; ++pr) {
           uint32_t a0;
           const int slot = wait_slot(a0);
           if (slot < 0) return false;
+          const uint32_t a_lo = dring.lo + ((slot * kPairBytes) >> 4);
+#pragma unroll
           for (int j = 0; j < 2; ++j) {
             const int c = 2 * pr + j;
-            if (c >= kNumChunks) break;
+            if (c < kNumChunks) {
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t ad = ptx::smem_desc(a0 + j * kSubChunk + kk * 32, 16, 1024,
-                                                 ptx::kLayoutSW128);
-              const uint64_t bd = ptx::smem_desc(q_addr + c * (kRowsPerCta * 128) + kk * 32, 16,
-                                                 1024, ptx::kLayoutSW128);
-              ptx::umma_f16_ss(d_tmem, ad, bd, idesc_qk, (c | kk) ? 1u : 0u);
+              for (int kk = 0; kk < 4; ++kk)
+                ptx::umma_f16_ss_w(d_tmem, a_lo + ((j * kSubChunk + kk * 32) >> 4), dring.hi,
+                                   dq.lo + ((c * (kRowsPerCta * 128) + kk * 32) >> 4), dq.hi,
+                                   idesc_qk, (c | kk) ? 1u : 0u);
             }
           }
           ptx::umma_commit(&C.slot_empty[slot]);
@@ -478,23 +494,23 @@ __global__ void __launch_bounds__(Threads<kMode>::value, 1)
         const int pb = g % NPm;
         if (!ptx::mbar_wait(&C.p_full[pb], (g / NPm) & 1, 0x13)) return false;
         ptx::tc_fence_after();
-        const uint32_t pbuf = p_addr + pb * kPBytes;
+        const uint32_t b_lo = dp.lo + ((pb * kPBytes) >> 4);
         for (int pr = 0; pr < nv_pairs; ++pr) {
           uint32_t a0;
           const int slot = wait_slot(a0);
           if (slot < 0) return false;
           const uint32_t d_tmem = tmem + kOCol + pr * kRowsPerCta;
+          const uint32_t a_lo = dv.lo + ((slot * kPairBytes) >> 4);
+          // first k-step of the unit's first tile starts the accumulator
+          ptx::umma_f16_ss_w(d_tmem, a_lo, dv.hi, b_lo, dp.hi, idesc_pv, first_of_unit ? 0u : 1u);
+          if (kPSplit) ptx::umma_f16_ss_w(d_tmem, a_lo, dv.hi, b_lo + (kPBytes >> 4), dp.hi, idesc_pv, 1u);
 #pragma unroll
-          for (int kk = 0; kk < kTileT / 16; ++kk) {
-            const uint64_t ad =
-                ptx::smem_desc(a0 + kk * 2048, kSubChunk, 1024, ptx::kLayoutSW128);
-            const uint64_t bd = ptx::smem_desc(pbuf + kk * 2048, 16, 1024, ptx::kLayoutSW128);
-            ptx::umma_f16_ss(d_tmem, ad, bd, idesc_pv, (first_of_unit && kk == 0) ? 0u : 1u);
-            if (kPSplit) {  // + V^T . P_lo^T
-              const uint64_t bl =
-                  ptx::smem_desc(pbuf + kPBytes + kk * 2048, 16, 1024, ptx::kLayoutSW128);
-              ptx::umma_f16_ss(d_tmem, ad, bl, idesc_pv, 1u);
-            }
+          for (int kk = 1; kk < kTileT / 16; ++kk) {
+            ptx::umma_f16_ss_w(d_tmem, a_lo + ((kk * 2048) >> 4), dv.hi, b_lo + ((kk * 2048) >> 4),
+                               dp.hi, idesc_pv, 1u);
+            if (kPSplit)  // + V^T . P_lo^T
+              ptx::umma_f16_ss_w(d_tmem, a_lo + ((kk * 2048) >> 4), dv.hi,
+                                 b_lo + ((kPBytes + kk * 2048) >> 4), dp.hi, idesc_pv, 1u);
           }
           ptx::umma_commit(&C.slot_empty[slot]);
         }

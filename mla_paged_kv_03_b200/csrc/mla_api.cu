@@ -14,6 +14,7 @@
 #include "../../include/mla.h"
 #include "combine_kernel.cuh"
 #include "decode_kernel.cuh"
+#include "pair_kernel.cuh"
 #include "mla_common.h"
 
 namespace {
@@ -144,6 +145,35 @@ int launch_decode(const CUtensorMap& tq, const CUtensorMap& tkv, const mla::Deco
   return MLA_OK;
 }
 
+// 2-CTA kernel for more than 64 query rows per KV head: clusters of two CTAs,
+// one pair per scheduler part and 128-row group.
+int launch_pair_decode(const CUtensorMap& tq, const CUtensorMap& tkv, const mla::DecodeParams& p,
+                       cudaStream_t st) {
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(mla::mla_pair_decode_kernel,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    mla::pcfg::kSmemBytes);
+  });
+  if (attr_err != cudaSuccess)
+    return fail(MLA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(attr_err));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * p.num_parts * p.n_groups), 1, 1);
+  cfg.blockDim = dim3(mla::pcfg::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = mla::pcfg::kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  MLA_CUDA(cudaLaunchKernelEx(&cfg, mla::mla_pair_decode_kernel, tq, tkv, p));
+  return MLA_OK;
+}
+
 int check_common_dense(const void* q, const void* kcache, const int32_t* block_table,
                        int max_pages, int num_blocks, const int32_t* cache_seqlens, int batch,
                        int h_q, float softmax_scale, const int32_t* metadata,
@@ -253,7 +283,7 @@ int mla_decode_fwd(const void* q, const void* kcache, const int32_t* block_table
                               h_q, softmax_scale, metadata, num_splits, num_sm_parts, workspace);
   if (rc != MLA_OK) return rc;
   MLA_CHECK_ARG(out && lse, "null output pointer");
-  MLA_CHECK_ARG(aligned(out, 8) && aligned(lse, 4), "out must be 8-byte aligned, lse 4-byte");
+  MLA_CHECK_ARG(aligned(out, 16) && aligned(lse, 4), "out must be 16-byte aligned, lse 4-byte");
   const int R = s_q * h_q;
   const WsLayout w = dense_ws_layout(batch, R, d_v, num_sm_parts);
   MLA_CHECK_ARG(workspace_bytes >= w.total, "workspace too small: %zu < %zu", workspace_bytes,
@@ -289,7 +319,12 @@ int mla_decode_fwd(const void* q, const void* kcache, const int32_t* block_table
   p.lse = lse;
   p.ws_o = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.o_off);
   p.ws_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.lse_off);
-  if ((rc = launch_decode<mla::kDense>(tq, tkv, p, st)) != MLA_OK) return rc;
+  if (R > mla::kRowsPerCta && d_v == 512) {
+    p.n_groups = mla::ceil_div(R, 2 * mla::kRowsPerCta);
+    if ((rc = launch_pair_decode(tq, tkv, p, st)) != MLA_OK) return rc;
+  } else if ((rc = launch_decode<mla::kDense>(tq, tkv, p, st)) != MLA_OK) {
+    return rc;
+  }
 
   mla::CombineParams cp{};
   cp.batch = batch;
