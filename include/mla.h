@@ -30,7 +30,8 @@
  * Conventions shared by every entry point
  *   - All tensor pointers are DEVICE pointers owned by the caller, unless an
  *     argument says "host".  The library allocates no device memory; scratch
- *     space is the caller's `workspace` (size from the *_size queries).
+ *     space is the caller's `workspace` (size from the *_size queries),
+ *     except for mla_decode_fwd_noalloc, which uses a fixed array of its own.
  *   - Layouts are dense, row-major, innermost dimension last:
  *       q            [batch, s_q, h_q, 576]        bf16 (16-byte aligned)
  *       kcache       [num_blocks, 64, 1, 576]      bf16 (16-byte aligned)
@@ -174,6 +175,32 @@ MLA_API int mla_sparse_decode(const void* q, const uint8_t* kcache_fp8, int64_t 
                       const int32_t* indices, int topk, int batch, int s_q, int h_q, int d_v,
                       float softmax_scale, int num_sm_parts, void* workspace,
                       size_t workspace_bytes, void* out, float* lse, void* stream);
+
+/* Dense decode without a caller workspace.  This entry point has no
+ * counterpart in the method's published interface; it exists for callers
+ * that cannot supply scratch memory at decode time (an embedder whose device
+ * memory belongs to another allocator, or a caller that must not allocate at
+ * that moment).  Arguments, layouts and results are those of mla_decode_fwd;
+ * the split planner runs inside the call.
+ *   Scratch   the split tables and fp32 partials live in one fixed array of
+ *             mla_noalloc_scratch_bytes() (32 MiB) bytes inside the
+ *             library's device image; this call allocates no device memory.
+ *   Limit     a problem whose tables + partials exceed that size
+ *             ((batch + parts) * s_q*h_q * d_v * 4 bytes dominate, parts =
+ *             mla_num_sm_parts(device, s_q*h_q, 1)) returns
+ *             MLA_ERR_INVALID_ARG with the bytes it would need.
+ *   Device    the current CUDA device; `stream` must belong to it.  The
+ *             first call on each device looks up the array's address once;
+ *             make that first call outside any stream capture.
+ *   Sharing   every call on a device uses the same array: calls that may
+ *             run at the same time on the GPU (unordered streams) race and
+ *             give wrong results.  Order them, e.g. on one stream.
+ *             Nothing in the array needs to be zeroed first. */
+MLA_API size_t mla_noalloc_scratch_bytes(void);
+MLA_API int mla_decode_fwd_noalloc(const void* q, const void* kcache, const int32_t* block_table,
+                           int max_pages, int num_blocks, const int32_t* cache_seqlens, int batch,
+                           int s_q, int h_q, int h_kv, int d_v, float softmax_scale, int causal,
+                           void* out, float* lse, void* stream);
 
 /* Reads the device status word that kernels set when a bounded wait expires
  * or an out-of-range block id / index is met: 0 = ok, else (code << 16) |

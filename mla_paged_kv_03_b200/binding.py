@@ -28,7 +28,7 @@ EXPORTED = [
     "mla_last_error", "mla_num_sms", "mla_num_sm_parts", "mla_metadata_size",
     "mla_get_metadata", "mla_get_metadata_host", "mla_workspace_size", "mla_decode_fwd",
     "mla_fused_norm_rope_attn_rope_cast", "mla_sparse_workspace_size", "mla_sparse_decode",
-    "mla_device_status",
+    "mla_device_status", "mla_noalloc_scratch_bytes", "mla_decode_fwd_noalloc",
 ]
 
 
@@ -70,9 +70,13 @@ def lib():
         L.mla_sparse_decode.argtypes = [vp, vp, i64, vp, i32, i32, i32, i32, i32, f32, i32, vp,
                                         sz, vp, vp, vp]
         L.mla_device_status.argtypes = [ip, i32]
+        L.mla_noalloc_scratch_bytes.argtypes = []
+        L.mla_decode_fwd_noalloc.argtypes = [vp, vp, vp, i32, i32, vp, i32, i32, i32, i32, i32,
+                                             f32, i32, vp, vp, vp]
         for name in EXPORTED:
-            if name != "mla_last_error":
+            if name not in ("mla_last_error", "mla_noalloc_scratch_bytes"):
                 getattr(L, name).restype = ctypes.c_int
+        L.mla_noalloc_scratch_bytes.restype = ctypes.c_size_t
         _lib = L
     return _lib
 
@@ -183,6 +187,38 @@ def mla_decode_fwd(q: torch.Tensor, kcache: torch.Tensor, block_table: torch.Ten
         s_q, h_q, h_kv, int(d_v), float(softmax_scale), int(bool(causal)), _ptr(metadata),
         _ptr(num_splits), int(num_sm_parts), _ptr(ws), ws.numel(), _ptr(out), _ptr(lse),
         _stream(q.device)))
+    return out, lse
+
+
+def mla_noalloc_scratch_bytes() -> int:
+    return int(lib().mla_noalloc_scratch_bytes())
+
+
+def mla_decode_fwd_noalloc(q: torch.Tensor, kcache: torch.Tensor, block_table: torch.Tensor,
+                           cache_seqlens: torch.Tensor, d_v: int, causal: bool = True,
+                           softmax_scale: Optional[float] = None, out=None, lse=None):
+    """Dense paged decode with the planner run inside the call and all scratch
+    in the library's fixed device array (no workspace argument).  The output
+    tensors are allocated here unless given; the C call itself allocates
+    nothing.  Calls on one device share the scratch array: keep them ordered."""
+    _require(q.dim() == 4 and q.shape[-1] == D_QK and q.dtype == torch.bfloat16,
+             "q must be [b, s_q, h_q, 576] bf16")
+    _require(kcache.dim() == 4 and kcache.shape[1] == 64 and kcache.shape[-1] == D_QK and
+             kcache.dtype == torch.bfloat16, "kcache must be [NB, 64, h_kv, 576] bf16")
+    b, s_q, h_q, _ = q.shape
+    q = q.contiguous()
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(D_QK)
+    if out is None:
+        out = torch.empty((b, s_q, h_q, d_v), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((b, s_q, h_q), dtype=torch.float32, device=q.device)
+    bt = block_table.contiguous()
+    with torch.cuda.device(q.device):
+        _check(lib().mla_decode_fwd_noalloc(
+            _ptr(q), _ptr(kcache), _ptr(bt), bt.shape[1], kcache.shape[0], _ptr(cache_seqlens),
+            b, s_q, h_q, kcache.shape[2], int(d_v), float(softmax_scale), int(bool(causal)),
+            _ptr(out), _ptr(lse), _stream(q.device)))
     return out, lse
 
 

@@ -198,9 +198,91 @@ int check_common_dense(const void* q, const void* kcache, const int32_t* block_t
   return MLA_OK;
 }
 
+// ------------------------------------------------- fixed-scratch decode
+//
+// Some callers cannot hand the library a workspace: an embedder whose device
+// memory is owned by another allocator (every byte pre-reserved for the KV
+// cache pool), or code that must not call an allocator at the moment it
+// decodes.  mla_decode_fwd_noalloc serves them from one scratch array that
+// lives in the library's own device image.  Every call on a device shares the
+// array, so calls whose work may overlap on the GPU (different streams, no
+// ordering between them) race on it; callers order them on one stream.
+// Nothing in the array needs to start at zero: the planner writes the split
+// tables and the decode kernel writes every partial the combine reads.
+
+constexpr size_t kStaticScratchBytes = static_cast<size_t>(32) << 20;
+constexpr int kStaticScratchMaxDevices = 64;
+
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+// Device address of g_static_scratch on the current device.  The first call
+// on a device looks the symbol up (once, with that device current); later
+// calls read the cached pointer.
+int static_scratch_ptr(void** ptr) {
+  int dev = -1;
+  MLA_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kStaticScratchMaxDevices)
+    return fail(MLA_ERR_UNSUPPORTED, "device ordinal %d beyond %d", dev, kStaticScratchMaxDevices);
+  static std::mutex mu;
+  static void* table[kStaticScratchMaxDevices] = {};
+  std::lock_guard<std::mutex> lk(mu);
+  if (!table[dev]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess || !p)
+      return fail(MLA_ERR_CUDA, "cudaGetSymbolAddress(scratch) on device %d: %s", dev,
+                  cudaGetErrorString(e));
+    table[dev] = p;
+  }
+  *ptr = table[dev];
+  return MLA_OK;
+}
+
 }  // namespace
 
 extern "C" {
+
+size_t mla_noalloc_scratch_bytes(void) { return kStaticScratchBytes; }
+
+int mla_decode_fwd_noalloc(const void* q, const void* kcache, const int32_t* block_table,
+                           int max_pages, int num_blocks, const int32_t* cache_seqlens, int batch,
+                           int s_q, int h_q, int h_kv, int d_v, float softmax_scale, int causal,
+                           void* out, float* lse, void* stream) {
+  if (h_kv != 1) return fail(MLA_ERR_UNSUPPORTED, "h_kv must be 1 (got %d)", h_kv);
+  MLA_CHECK_ARG(batch >= 0, "batch must be >= 0 (got %d)", batch);
+  MLA_CHECK_ARG(s_q >= 1 && h_q >= 1, "s_q and h_q must be >= 1");
+  MLA_CHECK_ARG(d_v == 512 || d_v == 576, "d_v must be 512 or 576 (got %d)", d_v);
+  if (batch == 0) return MLA_OK;
+  int dev = -1;
+  MLA_CUDA(cudaGetDevice(&dev));
+  const int R = s_q * h_q;
+  int parts = 0;
+  int rc = mla_num_sm_parts(dev, R, h_kv, &parts);
+  if (rc != MLA_OK) return rc;
+  // [metadata parts x 8 int32 | num_splits batch+1 int32 | decode workspace]
+  const size_t meta_bytes = align_up(static_cast<size_t>(parts) * mla::kMetaInts * 4, 256);
+  const size_t splits_bytes = align_up((static_cast<size_t>(batch) + 1) * 4, 256);
+  const size_t ws_bytes = dense_ws_layout(batch, R, d_v, parts).total;
+  const size_t need = meta_bytes + splits_bytes + ws_bytes;
+  if (need > kStaticScratchBytes)
+    return fail(MLA_ERR_INVALID_ARG,
+                "mla_decode_fwd_noalloc: batch %d x %d rows x d_v %d needs %zu scratch bytes, "
+                "above the fixed %zu; use mla_decode_fwd with a caller workspace",
+                batch, R, d_v, need, kStaticScratchBytes);
+  void* base = nullptr;
+  if ((rc = static_scratch_ptr(&base)) != MLA_OK) return rc;
+  uint8_t* b8 = static_cast<uint8_t*>(base);
+  int32_t* metadata = reinterpret_cast<int32_t*>(b8);
+  int32_t* num_splits = reinterpret_cast<int32_t*>(b8 + meta_bytes);
+  void* ws = b8 + meta_bytes + splits_bytes;
+  if ((rc = mla_get_metadata(cache_seqlens, batch, R, h_kv, parts, metadata, num_splits,
+                             stream)) != MLA_OK)
+    return rc;
+  return mla_decode_fwd(q, kcache, block_table, max_pages, num_blocks, cache_seqlens, batch, s_q,
+                        h_q, h_kv, d_v, softmax_scale, causal, metadata, num_splits, parts, ws,
+                        ws_bytes, out, lse, stream);
+}
+
 
 const char* mla_last_error(void) { return g_err.c_str(); }
 
