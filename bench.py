@@ -48,6 +48,34 @@ WORKLOAD_INFO = {
 }
 
 
+def kernel_source_hash():
+    """Hash of the CUDA sources; a stored ncu traffic figure is used only while
+    the kernels are unchanged since it was captured."""
+    import hashlib
+    d = os.path.join(ROOT, "mla_paged_kv_03_b200", "csrc")
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(d)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(d, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic(workload):
+    """dram bytes read + written per launch of the attention kernel from the
+    committed ncu summary, or None if absent or taken on other sources."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        e = d.get(workload)
+        if e and e.get("source_hash") == kernel_source_hash():
+            return e["bytes_per_launch"]
+    except Exception:
+        pass
+    return None
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -174,6 +202,67 @@ class GpuStep:
         return self.case.q_raw if self.kind == "fused" else self.case.q
 
 
+class ClockSampler:
+    """SM clock and throttle reasons of the bench's GPU sampled through NVML
+    every ~2 ms on a background thread while the timed region runs."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, dev):
+        import threading
+        self.samples = []
+        self.h = None
+        self.stop_flag = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(dev)
+            try:
+                bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+                self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(dev.index)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.reasons_fn = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                getattr(pynvml, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        except Exception:
+            self.h = None
+        self.thread = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        while not self.stop_flag.is_set():
+            try:
+                mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                self.samples.append((mhz, int(self.reasons_fn(self.h))))
+            except Exception:
+                return
+            time.sleep(0.002)
+
+    def start(self):
+        if self.h is not None:
+            self.thread.start()
+        return self
+
+    def stop(self):
+        if self.h is None:
+            return None
+        self.stop_flag.set()
+        self.thread.join(timeout=5)
+        if not self.samples:
+            return None
+        reasons = set()
+        for _, bits in self.samples:
+            for bit, name in self.REASONS.items():
+                if bits & bit:
+                    reasons.add(name)
+        mhz = [m for m, _ in self.samples]
+        return {"sm_mhz": statistics.median(mhz), "sm_min_mhz": min(mhz),
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(reasons),
+                "samples": len(mhz), "source": "nvml"}
+
+
 def sample_clocks_start(dev_index):
     path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{os.getpid()}.csv")
     try:
@@ -233,21 +322,33 @@ def run_gpu_arm(args, rank, world):
     if status != 0:
         raise RuntimeError(f"device status {status:#x} after warm-up")
 
+    # per-step event pairs around the attention kernel (the dominant launch),
+    # recorded by the library on the launching stream
+    k_start = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    k_stop = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    for e in k_start + k_stop:
+        e.record(st)  # creates the CUDA event behind the handle
+    torch.cuda.synchronize(dev)
+
     if world > 1:
         torch.distributed.barrier()
-    clk = sample_clocks_start(dev.index)
+    sampler = ClockSampler(dev).start()
+    clk = None if sampler.h is not None else sample_clocks_start(dev.index)
     torch.cuda.synchronize(dev)
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
     ev0.record(st)
-    for _ in range(args.steps):
+    for i in range(args.steps):
+        gs.B.mla_set_kernel_events(k_start[i], k_stop[i])
         gs.step()
     ev1.record(st)
     torch.cuda.synchronize(dev)
+    gs.B.mla_set_kernel_events(None, None)
     ms_total = ev0.elapsed_time(ev1)
+    ms_kernel = sum(a.elapsed_time(b) for a, b in zip(k_start, k_stop)) / args.steps
     if world > 1:
         torch.distributed.barrier()
-    clocks = sample_clocks_stop(clk)
+    clocks = sampler.stop() if clk is None else sample_clocks_stop(clk)
 
     # end to end through the same API with host buffers: H2D of the step's
     # query from pinned memory, the step, D2H of the outputs
@@ -279,12 +380,12 @@ def run_gpu_arm(args, rank, world):
         raise RuntimeError(f"device status {status:#x} after timing")
 
     ms_step = ms_total / args.steps
-    t = torch.tensor([ms_step, e2e_ms], dtype=torch.float64, device=dev)
+    t = torch.tensor([ms_step, e2e_ms, ms_kernel], dtype=torch.float64, device=dev)
     w = torch.tensor([flops, kv_bytes], dtype=torch.float64, device=dev)
     if world > 1:
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         torch.distributed.all_reduce(w, op=torch.distributed.ReduceOp.SUM)
-    ms_step, e2e_ms = float(t[0]), float(t[1])
+    ms_step, e2e_ms, ms_kernel = float(t[0]), float(t[1]), float(t[2])
     flops_all, kv_all = float(w[0]), float(w[1])
     if rank != 0:
         return None
@@ -293,21 +394,23 @@ def run_gpu_arm(args, rank, world):
     desc, bound = WORKLOAD_INFO[args.workload]
     tflops = flops_all / (ms_step * 1e-3) / 1e12
     gbs = kv_all / (ms_step * 1e-3) / 1e9
-    # dominant kernel: the decode call (decode + combine kernels), one per step
-    per_launch_s = ms_step * 1e-3
+    # dominant kernel: the attention kernel, one launch per step, timed alone
+    per_launch_s = ms_kernel * 1e-3
+    traffic = load_traffic(args.workload)
     if bound == "tensor":
         achieved = flops / per_launch_s / 1e12
         peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
         roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
                 "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                 "peak_source": f"{peak_src} bf16 sustained (burst {peaks['bf16_tflops']})",
-                "frac_of_burst": round(achieved / peaks["bf16_tflops"], 4), "traffic": None}
+                "frac_of_burst": round(achieved / peaks["bf16_tflops"], 4), "traffic": traffic,
+                "kernel_ms": round(ms_kernel, 5)}
     else:
         achieved = total_bytes / per_launch_s / 1e9
         peak = peaks["hbm_gbs"]
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "peak_source": f"{peak_src} hbm copy",
-                "traffic": None}
+                "traffic": traffic, "kernel_ms": round(ms_kernel, 5)}
     line = {
         "metric": METRIC,
         "value": round(tflops, 3),

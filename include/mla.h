@@ -202,6 +202,15 @@ MLA_API int mla_decode_fwd_noalloc(const void* q, const void* kcache, const int3
                            int s_q, int h_q, int h_kv, int d_v, float softmax_scale, int causal,
                            void* out, float* lse, void* stream);
 
+/* Profiling aid, with no counterpart in the method's published interface:
+ * while set, every decode entry point records `start_event` on its stream
+ * right before it launches its attention kernel and `stop_event` right after,
+ * so that a caller can time that kernel alone (cudaEventElapsedTime) next to
+ * the planner and combine launches of the same call.  Both are cudaEvent_t
+ * handles owned by the caller (NULL = do not record).  The setting belongs to
+ * the calling host thread; pass NULL, NULL to clear it. */
+MLA_API int mla_set_kernel_events(void* start_event, void* stop_event);
+
 /* Reads the device status word that kernels set when a bounded wait expires
  * or an out-of-range block id / index is met: 0 = ok, else (code << 16) |
  * site, code 1 = timeout, 2 = bad index.  Synchronises the device; reset != 0

@@ -29,6 +29,7 @@ EXPORTED = [
     "mla_get_metadata", "mla_get_metadata_host", "mla_workspace_size", "mla_decode_fwd",
     "mla_fused_norm_rope_attn_rope_cast", "mla_sparse_workspace_size", "mla_sparse_decode",
     "mla_device_status", "mla_noalloc_scratch_bytes", "mla_decode_fwd_noalloc",
+    "mla_set_kernel_events",
 ]
 
 
@@ -71,6 +72,7 @@ def lib():
                                         sz, vp, vp, vp]
         L.mla_device_status.argtypes = [ip, i32]
         L.mla_noalloc_scratch_bytes.argtypes = []
+        L.mla_set_kernel_events.argtypes = [vp, vp]
         L.mla_decode_fwd_noalloc.argtypes = [vp, vp, vp, i32, i32, vp, i32, i32, i32, i32, i32,
                                              f32, i32, vp, vp, vp]
         for name in EXPORTED:
@@ -188,6 +190,14 @@ def mla_decode_fwd(q: torch.Tensor, kcache: torch.Tensor, block_table: torch.Ten
         _ptr(num_splits), int(num_sm_parts), _ptr(ws), ws.numel(), _ptr(out), _ptr(lse),
         _stream(q.device)))
     return out, lse
+
+
+def mla_set_kernel_events(start: Optional[torch.cuda.Event], stop: Optional[torch.cuda.Event]):
+    """Record `start` / `stop` around the attention kernel of the following
+    decode calls of this thread (None, None clears)."""
+    _check(lib().mla_set_kernel_events(
+        None if start is None else ctypes.c_void_p(start.cuda_event),
+        None if stop is None else ctypes.c_void_p(stop.cuda_event)))
 
 
 def mla_noalloc_scratch_bytes() -> int:

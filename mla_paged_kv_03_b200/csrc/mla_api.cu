@@ -83,6 +83,25 @@ int make_latent_map(CUtensorMap* map, const void* base, long long rows) {
   return MLA_OK;
 }
 
+// 3-D bf16 view of the same rows: {64 dims, rows, 9 chunks of 64 dims}
+// (strides 1152 B and 128 B) with a {64, 64, box_chunks} box, 128-byte
+// swizzle; one copy lands [box_chunks][64 rows][64 dims] in shared memory.
+int make_latent_map3(CUtensorMap* map, const void* base, long long rows, int box_chunks) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(mla::kChunkD), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(mla::kNumChunks)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(mla::kD) * 2,
+                           static_cast<cuuint64_t>(mla::kChunkD) * 2};
+  cuuint32_t box[3] = {64, 64, static_cast<cuuint32_t>(box_chunks)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled (3-D) failed (%d)", (int)r);
+  return MLA_OK;
+}
+
 template <int kMode>
 int prepare_kernel() {
   static int done = 0;
@@ -133,22 +152,44 @@ int launch_combine(const mla::CombineParams& cp, bool fused, cudaStream_t st) {
   return MLA_OK;
 }
 
+// Events set by mla_set_kernel_events (per host thread), recorded around the
+// attention kernel of each decode entry point.
+thread_local cudaEvent_t t_kernel_start = nullptr;
+thread_local cudaEvent_t t_kernel_stop = nullptr;
+
+int record_start(cudaStream_t st) {
+  if (t_kernel_start) MLA_CUDA(cudaEventRecord(t_kernel_start, st));
+  return MLA_OK;
+}
+
+int record_stop(cudaStream_t st) {
+  if (t_kernel_stop) MLA_CUDA(cudaEventRecord(t_kernel_stop, st));
+  return MLA_OK;
+}
+
 template <int kMode>
 int launch_decode(const CUtensorMap& tq, const CUtensorMap& tkv, const mla::DecodeParams& p,
                   cudaStream_t st) {
   int rc = prepare_kernel<kMode>();
   if (rc != MLA_OK) return rc;
   const unsigned grid = static_cast<unsigned>(p.num_parts * p.n_groups);
+  if ((rc = record_start(st)) != MLA_OK) return rc;
   mla::mla_decode_kernel<kMode>
       <<<grid, mla::Threads<kMode>::value, mla::cfg::kSmemBytes, st>>>(tq, tkv, p);
   MLA_CUDA(cudaGetLastError());
-  return MLA_OK;
+  return record_stop(st);
 }
 
 // 2-CTA kernel for more than 64 query rows per KV head: clusters of two CTAs,
 // one pair per scheduler part and 128-row group.
-int launch_pair_decode(const CUtensorMap& tq, const CUtensorMap& tkv, const mla::DecodeParams& p,
-                       cudaStream_t st) {
+int launch_pair_decode(const void* q, const void* kcache, const CUtensorMap& tkv,
+                       const mla::DecodeParams& p, cudaStream_t st) {
+  CUtensorMap tq3, tv3;
+  int rc = make_latent_map3(&tq3, q, static_cast<long long>(p.batch) * p.R, mla::kNumChunks);
+  if (rc != MLA_OK) return rc;
+  if ((rc = make_latent_map3(&tv3, kcache, static_cast<long long>(p.num_blocks) * mla::kPage, 2)) !=
+      MLA_OK)
+    return rc;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
@@ -170,8 +211,9 @@ int launch_pair_decode(const CUtensorMap& tq, const CUtensorMap& tkv, const mla:
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  MLA_CUDA(cudaLaunchKernelEx(&cfg, mla::mla_pair_decode_kernel, tq, tkv, p));
-  return MLA_OK;
+  if ((rc = record_start(st)) != MLA_OK) return rc;
+  MLA_CUDA(cudaLaunchKernelEx(&cfg, mla::mla_pair_decode_kernel, tq3, tkv, tv3, p));
+  return record_stop(st);
 }
 
 int check_common_dense(const void* q, const void* kcache, const int32_t* block_table,
@@ -325,7 +367,7 @@ int mla_get_metadata(const int32_t* cache_seqlens, int batch, int heads_per_kv, 
   // For batches beyond the kernel's shared-memory staging, num_splits[1..]
   // doubles as the tile-count scratch: each entry is read before the planner
   // overwrites it with the prefix sum.
-  mla::mla_plan_kernel<<<1, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+  mla::mla_plan_kernel<<<1, mla::kPlanThreads, 0, static_cast<cudaStream_t>(stream)>>>(
       cache_seqlens, batch, num_sm_parts, num_splits + 1, metadata, num_splits);
   MLA_CUDA(cudaGetLastError());
   return MLA_OK;
@@ -403,7 +445,7 @@ int mla_decode_fwd(const void* q, const void* kcache, const int32_t* block_table
   p.ws_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.lse_off);
   if (R > mla::kRowsPerCta && d_v == 512) {
     p.n_groups = mla::ceil_div(R, 2 * mla::kRowsPerCta);
-    if ((rc = launch_pair_decode(tq, tkv, p, st)) != MLA_OK) return rc;
+    if ((rc = launch_pair_decode(q, kcache, tkv, p, st)) != MLA_OK) return rc;
   } else if ((rc = launch_decode<mla::kDense>(tq, tkv, p, st)) != MLA_OK) {
     return rc;
   }
@@ -532,7 +574,7 @@ int mla_sparse_decode(const void* q, const uint8_t* kcache_fp8, int64_t num_slot
   int32_t* meta = reinterpret_cast<int32_t*>(ws + w.meta_off);
   int32_t* splits = reinterpret_cast<int32_t*>(ws + w.splits_off);
   int32_t* lens = reinterpret_cast<int32_t*>(ws + w.lens_off);
-  mla::mla_plan_uniform_kernel<<<1, 256, 0, st>>>(topk, pairs, num_sm_parts, lens, meta, splits);
+  mla::mla_plan_uniform_kernel<<<1, mla::kPlanThreads, 0, st>>>(topk, pairs, num_sm_parts, lens, meta, splits);
   MLA_CUDA(cudaGetLastError());
 
   CUtensorMap tq;
@@ -575,6 +617,12 @@ int mla_sparse_decode(const void* q, const uint8_t* kcache_fp8, int64_t num_slot
   cp.out = p.out;
   cp.lse = lse;
   return launch_combine(cp, false, st);
+}
+
+int mla_set_kernel_events(void* start_event, void* stop_event) {
+  t_kernel_start = static_cast<cudaEvent_t>(start_event);
+  t_kernel_stop = static_cast<cudaEvent_t>(stop_event);
+  return MLA_OK;
 }
 
 int mla_device_status(int* status, int reset) {

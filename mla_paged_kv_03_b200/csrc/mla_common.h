@@ -92,47 +92,93 @@ MLA_HD inline int deal_tiles(const int32_t* tiles, int batch, long long target, 
   return part_open ? p + 1 : p;
 }
 
+// Parts used by the greedy dealing of deal_tiles() with cost cap `target`,
+// one arithmetic step per sequence: after the sequence's first segment fills
+// the open part, every further segment takes a fresh part of target - overhead
+// tiles.  Returns max_parts + 1 as soon as the count exceeds max_parts.
+MLA_HD inline int count_parts(const int32_t* tiles, int batch, long long target, int max_parts) {
+  const long long o = kSegmentOverheadTiles;
+  const long long full = target - o;  // tiles of a segment that fills a part
+  long long p = 0, used = 0;
+  bool open = false;
+  for (int b = 0; b < batch; ++b) {
+    const long long n = tiles[b];
+    if (open && used + o + 1 > target) {
+      ++p;
+      used = 0;
+      if (p >= max_parts) return max_parts + 1;
+    }
+    const long long avail = target - used - o;
+    open = true;
+    if (n <= avail) {
+      used += n + o;
+      continue;
+    }
+    const long long r = n - avail;           // tiles left after filling the open part
+    const long long k = (r + full - 1) / full;  // further segments, one part each
+    p += k;
+    if (p >= max_parts) return max_parts + 1;
+    used = r - (k - 1) * full + o;
+  }
+  return static_cast<int>(open ? p + 1 : p);
+}
+
+// Caps checked one by one above the lower bound before the planner falls
+// back to bisection (the device planner checks them in parallel).
+constexpr int kPlanWindow = 256;
+
+// Smallest cap >= lo in the window for which the dealing fits, else the
+// bisection boundary beyond it (the whole load in one part always fits).
+MLA_HD inline long long plan_cap_beyond_window(const int32_t* tiles, int batch, int num_parts,
+                                               long long lo, long long total) {
+  long long a = lo + kPlanWindow;
+  long long b = total > a ? total : a;
+  while (a < b) {
+    const long long mid = a + (b - a) / 2;
+    if (count_parts(tiles, batch, mid, num_parts) <= num_parts)
+      b = mid;
+    else
+      a = mid + 1;
+  }
+  return a;
+}
+
+// Lower bound of the cap: the mean cost per part, at least one tile.
+MLA_HD inline long long plan_lower_bound(long long total, int num_parts) {
+  long long lo = (total + num_parts - 1) / num_parts;
+  return lo < kSegmentOverheadTiles + 1 ? kSegmentOverheadTiles + 1 : lo;
+}
+
+MLA_HD inline void plan_mark_empty(int32_t* m, int batch) {
+  m[0] = batch;  // empty part: begins after every sequence
+  m[1] = 0;
+  m[2] = batch - 1;
+  m[3] = 0;
+  m[4] = m[5] = m[6] = m[7] = 0;
+}
+
 // Split-KV planner.  Finds the smallest per-part cost cap for which the
 // greedy dealing (sequences in order, tiles of 128 tokens, a segment costing
 // its tiles plus kSegmentOverheadTiles) fits in `num_parts` parts, then
 // writes metadata[num_parts][8] and the prefix sums num_splits[batch + 1]
 // (num_splits[b+1] - num_splits[b] = number of parts holding tiles of
 // sequence b).  Each part covers one contiguous run of (sequence, tile)
-// pairs; unused parts are marked empty (begin_seq > end_seq).  The search
-// starts at the lower bound ceil(total / num_parts), which usually fits after
-// a few steps, and falls back to bisection.  `tiles` holds tiles_of() of every
-// sequence.  Runs identically on host and device.
+// pairs; unused parts are marked empty (begin_seq > end_seq).  The caps
+// lo .. lo + kPlanWindow - 1 above the lower bound are tried in order
+// (the optimum lies within a few tiles of the bound), then bisection.
+// `tiles` holds tiles_of() of every sequence.  The device planner
+// (mla_plan_kernel) reaches the same cap.
 MLA_HD inline void plan_splits_tiles(const int32_t* tiles, int batch, int num_parts,
                                      int32_t* metadata, int32_t* num_splits) {
-  for (int p = 0; p < num_parts; ++p) {
-    int32_t* m = metadata + p * kMetaInts;
-    m[0] = batch;  // empty part: begins after every sequence
-    m[1] = 0;
-    m[2] = batch - 1;
-    m[3] = 0;
-    m[4] = m[5] = m[6] = m[7] = 0;
-  }
+  for (int p = 0; p < num_parts; ++p) plan_mark_empty(metadata + p * kMetaInts, batch);
   long long total = 0;
   for (int b = 0; b < batch; ++b) total += tiles[b] + kSegmentOverheadTiles;
-  long long lo = (total + num_parts - 1) / num_parts;
-  if (lo < kSegmentOverheadTiles + 1) lo = kSegmentOverheadTiles + 1;
-  long long hi = total > lo ? total : lo;  // one part holding everything always fits
-  // linear probe from the lower bound, then bisection on what remains
-  for (int probe = 0; probe < 4 && lo < hi; ++probe) {
-    if (deal_tiles(tiles, batch, lo, num_parts, nullptr, nullptr) <= num_parts) {
-      hi = lo;
-      break;
-    }
-    ++lo;
-  }
-  while (lo < hi) {
-    const long long mid = lo + (hi - lo) / 2;
-    if (deal_tiles(tiles, batch, mid, num_parts, nullptr, nullptr) <= num_parts)
-      hi = mid;
-    else
-      lo = mid + 1;
-  }
-  deal_tiles(tiles, batch, lo, num_parts, metadata, num_splits);
+  const long long lo = plan_lower_bound(total, num_parts);
+  long long cap = -1;
+  for (int k = 0; k < kPlanWindow && cap < 0; ++k)
+    if (count_parts(tiles, batch, lo + k, num_parts) <= num_parts) cap = lo + k;
+  if (cap < 0) cap = plan_cap_beyond_window(tiles, batch, num_parts, lo, total);
+  deal_tiles(tiles, batch, cap, num_parts, metadata, num_splits);
 }
 
 }  // namespace mla

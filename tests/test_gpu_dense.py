@@ -34,10 +34,13 @@ def check_full(case, num_sm_parts=None):
     assert_lse_close(lse, rl)
 
 
-def test_device_planner_matches_host_planner():
-    rng = np.random.default_rng(0)
+@pytest.mark.parametrize("batch", [97, 2048, 2049, 5000])
+def test_device_planner_matches_host_planner(batch):
+    # 2048 is the largest batch the device planner deals in parallel; above it
+    # one thread deals serially.
+    rng = np.random.default_rng(batch)
     for parts in (1, 7, 74, 148):
-        sl = rng.integers(0, 20000, size=97).astype(np.int32)
+        sl = rng.integers(0, 20000, size=batch).astype(np.int32)
         sl[:5] = [0, 1, 64, 65, 128]
         hm, hn = B.mla_get_metadata_host(sl, 16, parts)
         dm, dn, _ = B.mla_get_metadata(torch.tensor(sl, device="cuda"), 16, 1, parts)
