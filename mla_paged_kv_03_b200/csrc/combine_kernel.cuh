@@ -51,6 +51,7 @@ __global__ void __launch_bounds__(kCombineThreads) mla_combine_kernel(const Comb
   __shared__ float s_w[kCombineMaxSplits];
   __shared__ float s_red[kCombineThreads / 32];
   __shared__ float s_lse;
+  ptx::grid_dep_wait();  // the decode kernel's partials are complete
   const int row_id = blockIdx.x;
   const int b = row_id / P.R;
   const int r = row_id % P.R;
@@ -179,135 +180,84 @@ __global__ void __launch_bounds__(kCombineThreads) mla_combine_kernel(const Comb
 // Device-side planner: the block stages tiles_of(seqlens) in shared memory
 // (or, for very large batches, in the caller's scratch), then one thread runs
 // the same planner the host uses.
-constexpr int kPlanThreads = kPlanWindow;
-constexpr int kPlanSmemBatch = 2048;
+constexpr int kPlanThreads = 256;
+constexpr int kPlanMaxBatch = 8192;  // prefix sums live in shared memory
 
-// Split-KV planner of one CTA (same result as plan_splits_tiles): every
-// thread checks one cap of the window above the lower bound; then one thread
-// replays the dealing with the chosen cap to find each sequence's first part
-// and segment count, and all threads write the metadata rows in parallel.
-// `tiles` is filled by the caller's threads (shared memory, or the scratch
-// for batches above kPlanSmemBatch); `my_total` is each thread's share of
-// sum(tiles + overhead).
-__device__ void plan_block(int32_t* tiles, int batch, int num_parts, long long my_total,
+// Block-wide exclusive prefix sum of one value per thread; returns the
+// thread's exclusive sum, and the block total through *total.
+__device__ __forceinline__ int block_exclusive_scan(int v, int* total) {
+  __shared__ int s_warp[kPlanThreads / 32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, off);
+    if (lane >= off) x += y;
+  }
+  if (lane == 31) s_warp[warp] = x;
+  __syncthreads();
+  int before = 0, all = 0;
+#pragma unroll
+  for (int w = 0; w < kPlanThreads / 32; ++w) {
+    const int t = s_warp[w];
+    before += w < warp ? t : 0;
+    all += t;
+  }
+  __syncthreads();  // s_warp reusable
+  *total = all;
+  return before + x - v;
+}
+
+// Split-KV planner of one CTA: the closed forms of mla_common.h evaluated in
+// parallel (prefix sums by block scans, one metadata row per thread).
+// len_or_neg < 0: lengths from seqlens; else every sequence has that length.
+__device__ void plan_block(const int32_t* seqlens, int len_or_neg, int batch, int num_parts,
                            int32_t* metadata, int32_t* num_splits) {
-  __shared__ long long s_part[kPlanThreads / 32];
-  __shared__ int s_best;
-  __shared__ long long s_cap;
-  __shared__ int32_t s_first_part[kPlanSmemBatch];  // part of the sequence's first segment
-  __shared__ int32_t s_take0[kPlanSmemBatch];       // tiles of its first segment
-  __shared__ int32_t s_nseg[kPlanSmemBatch];        // its segments
-  __shared__ uint8_t s_opens[kPlanSmemBatch];       // its first segment opens a part
+  __shared__ int32_t C[kPlanMaxBatch + 1];
   const int tid = threadIdx.x;
-  for (int off = 16; off > 0; off >>= 1) my_total += __shfl_down_sync(0xffffffffu, my_total, off);
-  if ((tid & 31) == 0) s_part[tid >> 5] = my_total;
-  if (tid == 0) s_best = kPlanWindow;
-  for (int p = tid; p < num_parts; p += blockDim.x) plan_mark_empty(metadata + p * kMetaInts, batch);
-  __syncthreads();
-  long long total = 0;
-  for (int w = 0; w < kPlanThreads / 32; ++w) total += s_part[w];
-  const long long lo = plan_lower_bound(total, num_parts);
-  if (count_parts(tiles, batch, lo + tid, num_parts) <= num_parts) atomicMin(&s_best, tid);
-  __syncthreads();
-  if (tid == 0)
-    s_cap = s_best < kPlanWindow ? lo + s_best
-                                 : plan_cap_beyond_window(tiles, batch, num_parts, lo, total);
-  __syncthreads();
-  const long long cap = s_cap;
-  if (batch > kPlanSmemBatch) {  // large batch: serial dealing
-    if (tid == 0) deal_tiles(tiles, batch, cap, num_parts, metadata, num_splits);
-    return;
+  int carry = 0;
+  for (int base = 0; base < batch; base += kPlanThreads) {
+    const int b = base + tid;
+    const int L = b < batch ? (len_or_neg < 0 ? seqlens[b] : len_or_neg) : 0;
+    const int v = b < batch ? tiles_of(L) + kSegmentOverheadTiles : 0;
+    int chunk_total;
+    const int ex = block_exclusive_scan(v, &chunk_total);
+    if (b < batch) C[b] = carry + ex;
+    carry += chunk_total;
   }
-  const long long o = kSegmentOverheadTiles;
-  const long long full = cap - o;
-  if (tid == 0) {  // replay of count_parts with the per-sequence state kept
-    long long p = 0, used = 0;
-    bool open = false;
-    int32_t splits = 0;
-    num_splits[0] = 0;
-    for (int b = 0; b < batch; ++b) {
-      const long long n = tiles[b];
-      bool opens = !open;
-      if (open && used + o + 1 > cap) {
-        ++p;
-        used = 0;
-        opens = true;
-      }
-      const long long avail = cap - used - o;
-      s_first_part[b] = static_cast<int32_t>(p);
-      s_opens[b] = opens ? 1 : 0;
-      open = true;
-      if (n <= avail) {
-        used += n + o;
-        s_take0[b] = static_cast<int32_t>(n);
-        s_nseg[b] = 1;
-      } else {
-        const long long r = n - avail;
-        const long long k = (r + full - 1) / full;
-        s_take0[b] = static_cast<int32_t>(avail);
-        s_nseg[b] = static_cast<int32_t>(k + 1);
-        p += k;
-        used = r - (k - 1) * full + o;
-      }
-      splits += s_nseg[b];
-      num_splits[b + 1] = splits;
-    }
-  }
+  if (tid == 0) C[batch] = carry;
   __syncthreads();
-  // segment j of sequence b: part first_part + j, tiles [t0, t1)
-  for (int b = tid; b < batch; b += blockDim.x) {
-    const int nseg = s_nseg[b];
-    const int n = tiles[b];
-    const bool last_in_part_next = (b + 1 == batch) || s_opens[b + 1];
-    for (int j = 0; j < nseg; ++j) {
-      const int part = s_first_part[b] + j;
-      const int t0 = j == 0 ? 0 : s_take0[b] + (j - 1) * static_cast<int>(full);
-      const int t1 = j + 1 == nseg ? n : s_take0[b] + j * static_cast<int>(full);
-      int32_t* m = metadata + part * kMetaInts;
-      if (j > 0 || s_opens[b]) {  // opens the part
-        m[0] = b;
-        m[1] = t0;
-        m[4] = j;
-      }
-      if (j + 1 < nseg || last_in_part_next) {  // closes the part
-        m[2] = b;
-        m[3] = t1;
-      }
-    }
+  const int w = plan_width(carry, num_parts);
+  for (int p = tid; p < num_parts; p += kPlanThreads)
+    plan_part_row(C, batch, w, p, metadata + p * kMetaInts);
+  int nsum = 0;
+  if (tid == 0) num_splits[0] = 0;
+  for (int base = 0; base < batch; base += kPlanThreads) {
+    const int b = base + tid;
+    const int v = b < batch ? plan_last_part(C, b, w) - plan_first_part(C, b, w) + 1 : 0;
+    int chunk_total;
+    const int ex = block_exclusive_scan(v, &chunk_total);
+    if (b < batch) num_splits[b + 1] = nsum + ex + v;
+    nsum += chunk_total;
   }
 }
 
 __global__ void __launch_bounds__(kPlanThreads) mla_plan_kernel(const int32_t* seqlens, int batch,
-                                                               int num_parts,
-                                                               int32_t* tiles_scratch,
-                                                               int32_t* metadata,
+                                                               int num_parts, int32_t* metadata,
                                                                int32_t* num_splits) {
-  __shared__ int32_t s_tiles[kPlanSmemBatch];
-  int32_t* tiles = batch <= kPlanSmemBatch ? s_tiles : tiles_scratch;
-  long long mine = 0;
-  for (int i = threadIdx.x; i < batch; i += blockDim.x) {
-    tiles[i] = tiles_of(seqlens[i]);
-    mine += tiles[i] + kSegmentOverheadTiles;
-  }
-  __syncthreads();
-  plan_block(tiles, batch, num_parts, mine, metadata, num_splits);
+  ptx::grid_dep_wait();
+  ptx::grid_dep_launch();  // the decode grid waits for this one at its start
+  plan_block(seqlens, -1, batch, num_parts, metadata, num_splits);
 }
 
 // Planner over `batch` items of equal length `len` (sparse decode).
 __global__ void __launch_bounds__(kPlanThreads) mla_plan_uniform_kernel(int len, int batch,
                                                                        int num_parts,
-                                                                       int32_t* tiles_scratch,
                                                                        int32_t* metadata,
                                                                        int32_t* num_splits) {
-  __shared__ int32_t s_tiles[kPlanSmemBatch];
-  int32_t* tiles = batch <= kPlanSmemBatch ? s_tiles : tiles_scratch;
-  long long mine = 0;
-  for (int i = threadIdx.x; i < batch; i += blockDim.x) {
-    tiles[i] = tiles_of(len);
-    mine += tiles[i] + kSegmentOverheadTiles;
-  }
-  __syncthreads();
-  plan_block(tiles, batch, num_parts, mine, metadata, num_splits);
+  ptx::grid_dep_wait();
+  ptx::grid_dep_launch();
+  plan_block(nullptr, len, batch, num_parts, metadata, num_splits);
 }
 
 }  // namespace mla

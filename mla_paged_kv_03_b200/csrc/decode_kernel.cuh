@@ -299,6 +299,8 @@ __global__ void __launch_bounds__(Threads<kMode>::value, 1)
   constexpr int NPm = kPSplit ? 1 : kNP;
   static_assert(!kPSplit || kNP >= 2, "the hi/lo P pair needs two P buffer regions");
 
+  ptx::grid_dep_wait();    // the planner's metadata is complete
+  ptx::grid_dep_launch();  // the combine grid may be scheduled as CTAs retire
   const int32_t* meta = P.metadata + part * kMetaInts;
   if (meta[0] > meta[2]) return;  // empty part: nothing to do (uniform exit)
 

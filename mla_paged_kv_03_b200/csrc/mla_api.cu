@@ -120,7 +120,7 @@ int prepare_kernel() {
 }
 
 struct WsLayout {
-  size_t o_off, lse_off, meta_off, splits_off, lens_off, total;
+  size_t o_off, lse_off, meta_off, splits_off, total;
 };
 
 WsLayout dense_ws_layout(int batch, int R, int d_v, int parts) {
@@ -136,19 +136,43 @@ WsLayout sparse_ws_layout(int pairs, int R, int d_v, int parts) {
   WsLayout w = dense_ws_layout(pairs, R, d_v, parts);
   w.meta_off = w.total;
   w.splits_off = w.meta_off + align_up(static_cast<size_t>(parts) * mla::kMetaInts * 4, 256);
-  w.lens_off = w.splits_off + align_up((static_cast<size_t>(pairs) + 1) * 4, 256);
-  w.total = w.lens_off + align_up(static_cast<size_t>(pairs) * 4, 256);
+  w.total = w.splits_off + align_up((static_cast<size_t>(pairs) + 1) * 4, 256);
   return w;
 }
+
+// Launch configuration with programmatic dependent launch: the kernel may
+// be scheduled before the preceding grid of the stream has finished and
+// waits for it in its first instruction (griddepcontrol.wait).
+struct PdlLaunch {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  PdlLaunch(dim3 grid, dim3 block, size_t smem, cudaStream_t st, int cluster_x = 1) {
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.numAttrs = 1;
+    if (cluster_x > 1) {
+      attr[1].id = cudaLaunchAttributeClusterDimension;
+      attr[1].val.clusterDim.x = cluster_x;
+      attr[1].val.clusterDim.y = 1;
+      attr[1].val.clusterDim.z = 1;
+      cfg.numAttrs = 2;
+    }
+    cfg.attrs = attr;
+  }
+};
 
 int launch_combine(const mla::CombineParams& cp, bool fused, cudaStream_t st) {
   const long long rows = static_cast<long long>(cp.batch) * cp.R;
   if (rows == 0) return MLA_OK;
+  PdlLaunch L(dim3(static_cast<unsigned>(rows)), dim3(mla::kCombineThreads), 0, st);
   if (fused)
-    mla::mla_combine_kernel<true><<<static_cast<unsigned>(rows), mla::kCombineThreads, 0, st>>>(cp);
+    MLA_CUDA(cudaLaunchKernelEx(&L.cfg, mla::mla_combine_kernel<true>, cp));
   else
-    mla::mla_combine_kernel<false><<<static_cast<unsigned>(rows), mla::kCombineThreads, 0, st>>>(cp);
-  MLA_CUDA(cudaGetLastError());
+    MLA_CUDA(cudaLaunchKernelEx(&L.cfg, mla::mla_combine_kernel<false>, cp));
   return MLA_OK;
 }
 
@@ -174,9 +198,8 @@ int launch_decode(const CUtensorMap& tq, const CUtensorMap& tkv, const mla::Deco
   if (rc != MLA_OK) return rc;
   const unsigned grid = static_cast<unsigned>(p.num_parts * p.n_groups);
   if ((rc = record_start(st)) != MLA_OK) return rc;
-  mla::mla_decode_kernel<kMode>
-      <<<grid, mla::Threads<kMode>::value, mla::cfg::kSmemBytes, st>>>(tq, tkv, p);
-  MLA_CUDA(cudaGetLastError());
+  PdlLaunch L(dim3(grid), dim3(mla::Threads<kMode>::value), mla::cfg::kSmemBytes, st);
+  MLA_CUDA(cudaLaunchKernelEx(&L.cfg, mla::mla_decode_kernel<kMode>, tq, tkv, p));
   return record_stop(st);
 }
 
@@ -199,20 +222,10 @@ int launch_pair_decode(const void* q, const void* kcache, const CUtensorMap& tkv
   });
   if (attr_err != cudaSuccess)
     return fail(MLA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(attr_err));
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(2 * p.num_parts * p.n_groups), 1, 1);
-  cfg.blockDim = dim3(mla::pcfg::kThreads, 1, 1);
-  cfg.dynamicSmemBytes = mla::pcfg::kSmemBytes;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  PdlLaunch L(dim3(static_cast<unsigned>(2 * p.num_parts * p.n_groups)), dim3(mla::pcfg::kThreads),
+              mla::pcfg::kSmemBytes, st, 2);
   if ((rc = record_start(st)) != MLA_OK) return rc;
-  MLA_CUDA(cudaLaunchKernelEx(&cfg, mla::mla_pair_decode_kernel, tq3, tkv, tv3, p));
+  MLA_CUDA(cudaLaunchKernelEx(&L.cfg, mla::mla_pair_decode_kernel, tq3, tkv, tv3, p));
   return record_stop(st);
 }
 
@@ -364,11 +377,10 @@ int mla_get_metadata(const int32_t* cache_seqlens, int batch, int heads_per_kv, 
   MLA_CHECK_ARG(heads_per_kv >= 1, "heads_per_kv must be >= 1");
   if (h_kv != 1) return fail(MLA_ERR_UNSUPPORTED, "h_kv must be 1 (got %d)", h_kv);
   MLA_CHECK_ARG(metadata && num_splits && (cache_seqlens || batch == 0), "null device pointer");
-  // For batches beyond the kernel's shared-memory staging, num_splits[1..]
-  // doubles as the tile-count scratch: each entry is read before the planner
-  // overwrites it with the prefix sum.
+  MLA_CHECK_ARG(batch <= mla::kPlanMaxBatch, "the device planner takes at most %d sequences (got %d)",
+                mla::kPlanMaxBatch, batch);
   mla::mla_plan_kernel<<<1, mla::kPlanThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-      cache_seqlens, batch, num_sm_parts, num_splits + 1, metadata, num_splits);
+      cache_seqlens, batch, num_sm_parts, metadata, num_splits);
   MLA_CUDA(cudaGetLastError());
   return MLA_OK;
 }
@@ -382,8 +394,15 @@ int mla_get_metadata_host(const int32_t* cache_seqlens, int batch, int heads_per
   for (int b = 0; b < batch; ++b)
     MLA_CHECK_ARG(cache_seqlens[b] >= 0, "cache_seqlens[%d] = %d is negative", b, cache_seqlens[b]);
   std::vector<int32_t> tiles(static_cast<size_t>(batch));
-  for (int b = 0; b < batch; ++b) tiles[b] = mla::tiles_of(cache_seqlens[b]);
-  mla::plan_splits_tiles(tiles.data(), batch, num_sm_parts, metadata, num_splits);
+  long long total = 0;
+  for (int b = 0; b < batch; ++b) {
+    tiles[b] = mla::tiles_of(cache_seqlens[b]);
+    total += tiles[b] + mla::kSegmentOverheadTiles;
+  }
+  MLA_CHECK_ARG(total <= mla::kPlanMaxTotal, "total planner cost %lld above %lld", total,
+                mla::kPlanMaxTotal);
+  std::vector<int32_t> prefix(static_cast<size_t>(batch) + 1);
+  mla::plan_splits_host(tiles.data(), batch, num_sm_parts, metadata, num_splits, prefix.data());
   return MLA_OK;
 }
 
@@ -573,8 +592,10 @@ int mla_sparse_decode(const void* q, const uint8_t* kcache_fp8, int64_t num_slot
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   int32_t* meta = reinterpret_cast<int32_t*>(ws + w.meta_off);
   int32_t* splits = reinterpret_cast<int32_t*>(ws + w.splits_off);
-  int32_t* lens = reinterpret_cast<int32_t*>(ws + w.lens_off);
-  mla::mla_plan_uniform_kernel<<<1, mla::kPlanThreads, 0, st>>>(topk, pairs, num_sm_parts, lens, meta, splits);
+  MLA_CHECK_ARG(pairs <= mla::kPlanMaxBatch, "at most %d (batch, query) pairs (got %d)",
+                mla::kPlanMaxBatch, pairs);
+  mla::mla_plan_uniform_kernel<<<1, mla::kPlanThreads, 0, st>>>(topk, pairs, num_sm_parts, meta,
+                                                                 splits);
   MLA_CUDA(cudaGetLastError());
 
   CUtensorMap tq;

@@ -48,106 +48,46 @@ MLA_HD inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
 // O = 0, LSE = -inf result.
 MLA_HD inline int tiles_of(int L) { return L > 0 ? ceil_div(L, kTileT) : 1; }
 
-// Greedy dealing of tiles to parts with a cost cap `target` per part; a
-// segment costs its tiles plus kSegmentOverheadTiles.  `tiles[b]` is
-// tiles_of(seqlens[b]).  Returns the number of parts used (stops counting at
-// max_parts + 1); writes the plan when metadata != nullptr.
-MLA_HD inline int deal_tiles(const int32_t* tiles, int batch, long long target, int max_parts,
-                             int32_t* metadata, int32_t* num_splits) {
-  int p = 0;
-  long long used = 0;
-  bool part_open = false;
-  if (num_splits) num_splits[0] = 0;
-  for (int b = 0; b < batch; ++b) {
-    const int n = tiles[b];
-    int t = 0;
-    int splits = 0;
-    while (t < n) {
-      if (part_open && used + kSegmentOverheadTiles + 1 > target) {
-        ++p;
-        used = 0;
-        part_open = false;
-        if (!metadata && p >= max_parts) return max_parts + 1;  // does not fit
-      }
-      const long long avail = target - used - kSegmentOverheadTiles;
-      int take = static_cast<int>(avail < 1 ? 1 : (avail < n - t ? avail : n - t));
-      if (metadata && p >= max_parts - 1) take = n - t;  // the last part takes the rest
-      if (metadata) {
-        int32_t* m = metadata + p * kMetaInts;
-        if (!part_open) {
-          m[0] = b;
-          m[1] = t;
-          m[4] = splits;
-        }
-        m[2] = b;
-        m[3] = t + take;
-      }
-      part_open = true;
-      used += take + kSegmentOverheadTiles;
-      t += take;
-      ++splits;
-    }
-    if (num_splits) num_splits[b + 1] = num_splits[b] + splits;
-  }
-  return part_open ? p + 1 : p;
+// The planner counts in int32: the total cost sum(tiles + overhead) of a
+// call must stay below this (checked by the entry points).
+constexpr long long kPlanMaxTotal = (1LL << 30);
+
+// ------------------------------------------------------- split-KV planner
+//
+// The sequences' work is laid out on one cost line: sequence b occupies
+// [C[b], C[b+1]) with C[b+1] = C[b] + kSegmentOverheadTiles + tiles_of(L_b);
+// its overhead positions come first and tile t sits at C[b] + overhead + t.
+// The line is cut into num_parts intervals of width W = ceil(total /
+// num_parts); part p takes the tiles whose positions fall in [pW, (p+1)W).
+// Each part therefore covers one contiguous run of (sequence, tile) pairs and
+// costs at most W plus one segment overhead (that of a sequence continued
+// from the previous part).  Every quantity below is a closed form of C, so
+// the device planner computes all parts and sequences in parallel and the
+// host planner reaches the identical result with plain loops.
+
+MLA_HD inline int plan_width(int total, int num_parts) {
+  const int w = (total + num_parts - 1) / num_parts;
+  return w < 1 ? 1 : w;
 }
 
-// Parts used by the greedy dealing of deal_tiles() with cost cap `target`,
-// one arithmetic step per sequence: after the sequence's first segment fills
-// the open part, every further segment takes a fresh part of target - overhead
-// tiles.  Returns max_parts + 1 as soon as the count exceeds max_parts.
-MLA_HD inline int count_parts(const int32_t* tiles, int batch, long long target, int max_parts) {
-  const long long o = kSegmentOverheadTiles;
-  const long long full = target - o;  // tiles of a segment that fills a part
-  long long p = 0, used = 0;
-  bool open = false;
-  for (int b = 0; b < batch; ++b) {
-    const long long n = tiles[b];
-    if (open && used + o + 1 > target) {
-      ++p;
-      used = 0;
-      if (p >= max_parts) return max_parts + 1;
-    }
-    const long long avail = target - used - o;
-    open = true;
-    if (n <= avail) {
-      used += n + o;
-      continue;
-    }
-    const long long r = n - avail;           // tiles left after filling the open part
-    const long long k = (r + full - 1) / full;  // further segments, one part each
-    p += k;
-    if (p >= max_parts) return max_parts + 1;
-    used = r - (k - 1) * full + o;
-  }
-  return static_cast<int>(open ? p + 1 : p);
-}
-
-// Caps checked one by one above the lower bound before the planner falls
-// back to bisection (the device planner checks them in parallel).
-constexpr int kPlanWindow = 256;
-
-// Smallest cap >= lo in the window for which the dealing fits, else the
-// bisection boundary beyond it (the whole load in one part always fits).
-MLA_HD inline long long plan_cap_beyond_window(const int32_t* tiles, int batch, int num_parts,
-                                               long long lo, long long total) {
-  long long a = lo + kPlanWindow;
-  long long b = total > a ? total : a;
-  while (a < b) {
-    const long long mid = a + (b - a) / 2;
-    if (count_parts(tiles, batch, mid, num_parts) <= num_parts)
-      b = mid;
+// Sequence b with C[b] <= x < C[b+1] (C holds batch + 1 prefix sums).
+MLA_HD inline int plan_seq_at(const int32_t* C, int batch, int x) {
+  int lo = 0, hi = batch - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (C[mid] <= x)
+      lo = mid;
     else
-      a = mid + 1;
+      hi = mid - 1;
   }
-  return a;
+  return lo;
 }
 
-// Lower bound of the cap: the mean cost per part, at least one tile.
-MLA_HD inline long long plan_lower_bound(long long total, int num_parts) {
-  long long lo = (total + num_parts - 1) / num_parts;
-  return lo < kSegmentOverheadTiles + 1 ? kSegmentOverheadTiles + 1 : lo;
+// Parts holding tiles of sequence b: [plan_first_part(b), plan_last_part(b)].
+MLA_HD inline int plan_first_part(const int32_t* C, int b, int w) {
+  return (C[b] + kSegmentOverheadTiles) / w;
 }
+MLA_HD inline int plan_last_part(const int32_t* C, int b, int w) { return (C[b + 1] - 1) / w; }
 
 MLA_HD inline void plan_mark_empty(int32_t* m, int batch) {
   m[0] = batch;  // empty part: begins after every sequence
@@ -157,28 +97,50 @@ MLA_HD inline void plan_mark_empty(int32_t* m, int batch) {
   m[4] = m[5] = m[6] = m[7] = 0;
 }
 
-// Split-KV planner.  Finds the smallest per-part cost cap for which the
-// greedy dealing (sequences in order, tiles of 128 tokens, a segment costing
-// its tiles plus kSegmentOverheadTiles) fits in `num_parts` parts, then
-// writes metadata[num_parts][8] and the prefix sums num_splits[batch + 1]
-// (num_splits[b+1] - num_splits[b] = number of parts holding tiles of
-// sequence b).  Each part covers one contiguous run of (sequence, tile)
-// pairs; unused parts are marked empty (begin_seq > end_seq).  The caps
-// lo .. lo + kPlanWindow - 1 above the lower bound are tried in order
-// (the optimum lies within a few tiles of the bound), then bisection.
-// `tiles` holds tiles_of() of every sequence.  The device planner
-// (mla_plan_kernel) reaches the same cap.
-MLA_HD inline void plan_splits_tiles(const int32_t* tiles, int batch, int num_parts,
-                                     int32_t* metadata, int32_t* num_splits) {
-  for (int p = 0; p < num_parts; ++p) plan_mark_empty(metadata + p * kMetaInts, batch);
-  long long total = 0;
-  for (int b = 0; b < batch; ++b) total += tiles[b] + kSegmentOverheadTiles;
-  const long long lo = plan_lower_bound(total, num_parts);
-  long long cap = -1;
-  for (int k = 0; k < kPlanWindow && cap < 0; ++k)
-    if (count_parts(tiles, batch, lo + k, num_parts) <= num_parts) cap = lo + k;
-  if (cap < 0) cap = plan_cap_beyond_window(tiles, batch, num_parts, lo, total);
-  deal_tiles(tiles, batch, cap, num_parts, metadata, num_splits);
+// Metadata row of part p: {begin_b, begin_tile, end_b, end_tile (exclusive),
+// first_split, 0, 0, 0}, or an empty row.
+MLA_HD inline void plan_part_row(const int32_t* C, int batch, int w, int p, int32_t* m) {
+  const int o = kSegmentOverheadTiles;
+  const int total = C[batch];
+  const long long s64 = static_cast<long long>(p) * w;
+  if (batch == 0 || s64 >= total) {
+    plan_mark_empty(m, batch);
+    return;
+  }
+  const int s = static_cast<int>(s64);
+  const int e = (total - s > w) ? s + w : total;  // interval [s, e)
+  const int b0 = plan_seq_at(C, batch, s);
+  int t0 = s - C[b0] - o;
+  if (t0 < 0) t0 = 0;  // s inside b0's overhead: its first tile
+  int b1 = plan_seq_at(C, batch, e - 1);
+  int t1 = e - 1 - C[b1] - o;  // last tile in the interval
+  if (t1 < 0) {                // e - 1 inside b1's overhead: the previous sequence's last tile
+    --b1;
+    if (b1 >= 0) t1 = C[b1 + 1] - C[b1] - o - 1;
+  }
+  if (b1 < b0 || (b1 == b0 && t1 < t0)) {  // only overhead positions
+    plan_mark_empty(m, batch);
+    return;
+  }
+  m[0] = b0;
+  m[1] = t0;
+  m[2] = b1;
+  m[3] = t1 + 1;
+  m[4] = p - plan_first_part(C, b0, w);
+  m[5] = m[6] = m[7] = 0;
+}
+
+// Host planner: metadata[num_parts][8] and num_splits[batch + 1] from the
+// per-sequence tile counts (same result as the device planner).
+inline void plan_splits_host(const int32_t* tiles, int batch, int num_parts, int32_t* metadata,
+                             int32_t* num_splits, int32_t* C /* batch + 1 scratch */) {
+  C[0] = 0;
+  for (int b = 0; b < batch; ++b) C[b + 1] = C[b] + tiles[b] + kSegmentOverheadTiles;
+  const int w = plan_width(C[batch], num_parts);
+  for (int p = 0; p < num_parts; ++p) plan_part_row(C, batch, w, p, metadata + p * kMetaInts);
+  num_splits[0] = 0;
+  for (int b = 0; b < batch; ++b)
+    num_splits[b + 1] = num_splits[b] + plan_last_part(C, b, w) - plan_first_part(C, b, w) + 1;
 }
 
 }  // namespace mla

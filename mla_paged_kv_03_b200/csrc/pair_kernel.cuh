@@ -119,6 +119,8 @@ __global__ void __launch_bounds__(pcfg::kThreads, 1)
   const int part = pair / P.n_groups;
   const int grp = pair % P.n_groups;  // 128-row group
 
+  ptx::grid_dep_wait();    // the planner's metadata is complete
+  ptx::grid_dep_launch();  // the combine grid may be scheduled as CTAs retire
   const int32_t* meta = P.metadata + part * kMetaInts;
   if (meta[0] > meta[2]) return;  // empty part: both CTAs of the pair leave together
 

@@ -236,6 +236,14 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t local_addr, uint32_t ra
 }
 
 // Arrive on an mbarrier given by a shared::cluster address (possibly remote).
+// Programmatic dependent launch: wait until the preceding grid in the stream
+// has completed and its writes are visible (a no-op when the kernel was not
+// launched as a dependent), and let the following grid be scheduled early.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // True in exactly one active lane of a fully converged warp.  Issue loops
 // run warp-wide (their address arithmetic stays warp-uniform) and let the
 // elected lane issue the tcgen05 / TMA instructions.
