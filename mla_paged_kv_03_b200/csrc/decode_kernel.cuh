@@ -114,10 +114,22 @@ constexpr int kSoftmaxGroups = 2;
 constexpr int kBarAllSoftmax = 7;
 constexpr int kGatherThreads = 64;  // sparse: each gather thread fills two token rows
 
+// TMA loader warps filling the ring round-robin (one issuing warp sustains
+// only about 25 B/clk): warp 0, then warps 10, 11 after the softmax groups.
+// The sparse variant fills its ring from the gather warps instead.
+#ifndef MLA_DECODE_LOADERS
+#define MLA_DECODE_LOADERS 3
+#endif
+template <int kMode>
+struct Loaders {
+  static constexpr int value = kMode == kSparse ? 1 : MLA_DECODE_LOADERS;
+};
+
 template <int kMode>
 struct Threads {
-  // loader + MMA warps, softmax groups, and for sparse two gather warps
-  static constexpr int value = 64 + 128 * kSoftmaxGroups + (kMode == kSparse ? kGatherThreads : 0);
+  // loader + MMA warps, softmax groups, extra loaders, and for sparse two gather warps
+  static constexpr int value = 64 + 128 * kSoftmaxGroups + 32 * (Loaders<kMode>::value - 1) +
+                               (kMode == kSparse ? kGatherThreads : 0);
 };
 
 // Shared-memory control block (at kBarOff).
@@ -340,25 +352,30 @@ __global__ void __launch_bounds__(Threads<kMode>::value, 1)
   UnitIter it;
   it.init(meta);
 
-  if (warp == 0) {
-    // ============================== loader ==============================
-    // Lane 0 issues the TMA loads.  For the fused variant the whole warp also
-    // computes, per unit, the cos/sin table of the query position:
-    // theta_k = pos * base^(-2k/64), pos = positions[b] or L - 1.  A unit's
-    // table may be overwritten once the previous unit's QK finished
+  constexpr int kL = Loaders<kMode>::value;
+  constexpr int kFirstExtraLoader = 2 + 4 * kSoftmaxGroups;
+  if (warp == 0 || (kMode != kSparse && warp >= kFirstExtraLoader)) {
+    // ============================== loaders ==============================
+    // Pair slot j of the ring is filled by loader warp j % kL (whole warp,
+    // one elected lane issues the copies).  Warp 0 also loads Q; for the fused
+    // variant it computes, per unit, the cos/sin table of the query
+    // position: theta_k = pos * base^(-2k/64), pos = positions[b] or L - 1.
+    // A unit's table may be overwritten once the previous unit's QK finished
     // (q_empty), which implies the prologue that read it is done.
+    const int role = warp == 0 ? 0 : warp - kFirstExtraLoader + 1;
     uint32_t ring_it = 0;
     int u_idx = 0;
     Unit u;
     bool ok = true;
     auto load_pair = [&](const Unit& un, int tile, int pair) -> bool {
-      const int slot = ring_it % kNPair;
-      const uint32_t round = ring_it / kNPair;
-      ++ring_it;
-      if (!ptx::mbar_wait(&C.slot_empty[slot], (round & 1) ^ 1, 0x01)) return false;
+      const uint32_t idx = ring_it++;
+      if (static_cast<int>(idx % kL) != role) return true;
+      const int slot = idx % kNPair;
+      const uint32_t round = idx / kNPair;
+      bool w = ptx::mbar_wait(&C.slot_empty[slot], (round & 1) ^ 1, 0x01);
+      if (!__all_sync(0xffffffffu, w)) return false;
       const int c0 = 2 * pair;
       const int nch = (c0 + 1 < kNumChunks) ? 2 : 1;
-      ptx::mbar_arrive_expect_tx(&C.slot_full[slot], nch * kSubChunk);
       const int tok0 = tile * kTileT;
       int npg = (un.L + kPage - 1) / kPage;
       if (npg > P.max_pages) {
@@ -370,27 +387,21 @@ __global__ void __launch_bounds__(Threads<kMode>::value, 1)
       int blk1 = (p0 + 1 < npg) ? P.block_table[(size_t)un.b * P.max_pages + p0 + 1] : blk0;
       blk0 = clamp_block(blk0, P.num_blocks);
       blk1 = clamp_block(blk1, P.num_blocks);
-      uint8_t* dst = sRing + slot * kPairBytes;
-      for (int j = 0; j < nch; ++j) {
-        const int x = (c0 + j) * kChunkD;
-        ptx::tma_load_2d(dst + j * kSubChunk, &tm_kv, &C.slot_full[slot], x, blk0 * kPage);
-        ptx::tma_load_2d(dst + j * kSubChunk + kSubChunk / 2, &tm_kv, &C.slot_full[slot], x,
-                         blk1 * kPage);
+      if (ptx::elect_one_sync()) {
+        ptx::mbar_arrive_expect_tx(&C.slot_full[slot], nch * kSubChunk);
+        uint8_t* dst = sRing + slot * kPairBytes;
+        for (int j = 0; j < nch; ++j) {
+          const int x = (c0 + j) * kChunkD;
+          ptx::tma_load_2d(dst + j * kSubChunk, &tm_kv, &C.slot_full[slot], x, blk0 * kPage);
+          ptx::tma_load_2d(dst + j * kSubChunk + kSubChunk / 2, &tm_kv, &C.slot_full[slot], x,
+                           blk1 * kPage);
+        }
       }
+      __syncwarp();
       return true;
     };
-    // Pull both pages of a tile into L2 ahead of the TMA loads (a page is one
-    // contiguous 64 x 1152-byte block).
-    auto prefetch_tile = [&](const Unit& un, int tile) {
-      const int npg = min((un.L + kPage - 1) / kPage, P.max_pages);
-      for (int pg = 2 * tile; pg < 2 * tile + 2 && pg < npg; ++pg) {
-        const int blk = P.block_table[(size_t)un.b * P.max_pages + pg];
-        if (blk >= 0 && blk < P.num_blocks)
-          ptx::prefetch_l2_bulk(P.kcache + (size_t)blk * (kPage * kD * 2), kPage * kD * 2);
-      }
-    };
     while (ok && it.template next<kMode>(P, u)) {
-      if (kMode == kFused) {
+      if (kMode == kFused && role == 0) {
         ok = ptx::mbar_wait(&C.q_empty, (u_idx & 1) ^ 1, 0x06);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
@@ -402,79 +413,78 @@ __global__ void __launch_bounds__(Threads<kMode>::value, 1)
         C.rope_cs[lane][1] = sn;
         ptx::mbar_arrive(&C.rope_full);
       }
-      if (lane == 0) {
-        if (kMode != kFused) {
-          // Q rows [64*grp, 64*grp+64) of this sequence (or query pair)
-          ok = ptx::mbar_wait(&C.q_empty, (u_idx & 1) ^ 1, 0x02);
-          if (ok) {
-            ptx::mbar_arrive_expect_tx(&C.q_full, kQBytes);
-            const int row0 = u.b * P.R + grp * kRowsPerCta;
-            for (int c = 0; c < kNumChunks; ++c)
-              ptx::tma_load_2d(sQ + c * (kRowsPerCta * 128), &tm_q, &C.q_full, c * kChunkD, row0);
-          }
+      if (kMode != kFused && role == 0) {
+        // Q rows [64*grp, 64*grp+64) of this sequence (or query pair)
+        ok = __all_sync(0xffffffffu, ptx::mbar_wait(&C.q_empty, (u_idx & 1) ^ 1, 0x02));
+        if (ok && ptx::elect_one_sync()) {
+          ptx::mbar_arrive_expect_tx(&C.q_full, kQBytes);
+          const int row0 = u.b * P.R + grp * kRowsPerCta;
+          for (int c = 0; c < kNumChunks; ++c)
+            ptx::tma_load_2d(sQ + c * (kRowsPerCta * 128), &tm_q, &C.q_full, c * kChunkD, row0);
         }
-        if (kMode != kSparse && ok) {
-          const int n = u.hi - u.lo;
-          for (int k = 0; k < kPrefetchTiles && k < n; ++k) prefetch_tile(u, u.lo + k);
-          for (int k = 0; k < n && ok; ++k) {
-            if (k + kPrefetchTiles < n) prefetch_tile(u, u.lo + k + kPrefetchTiles);
-            for (int pr = 0; pr < 5 && ok; ++pr) ok = load_pair(u, u.lo + k, pr);
-            if (k >= 1)
-              for (int pr = 0; pr < nv_pairs && ok; ++pr) ok = load_pair(u, u.lo + k - 1, pr);
-          }
-          for (int pr = 0; pr < nv_pairs && ok; ++pr) ok = load_pair(u, u.hi - 1, pr);
-        }
+        __syncwarp();
       }
-      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (kMode != kSparse && ok) {
+        const int n = u.hi - u.lo;
+        for (int k = 0; k < n && ok; ++k) {
+          for (int pr = 0; pr < 5 && ok; ++pr) ok = load_pair(u, u.lo + k, pr);
+          if (k >= 1)
+            for (int pr = 0; pr < nv_pairs && ok; ++pr) ok = load_pair(u, u.lo + k - 1, pr);
+        }
+        for (int pr = 0; pr < nv_pairs && ok; ++pr) ok = load_pair(u, u.hi - 1, pr);
+      }
       ++u_idx;
     }
-    if (lane == 0) {
-      // Never leave a TMA write in flight: wait (bounded) for the last load
-      // issued into each slot.  In the normal path these phases completed
-      // long ago and the waits return at once.
-      for (int i = 0; i < kNPair && i < static_cast<int>(ring_it); ++i) {
-        const uint32_t last = ring_it - 1 - i;
-        ptx::mbar_wait(&C.slot_full[last % kNPair], (last / kNPair) & 1, 0x03);
-      }
-      if (kMode != kFused && u_idx > 0) ptx::mbar_wait(&C.q_full, (u_idx - 1) & 1, 0x04);
+    // Never leave a TMA write in flight: wait (bounded) for the final load of
+    // each slot if this warp issued it (an earlier load into a slot completed
+    // before the slot could be reused).  In the normal path these phases
+    // completed long ago and the waits return at once.
+    for (int i = 0; i < kNPair && i < static_cast<int>(ring_it); ++i) {
+      const uint32_t last = ring_it - 1 - i;
+      if (static_cast<int>(last % kL) != role) continue;
+      ptx::mbar_wait(&C.slot_full[last % kNPair], (last / kNPair) & 1, 0x03);
     }
+    if (kMode != kFused && role == 0 && u_idx > 0) ptx::mbar_wait(&C.q_full, (u_idx - 1) & 1, 0x04);
     __syncwarp();
   } else if (warp == 1) {
     // ============================== MMA issuer ==============================
-    if (lane == 0) {
-      const uint32_t idesc_qk = ptx::idesc_bf16_f32(128, kRowsPerCta, 0, 0);
-      const uint32_t idesc_pv = ptx::idesc_bf16_f32(128, kRowsPerCta, 1, 1);
-      const uint32_t q_addr = ptx::smem_u32(sQ);
-      const uint32_t ring_addr = ptx::smem_u32(sRing);
-      const uint32_t p_addr = ptx::smem_u32(sP);
-      uint32_t ring_it = 0, gt = 0;
-      int u_idx = 0;
-      Unit u;
-      bool ok = true;
-      auto wait_slot = [&](uint32_t& addr) -> int {
-        const int slot = ring_it % kNPair;
-        const uint32_t round = ring_it / kNPair;
-        ++ring_it;
-        if (!ptx::mbar_wait(&C.slot_full[slot], round & 1, 0x11)) return -1;
-        ptx::tc_fence_after();
-        addr = ring_addr + slot * kPairBytes;
-        return slot;
-      };
-      // Descriptor words of each operand's base; inner loops only add offsets.
-      const ptx::DescWords dq = ptx::desc_words(q_addr, 16, 1024, ptx::kLayoutSW128);
-      const ptx::DescWords dring = ptx::desc_words(ring_addr, 16, 1024, ptx::kLayoutSW128);
-      const ptx::DescWords dv = ptx::desc_words(ring_addr, kSubChunk, 1024, ptx::kLayoutSW128);
-      const ptx::DescWords dp = ptx::desc_words(p_addr, 16, 1024, ptx::kLayoutSW128);
-      auto do_qk = [&](uint32_t g) -> bool {
-        const int sb = g & 1;
-        if (!ptx::mbar_wait(&C.s_empty[sb], ((g >> 1) & 1) ^ 1, 0x12)) return false;
-        ptx::tc_fence_after();
-        const uint32_t d_tmem = tmem + kSCol + sb * kRowsPerCta;
+    // The whole warp runs the loop (its address arithmetic stays warp-uniform)
+    // and one elected lane issues each slot's UMMAs and commits.
+    const uint32_t idesc_qk = ptx::idesc_bf16_f32(128, kRowsPerCta, 0, 0);
+    const uint32_t idesc_pv = ptx::idesc_bf16_f32(128, kRowsPerCta, 1, 1);
+    const uint32_t q_addr = ptx::smem_u32(sQ);
+    const uint32_t ring_addr = ptx::smem_u32(sRing);
+    const uint32_t p_addr = ptx::smem_u32(sP);
+    uint32_t ring_it = 0, gt = 0;
+    int u_idx = 0;
+    Unit u;
+    bool ok = true;
+    auto warp_wait = [&](uint64_t* bar, uint32_t parity, int site) -> bool {
+      return __all_sync(0xffffffffu, ptx::mbar_wait(bar, parity, site));
+    };
+    auto wait_slot = [&]() -> int {
+      const int slot = ring_it % kNPair;
+      const uint32_t round = ring_it / kNPair;
+      ++ring_it;
+      if (!warp_wait(&C.slot_full[slot], round & 1, 0x11)) return -1;
+      ptx::tc_fence_after();
+      return slot;
+    };
+    // Descriptor words of each operand's base; inner loops only add offsets.
+    const ptx::DescWords dq = ptx::desc_words(q_addr, 16, 1024, ptx::kLayoutSW128);
+    const ptx::DescWords dring = ptx::desc_words(ring_addr, 16, 1024, ptx::kLayoutSW128);
+    const ptx::DescWords dv = ptx::desc_words(ring_addr, kSubChunk, 1024, ptx::kLayoutSW128);
+    const ptx::DescWords dp = ptx::desc_words(p_addr, 16, 1024, ptx::kLayoutSW128);
+    auto do_qk = [&](uint32_t g) -> bool {
+      const int sb = g & 1;
+      if (!warp_wait(&C.s_empty[sb], ((g >> 1) & 1) ^ 1, 0x12)) return false;
+      ptx::tc_fence_after();
+      const uint32_t d_tmem = tmem + kSCol + sb * kRowsPerCta;
 #pragma unroll
-        for (int pr = 0; pr < 5; ++pr) {
-          uint32_t a0;
-          const int slot = wait_slot(a0);
-          if (slot < 0) return false;
+      for (int pr = 0; pr < 5; ++pr) {
+        const int slot = wait_slot();
+        if (slot < 0) return false;
+        if (ptx::elect_one_sync()) {
           const uint32_t a_lo = dring.lo + ((slot * kPairBytes) >> 4);
 #pragma unroll
           for (int j = 0; j < 2; ++j) {
@@ -488,24 +498,27 @@ __global__ void __launch_bounds__(Threads<kMode>::value, 1)
             }
           }
           ptx::umma_commit(&C.slot_empty[slot]);
+          if (pr == 4) ptx::umma_commit(&C.s_full[sb]);
         }
-        ptx::umma_commit(&C.s_full[sb]);
-        return true;
-      };
-      auto do_pv = [&](uint32_t g, bool first_of_unit) -> bool {
-        const int pb = g % NPm;
-        if (!ptx::mbar_wait(&C.p_full[pb], (g / NPm) & 1, 0x13)) return false;
-        ptx::tc_fence_after();
-        const uint32_t b_lo = dp.lo + ((pb * kPBytes) >> 4);
-        for (int pr = 0; pr < nv_pairs; ++pr) {
-          uint32_t a0;
-          const int slot = wait_slot(a0);
-          if (slot < 0) return false;
+        __syncwarp();
+      }
+      return true;
+    };
+    auto do_pv = [&](uint32_t g, bool first_of_unit) -> bool {
+      const int pb = g % NPm;
+      if (!warp_wait(&C.p_full[pb], (g / NPm) & 1, 0x13)) return false;
+      ptx::tc_fence_after();
+      const uint32_t b_lo = dp.lo + ((pb * kPBytes) >> 4);
+      for (int pr = 0; pr < nv_pairs; ++pr) {
+        const int slot = wait_slot();
+        if (slot < 0) return false;
+        if (ptx::elect_one_sync()) {
           const uint32_t d_tmem = tmem + kOCol + pr * kRowsPerCta;
           const uint32_t a_lo = dv.lo + ((slot * kPairBytes) >> 4);
           // first k-step of the unit's first tile starts the accumulator
           ptx::umma_f16_ss_w(d_tmem, a_lo, dv.hi, b_lo, dp.hi, idesc_pv, first_of_unit ? 0u : 1u);
-          if (kPSplit) ptx::umma_f16_ss_w(d_tmem, a_lo, dv.hi, b_lo + (kPBytes >> 4), dp.hi, idesc_pv, 1u);
+          if (kPSplit)
+            ptx::umma_f16_ss_w(d_tmem, a_lo, dv.hi, b_lo + (kPBytes >> 4), dp.hi, idesc_pv, 1u);
 #pragma unroll
           for (int kk = 1; kk < kTileT / 16; ++kk) {
             ptx::umma_f16_ss_w(d_tmem, a_lo + ((kk * 2048) >> 4), dv.hi, b_lo + ((kk * 2048) >> 4),
@@ -515,34 +528,45 @@ __global__ void __launch_bounds__(Threads<kMode>::value, 1)
                                  b_lo + ((kPBytes + kk * 2048) >> 4), dp.hi, idesc_pv, 1u);
           }
           ptx::umma_commit(&C.slot_empty[slot]);
+          if (pr == nv_pairs - 1) ptx::umma_commit(&C.p_empty[pb]);
         }
-        ptx::umma_commit(&C.p_empty[pb]);
-        return true;
-      };
-      while (ok && it.template next<kMode>(P, u)) {
-        if (!ptx::mbar_wait(&C.q_full, u_idx & 1, 0x14)) break;
-        ptx::tc_fence_after();
-        const int n = u.hi - u.lo;
-        const uint32_t g0 = gt;
-        for (int k = 0; k < n && ok; ++k) {
-          ok = do_qk(g0 + k);
-          if (ok && k == n - 1) ptx::umma_commit(&C.q_empty);
-          if (ok && k >= 1) {
-            if (k == 1 && !ptx::mbar_wait(&C.o_free, (u_idx & 1) ^ 1, 0x15)) { ok = false; break; }
-            ok = do_pv(g0 + k - 1, k == 1);
-          }
-        }
-        if (ok) {
-          if (n == 1 && !ptx::mbar_wait(&C.o_free, (u_idx & 1) ^ 1, 0x16)) { ok = false; break; }
-          ok = do_pv(g0 + n - 1, n == 1);
-        }
-        gt += n;
-        ++u_idx;
+        __syncwarp();
       }
-      // Drain the tensor pipe before TMEM is released.
-      ptx::umma_commit(&C.drain);
-      ptx::mbar_wait(&C.drain, 0, 0x17);
+      return true;
+    };
+    while (ok && it.template next<kMode>(P, u)) {
+      if (!warp_wait(&C.q_full, u_idx & 1, 0x14)) break;
+      ptx::tc_fence_after();
+      const int n = u.hi - u.lo;
+      const uint32_t g0 = gt;
+      for (int k = 0; k < n && ok; ++k) {
+        ok = do_qk(g0 + k);
+        if (ok && k == n - 1) {
+          if (ptx::elect_one_sync()) ptx::umma_commit(&C.q_empty);
+          __syncwarp();
+        }
+        if (ok && k >= 1) {
+          if (k == 1 && !warp_wait(&C.o_free, (u_idx & 1) ^ 1, 0x15)) {
+            ok = false;
+            break;
+          }
+          ok = do_pv(g0 + k - 1, k == 1);
+        }
+      }
+      if (ok) {
+        if (n == 1 && !warp_wait(&C.o_free, (u_idx & 1) ^ 1, 0x16)) {
+          ok = false;
+          break;
+        }
+        ok = do_pv(g0 + n - 1, n == 1);
+      }
+      gt += n;
+      ++u_idx;
     }
+    // Drain the tensor pipe before TMEM is released.
+    if (ptx::elect_one_sync()) ptx::umma_commit(&C.drain);
+    __syncwarp();
+    ptx::mbar_wait(&C.drain, 0, 0x17);
     __syncwarp();
   } else if (warp >= 2 && warp < 2 + 4 * kSoftmaxGroups) {
     // ============================== softmax / epilogue ==============================
