@@ -176,7 +176,8 @@ class GpuStep:
             self.ns = torch.empty((b + 1,), dtype=torch.int32, device=dev)
 
     def launches_per_step(self):
-        return 3  # planner + decode + combine
+        # planner + attention kernel + combine (+ the FP8 gather for sparse)
+        return 4 if self.kind == "sparse" else 3
 
     def step(self, q=None):
         B, c = self.B, self.case

@@ -210,15 +210,14 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* total) {
 
 // Split-KV planner of one CTA: the closed forms of mla_common.h evaluated in
 // parallel (prefix sums by block scans, one metadata row per thread).
-// len_or_neg < 0: lengths from seqlens; else every sequence has that length.
-__device__ void plan_block(const int32_t* seqlens, int len_or_neg, int batch, int num_parts,
+__device__ void plan_block(const int32_t* seqlens, int batch, int num_parts,
                            int32_t* metadata, int32_t* num_splits) {
   __shared__ int32_t C[kPlanMaxBatch + 1];
   const int tid = threadIdx.x;
   int carry = 0;
   for (int base = 0; base < batch; base += kPlanThreads) {
     const int b = base + tid;
-    const int L = b < batch ? (len_or_neg < 0 ? seqlens[b] : len_or_neg) : 0;
+    const int L = b < batch ? seqlens[b] : 0;
     const int v = b < batch ? tiles_of(L) + kSegmentOverheadTiles : 0;
     int chunk_total;
     const int ex = block_exclusive_scan(v, &chunk_total);
@@ -247,17 +246,7 @@ __global__ void __launch_bounds__(kPlanThreads) mla_plan_kernel(const int32_t* s
                                                                int32_t* num_splits) {
   ptx::grid_dep_wait();
   ptx::grid_dep_launch();  // the decode grid waits for this one at its start
-  plan_block(seqlens, -1, batch, num_parts, metadata, num_splits);
-}
-
-// Planner over `batch` items of equal length `len` (sparse decode).
-__global__ void __launch_bounds__(kPlanThreads) mla_plan_uniform_kernel(int len, int batch,
-                                                                       int num_parts,
-                                                                       int32_t* metadata,
-                                                                       int32_t* num_splits) {
-  ptx::grid_dep_wait();
-  ptx::grid_dep_launch();
-  plan_block(nullptr, len, batch, num_parts, metadata, num_splits);
+  plan_block(seqlens, batch, num_parts, metadata, num_splits);
 }
 
 }  // namespace mla

@@ -21,10 +21,10 @@
 // ..., so the softmax of tile k overlaps QK of tile k+1.  V chunks are fetched
 // a second time for PV (an L2 hit) instead of holding a whole 144 KB tile.
 //
-// Roles (warps):  0 = loader (TMA),  1 = MMA issuer + TMEM owner,
-//   2..5 = softmax warpgroup (one thread per token lane of the tile; also the
-//   epilogue and, for the fused variant, the Q RMSNorm + RoPE prologue),
-//   6..9 = FP8 gather/dequant warpgroup (sparse variant only).
+// Roles (warps):  0, 10, 11 = TMA loaders (0 also loads Q),  1 = MMA issuer +
+//   TMEM owner,  2..9 = two softmax warpgroups (one thread per token lane of
+//   the tile and 32 query-row columns each; also the epilogue and, for the
+//   fused variant, the Q RMSNorm + RoPE prologue).
 //
 // Softmax uses a lazily updated per-row reference max m: scores are
 // exponentiated against m until some score exceeds m by more than 8 (log2
@@ -42,12 +42,12 @@
 
 namespace mla {
 
-enum Mode : int { kDense = 0, kFused = 1, kSparse = 2 };
+enum Mode : int { kDense = 0, kFused = 1 };
 
 struct DecodeParams {
-  int batch;       // sequences (dense/fused) or (sequence, query) pairs (sparse)
+  int batch;       // sequences
   int s_q, h_q;    // query tokens per sequence and heads
-  int R;           // rows sharing one KV head: s_q*h_q (dense/fused), h_q (sparse)
+  int R;           // rows sharing one KV head: s_q*h_q
   int d_v;         // 512 or 576
   int n_groups;    // ceil(R / 64)
   int num_parts;   // scheduler parts; grid = num_parts * n_groups
@@ -72,11 +72,6 @@ struct DecodeParams {
   float rope_base;
   const int32_t* positions;  // nullable: position = L - 1
   double inv_freq[kRope / 2];  // base^(-2k/64), computed on the host in fp64
-  // sparse
-  const uint8_t* cache656;  // [num_slots, 656]
-  const int32_t* indices;   // [batch(pairs), topk]
-  int topk;
-  long long num_slots;
 };
 
 namespace cfg {
@@ -112,24 +107,21 @@ constexpr int kPrefetchTiles = MLA_PREFETCH_TILES;  // pages of tile k + this ar
 // spans all of them (ids 1..6 are per-group).
 constexpr int kSoftmaxGroups = 2;
 constexpr int kBarAllSoftmax = 7;
-constexpr int kGatherThreads = 64;  // sparse: each gather thread fills two token rows
 
 // TMA loader warps filling the ring round-robin (one issuing warp sustains
 // only about 25 B/clk): warp 0, then warps 10, 11 after the softmax groups.
-// The sparse variant fills its ring from the gather warps instead.
 #ifndef MLA_DECODE_LOADERS
 #define MLA_DECODE_LOADERS 3
 #endif
 template <int kMode>
 struct Loaders {
-  static constexpr int value = kMode == kSparse ? 1 : MLA_DECODE_LOADERS;
+  static constexpr int value = MLA_DECODE_LOADERS;
 };
 
 template <int kMode>
 struct Threads {
-  // loader + MMA warps, softmax groups, extra loaders, and for sparse two gather warps
-  static constexpr int value = 64 + 128 * kSoftmaxGroups + 32 * (Loaders<kMode>::value - 1) +
-                               (kMode == kSparse ? kGatherThreads : 0);
+  // loader + MMA warps, softmax groups, extra loaders
+  static constexpr int value = 64 + 128 * kSoftmaxGroups + 32 * (Loaders<kMode>::value - 1);
 };
 
 // Shared-memory control block (at kBarOff).
@@ -170,7 +162,7 @@ struct UnitIter {
   __device__ bool next(const DecodeParams& P, Unit& u) {
     while (b <= b_end) {
       const int bb = b++;
-      const int L = (kMode == kSparse) ? P.topk : P.seqlens[bb];
+      const int L = P.seqlens[bb];
       const int lo = (bb == b_first) ? t_begin : 0;
       const int hi = (bb == b_end) ? t_end : tiles_of(L);
       if (lo >= hi) continue;
@@ -234,58 +226,6 @@ __device__ __forceinline__ int clamp_block(int blk, int num_blocks) {
 }
 
 // --------------------------------------------------------------------------
-// Sparse gather: dequantise one token's chunks of a pair slot into the
-// swizzled bf16 layout.  Row layout: [512 e4m3][4 fp32 scales][64 bf16].
-// [FlashMLA (AI Wiki), "The FP8 and FP4 KV cache"]
-__device__ __forceinline__ void sparse_fill_pair(uint8_t* slot, int t, const uint8_t* row,
-                                                 bool valid, int pair) {
-  const int sw = t & 7;
-  uint8_t* rowbase = slot + t * 128;
-#pragma unroll
-  for (int j = 0; j < 2; ++j) {
-    const int c = 2 * pair + j;
-    if (c >= kNumChunks) break;
-    uint8_t* dst = rowbase + j * cfg::kSubChunk;
-    if (!valid) {
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-        *reinterpret_cast<uint4*>(dst + ((u ^ sw) << 4)) = make_uint4(0, 0, 0, 0);
-      continue;
-    }
-    if (c == kNumChunks - 1) {
-      // RoPE dims: bf16 copy
-      const uint4* src = reinterpret_cast<const uint4*>(row + kNope + 16);
-#pragma unroll
-      for (int u = 0; u < 8; ++u) *reinterpret_cast<uint4*>(dst + ((u ^ sw) << 4)) = __ldg(src + u);
-    } else {
-      const float sc = __ldg(reinterpret_cast<const float*>(row + kNope) + (c >> 1));
-      const uint4* src = reinterpret_cast<const uint4*>(row + c * 64);
-#pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        const uint4 w = __ldg(src + v);  // 16 codes -> two 16-byte output units
-        const uint32_t words[4] = {w.x, w.y, w.z, w.w};
-        uint32_t o[8];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint16_t lo16 = static_cast<uint16_t>(words[q] & 0xFFFF);
-          const uint16_t hi16 = static_cast<uint16_t>(words[q] >> 16);
-          uint32_t h0, h1;
-          asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h0) : "h"(lo16));
-          asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h1) : "h"(hi16));
-          const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&h0));
-          const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&h1));
-          o[2 * q] = ptx::pack_bf16x2(f0.x * sc, f0.y * sc);
-          o[2 * q + 1] = ptx::pack_bf16x2(f1.x * sc, f1.y * sc);
-        }
-        const int u0 = 2 * v, u1 = 2 * v + 1;
-        *reinterpret_cast<uint4*>(dst + ((u0 ^ sw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-        *reinterpret_cast<uint4*>(dst + ((u1 ^ sw) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
-      }
-    }
-  }
-}
-
-// --------------------------------------------------------------------------
 template <int kMode>
 __global__ void __launch_bounds__(Threads<kMode>::value, 1)
     mla_decode_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -318,7 +258,7 @@ __global__ void __launch_bounds__(Threads<kMode>::value, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kNPair; ++i) {
-      ptx::mbar_init(&C.slot_full[i], kMode == kSparse ? kGatherThreads : 1);
+      ptx::mbar_init(&C.slot_full[i], 1);
       ptx::mbar_init(&C.slot_empty[i], 1);
     }
     ptx::mbar_init(&C.q_full, kMode == kFused ? 128 * kSoftmaxGroups : 1);
@@ -342,7 +282,7 @@ __global__ void __launch_bounds__(Threads<kMode>::value, 1)
   }
   if (warp == 0 && lane == 0) {
     if (kMode != kFused) ptx::prefetch_tmap(&tm_q);
-    if (kMode != kSparse) ptx::prefetch_tmap(&tm_kv);
+    ptx::prefetch_tmap(&tm_kv);
   }
   ptx::tc_fence_before();
   __syncthreads();
@@ -354,7 +294,7 @@ __global__ void __launch_bounds__(Threads<kMode>::value, 1)
 
   constexpr int kL = Loaders<kMode>::value;
   constexpr int kFirstExtraLoader = 2 + 4 * kSoftmaxGroups;
-  if (warp == 0 || (kMode != kSparse && warp >= kFirstExtraLoader)) {
+  if (warp == 0 || warp >= kFirstExtraLoader) {
     // ============================== loaders ==============================
     // Pair slot j of the ring is filled by loader warp j % kL (whole warp,
     // one elected lane issues the copies).  Warp 0 also loads Q; for the fused
@@ -424,7 +364,7 @@ __global__ void __launch_bounds__(Threads<kMode>::value, 1)
         }
         __syncwarp();
       }
-      if (kMode != kSparse && ok) {
+      if (ok) {
         const int n = u.hi - u.lo;
         for (int k = 0; k < n && ok; ++k) {
           for (int pr = 0; pr < 5 && ok; ++pr) ok = load_pair(u, u.lo + k, pr);
@@ -589,7 +529,7 @@ __global__ void __launch_bounds__(Threads<kMode>::value, 1)
         const int rg = grp * kRowsPerCta + cb + wt;
         int lim = 0;
         if (rg < P.R) {
-          if (kMode == kSparse || !P.causal) {
+          if (!P.causal) {
             lim = u.L;
           } else {
             lim = u.L - P.s_q + 1 + rg / P.h_q;
@@ -694,17 +634,12 @@ __global__ void __launch_bounds__(Threads<kMode>::value, 1)
 
         const int tile_tok0 = (u.lo + k) * kTileT;
         const int T = tile_tok0 + t;
-        bool tok_valid = true;
-        if (kMode == kSparse) {
-          const int idx = (T < P.topk) ? __ldg(P.indices + (size_t)u.b * P.topk + T) : -1;
-          tok_valid = idx >= 0 && static_cast<long long>(idx) < P.num_slots;
-        }
-        const bool need_mask = (tile_tok0 + kTileT > min_lim) || !tok_valid;
+        const bool need_mask = tile_tok0 + kTileT > min_lim;
         int need = 0;
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
           float v = x[c] * P.scale_log2;
-          if (need_mask && (!tok_valid || T >= C.lim[cb + c])) v = -INFINITY;
+          if (need_mask && T >= C.lim[cb + c]) v = -INFINITY;
           x[c] = v;
           need |= (v > C.m[cb + c] + kRescaleThreshold);
         }
@@ -848,43 +783,6 @@ __global__ void __launch_bounds__(Threads<kMode>::value, 1)
       ptx::named_bar_sync(bar_sync, 128);  // C.alpha / C.red / C.lim reusable
       gt += n;
       ++u_idx;
-    }
-  } else if (kMode == kSparse && warp >= 2 + 4 * kSoftmaxGroups) {
-    // ============================== FP8 gather / dequant ==============================
-    const int t0 = threadIdx.x - (64 + 128 * kSoftmaxGroups);  // token lanes t0, t0 + 64
-    uint32_t ring_it = 0;
-    Unit u;
-    bool ok = true;
-    auto fill = [&](const Unit& un, int tile, int pair) -> bool {
-      const int slot = ring_it % kNPair;
-      const uint32_t round = ring_it / kNPair;
-      ++ring_it;
-      if (!ptx::mbar_wait(&C.slot_empty[slot], (round & 1) ^ 1, 0x31)) return false;
-#pragma unroll 1
-      for (int h = 0; h < kTileT / kGatherThreads; ++h) {
-        const int t = t0 + h * kGatherThreads;
-        const int j = tile * kTileT + t;
-        const int idx = (j < P.topk) ? __ldg(P.indices + (size_t)un.b * P.topk + j) : -1;
-        bool valid = idx >= 0;
-        if (valid && static_cast<long long>(idx) >= P.num_slots) {
-          ptx::set_error(MLA_DEVERR_BAD_INDEX, 0x32);
-          valid = false;
-        }
-        const uint8_t* row = P.cache656 + (valid ? (size_t)idx * kRow656 : 0);
-        sparse_fill_pair(sRing + slot * kPairBytes, t, row, valid, pair);
-      }
-      ptx::fence_proxy_async_smem();
-      ptx::mbar_arrive(&C.slot_full[slot]);
-      return true;
-    };
-    while (ok && it.template next<kMode>(P, u)) {
-      const int n = u.hi - u.lo;
-      for (int k = 0; k < n && ok; ++k) {
-        for (int pr = 0; pr < 5 && ok; ++pr) ok = fill(u, u.lo + k, pr);
-        if (k >= 1)
-          for (int pr = 0; pr < nv_pairs && ok; ++pr) ok = fill(u, u.lo + k - 1, pr);
-      }
-      for (int pr = 0; pr < nv_pairs && ok; ++pr) ok = fill(u, u.hi - 1, pr);
     }
   }
 

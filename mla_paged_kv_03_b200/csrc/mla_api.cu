@@ -15,6 +15,7 @@
 #include "combine_kernel.cuh"
 #include "decode_kernel.cuh"
 #include "pair_kernel.cuh"
+#include "sparse_gather.cuh"
 #include "mla_common.h"
 
 namespace {
@@ -120,7 +121,7 @@ int prepare_kernel() {
 }
 
 struct WsLayout {
-  size_t o_off, lse_off, meta_off, splits_off, total;
+  size_t o_off, lse_off, total;
 };
 
 WsLayout dense_ws_layout(int batch, int R, int d_v, int parts) {
@@ -132,11 +133,26 @@ WsLayout dense_ws_layout(int batch, int R, int d_v, int parts) {
   return w;
 }
 
-WsLayout sparse_ws_layout(int pairs, int R, int d_v, int parts) {
-  WsLayout w = dense_ws_layout(pairs, R, d_v, parts);
-  w.meta_off = w.total;
+// Sparse decode workspace: the gathered bf16 rows (a dense paged buffer of
+// pages_per_pair pages per (sequence, query) pair), its block table and
+// lengths, the split tables, then the dense decode workspace.
+struct SparseWs {
+  size_t rows_off, bt_off, len_off, meta_off, splits_off, dense_off, dense_bytes, total;
+  int pages_per_pair;
+};
+
+SparseWs sparse_ws_layout(int pairs, int topk, int R, int d_v, int parts) {
+  SparseWs w{};
+  w.pages_per_pair = mla::ceil_div(topk, mla::kPage);
+  const size_t pages = static_cast<size_t>(pairs) * w.pages_per_pair;
+  w.rows_off = 0;
+  w.bt_off = align_up(pages * mla::kPage * mla::kD * 2, 256);
+  w.len_off = w.bt_off + align_up(pages * 4, 256);
+  w.meta_off = w.len_off + align_up(static_cast<size_t>(pairs) * 4, 256);
   w.splits_off = w.meta_off + align_up(static_cast<size_t>(parts) * mla::kMetaInts * 4, 256);
-  w.total = w.splits_off + align_up((static_cast<size_t>(pairs) + 1) * 4, 256);
+  w.dense_off = w.splits_off + align_up((static_cast<size_t>(pairs) + 1) * 4, 256);
+  w.dense_bytes = dense_ws_layout(pairs, R, d_v, parts).total;
+  w.total = w.dense_off + w.dense_bytes;
   return w;
 }
 
@@ -563,7 +579,7 @@ int mla_sparse_workspace_size(int batch, int s_q, int h_q, int topk, int d_v, in
   MLA_CHECK_ARG(batch >= 0 && s_q >= 1 && h_q >= 1 && topk >= 1 && num_sm_parts >= 1,
                 "bad sizes");
   MLA_CHECK_ARG(d_v == 512, "sparse decode supports d_v = 512 (got %d)", d_v);
-  *bytes = sparse_ws_layout(batch * s_q, h_q, d_v, num_sm_parts).total;
+  *bytes = sparse_ws_layout(batch * s_q, topk, h_q, d_v, num_sm_parts).total;
   return MLA_OK;
 }
 
@@ -584,61 +600,41 @@ int mla_sparse_decode(const void* q, const uint8_t* kcache_fp8, int64_t num_slot
   MLA_CHECK_ARG(aligned(workspace, 256), "workspace must be 256-byte aligned");
   MLA_CHECK_ARG(aligned(out, 8) && aligned(lse, 4) && aligned(indices, 4), "misaligned output");
   const int pairs = batch * s_q;
-  const WsLayout w = sparse_ws_layout(pairs, h_q, d_v, num_sm_parts);
+  MLA_CHECK_ARG(aligned(out, 16), "out must be 16-byte aligned");
+  const SparseWs w = sparse_ws_layout(pairs, topk, h_q, d_v, num_sm_parts);
   MLA_CHECK_ARG(workspace_bytes >= w.total, "workspace too small: %zu < %zu", workspace_bytes,
                 w.total);
+  MLA_CHECK_ARG(pairs <= mla::kPlanMaxBatch, "at most %d (batch, query) pairs (got %d)",
+                mla::kPlanMaxBatch, pairs);
+  const long long pages = static_cast<long long>(pairs) * w.pages_per_pair;
+  MLA_CHECK_ARG(pages * mla::kPage < (1LL << 31), "pairs * topk too large");
   if (batch == 0) return MLA_OK;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  int32_t* meta = reinterpret_cast<int32_t*>(ws + w.meta_off);
-  int32_t* splits = reinterpret_cast<int32_t*>(ws + w.splits_off);
-  MLA_CHECK_ARG(pairs <= mla::kPlanMaxBatch, "at most %d (batch, query) pairs (got %d)",
-                mla::kPlanMaxBatch, pairs);
-  mla::mla_plan_uniform_kernel<<<1, mla::kPlanThreads, 0, st>>>(topk, pairs, num_sm_parts, meta,
-                                                                 splits);
+
+  // 1. gather + dequantise + compact the valid tokens of every pair
+  mla::GatherParams g{};
+  g.cache656 = kcache_fp8;
+  g.num_slots = num_slots;
+  g.indices = indices;
+  g.topk = topk;
+  g.pages_per_pair = w.pages_per_pair;
+  g.rows = reinterpret_cast<__nv_bfloat16*>(ws + w.rows_off);
+  g.block_table = reinterpret_cast<int32_t*>(ws + w.bt_off);
+  g.seqlens = reinterpret_cast<int32_t*>(ws + w.len_off);
+  mla::mla_sparse_gather_kernel<<<dim3(w.pages_per_pair, pairs), mla::kGatherCtaThreads, 0, st>>>(g);
   MLA_CUDA(cudaGetLastError());
 
-  CUtensorMap tq;
-  int rc = make_latent_map(&tq, q, static_cast<long long>(pairs) * h_q);
+  // 2. dense decode over the compacted rows: no causal mask, lengths = valid counts
+  int32_t* meta = reinterpret_cast<int32_t*>(ws + w.meta_off);
+  int32_t* splits = reinterpret_cast<int32_t*>(ws + w.splits_off);
+  int rc = mla_get_metadata(g.seqlens, pairs, h_q, 1, num_sm_parts, meta, splits, stream);
   if (rc != MLA_OK) return rc;
-
-  mla::DecodeParams p{};
-  p.batch = pairs;
-  p.s_q = 1;
-  p.h_q = h_q;
-  p.R = h_q;
-  p.d_v = d_v;
-  p.n_groups = mla::ceil_div(h_q, mla::kRowsPerCta);
-  p.num_parts = num_sm_parts;
-  p.num_blocks = 1;
-  p.max_pages = 1;
-  p.causal = 0;
-  p.always_partial = 0;
-  p.scale_log2 = softmax_scale * 1.4426950408889634f;
-  p.metadata = meta;
-  p.num_splits = splits;
-  p.out = static_cast<__nv_bfloat16*>(out);
-  p.lse = lse;
-  p.ws_o = reinterpret_cast<float*>(ws + w.o_off);
-  p.ws_lse = reinterpret_cast<float*>(ws + w.lse_off);
-  p.cache656 = kcache_fp8;
-  p.indices = indices;
-  p.topk = topk;
-  p.num_slots = num_slots;
-  if ((rc = launch_decode<mla::kSparse>(tq, tq, p, st)) != MLA_OK) return rc;
-
-  mla::CombineParams cp{};
-  cp.batch = pairs;
-  cp.R = h_q;
-  cp.d_v = d_v;
-  cp.h_q = h_q;
-  cp.num_splits = splits;
-  cp.ws_o = p.ws_o;
-  cp.ws_lse = p.ws_lse;
-  cp.out = p.out;
-  cp.lse = lse;
-  return launch_combine(cp, false, st);
+  return mla_decode_fwd(q, g.rows, g.block_table, w.pages_per_pair, static_cast<int>(pages),
+                        g.seqlens, pairs, 1, h_q, 1, d_v, softmax_scale, 0, meta, splits,
+                        num_sm_parts, ws + w.dense_off, w.dense_bytes, out, lse, stream);
 }
+
 
 int mla_set_kernel_events(void* start_event, void* stop_event) {
   t_kernel_start = static_cast<cudaEvent_t>(start_event);

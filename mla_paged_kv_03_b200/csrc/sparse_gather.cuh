@@ -1,0 +1,143 @@
+// sparse_gather.cuh -- first step of token-level sparse decode: gather the
+// selected rows of the 656-byte FP8 latent cache, dequantise them to bf16 and
+// compact each query's valid tokens into a dense paged buffer that the dense
+// decode kernels then attend over.
+//
+// Cache row (per token): [512 x E4M3 codes][4 x fp32 scale, one per 128
+// codes][64 x bf16 RoPE dims]; a nope value is code * scale.
+// [FlashMLA (AI Wiki), "The FP8 and FP4 KV cache"]
+// Indices (per (sequence, query) pair): physical slots, -1 (or any value
+// outside [0, num_slots)) marks an unused entry; the block table of the cache
+// is not used.  [FlashMLA (AI Wiki), "Interfaces"]
+//
+// Attention is invariant to the order of the attended tokens, so the valid
+// tokens of pair b are written in index order to rows [0, n_b) of b's region
+// of the buffer (pages of 64 rows, b's pages numbered b * pages_per_pair + p),
+// n_b goes to seqlens[b], and the dense kernels run with that identity block
+// table, no causal mask and lengths n_b.  A pair without valid tokens gets
+// n_b = 0, hence O = 0 and LSE = -inf.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cstdint>
+
+#include "mla_common.h"
+#include "ptx.cuh"
+
+namespace mla {
+
+constexpr int kGatherTokens = 64;  // tokens per CTA = one page of the buffer
+constexpr int kGatherCtaThreads = 256;
+constexpr int kRowUnits = kD / 8;  // 16-byte bf16 output units per row (72)
+
+struct GatherParams {
+  const uint8_t* cache656;  // [num_slots, 656]
+  long long num_slots;
+  const int32_t* indices;   // [pairs, topk]
+  int topk;
+  int pages_per_pair;       // ceil(topk / 64)
+  __nv_bfloat16* rows;      // [pairs * pages_per_pair * 64, 576]
+  int32_t* block_table;     // [pairs, pages_per_pair]
+  int32_t* seqlens;         // [pairs]
+};
+
+__device__ __forceinline__ bool gather_valid(int idx, long long num_slots) {
+  return idx >= 0 && static_cast<long long>(idx) < num_slots;
+}
+
+// grid (pages_per_pair, pairs): CTA (c, b) handles indices [64c, 64c + 64) of pair b.
+__global__ void __launch_bounds__(kGatherCtaThreads)
+    mla_sparse_gather_kernel(const GatherParams G) {
+  __shared__ int s_red[kGatherCtaThreads / 32];
+  __shared__ int s_idx[kGatherTokens];
+  __shared__ int s_dst[kGatherTokens];  // destination row within the pair, or -1
+  __shared__ int s_base;
+  ptx::grid_dep_wait();
+  const int c = blockIdx.x, b = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int32_t* idx_b = G.indices + (size_t)b * G.topk;
+
+  // valid tokens in the pair's earlier chunks: this chunk's first output row
+  int cnt = 0;
+  for (int j = tid; j < c * kGatherTokens; j += kGatherCtaThreads)
+    cnt += gather_valid(__ldg(idx_b + j), G.num_slots) ? 1 : 0;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+  if (lane == 0) s_red[warp] = cnt;
+
+  // this chunk: validity and rank among the chunk's valid tokens (warps 0, 1)
+  if (tid < kGatherTokens) {
+    const int j = c * kGatherTokens + tid;
+    const int idx = j < G.topk ? __ldg(idx_b + j) : -1;
+    bool v = gather_valid(idx, G.num_slots);
+    if (j < G.topk && idx >= 0 && !v) ptx::set_error(MLA_DEVERR_BAD_INDEX, 0x80);
+    const unsigned m = __ballot_sync(0xffffffffu, v);
+    s_idx[tid] = idx;
+    s_dst[tid] = v ? __popc(m & ((1u << lane) - 1)) : -1;  // rank within the warp
+    if (tid == 0) s_base = __popc(m);  // valid tokens among the chunk's first 32
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int before = 0;
+    for (int w = 0; w < kGatherCtaThreads / 32; ++w) before += s_red[w];
+    s_red[0] = before;
+  }
+  __syncthreads();
+  const int before = s_red[0];
+  if (tid < kGatherTokens && s_dst[tid] >= 0)
+    s_dst[tid] += before + (tid >= 32 ? s_base : 0);
+  __syncthreads();
+
+  __nv_bfloat16* out_b = G.rows + (size_t)b * G.pages_per_pair * kGatherTokens * kD;
+  if (tid == 0) G.block_table[(size_t)b * G.pages_per_pair + c] = b * G.pages_per_pair + c;
+  if (c == G.pages_per_pair - 1) {
+    // the pair's length, and zeros for the rest of its last page: the decode
+    // kernel masks those tokens, but multiplies their rows by P = 0
+    __shared__ int s_n;
+    if (tid == 0) {
+      int n = 0;
+      for (int t = 0; t < kGatherTokens; ++t) n += s_dst[t] >= 0 ? 1 : 0;
+      s_n = before + n;
+      G.seqlens[b] = s_n;
+    }
+    __syncthreads();
+    const int n = s_n;
+    const int end = (n + kGatherTokens - 1) / kGatherTokens * kGatherTokens;
+    for (int item = tid; item < (end - n) * kRowUnits; item += kGatherCtaThreads)
+      *reinterpret_cast<uint4*>(out_b + (size_t)(n + item / kRowUnits) * kD + 8 * (item % kRowUnits)) =
+          make_uint4(0, 0, 0, 0);
+  }
+
+  // dequantise: 64 tokens x 72 output units of 8 bf16
+  for (int item = tid; item < kGatherTokens * kRowUnits; item += kGatherCtaThreads) {
+    const int t = item / kRowUnits, u = item % kRowUnits;
+    const int dst = s_dst[t];
+    if (dst < 0) continue;
+    const uint8_t* row = G.cache656 + (size_t)s_idx[t] * kRow656;
+    uint4 o;
+    if (u < kNope / 8) {
+      const float sc = __ldg(reinterpret_cast<const float*>(row + kNope) + (u >> 4));
+      const uint2 w = __ldg(reinterpret_cast<const uint2*>(row + 8 * u));
+      const uint32_t words[2] = {w.x, w.y};
+      uint32_t r[4];
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        uint32_t h0, h1;
+        const uint16_t lo16 = static_cast<uint16_t>(words[q] & 0xFFFF);
+        const uint16_t hi16 = static_cast<uint16_t>(words[q] >> 16);
+        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h0) : "h"(lo16));
+        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h1) : "h"(hi16));
+        const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&h0));
+        const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&h1));
+        r[2 * q] = ptx::pack_bf16x2(f0.x * sc, f0.y * sc);
+        r[2 * q + 1] = ptx::pack_bf16x2(f1.x * sc, f1.y * sc);
+      }
+      o = make_uint4(r[0], r[1], r[2], r[3]);
+    } else {
+      o = __ldg(reinterpret_cast<const uint4*>(row + kNope + 16) + (u - kNope / 8));
+    }
+    *reinterpret_cast<uint4*>(out_b + (size_t)dst * kD + 8 * u) = o;
+  }
+}
+
+}  // namespace mla
