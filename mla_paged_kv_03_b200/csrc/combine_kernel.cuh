@@ -32,6 +32,7 @@ struct CombineParams {
   const int32_t* seqlens;
   const int32_t* positions;   // nullable: L - 1
   double inv_freq[kRope / 2]; // base^(-2k/64), computed on the host in fp64
+  int row_per_cta;            // 1: a CTA's warps share one row's splits (few rows)
 };
 
 __device__ __forceinline__ uint32_t cvt_e4m3x4(float a, float b, float c, float d) {
@@ -41,137 +42,151 @@ __device__ __forceinline__ uint32_t cvt_e4m3x4(float a, float b, float c, float 
   return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
 }
 
-// One CTA per row; thread i owns the float4 group i of the row (d_v / 4 = 128
-// or 144 threads).  The split weights are formed once in shared memory.
+// One warp per row: lane l owns the float4 groups l, l + 32, ... of the row
+// (d_v / 4 = 128 or 144 groups); split weights are formed 32 at a time, one
+// per lane, and broadcast with shuffles.  With few rows and many splits
+// (row_per_cta) the CTA's warps take every kCombineWarps-th split of one row
+// and add their sums in shared memory.
 constexpr int kCombineMaxSplits = 1024;  // splits of one sequence (<= SM parts)
-constexpr int kCombineThreads = 160;
+constexpr int kCombineWarps = 8;
+constexpr int kCombineThreads = 32 * kCombineWarps;
+constexpr int kCombineGroups = (kD / 4 + 31) / 32;  // float4 groups per lane (5)
 
 template <bool kFusedOut>
 __global__ void __launch_bounds__(kCombineThreads) mla_combine_kernel(const CombineParams P) {
-  __shared__ float s_w[kCombineMaxSplits];
-  __shared__ float s_red[kCombineThreads / 32];
-  __shared__ float s_lse;
+  __shared__ float4 s_acc[kCombineWarps - 1][kD / 4];
   ptx::grid_dep_wait();  // the decode kernel's partials are complete
-  const int row_id = blockIdx.x;
-  const int b = row_id / P.R;
-  const int r = row_id % P.R;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool shared_row = P.row_per_cta != 0;
+  const long long row_id =
+      shared_row ? blockIdx.x : static_cast<long long>(blockIdx.x) * kCombineWarps + warp;
+  if (row_id >= static_cast<long long>(P.batch) * P.R) return;
+  const int b = static_cast<int>(row_id / P.R);
+  const int r = static_cast<int>(row_id % P.R);
   const int base = P.num_splits[b];
   const int n = P.num_splits[b + 1] - base;
   if (!kFusedOut && n <= 1) return;  // written directly by the decode kernel
-  const int tid = threadIdx.x;
-  const int lane = tid & 31, warp = tid >> 5;
-  constexpr int kWarps = kCombineThreads / 32;
 
-  // max over the split LSEs
+  // LSE of the merged row: max-subtracted log-sum-exp of the split LSEs
+  const float* lse_i = P.ws_lse + (size_t)base * P.R + r;
   float m = -INFINITY;
-  for (int i = tid; i < n; i += kCombineThreads) {
-    const float li = P.ws_lse[(size_t)(base + i) * P.R + r];
-    s_w[i] = li;
-    m = fmaxf(m, li);
-  }
+  for (int i = lane; i < n; i += 32) m = fmaxf(m, lse_i[(size_t)i * P.R]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  if (lane == 0) s_red[warp] = m;
-  __syncthreads();
-  m = s_red[0];
-#pragma unroll
-  for (int w = 1; w < kWarps; ++w) m = fmaxf(m, s_red[w]);
-  __syncthreads();
   float sum = 0.f;
   if (m != -INFINITY)
-    for (int i = tid; i < n; i += kCombineThreads) sum += expf(s_w[i] - m);
+    for (int i = lane; i < n; i += 32) sum += expf(lse_i[(size_t)i * P.R] - m);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-  if (lane == 0) s_red[warp] = sum;
-  __syncthreads();
-  if (tid == 0) {
-    float t = 0.f;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) t += s_red[w];
-    s_lse = (m == -INFINITY) ? -INFINITY : m + logf(t);
-  }
-  __syncthreads();
-  const float lse = s_lse;
-  for (int i = tid; i < n; i += kCombineThreads)
-    s_w[i] = (lse == -INFINITY || s_w[i] == -INFINITY) ? 0.f : expf(s_w[i] - lse);
-  __syncthreads();
+  const float lse = (m == -INFINITY) ? -INFINITY : m + logf(sum);
 
+  // O = sum_i exp(LSE_i - LSE) O_i
   const int ngroups = P.d_v / 4;
-  const int g = tid;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (g < ngroups) {
-    const float4* src = reinterpret_cast<const float4*>(P.ws_o + ((size_t)base * P.R + r) * P.d_v) + g;
-    const size_t stride = (size_t)P.R * P.d_v / 4;  // float4s between consecutive splits
-    int i = 0;
-    for (; i + 4 <= n; i += 4) {
-      const float4 v0 = src[(i + 0) * stride], v1 = src[(i + 1) * stride];
-      const float4 v2 = src[(i + 2) * stride], v3 = src[(i + 3) * stride];
-      const float w0 = s_w[i], w1 = s_w[i + 1], w2 = s_w[i + 2], w3 = s_w[i + 3];
-      acc.x += w0 * v0.x + w1 * v1.x + w2 * v2.x + w3 * v3.x;
-      acc.y += w0 * v0.y + w1 * v1.y + w2 * v2.y + w3 * v3.y;
-      acc.z += w0 * v0.z + w1 * v1.z + w2 * v2.z + w3 * v3.z;
-      acc.w += w0 * v0.w + w1 * v1.w + w2 * v2.w + w3 * v3.w;
+  const float4* src0 = reinterpret_cast<const float4*>(P.ws_o + ((size_t)base * P.R + r) * P.d_v);
+  const size_t stride = (size_t)P.R * P.d_v / 4;  // float4s between consecutive splits
+  float4 acc[kCombineGroups];
+#pragma unroll
+  for (int j = 0; j < kCombineGroups; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+  const int k_first = shared_row ? warp : 0;
+  const int k_step = shared_row ? kCombineWarps : 1;
+  for (int c0 = 0; c0 < n; c0 += 32) {
+    float wl = 0.f;
+    if (c0 + lane < n) {
+      const float li = lse_i[(size_t)(c0 + lane) * P.R];
+      wl = (lse == -INFINITY || li == -INFINITY) ? 0.f : expf(li - lse);
     }
-    for (; i < n; ++i) {
-      const float4 v = src[i * stride];
-      const float w = s_w[i];
-      acc.x += w * v.x;
-      acc.y += w * v.y;
-      acc.z += w * v.z;
-      acc.w += w * v.w;
+    const int cn = min(32, n - c0);
+    for (int k = k_first; k < cn; k += k_step) {
+      const float w = __shfl_sync(0xffffffffu, wl, k);
+      const float4* src = src0 + (size_t)(c0 + k) * stride;
+#pragma unroll
+      for (int j = 0; j < kCombineGroups; ++j) {
+        const int g = lane + 32 * j;
+        if (g < ngroups) {
+          const float4 v = src[g];
+          acc[j].x += w * v.x;
+          acc[j].y += w * v.y;
+          acc[j].z += w * v.z;
+          acc[j].w += w * v.w;
+        }
+      }
+    }
+  }
+
+  if (shared_row) {  // add the warps' partial sums; warp 0 finishes the row
+    if (warp > 0) {
+#pragma unroll
+      for (int j = 0; j < kCombineGroups; ++j)
+        if (lane + 32 * j < ngroups) s_acc[warp - 1][lane + 32 * j] = acc[j];
+    }
+    __syncthreads();
+    if (warp > 0) return;
+#pragma unroll
+    for (int j = 0; j < kCombineGroups; ++j) {
+      const int g = lane + 32 * j;
+      if (g < ngroups)
+        for (int w = 0; w < kCombineWarps - 1; ++w) {
+          const float4 v = s_acc[w][g];
+          acc[j].x += v.x;
+          acc[j].y += v.y;
+          acc[j].z += v.z;
+          acc[j].w += v.w;
+        }
     }
   }
 
   const size_t row = (size_t)b * P.R + r;
   if (!kFusedOut) {
-    if (g < ngroups) {
-      __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
-      __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
-      uint2 pk;
-      pk.x = *reinterpret_cast<uint32_t*>(&lo);
-      pk.y = *reinterpret_cast<uint32_t*>(&hi);
-      *reinterpret_cast<uint2*>(P.out + row * P.d_v + 4 * g) = pk;
+#pragma unroll
+    for (int j = 0; j < kCombineGroups; ++j) {
+      const int g = lane + 32 * j;
+      if (g < ngroups) {
+        uint2 pk;
+        pk.x = ptx::pack_bf16x2(acc[j].x, acc[j].y);
+        pk.y = ptx::pack_bf16x2(acc[j].z, acc[j].w);
+        *reinterpret_cast<uint2*>(P.out + row * P.d_v + 4 * g) = pk;
+      }
     }
-    if (tid == 0) P.lse[row] = lse;
+    if (lane == 0) P.lse[row] = lse;
     return;
   }
 
   // ---- fused epilogue: conjugate RoPE on dims 512..575, absmax, E4M3 cast
-  if (g < ngroups && 4 * g >= kNope) {
-    const int L = P.seqlens[b];
-    const double pos =
-        P.positions ? static_cast<double>(P.positions[b]) : static_cast<double>(L - 1);
-    const int k0 = (4 * g - kNope) / 2;  // pair index of (x, y); (z, w) is k0 + 1
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      float sn, c;
-      rope_sincos(pos, P.inv_freq[k0 + e], &sn, &c);
-      float& a = e ? acc.z : acc.x;
-      float& bb = e ? acc.w : acc.y;
-      const float na = a * c + bb * sn;  // rotate by -theta
-      const float nb = -a * sn + bb * c;
-      a = na;
-      bb = nb;
-    }
-  }
+  const int L = P.seqlens[b];
+  const double pos = P.positions ? static_cast<double>(P.positions[b]) : static_cast<double>(L - 1);
   float amax = 0.f;
-  if (g < ngroups)
-    amax = fmaxf(fmaxf(fabsf(acc.x), fabsf(acc.y)), fmaxf(fabsf(acc.z), fabsf(acc.w)));
+#pragma unroll
+  for (int j = 0; j < kCombineGroups; ++j) {
+    const int g = lane + 32 * j;
+    if (g < ngroups && 4 * g >= kNope) {
+      const int k0 = (4 * g - kNope) / 2;  // pair index of (x, y); (z, w) is k0 + 1
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        float sn, c;
+        rope_sincos(pos, P.inv_freq[k0 + e], &sn, &c);
+        float& a = e ? acc[j].z : acc[j].x;
+        float& bb = e ? acc[j].w : acc[j].y;
+        const float na = a * c + bb * sn;  // rotate by -theta
+        const float nb = -a * sn + bb * c;
+        a = na;
+        bb = nb;
+      }
+    }
+    if (g < ngroups)
+      amax = fmaxf(amax, fmaxf(fmaxf(fabsf(acc[j].x), fabsf(acc[j].y)),
+                               fmaxf(fabsf(acc[j].z), fabsf(acc[j].w))));
+  }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  __syncthreads();
-  if (lane == 0) s_red[warp] = amax;
-  __syncthreads();
-  amax = s_red[0];
-#pragma unroll
-  for (int w = 1; w < kWarps; ++w) amax = fmaxf(amax, s_red[w]);
   const float scale = amax > 0.f ? amax / 448.0f : 1.0f;
-  if (g < ngroups) {
-    const uint32_t codes =
-        cvt_e4m3x4(acc.x / scale, acc.y / scale, acc.z / scale, acc.w / scale);
-    *reinterpret_cast<uint32_t*>(P.out_fp8 + row * kD + 4 * g) = codes;
+#pragma unroll
+  for (int j = 0; j < kCombineGroups; ++j) {
+    const int g = lane + 32 * j;
+    if (g < ngroups)
+      *reinterpret_cast<uint32_t*>(P.out_fp8 + row * kD + 4 * g) =
+          cvt_e4m3x4(acc[j].x / scale, acc[j].y / scale, acc[j].z / scale, acc[j].w / scale);
   }
-  if (tid == 0) {
+  if (lane == 0) {
     P.out_scale[row] = scale;
     P.lse[row] = lse;
   }

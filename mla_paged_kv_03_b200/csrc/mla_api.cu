@@ -184,11 +184,19 @@ struct PdlLaunch {
 int launch_combine(const mla::CombineParams& cp, bool fused, cudaStream_t st) {
   const long long rows = static_cast<long long>(cp.batch) * cp.R;
   if (rows == 0) return MLA_OK;
-  PdlLaunch L(dim3(static_cast<unsigned>(rows)), dim3(mla::kCombineThreads), 0, st);
+  // few rows (fewer warps than a few per SM): a CTA per row, warps share its splits
+  mla::CombineParams c = cp;
+  int num_sms = 148;
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
+  c.row_per_cta = rows < 8LL * num_sms ? 1 : 0;
+  const long long ctas = c.row_per_cta ? rows : (rows + mla::kCombineWarps - 1) / mla::kCombineWarps;
+  PdlLaunch L(dim3(static_cast<unsigned>(ctas)), dim3(mla::kCombineThreads), 0, st);
   if (fused)
-    MLA_CUDA(cudaLaunchKernelEx(&L.cfg, mla::mla_combine_kernel<true>, cp));
+    MLA_CUDA(cudaLaunchKernelEx(&L.cfg, mla::mla_combine_kernel<true>, c));
   else
-    MLA_CUDA(cudaLaunchKernelEx(&L.cfg, mla::mla_combine_kernel<false>, cp));
+    MLA_CUDA(cudaLaunchKernelEx(&L.cfg, mla::mla_combine_kernel<false>, c));
   return MLA_OK;
 }
 

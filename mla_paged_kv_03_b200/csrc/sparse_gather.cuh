@@ -108,20 +108,42 @@ __global__ void __launch_bounds__(kGatherCtaThreads)
           make_uint4(0, 0, 0, 0);
   }
 
-  // dequantise: 64 tokens x 72 output units of 8 bf16
-  for (int item = tid; item < kGatherTokens * kRowUnits; item += kGatherCtaThreads) {
-    const int t = item / kRowUnits, u = item % kRowUnits;
+  // dequantise: per token 32 units of 16 codes (two 16-byte bf16 outputs
+  // each) and 8 units of 8 bf16 RoPE dims; all loads of a thread are issued
+  // before any conversion so that they overlap
+  constexpr int kUnits = kNope / 16 + kRope / 8;  // 40
+  constexpr int kPer = kGatherTokens * kUnits / kGatherCtaThreads;  // 10
+  static_assert(kGatherTokens * kUnits % kGatherCtaThreads == 0, "even split");
+  uint4 raw[kPer];
+  float sc[kPer];
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) {
+    const int item = tid + k * kGatherCtaThreads;
+    const int t = item / kUnits, u = item % kUnits;
+    raw[k] = make_uint4(0, 0, 0, 0);
+    sc[k] = 0.f;
+    if (s_dst[t] >= 0) {
+      const uint8_t* row = G.cache656 + (size_t)s_idx[t] * kRow656;
+      if (u < kNope / 16) {
+        raw[k] = __ldg(reinterpret_cast<const uint4*>(row) + u);
+        sc[k] = __ldg(reinterpret_cast<const float*>(row + kNope) + (u >> 3));
+      } else {
+        raw[k] = __ldg(reinterpret_cast<const uint4*>(row + kNope + 16) + (u - kNope / 16));
+      }
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) {
+    const int item = tid + k * kGatherCtaThreads;
+    const int t = item / kUnits, u = item % kUnits;
     const int dst = s_dst[t];
     if (dst < 0) continue;
-    const uint8_t* row = G.cache656 + (size_t)s_idx[t] * kRow656;
-    uint4 o;
-    if (u < kNope / 8) {
-      const float sc = __ldg(reinterpret_cast<const float*>(row + kNope) + (u >> 4));
-      const uint2 w = __ldg(reinterpret_cast<const uint2*>(row + 8 * u));
-      const uint32_t words[2] = {w.x, w.y};
-      uint32_t r[4];
+    __nv_bfloat16* orow = out_b + (size_t)dst * kD;
+    if (u < kNope / 16) {
+      const uint32_t words[4] = {raw[k].x, raw[k].y, raw[k].z, raw[k].w};
+      uint32_t r[8];
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
+      for (int q = 0; q < 4; ++q) {
         uint32_t h0, h1;
         const uint16_t lo16 = static_cast<uint16_t>(words[q] & 0xFFFF);
         const uint16_t hi16 = static_cast<uint16_t>(words[q] >> 16);
@@ -129,14 +151,14 @@ __global__ void __launch_bounds__(kGatherCtaThreads)
         asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h1) : "h"(hi16));
         const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&h0));
         const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&h1));
-        r[2 * q] = ptx::pack_bf16x2(f0.x * sc, f0.y * sc);
-        r[2 * q + 1] = ptx::pack_bf16x2(f1.x * sc, f1.y * sc);
+        r[2 * q] = ptx::pack_bf16x2(f0.x * sc[k], f0.y * sc[k]);
+        r[2 * q + 1] = ptx::pack_bf16x2(f1.x * sc[k], f1.y * sc[k]);
       }
-      o = make_uint4(r[0], r[1], r[2], r[3]);
+      *reinterpret_cast<uint4*>(orow + 16 * u) = make_uint4(r[0], r[1], r[2], r[3]);
+      *reinterpret_cast<uint4*>(orow + 16 * u + 8) = make_uint4(r[4], r[5], r[6], r[7]);
     } else {
-      o = __ldg(reinterpret_cast<const uint4*>(row + kNope + 16) + (u - kNope / 8));
+      *reinterpret_cast<uint4*>(orow + kNope + 8 * (u - kNope / 16)) = raw[k];
     }
-    *reinterpret_cast<uint4*>(out_b + (size_t)dst * kD + 8 * u) = o;
   }
 }
 
