@@ -14,6 +14,7 @@
 #include "../../include/mla.h"
 #include "combine_kernel.cuh"
 #include "decode_kernel.cuh"
+#include "page_kernel.cuh"
 #include "pair_kernel.cuh"
 #include "sparse_gather.cuh"
 #include "mla_common.h"
@@ -85,16 +86,17 @@ int make_latent_map(CUtensorMap* map, const void* base, long long rows) {
 }
 
 // 3-D bf16 view of the same rows: {64 dims, rows, 9 chunks of 64 dims}
-// (strides 1152 B and 128 B) with a {64, 64, box_chunks} box, 128-byte
-// swizzle; one copy lands [box_chunks][64 rows][64 dims] in shared memory.
-int make_latent_map3(CUtensorMap* map, const void* base, long long rows, int box_chunks) {
+// (strides 1152 B and 128 B) with a {64, box_rows, box_chunks} box, 128-byte
+// swizzle; one copy lands [box_chunks][box_rows][64 dims] in shared memory.
+int make_latent_map3(CUtensorMap* map, const void* base, long long rows, int box_chunks,
+                     int box_rows = 64) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(mla::kChunkD), static_cast<cuuint64_t>(rows),
                         static_cast<cuuint64_t>(mla::kNumChunks)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(mla::kD) * 2,
                            static_cast<cuuint64_t>(mla::kChunkD) * 2};
-  cuuint32_t box[3] = {64, 64, static_cast<cuuint32_t>(box_chunks)};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), static_cast<cuuint32_t>(box_chunks)};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -224,6 +226,32 @@ int launch_decode(const CUtensorMap& tq, const CUtensorMap& tkv, const mla::Deco
   if ((rc = record_start(st)) != MLA_OK) return rc;
   PdlLaunch L(dim3(grid), dim3(mla::Threads<kMode>::value), mla::cfg::kSmemBytes, st);
   MLA_CUDA(cudaLaunchKernelEx(&L.cfg, mla::mla_decode_kernel<kMode>, tq, tkv, p));
+  return record_stop(st);
+}
+
+// Page-resident kernel for up to 32 query rows per KV head (d_v 512).
+int launch_page_decode(const void* q, const void* kcache, const mla::DecodeParams& p,
+                       cudaStream_t st) {
+  CUtensorMap tq3, tpage;
+  int rc = make_latent_map3(&tq3, q, static_cast<long long>(p.batch) * p.R, mla::kNumChunks,
+                            mla::gcfg::kRows);
+  if (rc != MLA_OK) return rc;
+  if ((rc = make_latent_map3(&tpage, kcache, static_cast<long long>(p.num_blocks) * mla::kPage,
+                             mla::kNumChunks)) != MLA_OK)
+    return rc;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(mla::mla_page_decode_kernel,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    mla::gcfg::kSmemBytes);
+  });
+  if (attr_err != cudaSuccess)
+    return fail(MLA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(attr_err));
+  PdlLaunch L(dim3(static_cast<unsigned>(p.num_parts)), dim3(mla::gcfg::kThreads),
+              mla::gcfg::kSmemBytes, st);
+  if ((rc = record_start(st)) != MLA_OK) return rc;
+  MLA_CUDA(cudaLaunchKernelEx(&L.cfg, mla::mla_page_decode_kernel, tq3, tpage, p));
   return record_stop(st);
 }
 
@@ -486,7 +514,10 @@ int mla_decode_fwd(const void* q, const void* kcache, const int32_t* block_table
   p.lse = lse;
   p.ws_o = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.o_off);
   p.ws_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.lse_off);
-  if (R > mla::kRowsPerCta && d_v == 512) {
+  if (R <= mla::gcfg::kRows && d_v == 512) {
+    p.n_groups = 1;
+    if ((rc = launch_page_decode(q, kcache, p, st)) != MLA_OK) return rc;
+  } else if (R > mla::kRowsPerCta && d_v == 512) {
     p.n_groups = mla::ceil_div(R, 2 * mla::kRowsPerCta);
     if ((rc = launch_pair_decode(q, kcache, tkv, p, st)) != MLA_OK) return rc;
   } else if ((rc = launch_decode<mla::kDense>(tq, tkv, p, st)) != MLA_OK) {
