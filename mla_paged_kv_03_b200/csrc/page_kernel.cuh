@@ -13,8 +13,9 @@
 // alternate: while page k is multiplied, page k + 1 is loaded.
 //
 // TMEM: an M = 64 accumulator puts token t in lane 32 (t / 16) + t % 16, so
-// the softmax threads of lanes 0..15 of each warp own the 64 tokens of a page;
-// the M = 128 O^T accumulators put output dim d in lane d.
+// lanes 0..15 of the softmax warps receive the 64 tokens of a page (and share
+// each token's 32 columns with lanes 16..31); the M = 128 O^T accumulators
+// put output dim d in lane d.
 //
 // Roles (warps): 0 loader (Q, pages), 1 MMA issuer + TMEM owner,
 // 2..5 softmax / epilogue.
@@ -263,9 +264,13 @@ __global__ void __launch_bounds__(gcfg::kThreads, 1)
     __syncwarp();
   } else {
     // ============================== softmax / epilogue ==============================
+    // Lanes 0..15 of each warp receive the S^T rows of 16 tokens; lane l and
+    // lane l + 16 then share token 16 wq + l, lane l taking the query columns
+    // 0..15 and lane l + 16 the columns 16..31 (handed over by shuffles).
     const int wq = warp & 3;                   // TMEM lane quarter
     const int wt = threadIdx.x - 64;           // 0..127
-    const bool active = lane < 16;             // holds a token of the page
+    const int half = lane >> 4;                // column half of this lane
+    const int cb = 16 * half;                  // its first column
     const int t = 16 * wq + (lane & 15);       // token within the page
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     uint32_t gt = 0;
@@ -289,9 +294,9 @@ __global__ void __launch_bounds__(gcfg::kThreads, 1)
       int min_lim = 1 << 30;
       for (int c = 0; c < 32; ++c)
         if (c < P.R && C.lim[c] < min_lim) min_lim = C.lim[c];
-      float lsum[32];
+      float lsum[16];
 #pragma unroll
-      for (int c = 0; c < 32; ++c) lsum[c] = 0.f;
+      for (int i = 0; i < 16; ++i) lsum[i] = 0.f;
 
       for (int k = 0; k < np && ok; ++k) {
         const uint32_t g = gt + k;
@@ -301,22 +306,30 @@ __global__ void __launch_bounds__(gcfg::kThreads, 1)
           break;
         }
         ptx::tc_fence_after();
-        float x[32];
-        ptx::tmem_ld32(lane_addr + kSCol + 32 * sb, x);
-        ptx::tmem_ld_wait_regs(x);
+        float x[16];
+        {
+          float raw[32];
+          ptx::tmem_ld32(lane_addr + kSCol + 32 * sb, raw);
+          ptx::tmem_ld_wait_regs(raw);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float hi = __shfl_sync(0xffffffffu, raw[16 + i], lane & 15);
+            x[i] = half ? hi : raw[i];
+          }
+        }
         ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&C.s_empty[sb]);
 
         const int T = (p0 + k) * kPage + t;
-        const bool need_mask = !active || (p0 + k + 1) * kPage > min_lim;
+        const bool need_mask = (p0 + k + 1) * kPage > min_lim;
         int need = 0;
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          float v = x[c] * P.scale_log2;
-          if (need_mask && (!active || T >= C.lim[c])) v = -INFINITY;
-          x[c] = v;
-          need |= (v > C.m[c] + cfg::kRescaleThreshold);
+        for (int i = 0; i < 16; ++i) {
+          float v = x[i] * P.scale_log2;
+          if (need_mask && T >= C.lim[cb + i]) v = -INFINITY;
+          x[i] = v;
+          need |= (v > C.m[cb + i] + cfg::kRescaleThreshold);
         }
         uint32_t any_need;
         asm volatile(
@@ -329,11 +342,11 @@ __global__ void __launch_bounds__(gcfg::kThreads, 1)
         if (any_need) {
           // raise the reference max to this page's exact column max
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            float v = x[c];
+          for (int i = 0; i < 16; ++i) {
+            float v = x[i];
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-            if (lane == 0) C.red[wq][c] = v;
+            for (int o = 8; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+            if ((lane & 15) == 0) C.red[wq][cb + i] = v;
           }
           ptx::named_bar_sync(1, 128);
           if (wt < 32) {
@@ -345,7 +358,7 @@ __global__ void __launch_bounds__(gcfg::kThreads, 1)
           }
           ptx::named_bar_sync(1, 128);
 #pragma unroll
-          for (int c = 0; c < 32; ++c) lsum[c] *= C.alpha[c];
+          for (int i = 0; i < 16; ++i) lsum[i] *= C.alpha[cb + i];
           if (k > 0) {
             // O holds the sum through PV(g - 1): wait for it, rescale this dim lane
             const uint32_t gp = g - 1;
@@ -372,23 +385,24 @@ __global__ void __launch_bounds__(gcfg::kThreads, 1)
           ok = false;
           break;
         }
-        if (active) {
+        {
           uint8_t* prow = sP + pb * kPBytes + t * 128;
 #pragma unroll
-          for (int uu = 0; uu < 4; ++uu) {
+          for (int uu = 0; uu < 2; ++uu) {
             uint32_t pk[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const int c = 8 * uu + 2 * e;
-              const volatile float* mv = &C.m[c];
+              const int i = 8 * uu + 2 * e;
+              const volatile float* mv = &C.m[cb + i];
               const float m0 = mv[0], m1 = mv[1];
-              const float q0 = (x[c] == -INFINITY) ? 0.f : ex2(x[c] - m0);
-              const float q1 = (x[c + 1] == -INFINITY) ? 0.f : ex2(x[c + 1] - m1);
+              const float q0 = (x[i] == -INFINITY) ? 0.f : ex2(x[i] - m0);
+              const float q1 = (x[i + 1] == -INFINITY) ? 0.f : ex2(x[i + 1] - m1);
               pk[e] = ptx::pack_bf16x2(q0, q1);
-              lsum[c] += q0;
-              lsum[c + 1] += q1;
+              lsum[i] += q0;
+              lsum[i + 1] += q1;
             }
-            *reinterpret_cast<uint4*>(prow + ((uu ^ (t & 7)) << 4)) =
+            const int unit = 2 * half + uu;  // 16-byte unit = columns 8 unit .. 8 unit + 7
+            *reinterpret_cast<uint4*>(prow + ((unit ^ (t & 7)) << 4)) =
                 make_uint4(pk[0], pk[1], pk[2], pk[3]);
           }
         }
@@ -401,11 +415,11 @@ __global__ void __launch_bounds__(gcfg::kThreads, 1)
 
       // ---- epilogue: l = column sums over the page tokens
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        float v = lsum[c];
+      for (int i = 0; i < 16; ++i) {
+        float v = lsum[i];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if (lane == 0) C.red[wq][c] = v;
+        for (int o = 8; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if ((lane & 15) == 0) C.red[wq][cb + i] = v;
       }
       ptx::named_bar_sync(1, 128);
       const bool partial = P.always_partial || u.nsplit > 1;
