@@ -548,43 +548,54 @@ __global__ void __launch_bounds__(Threads<kMode>::value, 1)
           ok = false;
           break;
         }
-        // RMSNorm and RoPE in fp64; one bf16 rounding at the end.
+        // RMSNorm and RoPE in fp64; one bf16 rounding at the end.  Each warp
+        // takes every 8th row; a row's 72 16-byte units are loaded once (3 per
+        // lane) and the next row's units are in flight while this one is
+        // transformed.
         const int wl = (threadIdx.x - 64) >> 5;  // warp within both groups (0..7)
-        for (int r = wl; r < kRowsPerCta; r += 4 * kSoftmaxGroups) {
+        constexpr int kRowStep = 4 * kSoftmaxGroups;
+        auto load_row = [&](int r, uint4* w) {
           const int rg = grp * kRowsPerCta + r;
-          const bool valid = rg < P.R;
-          const __nv_bfloat16* src = P.q_raw + ((size_t)u.b * P.R + (valid ? rg : 0)) * kD;
-          double ss = 0.0;
+          const __nv_bfloat16* src = P.q_raw + ((size_t)u.b * P.R + (rg < P.R ? rg : 0)) * kD;
 #pragma unroll
           for (int j = 0; j < 3; ++j) {
             const int uu = lane + 32 * j;
-            if (uu < kD / 8) {
-              const uint4 w = *reinterpret_cast<const uint4*>(src + uu * 8);
-              const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
+            w[j] = uu < kD / 8 ? *reinterpret_cast<const uint4*>(src + uu * 8) : make_uint4(0, 0, 0, 0);
+          }
+        };
+        uint4 wcur[3], wnext[3];
+        load_row(wl, wcur);
+        for (int r = wl; r < kRowsPerCta; r += kRowStep) {
+          if (r + kRowStep < kRowsPerCta) load_row(r + kRowStep, wnext);
+          const bool valid = grp * kRowsPerCta + r < P.R;
+          double ss = 0.0;
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const float2 f = __bfloat1622float2(h[e]);
-                ss = fma(static_cast<double>(f.x), static_cast<double>(f.x), ss);
-                ss = fma(static_cast<double>(f.y), static_cast<double>(f.y), ss);
-              }
+          for (int j = 0; j < 3; ++j) {
+            const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&wcur[j]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = __bfloat1622float2(h[e]);
+              ss = fma(static_cast<double>(f.x), static_cast<double>(f.x), ss);
+              ss = fma(static_cast<double>(f.y), static_cast<double>(f.y), ss);
             }
           }
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
           const double inv = valid ? 1.0 / sqrt(ss / static_cast<double>(kD) + P.eps) : 0.0;
-#pragma unroll 1
+#pragma unroll
           for (int j = 0; j < 3; ++j) {
             const int uu = lane + 32 * j;
             if (uu < kD / 8) {
-              const uint4 w = *reinterpret_cast<const uint4*>(src + uu * 8);
-              const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
+              const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&wcur[j]);
+              const float4 g0 = __ldg(reinterpret_cast<const float4*>(P.gain + uu * 8));
+              const float4 g1 = __ldg(reinterpret_cast<const float4*>(P.gain + uu * 8 + 4));
+              const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
               double y[8];
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
                 const float2 f = __bfloat1622float2(h[e]);
-                y[2 * e] = static_cast<double>(f.x) * inv * static_cast<double>(__ldg(P.gain + uu * 8 + 2 * e));
-                y[2 * e + 1] =
-                    static_cast<double>(f.y) * inv * static_cast<double>(__ldg(P.gain + uu * 8 + 2 * e + 1));
+                y[2 * e] = static_cast<double>(f.x) * inv * static_cast<double>(gv[2 * e]);
+                y[2 * e + 1] = static_cast<double>(f.y) * inv * static_cast<double>(gv[2 * e + 1]);
               }
               if (uu >= kNope / 8) {
 #pragma unroll
@@ -606,6 +617,8 @@ __global__ void __launch_bounds__(Threads<kMode>::value, 1)
                                         ((unit ^ (r & 7)) << 4)) = o;
             }
           }
+#pragma unroll
+          for (int j = 0; j < 3; ++j) wcur[j] = wnext[j];
         }
         ptx::fence_proxy_async_smem();
         ptx::mbar_arrive(&C.q_full);
