@@ -47,12 +47,22 @@ __device__ __forceinline__ uint32_t cvt_e4m3x4(float a, float b, float c, float 
 // per lane, and broadcast with shuffles.  With few rows and many splits
 // (row_per_cta) the CTA's warps take every kCombineWarps-th split of one row
 // and add their sums in shared memory.
+__device__ __forceinline__ void fma_acc(float4& a, float w, const float4 v) {
+  a.x += w * v.x;
+  a.y += w * v.y;
+  a.z += w * v.z;
+  a.w += w * v.w;
+}
+
 constexpr int kCombineMaxSplits = 1024;  // splits of one sequence (<= SM parts)
 constexpr int kCombineWarps = 8;
 constexpr int kCombineThreads = 32 * kCombineWarps;
 constexpr int kCombineGroups = (kD / 4 + 31) / 32;  // float4 groups per lane (5)
 
-template <bool kFusedOut>
+// kPairs: splits are taken two at a time (both loads in flight before the
+// FMAs).  It needs more registers (two CTAs per SM instead of four), so the
+// host selects it only when the grid fits in one wave at that occupancy.
+template <bool kFusedOut, bool kPairs>
 __global__ void __launch_bounds__(kCombineThreads) mla_combine_kernel(const CombineParams P) {
   __shared__ float4 s_acc[kCombineWarps - 1][kD / 4];
   ptx::grid_dep_wait();  // the decode kernel's partials are complete
@@ -96,19 +106,36 @@ __global__ void __launch_bounds__(kCombineThreads) mla_combine_kernel(const Comb
       wl = (lse == -INFINITY || li == -INFINITY) ? 0.f : expf(li - lse);
     }
     const int cn = min(32, n - c0);
-    for (int k = k_first; k < cn; k += k_step) {
+    int k = k_first;
+    for (; kPairs && k + k_step < cn; k += 2 * k_step) {
+      const float w0 = __shfl_sync(0xffffffffu, wl, k);
+      const float w1 = __shfl_sync(0xffffffffu, wl, k + k_step);
+      const float4* s0 = src0 + (size_t)(c0 + k) * stride;
+      const float4* s1 = s0 + (size_t)k_step * stride;
+      float4 v0[kCombineGroups], v1[kCombineGroups];
+#pragma unroll
+      for (int j = 0; j < kCombineGroups; ++j) {
+        const int g = lane + 32 * j;
+        if (g < ngroups) {
+          v0[j] = s0[g];
+          v1[j] = s1[g];
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < kCombineGroups; ++j) {
+        if (lane + 32 * j < ngroups) {
+          fma_acc(acc[j], w0, v0[j]);
+          fma_acc(acc[j], w1, v1[j]);
+        }
+      }
+    }
+    for (; k < cn; k += k_step) {
       const float w = __shfl_sync(0xffffffffu, wl, k);
       const float4* src = src0 + (size_t)(c0 + k) * stride;
 #pragma unroll
       for (int j = 0; j < kCombineGroups; ++j) {
         const int g = lane + 32 * j;
-        if (g < ngroups) {
-          const float4 v = src[g];
-          acc[j].x += w * v.x;
-          acc[j].y += w * v.y;
-          acc[j].z += w * v.z;
-          acc[j].w += w * v.w;
-        }
+        if (g < ngroups) fma_acc(acc[j], w, src[g]);
       }
     }
   }

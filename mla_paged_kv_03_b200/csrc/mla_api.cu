@@ -194,11 +194,17 @@ int launch_combine(const mla::CombineParams& cp, bool fused, cudaStream_t st) {
     cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
   c.row_per_cta = rows < 8LL * num_sms ? 1 : 0;
   const long long ctas = c.row_per_cta ? rows : (rows + mla::kCombineWarps - 1) / mla::kCombineWarps;
+  // two splits per iteration when one wave at two CTAs per SM holds the grid
+  const bool pairs = ctas <= 2LL * num_sms;
   PdlLaunch L(dim3(static_cast<unsigned>(ctas)), dim3(mla::kCombineThreads), 0, st);
-  if (fused)
-    MLA_CUDA(cudaLaunchKernelEx(&L.cfg, mla::mla_combine_kernel<true>, c));
+  if (fused && pairs)
+    MLA_CUDA(cudaLaunchKernelEx(&L.cfg, mla::mla_combine_kernel<true, true>, c));
+  else if (fused)
+    MLA_CUDA(cudaLaunchKernelEx(&L.cfg, mla::mla_combine_kernel<true, false>, c));
+  else if (pairs)
+    MLA_CUDA(cudaLaunchKernelEx(&L.cfg, mla::mla_combine_kernel<false, true>, c));
   else
-    MLA_CUDA(cudaLaunchKernelEx(&L.cfg, mla::mla_combine_kernel<false>, c));
+    MLA_CUDA(cudaLaunchKernelEx(&L.cfg, mla::mla_combine_kernel<false, false>, c));
   return MLA_OK;
 }
 
