@@ -239,13 +239,25 @@ __global__ void __launch_bounds__(gcfg::kThreads, 1)
         return true;
       };
       const uint32_t g0 = gt, it0 = pg_it;
-      // PV(k) right after QK(k): a slot is released as soon as its page's
-      // softmax is done, so the load of page k + 2 starts early.  (Issuing
-      // QK(k + 1) first to overlap the softmax ties PV(k), and with it the
-      // slot, to page k + 1's load; measured slower with two slots.)
+      // PV(k) follows QK(k), so that a slot is released as soon as its
+      // page's softmax is done and the load of page k + 2 starts early.  QK(k
+      // + 1) goes in between only when page k + 1 has already landed: the
+      // tensor pipe then runs it during the softmax of page k, while PV(k)
+      // never waits for a load.  (Always issuing QK(k + 1) first ties PV(k),
+      // and with it the slot, to page k + 1's load; measured slower.)
+      bool qk_ahead = false;
       for (int k = 0; k < np && ok; ++k) {
         const uint32_t idx = it0 + k;
-        ok = do_qk(g0 + k, idx % kSlots, idx / kSlots);
+        if (!qk_ahead) ok = do_qk(g0 + k, idx % kSlots, idx / kSlots);
+        qk_ahead = false;
+        if (ok && k + 1 < np) {
+          const uint32_t nx = idx + 1;
+          const bool landed = ptx::mbar_test(&C.slot_full[nx % kSlots], (nx / kSlots) & 1);
+          if (__all_sync(0xffffffffu, landed)) {
+            ok = do_qk(g0 + k + 1, nx % kSlots, nx / kSlots);
+            qk_ahead = true;
+          }
+        }
         if (ok && k == 0) ok = wait_o_free();
         if (ok) ok = do_pv(g0 + k, idx % kSlots, k == 0);
       }
