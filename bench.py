@@ -202,6 +202,25 @@ class GpuStep:
     def query(self):
         return self.case.q_raw if self.kind == "fused" else self.case.q
 
+    def outputs(self):
+        return [self.out, self.lse] + ([self.scale] if self.kind == "fused" else [])
+
+    def capture(self):
+        """One step recorded as a CUDA graph (planner, attention kernel,
+        combine and, for sparse, the gather, with their programmatic launch
+        edges).  Replays run the same launches on the same buffers without
+        the host-side argument checks and launch calls of the API."""
+        side = torch.cuda.Stream(self.dev)
+        side.wait_stream(torch.cuda.current_stream(self.dev))
+        with torch.cuda.stream(side):
+            for _ in range(2):
+                self.step()
+        torch.cuda.current_stream(self.dev).wait_stream(side)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self.step()
+        return g
+
 
 class ClockSampler:
     """SM clock and throttle reasons of the bench's GPU sampled through NVML
@@ -336,11 +355,29 @@ def run_gpu_arm(args, rank, world):
     sampler = ClockSampler(dev).start()
     clk = None if sampler.h is not None else sample_clocks_start(dev.index)
     torch.cuda.synchronize(dev)
+    # the timed step: a CUDA graph replay of one API step (the direct calls
+    # with --graph 0); a replay must reproduce the direct call's outputs
+    run = gs.step
+    if args.graph:
+        gs.step()
+        torch.cuda.synchronize(dev)
+        ref = [t.clone() for t in gs.outputs()]
+        graph = gs.capture()
+        for t in gs.outputs():
+            t.zero_()
+        graph.replay()
+        torch.cuda.synchronize(dev)
+        if not all(torch.equal(a, b) for a, b in zip(ref, gs.outputs())):
+            raise RuntimeError("CUDA graph replay differs from the direct call")
+        for _ in range(3):
+            graph.replay()
+        run = graph.replay
+    torch.cuda.synchronize(dev)
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
     ev0.record(st)
     for i in range(args.steps):
-        gs.step()
+        run()
     ev1.record(st)
     torch.cuda.synchronize(dev)
     ms_total = ev0.elapsed_time(ev1)
@@ -436,7 +473,9 @@ def run_gpu_arm(args, rank, world):
         "dtype": "bf16" if args.workload != "sparse" else "bf16 (fp8 cache dequantised)",
         "data": "synthetic",
         "config": {"workload": desc, "name": args.workload,
-                   "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas x{world}"},
+                   "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas x{world}",
+                   "launch": "CUDA graph replay of one API step" if args.graph
+                   else "direct API calls"},
         "e2e": {"value": round(flops_all / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOPS",
                 "h2d_bytes_per_step": int(q_dev.numel() * q_dev.element_size()),
                 "d2h_bytes_per_step": int(gs.out.numel() * gs.out.element_size() +
@@ -570,6 +609,8 @@ def main():
     ap.add_argument("--workload", default="compute", choices=sorted(WORKLOAD_INFO))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--graph", type=int, default=1,
+                    help="time CUDA graph replays of the step (0: direct API calls)")
     ap.add_argument("--cpu-baseline", dest="cpu_baseline", type=int, default=1)
     ap.add_argument("--cpu-budget", dest="cpu_budget", type=float, default=15.0)
     args = ap.parse_args()
