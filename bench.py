@@ -329,6 +329,18 @@ def sample_clocks_stop(handle):
             "samples": len(sm)}
 
 
+def reduce_over_ranks(times, work, world, device):
+    """Whole-job figures of a replicas-only run: every per-step time is the
+    maximum over the ranks (the slowest replica ends the step) and the work is
+    the sum over the ranks.  Every rank takes the same two collectives."""
+    t = torch.tensor(times, dtype=torch.float64, device=device)
+    w = torch.tensor(work, dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        torch.distributed.all_reduce(w, op=torch.distributed.ReduceOp.SUM)
+    return [float(x) for x in t], [float(x) for x in w]
+
+
 def run_gpu_arm(args, rank, world):
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
@@ -427,13 +439,8 @@ def run_gpu_arm(args, rank, world):
         raise RuntimeError(f"device status {status:#x} after timing")
 
     ms_step = ms_total / args.steps
-    t = torch.tensor([ms_step, e2e_ms, ms_kernel], dtype=torch.float64, device=dev)
-    w = torch.tensor([flops, kv_bytes], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        torch.distributed.all_reduce(w, op=torch.distributed.ReduceOp.SUM)
-    ms_step, e2e_ms, ms_kernel = float(t[0]), float(t[1]), float(t[2])
-    flops_all, kv_all = float(w[0]), float(w[1])
+    (ms_step, e2e_ms, ms_kernel), (flops_all, kv_all) = reduce_over_ranks(
+        [ms_step, e2e_ms, ms_kernel], [flops, kv_bytes], world, dev)
     if rank != 0:
         return None
 
