@@ -16,6 +16,9 @@ Workloads (shapes and distributions as specified for this library):
 * ``sparse``    b=32, s_q=1, h_q=128, 65536-token cache per sequence, topk=2048
                 indices drawn without replacement, round(5%) of slots = -1,
                 656-byte FP8 rows.
+* ``sparse_v41`` the same shapes over the 528-byte V4.1 FP8 cache: a 512-dim
+                latent, 512 e4m3 codes + 16 e8m0 (power-of-two) scales per row,
+                q [b, s_q, h_q, 512].
 
 The cache of the fused workload is specified as "already rotated at its own
 positions".  A rotation of an isotropic Gaussian pair is again an isotropic
@@ -40,6 +43,8 @@ D_NOPE = 512
 D_ROPE = 64
 PAGE = 64
 ROW656 = 656
+ROW528 = 528  # V4.1 FP8 row: 512 e4m3 codes + 16 e8m0 scales
+D_V41 = 512   # V4.1 latent width (RoPE dims included)
 
 
 def _gen(seed: int, device) -> torch.Generator:
@@ -88,8 +93,8 @@ class FusedCase:
 
 @dataclass
 class SparseCase:
-    q: torch.Tensor            # [b, s_q, h_q, 576] bf16
-    kcache: torch.Tensor       # [num_blocks, 64, 656] uint8
+    q: torch.Tensor            # [b, s_q, h_q, 576] bf16 (512 for the V4.1 format)
+    kcache: torch.Tensor       # [num_blocks, 64, 656] uint8 (528 for the V4.1 format)
     indices: torch.Tensor      # [b, s_q, topk] int32, physical slot or -1
     h_q: int
     s_q: int
@@ -219,6 +224,26 @@ def quantize_rows656(x_nope: torch.Tensor, rope_bf16: torch.Tensor) -> torch.Ten
     return out
 
 
+def _sparse_indices(sl, bt, s_q, topk, invalid_frac, g):
+    """Per (sequence, query): min(topk, L) logical tokens drawn without
+    replacement from [0, L), mapped through the block table to physical slots
+    (block * 64 + offset); round(invalid_frac * topk) random entries -> -1."""
+    n_bad = int(round(invalid_frac * topk))
+    idx = torch.empty((len(sl), s_q, topk), dtype=torch.int32, device=g.device)
+    for b, L in enumerate(sl):
+        for i in range(s_q):
+            k = min(topk, L)
+            logical = torch.randperm(L, generator=g, device=g.device)[:k].to(torch.int64)
+            phys = bt[b].to(torch.int64)[logical // PAGE] * PAGE + logical % PAGE
+            row = torch.full((topk,), -1, dtype=torch.int64, device=g.device)
+            row[:k] = phys
+            if n_bad:
+                bad = torch.randperm(topk, generator=g, device=g.device)[:n_bad]
+                row[bad] = -1
+            idx[b, i] = row.to(torch.int32)
+    return idx
+
+
 def sparse(seed=0, device="cpu", batch=32, h_q=128, s_q=1, seqlen=65536, topk=2048,
            invalid_frac=0.05, seqlens=None):
     """Sparse FP8 case.  Each sequence owns ceil(seqlen/64) physical blocks of
@@ -239,23 +264,52 @@ def sparse(seed=0, device="cpu", batch=32, h_q=128, s_q=1, seqlen=65536, topk=20
                            dtype=torch.float32).to(torch.bfloat16)
         cache[r0:r1] = quantize_rows656(x, rope)
     q = _randn_bf16((len(sl), s_q, h_q, D_QK), g)
-    n_bad = int(round(invalid_frac * topk))
-    idx = torch.empty((len(sl), s_q, topk), dtype=torch.int32, device=g.device)
-    for b, L in enumerate(sl):
-        for i in range(s_q):
-            k = min(topk, L)
-            logical = torch.randperm(L, generator=g, device=g.device)[:k].to(torch.int64)
-            phys = bt[b].to(torch.int64)[logical // PAGE] * PAGE + logical % PAGE
-            row = torch.full((topk,), -1, dtype=torch.int64, device=g.device)
-            row[:k] = phys
-            if n_bad:
-                bad = torch.randperm(topk, generator=g, device=g.device)[:n_bad]
-                row[bad] = -1
-            idx[b, i] = row.to(torch.int32)
+    idx = _sparse_indices(sl, bt, s_q, topk, invalid_frac, g)
     return SparseCase(q=q.to(device), kcache=cache.view(nb, PAGE, ROW656).to(device),
                       indices=idx.to(device), h_q=h_q, s_q=s_q, d_v=D_NOPE,
                       softmax_scale=default_scale(), topk=topk, seqlen=max(sl),
                       block_table=bt.to(device), name="sparse")
+
+
+def quantize_rows528(x: torch.Tensor) -> torch.Tensor:
+    """Cache-writer layout of the 528-byte V4.1 row from fp32 values [n, 512]:
+    per 32-value group a power-of-two scale 2^e with e = ceil(log2(absmax/448))
+    (e = 0 for an all-zero group), stored as the E8M0 byte e + 127 after the
+    512 codes; codes = float8_e4m3fn cast of x / 2^e."""
+    n = x.shape[0]
+    grp = x.view(n, 16, 32)
+    amax = grp.abs().amax(dim=2, keepdim=True)
+    e = torch.where(amax > 0, torch.ceil(torch.log2(amax / 448.0)), torch.zeros_like(amax))
+    e = e.clamp(-127.0, 127.0)
+    codes = (grp / torch.exp2(e)).to(torch.float8_e4m3fn).view(torch.uint8).view(n, 512)
+    out = torch.empty((n, ROW528), dtype=torch.uint8, device=x.device)
+    out[:, :512] = codes
+    out[:, 512:] = (e + 127.0).to(torch.uint8).view(n, 16)
+    return out
+
+
+def sparse_v41(seed=0, device="cpu", batch=32, h_q=128, s_q=1, seqlen=65536, topk=2048,
+               invalid_frac=0.05, seqlens=None):
+    """Sparse case over the 528-byte V4.1 FP8 cache: a 512-dim latent (RoPE
+    dims included), q [b, s_q, h_q, 512] ~ N(0,1), cache values ~ N(0,1)
+    before quantisation, indices drawn as in ``sparse``; softmax scale
+    1/sqrt(512), d_v = 512."""
+    g = _gen(seed, device)
+    sl = seqlens if seqlens is not None else [seqlen] * batch
+    bt, nb = paged_block_table(sl, g, device=g.device)
+    n_rows = nb * PAGE
+    cache = torch.empty((n_rows, ROW528), dtype=torch.uint8, device=g.device)
+    step = 1 << 16
+    for r0 in range(0, n_rows, step):
+        r1 = min(n_rows, r0 + step)
+        x = torch.randn((r1 - r0, D_V41), generator=g, device=g.device, dtype=torch.float32)
+        cache[r0:r1] = quantize_rows528(x)
+    q = _randn_bf16((len(sl), s_q, h_q, D_V41), g)
+    idx = _sparse_indices(sl, bt, s_q, topk, invalid_frac, g)
+    return SparseCase(q=q.to(device), kcache=cache.view(nb, PAGE, ROW528).to(device),
+                      indices=idx.to(device), h_q=h_q, s_q=s_q, d_v=D_V41,
+                      softmax_scale=1.0 / math.sqrt(D_V41), topk=topk, seqlen=max(sl),
+                      block_table=bt.to(device), name="sparse_v41")
 
 
 WORKLOADS = {
@@ -264,4 +318,5 @@ WORKLOADS = {
     "memory": memory_bound,
     "fused": fused,
     "sparse": sparse,
+    "sparse_v41": sparse_v41,
 }

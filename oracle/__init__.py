@@ -59,6 +59,14 @@ def lib():
         L.oracle_sparse_decode.argtypes = [
             u16p, u8p, ctypes.c_int64, i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
             ctypes.c_int, ctypes.c_int, ctypes.c_double, i64p, ctypes.c_int64, f64p, f64p]
+        L.oracle_e8m0_decode.restype = ctypes.c_double
+        L.oracle_e8m0_decode.argtypes = [ctypes.c_uint8]
+        L.oracle_decode_row528.restype = None
+        L.oracle_decode_row528.argtypes = [u8p, f64p]
+        L.oracle_sparse_decode_v41.restype = ctypes.c_int
+        L.oracle_sparse_decode_v41.argtypes = [
+            u16p, u8p, ctypes.c_int64, i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, ctypes.c_double, i64p, ctypes.c_int64, f64p, f64p]
         _LIB = L
     return _LIB
 
@@ -123,6 +131,22 @@ def decode_row656(row):
     assert r.size == 656
     out = np.zeros(_D, dtype=np.float64)
     lib().oracle_decode_row656(_ptr(r, ctypes.c_uint8), _ptr(out, ctypes.c_double))
+    return out
+
+
+def e8m0_decode(codes):
+    """oracle_e8m0_decode over an array of uint8 exponent bytes -> float64."""
+    c = _np(codes, np.uint8)
+    f = lib().oracle_e8m0_decode
+    return np.array([f(int(v)) for v in c.ravel()], dtype=np.float64).reshape(c.shape)
+
+
+def decode_row528(row):
+    """oracle_decode_row528: one 528-byte V4.1 FP8 cache row -> float64[512]."""
+    r = _np(row, np.uint8).ravel()
+    assert r.size == 528
+    out = np.zeros(512, dtype=np.float64)
+    lib().oracle_decode_row528(_ptr(r, ctypes.c_uint8), _ptr(out, ctypes.c_double))
     return out
 
 
@@ -244,4 +268,29 @@ def sparse_decode(q, kcache656, indices, d_v, softmax_scale, rows=None):
         raise ValueError("sparse index out of range")
     if ra is None:
         return out.reshape(b, s_q, h_q, d_v), lse.reshape(b, s_q, h_q)
+    return out, lse
+
+
+def sparse_decode_v41(q, kcache528, indices, softmax_scale, rows=None):
+    """oracle_sparse_decode_v41.  q [b, s_q, h_q, 512] bf16; kcache528 [..., 528]
+    uint8 (flattened to slots); indices [b, s_q, topk] int32 (-1 = invalid).
+    Returns O [.., 512] (V = the whole latent) and LSE."""
+    b, s_q, h_q, dq = q.shape
+    assert dq == 512
+    qa = _np(q, np.uint16)
+    ca = _np(kcache528, np.uint8).reshape(-1, 528)
+    ix = _np(indices, np.int32)
+    topk = ix.shape[-1]
+    ra = None if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    n = b * s_q * h_q if ra is None else ra.size
+    out = np.zeros((n, 512), dtype=np.float64)
+    lse = np.zeros(n, dtype=np.float64)
+    rc = lib().oracle_sparse_decode_v41(
+        _ptr(qa, ctypes.c_uint16), _ptr(ca, ctypes.c_uint8), ca.shape[0], _ptr(ix, ctypes.c_int32),
+        b, s_q, h_q, topk, float(softmax_scale), _ptr(ra, ctypes.c_int64), n,
+        _ptr(out, ctypes.c_double), _ptr(lse, ctypes.c_double))
+    if rc != 0:
+        raise ValueError("sparse index out of range")
+    if ra is None:
+        return out.reshape(b, s_q, h_q, 512), lse.reshape(b, s_q, h_q)
     return out, lse

@@ -30,6 +30,10 @@
  *  - The 656-byte FP8 cache row: 512 E4M3 codes, 4 fp32 tile scales (one per
  *    128 values), 64 bf16 RoPE dims.
  *      [FlashMLA (AI Wiki), "The FP8 and FP4 KV cache"]
+ *  - The 528-byte V4.1 FP8 cache row: 512 E4M3 codes covering every dim of a
+ *    512-dim latent (RoPE dims included), then 16 E8M0 scales, one per 32
+ *    consecutive codes.
+ *      [FlashMLA (AI Wiki), "The FP8 and FP4 KV cache", layout table]
  *
  * Readings where the pages are silent (each is listed in the design notes):
  *  - LSE is the natural log; an empty row gives O = 0 and LSE = -inf.
@@ -41,6 +45,9 @@
  *  - Fused path: the normalised, rotated query enters the attention in bf16
  *    (the tensor-core operand precision); the pages leave this precision
  *    open, and fixing it makes the FP8 code decisions comparable.
+ *  - V4.1 rows: the latent is 512 wide, q . K runs over all 512 dims and V is
+ *    the whole latent (d_v = 512).  An E8M0 byte e is the power of two
+ *    2^(e - 127); 0xFF is NaN.
  *  - FP8 output: scale = absmax/448 (scale := 1 when absmax == 0), code =
  *    E4M3 round-to-nearest-even with saturation to +-448 of (o / scale),
  *    where the ratio is rounded to fp32 before encoding (the kernel takes
@@ -57,6 +64,8 @@
 #define ORACLE_NOPE 512
 #define ORACLE_ROPE 64
 #define ORACLE_ROW656 656
+#define ORACLE_D41 512
+#define ORACLE_ROW528 528
 
 /* ---------------------------------------------------------------- formats */
 
@@ -182,13 +191,13 @@ void oracle_rope64(const double* x, double pos, double base, int sign, double* y
  * j-th attended token into out[576]. */
 typedef void (*row_fetch_fn)(const void* ctx, int j, double* out);
 
-/* Exact attention of one query row q[576] over n tokens:
+/* Exact attention of one query row q[d_qk] over n tokens:
  *   s_t = scale * q . K_t ;  LSE = m + ln sum exp(s_t - m) ;
  *   O   = sum_t exp(s_t - LSE) * K_t[0:d_v]
  * Two passes over the rows (scores, then the weighted sum); n == 0 gives
  * O = 0, LSE = -inf. */
-static void attend_rows(const double* q, row_fetch_fn fetch, const void* ctx, int n, int d_v,
-                        double scale, double* o, double* lse) {
+static void attend_rows_d(const double* q, int d_qk, row_fetch_fn fetch, const void* ctx, int n,
+                          int d_v, double scale, double* o, double* lse) {
   int t, d;
   double m = -INFINITY, sum = 0.0, l;
   double k[ORACLE_D];
@@ -202,7 +211,7 @@ static void attend_rows(const double* q, row_fetch_fn fetch, const void* ctx, in
   for (t = 0; t < n; ++t) {
     double acc = 0.0;
     fetch(ctx, t, k);
-    for (d = 0; d < ORACLE_D; ++d) acc += q[d] * k[d];
+    for (d = 0; d < d_qk; ++d) acc += q[d] * k[d];
     s[t] = scale * acc;
     if (s[t] > m) m = s[t];
   }
@@ -215,6 +224,11 @@ static void attend_rows(const double* q, row_fetch_fn fetch, const void* ctx, in
   }
   *lse = l;
   free(s);
+}
+
+static void attend_rows(const double* q, row_fetch_fn fetch, const void* ctx, int n, int d_v,
+                        double scale, double* o, double* lse) {
+  attend_rows_d(q, ORACLE_D, fetch, ctx, n, d_v, scale, o, lse);
 }
 
 /* Paged bf16 cache source: token j of the window is logical token lo + j of
@@ -440,6 +454,68 @@ int oracle_sparse_decode(const uint16_t* q, const uint8_t* cache, int64_t num_sl
     ctx.cache = cache;
     ctx.slots = slots;
     attend_rows(qv, fetch_fp8, &ctx, cnt, d_v, scale, out + (size_t)r * d_v, lse + r);
+    free(slots);
+  }
+  return bad ? -1 : 0;
+}
+
+/* ------------------------------------------------- V4.1 FP8 cache (528 B) */
+
+/* E8M0: an 8-bit biased exponent with no sign and no mantissa. */
+double oracle_e8m0_decode(uint8_t e) {
+  if (e == 0xFF) return NAN;
+  return ldexp(1.0, (int)e - 127);
+}
+
+/* Decode one 528-byte row: [512 e4m3 codes][16 e8m0 scales, one per 32]. */
+void oracle_decode_row528(const uint8_t* row, double* out) {
+  int d;
+  for (d = 0; d < ORACLE_D41; ++d)
+    out[d] = oracle_e4m3_decode(row[d]) * oracle_e8m0_decode(row[ORACLE_D41 + d / 32]);
+}
+
+static void fetch_row528(const void* vctx, int j, double* out) {
+  const fp8_ctx* c = (const fp8_ctx*)vctx;
+  oracle_decode_row528(c->cache + (size_t)c->slots[j] * ORACLE_ROW528, out);
+}
+
+/* Token-level sparse decode over the 528-byte V4.1 cache.
+ *  q        [b, s_q, h_q, 512] bf16 bits
+ *  cache    [num_slots, 528] bytes (slot = block*64 + offset)
+ *  indices  [b, s_q, topk] int32 physical slots, -1 = invalid (skipped)
+ *  out      [rows, 512]: V is the whole 512-dim latent.  No causal mask. */
+int oracle_sparse_decode_v41(const uint16_t* q, const uint8_t* cache, int64_t num_slots,
+                             const int32_t* indices, int batch, int s_q, int h_q, int topk,
+                             double scale, const int64_t* rows, int64_t n_rows, double* out,
+                             double* lse) {
+  int64_t total = (int64_t)batch * s_q * h_q;
+  int64_t n = rows ? n_rows : total;
+  int64_t r;
+  int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+  for (r = 0; r < n; ++r) {
+    int64_t flat = rows ? rows[r] : r;
+    int64_t bi = flat / h_q; /* (b, i) */
+    const int32_t* idx = indices + (size_t)bi * topk;
+    const uint16_t* qr = q + (size_t)flat * ORACLE_D41;
+    double qv[ORACLE_D41];
+    int32_t* slots = (int32_t*)malloc(sizeof(int32_t) * (size_t)(topk > 0 ? topk : 1));
+    fp8_ctx ctx;
+    int j, d, cnt = 0;
+    for (d = 0; d < ORACLE_D41; ++d) qv[d] = bf16_bits_to_f64(qr[d]);
+    for (j = 0; j < topk; ++j) {
+      int32_t s = idx[j];
+      if (s < 0) continue;
+      if ((int64_t)s >= num_slots) {
+        bad = 1;
+        continue;
+      }
+      slots[cnt++] = s;
+    }
+    ctx.cache = cache;
+    ctx.slots = slots;
+    attend_rows_d(qv, ORACLE_D41, fetch_row528, &ctx, cnt, ORACLE_D41, scale,
+                  out + (size_t)r * ORACLE_D41, lse + r);
     free(slots);
   }
   return bad ? -1 : 0;
