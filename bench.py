@@ -6,7 +6,7 @@ A step is one pass of the whole decode path over one batch of synthetic input:
 the split-KV planner, the decode kernel (page fetch, QK, online softmax, PV,
 finalize) and the split-combine kernel (for the fused workload also the
 RMSNorm/RoPE prologue and the conjugate-RoPE/FP8 epilogue; for the sparse
-workload the FP8 gather/dequant).  Inputs are resident in HBM before the timed
+workloads the FP8 gather/dequant).  Inputs are resident in HBM before the timed
 region; every workload's KV cache is larger than the 126 MB L2, so no L2 flush
 is inserted between steps.
 
@@ -42,6 +42,9 @@ WORKLOAD_INFO = {
               "L ~ U[2048, 32768], block 64", "hbm"),
     "fused_b1": ("Fused RMSNorm-RoPE-attn-conjRoPE-FP8 decode: batch 1, s_q 1, h_q 64, d 576, "
                  "d_v 576, L ~ U[2048, 32768], block 64", "hbm"),
+    "sparse_v41": ("Token-level sparse decode, V4.1 FP8 528-byte cache (512 e4m3 + 16 e8m0): "
+                   "batch 32, s_q 1, h_q 128, d_qk = d_v 512, 65536-token cache per sequence, "
+                   "topk 2048, 5% -1 slots", "tensor"),
     "sparse": ("Token-level sparse decode, FP8 656-byte cache: batch 32, s_q 1, h_q 128, d_v 512, "
                "65536-token cache per sequence, topk 2048, 5% -1 slots", "tensor"),
     "tiny": ("Tiny dense decode, bf16: batch 2, s_q 1, h_q 16, lengths {37, 200}", "tensor"),
@@ -114,10 +117,16 @@ def fused_work(case):
     return flops, kv_bytes, kv_bytes + io
 
 
+def sparse_dims(case):
+    """(latent width of q . k, bytes per cache row) of a sparse case."""
+    return (576, 656) if case.kcache.shape[-1] == 656 else (512, 528)
+
+
 def sparse_work(case):
     valid = int((case.indices >= 0).sum())  # (b, s_q) pairs x valid slots
-    flops = 2 * valid * (576 + case.d_v) * case.h_q
-    kv_bytes = valid * 656
+    d_qk, row_bytes = sparse_dims(case)
+    flops = 2 * valid * (d_qk + case.d_v) * case.h_q
+    kv_bytes = valid * row_bytes
     io = case.q.numel() * 2 + case.indices.numel() * 4 + \
         case.batch * case.s_q * case.h_q * (case.d_v * 2 + 4)
     return flops, kv_bytes, kv_bytes + io
@@ -144,8 +153,8 @@ class GpuStep:
             self.kind = "fused"
             self.work = fused_work(self.case)
             self.R = self.case.h_q
-        elif name == "sparse":
-            self.case = W.sparse(seed=seed, device=dev)
+        elif name in ("sparse", "sparse_v41"):
+            self.case = W.WORKLOADS[name](seed=seed, device=dev)
             self.kind = "sparse"
             self.work = sparse_work(self.case)
             self.R = self.case.h_q
@@ -168,9 +177,10 @@ class GpuStep:
         else:
             self.out = torch.empty((b, c.s_q, c.h_q, c.d_v), dtype=torch.bfloat16, device=dev)
             self.lse = torch.empty((b, c.s_q, c.h_q), dtype=torch.float32, device=dev)
-            self.ws = torch.empty((B.mla_sparse_workspace_size(b, c.s_q, c.h_q, c.topk, c.d_v,
-                                                               self.parts),),
-                                  dtype=torch.uint8, device=dev)
+            nbytes = (B.mla_sparse_workspace_size(b, c.s_q, c.h_q, c.topk, c.d_v, self.parts)
+                      if name == "sparse" else
+                      B.mla_sparse_v41_workspace_size(b, c.s_q, c.h_q, c.topk, self.parts))
+            self.ws = torch.empty((nbytes,), dtype=torch.uint8, device=dev)
         if self.kind != "sparse":
             self.meta = torch.empty((self.parts, 8), dtype=torch.int32, device=dev)
             self.ns = torch.empty((b + 1,), dtype=torch.int32, device=dev)
@@ -477,7 +487,7 @@ def run_gpu_arm(args, rank, world):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16" if args.workload != "sparse" else "bf16 (fp8 cache dequantised)",
+        "dtype": "bf16" if not args.workload.startswith("sparse") else "bf16 (fp8 cache dequantised)",
         "data": "synthetic",
         "config": {"workload": desc, "name": args.workload,
                    "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas x{world}",
@@ -517,8 +527,12 @@ def oracle_rows_timed(name, case, rows):
         return time.perf_counter() - t0
     c = case
     t0 = time.perf_counter()
-    oracle.sparse_decode(c.q.cpu(), c.kcache_cpu, c.indices.cpu(), c.d_v, c.softmax_scale,
-                         rows=rows)
+    if name == "sparse_v41":
+        oracle.sparse_decode_v41(c.q.cpu(), c.kcache_cpu, c.indices.cpu(), c.softmax_scale,
+                                 rows=rows)
+    else:
+        oracle.sparse_decode(c.q.cpu(), c.kcache_cpu, c.indices.cpu(), c.d_v, c.softmax_scale,
+                             rows=rows)
     return time.perf_counter() - t0
 
 
@@ -539,9 +553,17 @@ def row_flops(name, case, rows):
             f += 2 * sl[r // case.h_q] * 1152
     else:
         valid = (case.indices.cpu() >= 0).sum(-1).reshape(-1).tolist()
+        d_qk = sparse_dims(case)[0]
         for r in rows:
-            f += 2 * valid[r // case.h_q] * (576 + case.d_v)
+            f += 2 * valid[r // case.h_q] * (d_qk + case.d_v)
     return f
+
+
+def make_case(name, seed, device="cpu"):
+    """The named workload's seeded inputs."""
+    if name.startswith("fused"):
+        return W.fused(seed=seed, device=device, batch=32 if name == "fused" else 1)
+    return W.WORKLOADS[name](seed=seed, device=device)
 
 
 def cpu_baseline(name, seed=0, budget_s=15.0, case=None):
@@ -549,9 +571,7 @@ def cpu_baseline(name, seed=0, budget_s=15.0, case=None):
     import numpy as np
     import oracle
     if case is None:
-        case = (W.WORKLOADS[name](seed=seed) if name in ("compute", "memory", "tiny")
-                else W.fused(seed=seed, batch=32 if name == "fused" else 1) if name.startswith("fused")
-                else W.sparse(seed=seed))
+        case = make_case(name, seed)
     case.kcache_cpu = case.kcache.cpu()
     total_rows = case.batch * (case.s_q if hasattr(case, "s_q") else 1) * case.h_q
     rng = np.random.default_rng(seed)
@@ -573,9 +593,7 @@ def run_reference_arm(args, rank, world):
         return None
     desc, _ = WORKLOAD_INFO[args.workload]
     name = args.workload
-    case = (W.WORKLOADS[name](seed=args.seed) if name in ("compute", "memory", "tiny")
-            else W.fused(seed=args.seed, batch=32 if name == "fused" else 1)
-            if name.startswith("fused") else W.sparse(seed=args.seed))
+    case = make_case(name, args.seed)
     per_step = max(1.0, args.cpu_budget / max(1, args.steps + args.warmup))
     import numpy as np
     import oracle

@@ -176,6 +176,34 @@ MLA_API int mla_sparse_decode(const void* q, const uint8_t* kcache_fp8, int64_t 
                       float softmax_scale, int num_sm_parts, void* workspace,
                       size_t workspace_bytes, void* out, float* lse, void* stream);
 
+/* Workspace bytes for mla_sparse_decode_v41: those of mla_sparse_decode with
+ * d_v = 512, plus the query widened to 576 dims. */
+MLA_API int mla_sparse_v41_workspace_size(int batch, int s_q, int h_q, int topk, int num_sm_parts,
+                                  size_t* bytes);
+
+/* Token-level sparse decode over the 528-byte V4.1 FP8 latent cache
+ * [FlashMLA (AI Wiki), "The FP8 and FP4 KV cache", layout table].
+ *   q             [batch, s_q, h_q, 512] bf16: the latent is 512 wide, RoPE
+ *                 dims included
+ *   kcache_528    [num_slots, 528] bytes per row: 512 E4M3 codes covering all
+ *                 512 dims, then 16 E8M0 scales (one per 32 consecutive
+ *                 codes); a value is code * 2^(e - 127), e = 0xFF is NaN
+ *   num_slots     rows of kcache_528 (num_blocks * 64)
+ *   indices       int32[batch, s_q, topk]: physical slots; -1 (or any value
+ *                 outside [0, num_slots)) marks an unused entry
+ *   out, lse      [batch, s_q, h_q, 512] bf16 (V = the whole latent) and
+ *                 [batch, s_q, h_q] fp32
+ *   softmax_scale usually 1/sqrt(512)
+ *   num_sm_parts  from mla_num_sm_parts(device, h_q, 1)
+ * The dequantised rows (and the query) are widened to the 576-dim layout of
+ * the dense kernels with zero dims 512..575, which leaves q . k and the
+ * output unchanged.  Ownership, alignment (q, the cache and out 16-byte
+ * aligned, workspace 256-byte aligned) and errors as in mla_sparse_decode. */
+MLA_API int mla_sparse_decode_v41(const void* q, const uint8_t* kcache_528, int64_t num_slots,
+                          const int32_t* indices, int topk, int batch, int s_q, int h_q,
+                          float softmax_scale, int num_sm_parts, void* workspace,
+                          size_t workspace_bytes, void* out, float* lse, void* stream);
+
 /* Dense decode without a caller workspace.  This entry point has no
  * counterpart in the method's published interface; it exists for callers
  * that cannot supply scratch memory at decode time (an embedder whose device

@@ -29,7 +29,7 @@ EXPORTED = [
     "mla_get_metadata", "mla_get_metadata_host", "mla_workspace_size", "mla_decode_fwd",
     "mla_fused_norm_rope_attn_rope_cast", "mla_sparse_workspace_size", "mla_sparse_decode",
     "mla_device_status", "mla_noalloc_scratch_bytes", "mla_decode_fwd_noalloc",
-    "mla_set_kernel_events",
+    "mla_set_kernel_events", "mla_sparse_v41_workspace_size", "mla_sparse_decode_v41",
 ]
 
 
@@ -70,6 +70,9 @@ def lib():
         L.mla_sparse_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32, szp]
         L.mla_sparse_decode.argtypes = [vp, vp, i64, vp, i32, i32, i32, i32, i32, f32, i32, vp,
                                         sz, vp, vp, vp]
+        L.mla_sparse_v41_workspace_size.argtypes = [i32, i32, i32, i32, i32, szp]
+        L.mla_sparse_decode_v41.argtypes = [vp, vp, i64, vp, i32, i32, i32, i32, f32, i32, vp,
+                                            sz, vp, vp, vp]
         L.mla_device_status.argtypes = [ip, i32]
         L.mla_noalloc_scratch_bytes.argtypes = []
         L.mla_set_kernel_events.argtypes = [vp, vp]
@@ -150,6 +153,13 @@ def mla_sparse_workspace_size(batch, s_q, h_q, topk, d_v, num_sm_parts) -> int:
     _check(lib().mla_sparse_workspace_size(int(batch), int(s_q), int(h_q), int(topk), int(d_v),
                                            int(num_sm_parts), ctypes.byref(out)))
     return out.value
+
+
+def mla_sparse_v41_workspace_size(batch, s_q, h_q, topk, num_sm_parts) -> int:
+    out = ctypes.c_size_t(0)
+    _check(lib().mla_sparse_v41_workspace_size(int(batch), int(s_q), int(h_q), int(topk),
+                                               int(num_sm_parts), ctypes.byref(out)))
+    return int(out.value)
 
 
 def _workspace(nbytes, device, workspace):
@@ -265,20 +275,26 @@ def mla_fused_norm_rope_attn_rope_cast(q_raw, norm_gain, eps, rope_base, kcache,
 
 def mla_sparse_decode(q, kcache_fp8, indices, d_v=512, softmax_scale=None, num_sm_parts=None,
                       out=None, lse=None, workspace=None):
-    """Token-level sparse decode over the 656-byte FP8 cache.
-    q [b, s_q, h_q, 576] bf16; kcache_fp8 [..., 656] uint8; indices
-    [b, s_q, topk] int32 physical slots (-1 = unused).  Returns (out, lse)."""
-    _require(q.dim() == 4 and q.shape[-1] == D_QK and q.dtype == torch.bfloat16,
-             "q must be [b, s_q, h_q, 576] bf16")
-    _require(kcache_fp8.dtype == torch.uint8 and kcache_fp8.shape[-1] == 656,
-             "kcache_fp8 must be uint8 [..., 656]")
+    """Token-level sparse decode over an FP8 latent cache whose format is told
+    by its bytes per token, as the method's interface does:
+      656 bytes  q [b, s_q, h_q, 576] bf16 (mla_sparse_decode)
+      528 bytes  V4.1, q [b, s_q, h_q, 512] bf16, d_v = 512 (mla_sparse_decode_v41)
+    indices [b, s_q, topk] int32 physical slots (-1 = unused).  Returns
+    (out [b, s_q, h_q, d_v] bf16, lse [b, s_q, h_q] fp32)."""
+    _require(kcache_fp8.dtype == torch.uint8 and kcache_fp8.shape[-1] in (656, 528),
+             "kcache_fp8 must be uint8 [..., 656] or [..., 528]")
+    row = int(kcache_fp8.shape[-1])
+    width = D_QK if row == 656 else 512
+    _require(q.dim() == 4 and q.shape[-1] == width and q.dtype == torch.bfloat16,
+             f"q must be [b, s_q, h_q, {width}] bf16 for {row}-byte cache rows")
+    _require(row == 656 or d_v == 512, "the 528-byte format has d_v = 512")
     b, s_q, h_q, _ = q.shape
     q = q.contiguous()
     idx = indices.to(torch.int32).contiguous()
     topk = idx.shape[-1]
-    num_slots = kcache_fp8.numel() // 656
+    num_slots = kcache_fp8.numel() // row
     if softmax_scale is None:
-        softmax_scale = 1.0 / math.sqrt(D_QK)
+        softmax_scale = 1.0 / math.sqrt(width)
     if num_sm_parts is None:
         num_sm_parts = mla_num_sm_parts(h_q, 1, q.device)
     dev = q.device
@@ -286,12 +302,20 @@ def mla_sparse_decode(q, kcache_fp8, indices, d_v=512, softmax_scale=None, num_s
         out = torch.empty((b, s_q, h_q, d_v), dtype=torch.bfloat16, device=dev)
     if lse is None:
         lse = torch.empty((b, s_q, h_q), dtype=torch.float32, device=dev)
-    ws = _workspace(mla_sparse_workspace_size(b, s_q, h_q, topk, d_v, num_sm_parts), dev,
-                    workspace)
-    _check(lib().mla_sparse_decode(
-        _ptr(q), _ptr(kcache_fp8), num_slots, _ptr(idx), topk, b, s_q, h_q, int(d_v),
-        float(softmax_scale), int(num_sm_parts), _ptr(ws), ws.numel(), _ptr(out), _ptr(lse),
-        _stream(dev)))
+    if row == 656:
+        ws = _workspace(mla_sparse_workspace_size(b, s_q, h_q, topk, d_v, num_sm_parts), dev,
+                        workspace)
+        _check(lib().mla_sparse_decode(
+            _ptr(q), _ptr(kcache_fp8), num_slots, _ptr(idx), topk, b, s_q, h_q, int(d_v),
+            float(softmax_scale), int(num_sm_parts), _ptr(ws), ws.numel(), _ptr(out), _ptr(lse),
+            _stream(dev)))
+    else:
+        ws = _workspace(mla_sparse_v41_workspace_size(b, s_q, h_q, topk, num_sm_parts), dev,
+                        workspace)
+        _check(lib().mla_sparse_decode_v41(
+            _ptr(q), _ptr(kcache_fp8), num_slots, _ptr(idx), topk, b, s_q, h_q,
+            float(softmax_scale), int(num_sm_parts), _ptr(ws), ws.numel(), _ptr(out), _ptr(lse),
+            _stream(dev)))
     return out, lse
 
 

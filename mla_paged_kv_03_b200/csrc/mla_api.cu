@@ -139,11 +139,14 @@ WsLayout dense_ws_layout(int batch, int R, int d_v, int parts) {
 // pages_per_pair pages per (sequence, query) pair), its block table and
 // lengths, the split tables, then the dense decode workspace.
 struct SparseWs {
-  size_t rows_off, bt_off, len_off, meta_off, splits_off, dense_off, dense_bytes, total;
+  size_t rows_off, bt_off, len_off, meta_off, splits_off, dense_off, dense_bytes, q_off, total;
   int pages_per_pair;
 };
 
-SparseWs sparse_ws_layout(int pairs, int topk, int R, int d_v, int parts) {
+// Workspace of the sparse paths: the compacted bf16 rows, their identity
+// block table and lengths, the planner's output, the dense path's own
+// workspace and, for the 528-byte rows, the query widened to 576 dims.
+SparseWs sparse_ws_layout(int pairs, int topk, int R, int d_v, int parts, bool v41 = false) {
   SparseWs w{};
   w.pages_per_pair = mla::ceil_div(topk, mla::kPage);
   const size_t pages = static_cast<size_t>(pairs) * w.pages_per_pair;
@@ -154,7 +157,9 @@ SparseWs sparse_ws_layout(int pairs, int topk, int R, int d_v, int parts) {
   w.splits_off = w.meta_off + align_up(static_cast<size_t>(parts) * mla::kMetaInts * 4, 256);
   w.dense_off = w.splits_off + align_up((static_cast<size_t>(pairs) + 1) * 4, 256);
   w.dense_bytes = dense_ws_layout(pairs, R, d_v, parts).total;
-  w.total = w.dense_off + w.dense_bytes;
+  w.q_off = w.dense_off + align_up(w.dense_bytes, 256);
+  w.total = v41 ? w.q_off + align_up(static_cast<size_t>(pairs) * R * mla::kD * 2, 256)
+                : w.dense_off + w.dense_bytes;
   return w;
 }
 
@@ -352,6 +357,70 @@ int static_scratch_ptr(void** ptr) {
 }
 
 }  // namespace
+
+// Both sparse paths: gather + dequantise + compact the valid rows of every
+// (sequence, query) pair, then the dense planner and decode over them.
+static int sparse_decode_impl(int row_bytes, const void* q, const uint8_t* kcache, int64_t num_slots,
+                       const int32_t* indices, int topk, int batch, int s_q, int h_q, int d_v,
+                       float softmax_scale, int num_sm_parts, void* workspace,
+                       size_t workspace_bytes, void* out, float* lse, void* stream) {
+  const bool v41 = row_bytes == mla::kRow528;
+  MLA_CHECK_ARG(batch >= 0 && s_q >= 1 && h_q >= 1, "bad sizes");
+  MLA_CHECK_ARG(topk >= 1, "topk must be >= 1 (got %d)", topk);
+  MLA_CHECK_ARG(num_slots >= 1 && num_slots < (1LL << 31), "num_slots must be in [1, 2^31)");
+  MLA_CHECK_ARG(d_v == 512, "sparse decode supports d_v = 512 (got %d)", d_v);
+  MLA_CHECK_ARG(num_sm_parts >= 1 && num_sm_parts <= mla::kCombineMaxSplits,
+                "num_sm_parts must be in [1, %d]", mla::kCombineMaxSplits);
+  MLA_CHECK_ARG(std::isfinite(softmax_scale) && softmax_scale > 0.f,
+                "softmax_scale must be finite and > 0");
+  MLA_CHECK_ARG(q && kcache && indices && workspace && out && lse, "null device pointer");
+  MLA_CHECK_ARG(aligned(q, 16) && aligned(kcache, 16), "q and the cache must be 16-byte aligned");
+  MLA_CHECK_ARG(aligned(workspace, 256), "workspace must be 256-byte aligned");
+  MLA_CHECK_ARG(aligned(out, 8) && aligned(lse, 4) && aligned(indices, 4), "misaligned output");
+  const int pairs = batch * s_q;
+  MLA_CHECK_ARG(aligned(out, 16), "out must be 16-byte aligned");
+  const SparseWs w = sparse_ws_layout(pairs, topk, h_q, d_v, num_sm_parts, v41);
+  MLA_CHECK_ARG(workspace_bytes >= w.total, "workspace too small: %zu < %zu", workspace_bytes,
+                w.total);
+  MLA_CHECK_ARG(pairs <= mla::kPlanMaxBatch, "at most %d (batch, query) pairs (got %d)",
+                mla::kPlanMaxBatch, pairs);
+  const long long pages = static_cast<long long>(pairs) * w.pages_per_pair;
+  MLA_CHECK_ARG(pages * mla::kPage < (1LL << 31), "pairs * topk too large");
+  if (batch == 0) return MLA_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+
+  // 1. gather + dequantise + compact the valid tokens of every pair
+  mla::GatherParams g{};
+  g.cache = kcache;
+  g.num_slots = num_slots;
+  g.indices = indices;
+  g.topk = topk;
+  g.pages_per_pair = w.pages_per_pair;
+  g.rows = reinterpret_cast<__nv_bfloat16*>(ws + w.rows_off);
+  g.block_table = reinterpret_cast<int32_t*>(ws + w.bt_off);
+  g.seqlens = reinterpret_cast<int32_t*>(ws + w.len_off);
+  g.h_q = h_q;
+  const dim3 grid(w.pages_per_pair, pairs);
+  if (v41) {
+    g.q512 = static_cast<const __nv_bfloat16*>(q);
+    g.q576 = reinterpret_cast<__nv_bfloat16*>(ws + w.q_off);
+    mla::mla_sparse_gather_kernel<mla::kRow528><<<grid, mla::kGatherCtaThreads, 0, st>>>(g);
+  } else {
+    mla::mla_sparse_gather_kernel<mla::kRow656><<<grid, mla::kGatherCtaThreads, 0, st>>>(g);
+  }
+  MLA_CUDA(cudaGetLastError());
+
+  // 2. dense decode over the compacted rows: no causal mask, lengths = valid counts
+  int32_t* meta = reinterpret_cast<int32_t*>(ws + w.meta_off);
+  int32_t* splits = reinterpret_cast<int32_t*>(ws + w.splits_off);
+  int rc = mla_get_metadata(g.seqlens, pairs, h_q, 1, num_sm_parts, meta, splits, stream);
+  if (rc != MLA_OK) return rc;
+  const void* q_dense = v41 ? static_cast<const void*>(g.q576) : q;
+  return mla_decode_fwd(q_dense, g.rows, g.block_table, w.pages_per_pair, static_cast<int>(pages),
+                        g.seqlens, pairs, 1, h_q, 1, d_v, softmax_scale, 0, meta, splits,
+                        num_sm_parts, ws + w.dense_off, w.dense_bytes, out, lse, stream);
+}
 
 extern "C" {
 
@@ -628,56 +697,31 @@ int mla_sparse_workspace_size(int batch, int s_q, int h_q, int topk, int d_v, in
   return MLA_OK;
 }
 
+int mla_sparse_v41_workspace_size(int batch, int s_q, int h_q, int topk, int num_sm_parts,
+                                  size_t* bytes) {
+  MLA_CHECK_ARG(bytes, "bytes is null");
+  MLA_CHECK_ARG(batch >= 0 && s_q >= 1 && h_q >= 1 && topk >= 1 && num_sm_parts >= 1,
+                "bad sizes");
+  *bytes = sparse_ws_layout(batch * s_q, topk, h_q, 512, num_sm_parts, true).total;
+  return MLA_OK;
+}
+
 int mla_sparse_decode(const void* q, const uint8_t* kcache_fp8, int64_t num_slots,
                       const int32_t* indices, int topk, int batch, int s_q, int h_q, int d_v,
                       float softmax_scale, int num_sm_parts, void* workspace,
                       size_t workspace_bytes, void* out, float* lse, void* stream) {
-  MLA_CHECK_ARG(batch >= 0 && s_q >= 1 && h_q >= 1, "bad sizes");
-  MLA_CHECK_ARG(topk >= 1, "topk must be >= 1 (got %d)", topk);
-  MLA_CHECK_ARG(num_slots >= 1 && num_slots < (1LL << 31), "num_slots must be in [1, 2^31)");
-  MLA_CHECK_ARG(d_v == 512, "sparse decode supports d_v = 512 (got %d)", d_v);
-  MLA_CHECK_ARG(num_sm_parts >= 1 && num_sm_parts <= mla::kCombineMaxSplits,
-                "num_sm_parts must be in [1, %d]", mla::kCombineMaxSplits);
-  MLA_CHECK_ARG(std::isfinite(softmax_scale) && softmax_scale > 0.f,
-                "softmax_scale must be finite and > 0");
-  MLA_CHECK_ARG(q && kcache_fp8 && indices && workspace && out && lse, "null device pointer");
-  MLA_CHECK_ARG(aligned(q, 16) && aligned(kcache_fp8, 16), "q and kcache_fp8 must be 16-byte aligned");
-  MLA_CHECK_ARG(aligned(workspace, 256), "workspace must be 256-byte aligned");
-  MLA_CHECK_ARG(aligned(out, 8) && aligned(lse, 4) && aligned(indices, 4), "misaligned output");
-  const int pairs = batch * s_q;
-  MLA_CHECK_ARG(aligned(out, 16), "out must be 16-byte aligned");
-  const SparseWs w = sparse_ws_layout(pairs, topk, h_q, d_v, num_sm_parts);
-  MLA_CHECK_ARG(workspace_bytes >= w.total, "workspace too small: %zu < %zu", workspace_bytes,
-                w.total);
-  MLA_CHECK_ARG(pairs <= mla::kPlanMaxBatch, "at most %d (batch, query) pairs (got %d)",
-                mla::kPlanMaxBatch, pairs);
-  const long long pages = static_cast<long long>(pairs) * w.pages_per_pair;
-  MLA_CHECK_ARG(pages * mla::kPage < (1LL << 31), "pairs * topk too large");
-  if (batch == 0) return MLA_OK;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  return sparse_decode_impl(mla::kRow656, q, kcache_fp8, num_slots, indices, topk, batch, s_q, h_q,
+                            d_v, softmax_scale, num_sm_parts, workspace, workspace_bytes, out, lse,
+                            stream);
+}
 
-  // 1. gather + dequantise + compact the valid tokens of every pair
-  mla::GatherParams g{};
-  g.cache656 = kcache_fp8;
-  g.num_slots = num_slots;
-  g.indices = indices;
-  g.topk = topk;
-  g.pages_per_pair = w.pages_per_pair;
-  g.rows = reinterpret_cast<__nv_bfloat16*>(ws + w.rows_off);
-  g.block_table = reinterpret_cast<int32_t*>(ws + w.bt_off);
-  g.seqlens = reinterpret_cast<int32_t*>(ws + w.len_off);
-  mla::mla_sparse_gather_kernel<<<dim3(w.pages_per_pair, pairs), mla::kGatherCtaThreads, 0, st>>>(g);
-  MLA_CUDA(cudaGetLastError());
-
-  // 2. dense decode over the compacted rows: no causal mask, lengths = valid counts
-  int32_t* meta = reinterpret_cast<int32_t*>(ws + w.meta_off);
-  int32_t* splits = reinterpret_cast<int32_t*>(ws + w.splits_off);
-  int rc = mla_get_metadata(g.seqlens, pairs, h_q, 1, num_sm_parts, meta, splits, stream);
-  if (rc != MLA_OK) return rc;
-  return mla_decode_fwd(q, g.rows, g.block_table, w.pages_per_pair, static_cast<int>(pages),
-                        g.seqlens, pairs, 1, h_q, 1, d_v, softmax_scale, 0, meta, splits,
-                        num_sm_parts, ws + w.dense_off, w.dense_bytes, out, lse, stream);
+int mla_sparse_decode_v41(const void* q, const uint8_t* kcache_528, int64_t num_slots,
+                          const int32_t* indices, int topk, int batch, int s_q, int h_q,
+                          float softmax_scale, int num_sm_parts, void* workspace,
+                          size_t workspace_bytes, void* out, float* lse, void* stream) {
+  return sparse_decode_impl(mla::kRow528, q, kcache_528, num_slots, indices, topk, batch, s_q, h_q,
+                            512, softmax_scale, num_sm_parts, workspace, workspace_bytes, out, lse,
+                            stream);
 }
 
 

@@ -1,11 +1,16 @@
 // sparse_gather.cuh -- first step of token-level sparse decode: gather the
-// selected rows of the 656-byte FP8 latent cache, dequantise them to bf16 and
-// compact each query's valid tokens into a dense paged buffer that the dense
-// decode kernels then attend over.
+// selected rows of an FP8 latent cache, dequantise them to bf16 and compact
+// each query's valid tokens into a dense paged buffer that the dense decode
+// kernels then attend over.
 //
-// Cache row (per token): [512 x E4M3 codes][4 x fp32 scale, one per 128
-// codes][64 x bf16 RoPE dims]; a nope value is code * scale.
-// [FlashMLA (AI Wiki), "The FP8 and FP4 KV cache"]
+// Cache rows (per token), [FlashMLA (AI Wiki), "The FP8 and FP4 KV cache"]:
+//  - 656 bytes: [512 x E4M3 codes][4 x fp32 scale, one per 128 codes]
+//    [64 x bf16 RoPE dims]; a nope value is code * scale.
+//  - 528 bytes (V4.1): [512 x E4M3 codes over the whole 512-dim latent]
+//    [16 x E8M0 scale, one per 32 codes]; a value is code * 2^(e - 127).
+//    The buffer row stays 576 wide with dims 512..575 zero, and the 512-wide
+//    query rows are copied into a 576-wide buffer with zero dims 512..575, so
+//    that q . k and the first 512 dims of V are unchanged.
 // Indices (per (sequence, query) pair): physical slots, -1 (or any value
 // outside [0, num_slots)) marks an unused entry; the block table of the cache
 // is not used.  [FlashMLA (AI Wiki), "Interfaces"]
@@ -31,7 +36,7 @@ constexpr int kGatherCtaThreads = 256;
 constexpr int kRowUnits = kD / 8;  // 16-byte bf16 output units per row (72)
 
 struct GatherParams {
-  const uint8_t* cache656;  // [num_slots, 656]
+  const uint8_t* cache;     // [num_slots, 656] or [num_slots, 528]
   long long num_slots;
   const int32_t* indices;   // [pairs, topk]
   int topk;
@@ -39,15 +44,29 @@ struct GatherParams {
   __nv_bfloat16* rows;      // [pairs * pages_per_pair * 64, 576]
   int32_t* block_table;     // [pairs, pages_per_pair]
   int32_t* seqlens;         // [pairs]
+  // 528-byte format only: query rows [pairs * h_q, 512] -> [pairs * h_q, 576]
+  const __nv_bfloat16* q512;
+  __nv_bfloat16* q576;
+  int h_q;
 };
+
+// E8M0 byte -> fp32: 2^(e - 127) (e = 0 is the fp32 subnormal 2^-127),
+// 0xFF -> NaN.
+__device__ __forceinline__ float e8m0_to_float(uint32_t e) {
+  if (e == 0xFFu) return __int_as_float(0x7FC00000);
+  return e == 0u ? __int_as_float(0x00400000) : __int_as_float(static_cast<int>(e << 23));
+}
 
 __device__ __forceinline__ bool gather_valid(int idx, long long num_slots) {
   return idx >= 0 && static_cast<long long>(idx) < num_slots;
 }
 
 // grid (pages_per_pair, pairs): CTA (c, b) handles indices [64c, 64c + 64) of pair b.
+template <int kRowBytes>
 __global__ void __launch_bounds__(kGatherCtaThreads)
     mla_sparse_gather_kernel(const GatherParams G) {
+  static_assert(kRowBytes == kRow656 || kRowBytes == kRow528, "656- or 528-byte rows");
+  constexpr bool kV41 = kRowBytes == kRow528;
   __shared__ int s_red[kGatherCtaThreads / 32];
   __shared__ int s_idx[kGatherTokens];
   __shared__ int s_dst[kGatherTokens];  // destination row within the pair, or -1
@@ -108,9 +127,22 @@ __global__ void __launch_bounds__(kGatherCtaThreads)
           make_uint4(0, 0, 0, 0);
   }
 
+  if (kV41 && c == 0) {
+    // the pair's query rows, widened to 576 dims (72 16-byte units a row)
+    for (int item = tid; item < G.h_q * kRowUnits; item += kGatherCtaThreads) {
+      const size_t r = (size_t)b * G.h_q + item / kRowUnits;
+      const int uu = item % kRowUnits;
+      const uint4 v = uu < kNope / 8
+                          ? __ldg(reinterpret_cast<const uint4*>(G.q512 + r * kNope) + uu)
+                          : make_uint4(0, 0, 0, 0);
+      *reinterpret_cast<uint4*>(G.q576 + r * kD + 8 * uu) = v;
+    }
+  }
+
   // dequantise: per token 32 units of 16 codes (two 16-byte bf16 outputs
-  // each) and 8 units of 8 bf16 RoPE dims; all loads of a thread are issued
-  // before any conversion so that they overlap
+  // each) and 8 units of the dims 512..575 (bf16 RoPE dims, or zeros for the
+  // 528-byte rows); all loads of a thread are issued before any conversion so
+  // that they overlap
   constexpr int kUnits = kNope / 16 + kRope / 8;  // 40
   constexpr int kPer = kGatherTokens * kUnits / kGatherCtaThreads;  // 10
   static_assert(kGatherTokens * kUnits % kGatherCtaThreads == 0, "even split");
@@ -123,11 +155,14 @@ __global__ void __launch_bounds__(kGatherCtaThreads)
     raw[k] = make_uint4(0, 0, 0, 0);
     sc[k] = 0.f;
     if (s_dst[t] >= 0) {
-      const uint8_t* row = G.cache656 + (size_t)s_idx[t] * kRow656;
+      const uint8_t* row = G.cache + (size_t)s_idx[t] * kRowBytes;
       if (u < kNope / 16) {
         raw[k] = __ldg(reinterpret_cast<const uint4*>(row) + u);
-        sc[k] = __ldg(reinterpret_cast<const float*>(row + kNope) + (u >> 3));
-      } else {
+        if (kV41)
+          sc[k] = e8m0_to_float(__ldg(row + kNope + (u >> 1)));
+        else
+          sc[k] = __ldg(reinterpret_cast<const float*>(row + kNope) + (u >> 3));
+      } else if (!kV41) {
         raw[k] = __ldg(reinterpret_cast<const uint4*>(row + kNope + 16) + (u - kNope / 16));
       }
     }
