@@ -51,16 +51,29 @@ WORKLOAD_INFO = {
 }
 
 
-def kernel_source_hash():
-    """Hash of the CUDA sources; a stored ncu traffic figure is used only while
-    the kernels are unchanged since it was captured."""
+# Sources each workload's dominant (attention) kernel is built from, with the
+# launch code: its stored ncu traffic stays valid while these are unchanged.
+_KERNEL_SOURCES = {
+    "mla_pair_decode_kernel": ["pair_kernel.cuh", "decode_kernel.cuh"],
+    "mla_page_decode_kernel": ["page_kernel.cuh", "decode_kernel.cuh"],
+    "mla_decode_kernel": ["decode_kernel.cuh"],
+}
+_COMMON_SOURCES = ["ptx.cuh", "mla_common.h", "mla_api.cu"]
+
+
+def kernel_source_hash(kernel="mla_decode_kernel"):
+    """Hash of the CUDA sources of one kernel (its headers, the shared PTX and
+    constant headers, and the launch code); a stored ncu traffic figure is
+    used only while they are unchanged since it was captured."""
     import hashlib
     d = os.path.join(ROOT, "mla_paged_kv_03_b200", "csrc")
+    key = next((k for k in _KERNEL_SOURCES if kernel.startswith(k)), None)
+    names = sorted(_KERNEL_SOURCES[key] + _COMMON_SOURCES) if key else \
+        sorted(n for n in os.listdir(d) if n.endswith((".cu", ".cuh", ".h")))
     h = hashlib.sha256()
-    for name in sorted(os.listdir(d)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(d, name), "rb") as f:
-                h.update(name.encode() + b"\0" + f.read())
+    for name in names:
+        with open(os.path.join(d, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()[:16]
 
 
@@ -72,7 +85,7 @@ def load_traffic(workload):
         with open(p) as f:
             d = json.load(f)
         e = d.get(workload)
-        if e and e.get("source_hash") == kernel_source_hash():
+        if e and e.get("source_hash") == kernel_source_hash(e.get("kernel", "")):
             return e["bytes_per_launch"]
     except Exception:
         pass

@@ -127,9 +127,43 @@ __global__ void __launch_bounds__(kGatherCtaThreads)
           make_uint4(0, 0, 0, 0);
   }
 
-  if (kV41 && c == 0) {
-    // the pair's query rows, widened to 576 dims (72 16-byte units a row)
-    for (int item = tid; item < G.h_q * kRowUnits; item += kGatherCtaThreads) {
+  // dequantise: per token 32 units of 16 codes (two 16-byte bf16 outputs
+  // each) and 8 units of the dims 512..575 (bf16 RoPE dims, or zeros for the
+  // 528-byte rows); all loads of a thread are issued before any conversion so
+  // that they overlap
+  constexpr int kUnits = kNope / 16 + kRope / 8;  // 40
+  constexpr int kPer = kGatherTokens * kUnits / kGatherCtaThreads;  // 10
+  static_assert(kGatherTokens * kUnits % kGatherCtaThreads == 0, "even split");
+  uint4 raw[kPer];
+  float sc[kPer];      // 656-byte rows: the fp32 scale
+  uint32_t eb[kPer];   // 528-byte rows: the E8M0 byte, converted after all loads
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) {
+    const int item = tid + k * kGatherCtaThreads;
+    const int t = item / kUnits, u = item % kUnits;
+    raw[k] = make_uint4(0, 0, 0, 0);
+    sc[k] = 0.f;
+    eb[k] = 127u;
+    if (s_dst[t] >= 0) {
+      const uint8_t* row = G.cache + (size_t)s_idx[t] * kRowBytes;
+      if (u < kNope / 16) {
+        raw[k] = __ldg(reinterpret_cast<const uint4*>(row) + u);
+        if (kV41)
+          eb[k] = __ldg(row + kNope + (u >> 1));
+        else
+          sc[k] = __ldg(reinterpret_cast<const float*>(row + kNope) + (u >> 3));
+      } else if (!kV41) {
+        raw[k] = __ldg(reinterpret_cast<const uint4*>(row + kNope + 16) + (u - kNope / 16));
+      }
+    }
+  }
+  if (kV41) {
+    // the pair's query rows widened to 576 dims (72 16-byte units a row),
+    // spread over all pages_per_pair CTAs of the pair, while the row loads
+    // above are in flight
+    const int n_items = G.h_q * kRowUnits;
+    for (int item = c * kGatherCtaThreads + tid; item < n_items;
+         item += G.pages_per_pair * kGatherCtaThreads) {
       const size_t r = (size_t)b * G.h_q + item / kRowUnits;
       const int uu = item % kRowUnits;
       const uint4 v = uu < kNope / 8
@@ -139,34 +173,6 @@ __global__ void __launch_bounds__(kGatherCtaThreads)
     }
   }
 
-  // dequantise: per token 32 units of 16 codes (two 16-byte bf16 outputs
-  // each) and 8 units of the dims 512..575 (bf16 RoPE dims, or zeros for the
-  // 528-byte rows); all loads of a thread are issued before any conversion so
-  // that they overlap
-  constexpr int kUnits = kNope / 16 + kRope / 8;  // 40
-  constexpr int kPer = kGatherTokens * kUnits / kGatherCtaThreads;  // 10
-  static_assert(kGatherTokens * kUnits % kGatherCtaThreads == 0, "even split");
-  uint4 raw[kPer];
-  float sc[kPer];
-#pragma unroll
-  for (int k = 0; k < kPer; ++k) {
-    const int item = tid + k * kGatherCtaThreads;
-    const int t = item / kUnits, u = item % kUnits;
-    raw[k] = make_uint4(0, 0, 0, 0);
-    sc[k] = 0.f;
-    if (s_dst[t] >= 0) {
-      const uint8_t* row = G.cache + (size_t)s_idx[t] * kRowBytes;
-      if (u < kNope / 16) {
-        raw[k] = __ldg(reinterpret_cast<const uint4*>(row) + u);
-        if (kV41)
-          sc[k] = e8m0_to_float(__ldg(row + kNope + (u >> 1)));
-        else
-          sc[k] = __ldg(reinterpret_cast<const float*>(row + kNope) + (u >> 3));
-      } else if (!kV41) {
-        raw[k] = __ldg(reinterpret_cast<const uint4*>(row + kNope + 16) + (u - kNope / 16));
-      }
-    }
-  }
 #pragma unroll
   for (int k = 0; k < kPer; ++k) {
     const int item = tid + k * kGatherCtaThreads;
@@ -176,6 +182,7 @@ __global__ void __launch_bounds__(kGatherCtaThreads)
     __nv_bfloat16* orow = out_b + (size_t)dst * kD;
     if (u < kNope / 16) {
       const uint32_t words[4] = {raw[k].x, raw[k].y, raw[k].z, raw[k].w};
+      const float scl = kV41 ? e8m0_to_float(eb[k]) : sc[k];
       uint32_t r[8];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
@@ -186,8 +193,8 @@ __global__ void __launch_bounds__(kGatherCtaThreads)
         asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h1) : "h"(hi16));
         const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&h0));
         const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&h1));
-        r[2 * q] = ptx::pack_bf16x2(f0.x * sc[k], f0.y * sc[k]);
-        r[2 * q + 1] = ptx::pack_bf16x2(f1.x * sc[k], f1.y * sc[k]);
+        r[2 * q] = ptx::pack_bf16x2(f0.x * scl, f0.y * scl);
+        r[2 * q + 1] = ptx::pack_bf16x2(f1.x * scl, f1.y * scl);
       }
       *reinterpret_cast<uint4*>(orow + 16 * u) = make_uint4(r[0], r[1], r[2], r[3]);
       *reinterpret_cast<uint4*>(orow + 16 * u + 8) = make_uint4(r[4], r[5], r[6], r[7]);
