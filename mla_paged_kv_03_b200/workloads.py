@@ -19,6 +19,8 @@ Workloads (shapes and distributions as specified for this library):
 * ``sparse_v41`` the same shapes over the 528-byte V4.1 FP8 cache: a 512-dim
                 latent, 512 e4m3 codes + 16 e8m0 (power-of-two) scales per row,
                 q [b, s_q, h_q, 512].
+* ``sparse_v41_fp4`` the same over 288-byte V4.1 FP4 rows: 512 e2m1 codes
+                packed two per byte + 32 e4m3 scales (one per 16 values).
 
 The cache of the fused workload is specified as "already rotated at its own
 positions".  A rotation of an isotropic Gaussian pair is again an isotropic
@@ -44,6 +46,7 @@ D_ROPE = 64
 PAGE = 64
 ROW656 = 656
 ROW528 = 528  # V4.1 FP8 row: 512 e4m3 codes + 16 e8m0 scales
+ROW288 = 288  # V4.1 FP4 row: 512 e2m1 codes (256 bytes) + 32 e4m3 scales
 D_V41 = 512   # V4.1 latent width (RoPE dims included)
 
 
@@ -288,28 +291,62 @@ def quantize_rows528(x: torch.Tensor) -> torch.Tensor:
     return out
 
 
+E2M1_MAGNITUDES = (0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0)  # codes 0..7 of the format
+
+
+def quantize_rows288(x: torch.Tensor) -> torch.Tensor:
+    """Cache-writer layout of the 288-byte V4.1 FP4 row from fp32 values
+    [n, 512]: per 16-value group an e4m3 scale = float8_e4m3fn(absmax / 6)
+    (1 for an all-zero group), codes = the E2M1 magnitude nearest |x| / scale
+    (saturating at 6) with the sign bit; code 2i in the low nibble of byte i,
+    code 2i + 1 in the high nibble; the 32 scale bytes follow the 256 code
+    bytes."""
+    n = x.shape[0]
+    grp = x.view(n, 32, 16)
+    amax = grp.abs().amax(dim=2, keepdim=True)
+    scale8 = torch.where(amax > 0, amax / 6.0, torch.ones_like(amax)).to(torch.float8_e4m3fn)
+    scale = scale8.to(torch.float32)
+    scale = torch.where(scale > 0, scale, torch.ones_like(scale))
+    scale8 = scale.to(torch.float8_e4m3fn)
+    v = (grp / scale).abs().clamp(max=6.0)
+    mags = torch.tensor(E2M1_MAGNITUDES, dtype=torch.float32, device=x.device)
+    code = (v.unsqueeze(-1) - mags).abs().argmin(dim=-1).to(torch.uint8)
+    code = code | ((grp < 0).to(torch.uint8) << 3)
+    code = code.view(n, 256, 2)
+    out = torch.empty((n, ROW288), dtype=torch.uint8, device=x.device)
+    out[:, :256] = code[..., 0] | (code[..., 1] << 4)
+    out[:, 256:] = scale8.view(torch.uint8).view(n, 32)
+    return out
+
+
 def sparse_v41(seed=0, device="cpu", batch=32, h_q=128, s_q=1, seqlen=65536, topk=2048,
-               invalid_frac=0.05, seqlens=None):
-    """Sparse case over the 528-byte V4.1 FP8 cache: a 512-dim latent (RoPE
-    dims included), q [b, s_q, h_q, 512] ~ N(0,1), cache values ~ N(0,1)
-    before quantisation, indices drawn as in ``sparse``; softmax scale
-    1/sqrt(512), d_v = 512."""
+               invalid_frac=0.05, seqlens=None, fp4=False):
+    """Sparse case over the V4.1 cache: a 512-dim latent (RoPE dims
+    included) in 528-byte FP8 rows, or 288-byte FP4 rows with ``fp4``;
+    q [b, s_q, h_q, 512] ~ N(0,1), cache values ~ N(0,1) before quantisation,
+    indices drawn as in ``sparse``; softmax scale 1/sqrt(512), d_v = 512."""
     g = _gen(seed, device)
     sl = seqlens if seqlens is not None else [seqlen] * batch
     bt, nb = paged_block_table(sl, g, device=g.device)
     n_rows = nb * PAGE
-    cache = torch.empty((n_rows, ROW528), dtype=torch.uint8, device=g.device)
+    row_bytes = ROW288 if fp4 else ROW528
+    cache = torch.empty((n_rows, row_bytes), dtype=torch.uint8, device=g.device)
     step = 1 << 16
     for r0 in range(0, n_rows, step):
         r1 = min(n_rows, r0 + step)
         x = torch.randn((r1 - r0, D_V41), generator=g, device=g.device, dtype=torch.float32)
-        cache[r0:r1] = quantize_rows528(x)
+        cache[r0:r1] = quantize_rows288(x) if fp4 else quantize_rows528(x)
     q = _randn_bf16((len(sl), s_q, h_q, D_V41), g)
     idx = _sparse_indices(sl, bt, s_q, topk, invalid_frac, g)
-    return SparseCase(q=q.to(device), kcache=cache.view(nb, PAGE, ROW528).to(device),
+    return SparseCase(q=q.to(device), kcache=cache.view(nb, PAGE, row_bytes).to(device),
                       indices=idx.to(device), h_q=h_q, s_q=s_q, d_v=D_V41,
                       softmax_scale=1.0 / math.sqrt(D_V41), topk=topk, seqlen=max(sl),
-                      block_table=bt.to(device), name="sparse_v41")
+                      block_table=bt.to(device), name="sparse_v41_fp4" if fp4 else "sparse_v41")
+
+
+def sparse_v41_fp4(seed=0, device="cpu", **kw):
+    """``sparse_v41`` over 288-byte FP4 rows."""
+    return sparse_v41(seed=seed, device=device, fp4=True, **kw)
 
 
 WORKLOADS = {
@@ -319,4 +356,5 @@ WORKLOADS = {
     "fused": fused,
     "sparse": sparse,
     "sparse_v41": sparse_v41,
+    "sparse_v41_fp4": sparse_v41_fp4,
 }

@@ -63,6 +63,15 @@ def lib():
         L.oracle_e8m0_decode.argtypes = [ctypes.c_uint8]
         L.oracle_decode_row528.restype = None
         L.oracle_decode_row528.argtypes = [u8p, f64p]
+        L.oracle_e2m1_decode.restype = ctypes.c_double
+        L.oracle_e2m1_decode.argtypes = [ctypes.c_uint8]
+        L.oracle_decode_row288.restype = None
+        L.oracle_decode_row288.argtypes = [u8p, f64p]
+        for fn in (L.oracle_sparse_decode_v41, L.oracle_sparse_decode_v41_fp4):
+            fn.restype = ctypes.c_int
+            fn.argtypes = [
+                u16p, u8p, ctypes.c_int64, i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                ctypes.c_int, ctypes.c_double, i64p, ctypes.c_int64, f64p, f64p]
         L.oracle_sparse_decode_v41.restype = ctypes.c_int
         L.oracle_sparse_decode_v41.argtypes = [
             u16p, u8p, ctypes.c_int64, i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
@@ -147,6 +156,22 @@ def decode_row528(row):
     assert r.size == 528
     out = np.zeros(512, dtype=np.float64)
     lib().oracle_decode_row528(_ptr(r, ctypes.c_uint8), _ptr(out, ctypes.c_double))
+    return out
+
+
+def e2m1_decode(codes):
+    """oracle_e2m1_decode over an array of 4-bit codes (0..15) -> float64."""
+    c = _np(codes, np.uint8)
+    f = lib().oracle_e2m1_decode
+    return np.array([f(int(v)) for v in c.ravel()], dtype=np.float64).reshape(c.shape)
+
+
+def decode_row288(row):
+    """oracle_decode_row288: one 288-byte V4.1 FP4 cache row -> float64[512]."""
+    r = _np(row, np.uint8).ravel()
+    assert r.size == 288
+    out = np.zeros(512, dtype=np.float64)
+    lib().oracle_decode_row288(_ptr(r, ctypes.c_uint8), _ptr(out, ctypes.c_double))
     return out
 
 
@@ -271,21 +296,26 @@ def sparse_decode(q, kcache656, indices, d_v, softmax_scale, rows=None):
     return out, lse
 
 
-def sparse_decode_v41(q, kcache528, indices, softmax_scale, rows=None):
-    """oracle_sparse_decode_v41.  q [b, s_q, h_q, 512] bf16; kcache528 [..., 528]
-    uint8 (flattened to slots); indices [b, s_q, topk] int32 (-1 = invalid).
+def sparse_decode_v41(q, kcache, indices, softmax_scale, rows=None):
+    """oracle_sparse_decode_v41 (528-byte FP8 rows) or
+    oracle_sparse_decode_v41_fp4 (288-byte FP4 rows), told apart by the bytes
+    per row.  q [b, s_q, h_q, 512] bf16; kcache [..., 528 | 288] uint8
+    (flattened to slots); indices [b, s_q, topk] int32 (-1 = invalid).
     Returns O [.., 512] (V = the whole latent) and LSE."""
     b, s_q, h_q, dq = q.shape
     assert dq == 512
+    row = int(kcache.shape[-1])
+    assert row in (528, 288)
+    fn = lib().oracle_sparse_decode_v41 if row == 528 else lib().oracle_sparse_decode_v41_fp4
     qa = _np(q, np.uint16)
-    ca = _np(kcache528, np.uint8).reshape(-1, 528)
+    ca = _np(kcache, np.uint8).reshape(-1, row)
     ix = _np(indices, np.int32)
     topk = ix.shape[-1]
     ra = None if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
     n = b * s_q * h_q if ra is None else ra.size
     out = np.zeros((n, 512), dtype=np.float64)
     lse = np.zeros(n, dtype=np.float64)
-    rc = lib().oracle_sparse_decode_v41(
+    rc = fn(
         _ptr(qa, ctypes.c_uint16), _ptr(ca, ctypes.c_uint8), ca.shape[0], _ptr(ix, ctypes.c_int32),
         b, s_q, h_q, topk, float(softmax_scale), _ptr(ra, ctypes.c_int64), n,
         _ptr(out, ctypes.c_double), _ptr(lse, ctypes.c_double))

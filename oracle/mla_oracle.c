@@ -33,6 +33,8 @@
  *  - The 528-byte V4.1 FP8 cache row: 512 E4M3 codes covering every dim of a
  *    512-dim latent (RoPE dims included), then 16 E8M0 scales, one per 32
  *    consecutive codes.
+ *  - The 288-byte V4.1 FP4 cache row: 512 E2M1 codes packed two per byte
+ *    into 256 bytes, then 32 E4M3 scales, one per 16 consecutive codes.
  *      [FlashMLA (AI Wiki), "The FP8 and FP4 KV cache", layout table]
  *
  * Readings where the pages are silent (each is listed in the design notes):
@@ -47,7 +49,8 @@
  *    open, and fixing it makes the FP8 code decisions comparable.
  *  - V4.1 rows: the latent is 512 wide, q . K runs over all 512 dims and V is
  *    the whole latent (d_v = 512).  An E8M0 byte e is the power of two
- *    2^(e - 127); 0xFF is NaN.
+ *    2^(e - 127); 0xFF is NaN.  In the FP4 row, code 2i sits in the low
+ *    nibble of byte i and code 2i + 1 in the high nibble.
  *  - FP8 output: scale = absmax/448 (scale := 1 when absmax == 0), code =
  *    E4M3 round-to-nearest-even with saturation to +-448 of (o / scale),
  *    where the ratio is rounded to fp32 before encoding (the kernel takes
@@ -66,6 +69,7 @@
 #define ORACLE_ROW656 656
 #define ORACLE_D41 512
 #define ORACLE_ROW528 528
+#define ORACLE_ROW288 288
 
 /* ---------------------------------------------------------------- formats */
 
@@ -479,15 +483,40 @@ static void fetch_row528(const void* vctx, int j, double* out) {
   oracle_decode_row528(c->cache + (size_t)c->slots[j] * ORACLE_ROW528, out);
 }
 
-/* Token-level sparse decode over the 528-byte V4.1 cache.
+/* E2M1 (a 4-bit code): sign, 2 exponent bits with bias 1, 1 mantissa bit;
+ * exponent 0 holds the subnormals 0 and 0.5.  No inf or NaN. */
+double oracle_e2m1_decode(uint8_t c) {
+  int sign = (c >> 3) & 1, e = (c >> 1) & 3, m = c & 1;
+  double mag = e == 0 ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+  return sign ? -mag : mag;
+}
+
+/* Decode one 288-byte row: [256 bytes of E2M1 pairs][32 e4m3 scales, one per
+ * 16 codes]. */
+void oracle_decode_row288(const uint8_t* row, double* out) {
+  int d;
+  for (d = 0; d < ORACLE_D41; ++d) {
+    uint8_t byte = row[d / 2];
+    uint8_t code = (d % 2 == 0) ? (uint8_t)(byte & 0x0F) : (uint8_t)(byte >> 4);
+    out[d] = oracle_e2m1_decode(code) * oracle_e4m3_decode(row[ORACLE_D41 / 2 + d / 16]);
+  }
+}
+
+static void fetch_row288(const void* vctx, int j, double* out) {
+  const fp8_ctx* c = (const fp8_ctx*)vctx;
+  oracle_decode_row288(c->cache + (size_t)c->slots[j] * ORACLE_ROW288, out);
+}
+
+/* Token-level sparse decode over a 512-dim V4.1 cache of `row_bytes`-byte
+ * rows decoded by `fetch`.
  *  q        [b, s_q, h_q, 512] bf16 bits
- *  cache    [num_slots, 528] bytes (slot = block*64 + offset)
+ *  cache    [num_slots, row_bytes] (slot = block*64 + offset)
  *  indices  [b, s_q, topk] int32 physical slots, -1 = invalid (skipped)
  *  out      [rows, 512]: V is the whole 512-dim latent.  No causal mask. */
-int oracle_sparse_decode_v41(const uint16_t* q, const uint8_t* cache, int64_t num_slots,
-                             const int32_t* indices, int batch, int s_q, int h_q, int topk,
-                             double scale, const int64_t* rows, int64_t n_rows, double* out,
-                             double* lse) {
+static int sparse_decode_512(row_fetch_fn fetch, const uint16_t* q, const uint8_t* cache,
+                             int64_t num_slots, const int32_t* indices, int batch, int s_q,
+                             int h_q, int topk, double scale, const int64_t* rows, int64_t n_rows,
+                             double* out, double* lse) {
   int64_t total = (int64_t)batch * s_q * h_q;
   int64_t n = rows ? n_rows : total;
   int64_t r;
@@ -514,9 +543,27 @@ int oracle_sparse_decode_v41(const uint16_t* q, const uint8_t* cache, int64_t nu
     }
     ctx.cache = cache;
     ctx.slots = slots;
-    attend_rows_d(qv, ORACLE_D41, fetch_row528, &ctx, cnt, ORACLE_D41, scale,
+    attend_rows_d(qv, ORACLE_D41, fetch, &ctx, cnt, ORACLE_D41, scale,
                   out + (size_t)r * ORACLE_D41, lse + r);
     free(slots);
   }
   return bad ? -1 : 0;
+}
+
+/* Sparse decode over the 528-byte V4.1 FP8 rows. */
+int oracle_sparse_decode_v41(const uint16_t* q, const uint8_t* cache, int64_t num_slots,
+                             const int32_t* indices, int batch, int s_q, int h_q, int topk,
+                             double scale, const int64_t* rows, int64_t n_rows, double* out,
+                             double* lse) {
+  return sparse_decode_512(fetch_row528, q, cache, num_slots, indices, batch, s_q, h_q, topk,
+                           scale, rows, n_rows, out, lse);
+}
+
+/* Sparse decode over the 288-byte V4.1 FP4 rows. */
+int oracle_sparse_decode_v41_fp4(const uint16_t* q, const uint8_t* cache, int64_t num_slots,
+                                 const int32_t* indices, int batch, int s_q, int h_q, int topk,
+                                 double scale, const int64_t* rows, int64_t n_rows, double* out,
+                                 double* lse) {
+  return sparse_decode_512(fetch_row288, q, cache, num_slots, indices, batch, s_q, h_q, topk,
+                           scale, rows, n_rows, out, lse);
 }

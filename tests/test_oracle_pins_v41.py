@@ -1,8 +1,13 @@
-"""Pins of the oracle's V4.1 FP8 cache path (528-byte rows: 512 E4M3 codes over
-the whole 512-dim latent, then 16 E8M0 scales, one per 32 codes) against
-facts that do not come from the oracle: torch's float8_e4m3fn and
-float8_e8m0fnu casts, the quantisation error bound of the format, torch SDPA
-on independently dequantised rows, and the invariances of sparse attention."""
+"""Pins of the oracle's V4.1 cache paths against facts that do not come from
+the oracle:
+  - FP8, 528-byte rows (512 E4M3 codes over the whole 512-dim latent, then 16
+    E8M0 scales, one per 32 codes): torch's float8_e4m3fn and float8_e8m0fnu
+    casts, the quantisation error bound, the one-slot case and the
+    invariances of sparse attention;
+  - FP4, 288-byte rows (512 E2M1 codes two per byte, then 32 E4M3 scales, one
+    per 16 codes): the E2M1 value table of the format, torch's float8_e4m3fn
+    cast for the scales, exactly representable values coming back exactly;
+  - both: torch SDPA on independently dequantised rows."""
 import numpy as np
 import torch
 import torch.nn.functional as F
@@ -101,3 +106,65 @@ def test_sparse_v41_permutation_and_invalid_slots():
     o5, l5 = oracle.sparse_decode_v41(case.q, case.kcache, torch.full_like(ix, -1),
                                       case.softmax_scale)
     assert (o5 == 0).all() and np.isneginf(l5).all()
+
+
+# ------------------------------------------------------- V4.1 FP4 (288 B)
+
+# The E2M1 format's values for codes 0..7 (sign bit 3 negates them).
+E2M1_TABLE = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+
+def dequant288_torch(rows):
+    """[n, 288] uint8 -> fp64 [n, 512]: nibbles unpacked low-then-high with
+    the format's value table, scales by torch's float8_e4m3fn decoder."""
+    rows = rows.reshape(-1, 288)
+    b = rows[:, :256].to(torch.int64)
+    codes = torch.stack([b & 0xF, b >> 4], dim=-1).reshape(-1, 512)
+    table = torch.tensor(E2M1_TABLE + [-v for v in E2M1_TABLE], dtype=torch.float64)
+    vals = table[codes]
+    scale = rows[:, 256:].contiguous().view(torch.float8_e4m3fn).to(torch.float64)
+    return vals * scale.repeat_interleave(16, dim=1)
+
+
+def test_e2m1_decode_matches_format_table():
+    got = oracle.e2m1_decode(np.arange(16, dtype=np.uint8))
+    want = np.array(E2M1_TABLE + [-v for v in E2M1_TABLE])
+    np.testing.assert_array_equal(np.abs(got), np.abs(want))
+    assert (np.signbit(got[8:])).all() and not np.signbit(got[:8]).any()
+
+
+def test_row288_decode_matches_torch_and_exact_values_roundtrip():
+    g = torch.Generator().manual_seed(1)
+    x = torch.randn((48, 512), generator=g)
+    rows = W.quantize_rows288(x)
+    ref = dequant288_torch(rows)
+    dec = torch.stack([torch.tensor(oracle.decode_row288(rows[r])) for r in range(48)])
+    np.testing.assert_array_equal(dec.numpy(), ref.numpy())
+    # values that are exactly code * scale (absmax = 6 * scale) come back exactly
+    scales = torch.tensor([0.25, 1.0, 0.09375, 3.5], dtype=torch.float32)  # all e4m3 values
+    idx = torch.randint(0, 16, (4, 32, 16), generator=g)
+    table = torch.tensor(E2M1_TABLE + [-v for v in E2M1_TABLE])
+    vals = table[idx]
+    vals[..., 0] = 6.0  # pin each group's absmax so that absmax / 6 is the scale
+    group_scale = scales[torch.randint(0, 4, (4, 32), generator=g)].view(4, 32, 1)
+    exact = (vals * group_scale).reshape(4, 512)
+    rows2 = W.quantize_rows288(exact)
+    dec2 = torch.stack([torch.tensor(oracle.decode_row288(rows2[r])) for r in range(4)])
+    np.testing.assert_array_equal(dec2.numpy(), exact.to(torch.float64).numpy())
+
+
+def test_sparse_v41_fp4_matches_sdpa_on_dequantised_rows():
+    case = W.sparse_v41_fp4(seed=4, batch=2, h_q=3, s_q=2, seqlens=[300, 130], topk=96,
+                            invalid_frac=0.05)
+    o, lse = oracle.sparse_decode_v41(case.q, case.kcache, case.indices, case.softmax_scale)
+    K = dequant288_torch(case.kcache)
+    for b in range(case.batch):
+        for i in range(case.s_q):
+            idx = case.indices[b, i]
+            sel = K[idx[idx >= 0].long()]
+            q = case.q[b, i].to(torch.float64)
+            ro = F.scaled_dot_product_attention(q[None], sel[None], sel[None],
+                                                scale=case.softmax_scale)[0]
+            rl = torch.logsumexp((q @ sel.T) * case.softmax_scale, dim=-1)
+            np.testing.assert_allclose(o[b, i], ro.numpy(), rtol=1e-11, atol=1e-12)
+            np.testing.assert_allclose(lse[b, i], rl.numpy(), rtol=1e-12)
