@@ -45,6 +45,9 @@ WORKLOAD_INFO = {
     "sparse_v41": ("Token-level sparse decode, V4.1 FP8 528-byte cache (512 e4m3 + 16 e8m0): "
                    "batch 32, s_q 1, h_q 128, d_qk = d_v 512, 65536-token cache per sequence, "
                    "topk 2048, 5% -1 slots", "tensor"),
+    "sparse_v41_fp4": ("Token-level sparse decode, V4.1 FP4 288-byte cache (512 e2m1 + 32 e4m3): "
+                       "batch 32, s_q 1, h_q 128, d_qk = d_v 512, 65536-token cache per sequence, "
+                       "topk 2048, 5% -1 slots", "tensor"),
     "sparse": ("Token-level sparse decode, FP8 656-byte cache: batch 32, s_q 1, h_q 128, d_v 512, "
                "65536-token cache per sequence, topk 2048, 5% -1 slots", "tensor"),
     "tiny": ("Tiny dense decode, bf16: batch 2, s_q 1, h_q 16, lengths {37, 200}", "tensor"),
@@ -132,7 +135,8 @@ def fused_work(case):
 
 def sparse_dims(case):
     """(latent width of q . k, bytes per cache row) of a sparse case."""
-    return (576, 656) if case.kcache.shape[-1] == 656 else (512, 528)
+    row = int(case.kcache.shape[-1])
+    return (576 if row == 656 else 512), row
 
 
 def sparse_work(case):
@@ -166,7 +170,7 @@ class GpuStep:
             self.kind = "fused"
             self.work = fused_work(self.case)
             self.R = self.case.h_q
-        elif name in ("sparse", "sparse_v41"):
+        elif name in ("sparse", "sparse_v41", "sparse_v41_fp4"):
             self.case = W.WORKLOADS[name](seed=seed, device=dev)
             self.kind = "sparse"
             self.work = sparse_work(self.case)
@@ -500,7 +504,8 @@ def run_gpu_arm(args, rank, world):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16" if not args.workload.startswith("sparse") else "bf16 (fp8 cache dequantised)",
+        "dtype": "bf16" if not args.workload.startswith("sparse") else
+        "bf16 (fp4 cache dequantised)" if args.workload.endswith("fp4") else "bf16 (fp8 cache dequantised)",
         "data": "synthetic",
         "config": {"workload": desc, "name": args.workload,
                    "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas x{world}",
@@ -540,7 +545,7 @@ def oracle_rows_timed(name, case, rows):
         return time.perf_counter() - t0
     c = case
     t0 = time.perf_counter()
-    if name == "sparse_v41":
+    if name.startswith("sparse_v41"):
         oracle.sparse_decode_v41(c.q.cpu(), c.kcache_cpu, c.indices.cpu(), c.softmax_scale,
                                  rows=rows)
     else:

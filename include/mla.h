@@ -24,7 +24,9 @@
  *       [FlashMLA fused norm-RoPE-attention-RoPE-cast kernel card,
  *        "Arithmetic intensity"; deepseek-ai/FlashMLA README, "News"]
  *   - the 656-byte FP8 cache row: 512 E4M3 values with one fp32 scale per 128,
- *     then the 64 RoPE dims in bf16
+ *     then the 64 RoPE dims in bf16; the V4.1 rows of a 512-dim latent: 528
+ *     bytes (512 E4M3 + 16 E8M0 scales, one per 32) or 288 bytes (512 E2M1
+ *     packed two per byte + 32 E4M3 scales, one per 16)
  *       [FlashMLA (AI Wiki), "The FP8 and FP4 KV cache"]
  *
  * Conventions shared by every entry point
@@ -176,8 +178,9 @@ MLA_API int mla_sparse_decode(const void* q, const uint8_t* kcache_fp8, int64_t 
                       float softmax_scale, int num_sm_parts, void* workspace,
                       size_t workspace_bytes, void* out, float* lse, void* stream);
 
-/* Workspace bytes for mla_sparse_decode_v41: those of mla_sparse_decode with
- * d_v = 512, plus the query widened to 576 dims. */
+/* Workspace bytes for mla_sparse_decode_v41 and mla_sparse_decode_v41_fp4:
+ * those of mla_sparse_decode with d_v = 512, plus the query widened to 576
+ * dims. */
 MLA_API int mla_sparse_v41_workspace_size(int batch, int s_q, int h_q, int topk, int num_sm_parts,
                                   size_t* bytes);
 
@@ -203,6 +206,20 @@ MLA_API int mla_sparse_decode_v41(const void* q, const uint8_t* kcache_528, int6
                           const int32_t* indices, int topk, int batch, int s_q, int h_q,
                           float softmax_scale, int num_sm_parts, void* workspace,
                           size_t workspace_bytes, void* out, float* lse, void* stream);
+
+/* Token-level sparse decode over the 288-byte V4.1 FP4 latent cache
+ * [FlashMLA (AI Wiki), "The FP8 and FP4 KV cache", layout table].
+ *   kcache_288    [num_slots, 288] bytes per row: 512 E2M1 codes packed two
+ *                 per byte into 256 bytes (code 2i in the low nibble of byte
+ *                 i, code 2i + 1 in the high nibble), then 32 E4M3 scales,
+ *                 one per 16 consecutive codes; a value is code * scale
+ * Every other argument, the layouts, the workspace
+ * (mla_sparse_v41_workspace_size), ownership and errors are those of
+ * mla_sparse_decode_v41. */
+MLA_API int mla_sparse_decode_v41_fp4(const void* q, const uint8_t* kcache_288, int64_t num_slots,
+                              const int32_t* indices, int topk, int batch, int s_q, int h_q,
+                              float softmax_scale, int num_sm_parts, void* workspace,
+                              size_t workspace_bytes, void* out, float* lse, void* stream);
 
 /* Dense decode without a caller workspace.  This entry point has no
  * counterpart in the method's published interface; it exists for callers

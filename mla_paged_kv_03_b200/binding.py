@@ -30,6 +30,7 @@ EXPORTED = [
     "mla_fused_norm_rope_attn_rope_cast", "mla_sparse_workspace_size", "mla_sparse_decode",
     "mla_device_status", "mla_noalloc_scratch_bytes", "mla_decode_fwd_noalloc",
     "mla_set_kernel_events", "mla_sparse_v41_workspace_size", "mla_sparse_decode_v41",
+    "mla_sparse_decode_v41_fp4",
 ]
 
 
@@ -73,6 +74,7 @@ def lib():
         L.mla_sparse_v41_workspace_size.argtypes = [i32, i32, i32, i32, i32, szp]
         L.mla_sparse_decode_v41.argtypes = [vp, vp, i64, vp, i32, i32, i32, i32, f32, i32, vp,
                                             sz, vp, vp, vp]
+        L.mla_sparse_decode_v41_fp4.argtypes = L.mla_sparse_decode_v41.argtypes
         L.mla_device_status.argtypes = [ip, i32]
         L.mla_noalloc_scratch_bytes.argtypes = []
         L.mla_set_kernel_events.argtypes = [vp, vp]
@@ -278,16 +280,17 @@ def mla_sparse_decode(q, kcache_fp8, indices, d_v=512, softmax_scale=None, num_s
     """Token-level sparse decode over an FP8 latent cache whose format is told
     by its bytes per token, as the method's interface does:
       656 bytes  q [b, s_q, h_q, 576] bf16 (mla_sparse_decode)
-      528 bytes  V4.1, q [b, s_q, h_q, 512] bf16, d_v = 512 (mla_sparse_decode_v41)
+      528 bytes  V4.1 FP8, q [b, s_q, h_q, 512] bf16, d_v = 512 (mla_sparse_decode_v41)
+      288 bytes  V4.1 FP4, q as for 528 (mla_sparse_decode_v41_fp4)
     indices [b, s_q, topk] int32 physical slots (-1 = unused).  Returns
     (out [b, s_q, h_q, d_v] bf16, lse [b, s_q, h_q] fp32)."""
-    _require(kcache_fp8.dtype == torch.uint8 and kcache_fp8.shape[-1] in (656, 528),
-             "kcache_fp8 must be uint8 [..., 656] or [..., 528]")
+    _require(kcache_fp8.dtype == torch.uint8 and kcache_fp8.shape[-1] in (656, 528, 288),
+             "kcache_fp8 must be uint8 [..., 656], [..., 528] or [..., 288]")
     row = int(kcache_fp8.shape[-1])
     width = D_QK if row == 656 else 512
     _require(q.dim() == 4 and q.shape[-1] == width and q.dtype == torch.bfloat16,
              f"q must be [b, s_q, h_q, {width}] bf16 for {row}-byte cache rows")
-    _require(row == 656 or d_v == 512, "the 528-byte format has d_v = 512")
+    _require(row == 656 or d_v == 512, "the V4.1 formats have d_v = 512")
     b, s_q, h_q, _ = q.shape
     q = q.contiguous()
     idx = indices.to(torch.int32).contiguous()
@@ -312,7 +315,8 @@ def mla_sparse_decode(q, kcache_fp8, indices, d_v=512, softmax_scale=None, num_s
     else:
         ws = _workspace(mla_sparse_v41_workspace_size(b, s_q, h_q, topk, num_sm_parts), dev,
                         workspace)
-        _check(lib().mla_sparse_decode_v41(
+        fn = lib().mla_sparse_decode_v41 if row == 528 else lib().mla_sparse_decode_v41_fp4
+        _check(fn(
             _ptr(q), _ptr(kcache_fp8), num_slots, _ptr(idx), topk, b, s_q, h_q,
             float(softmax_scale), int(num_sm_parts), _ptr(ws), ws.numel(), _ptr(out), _ptr(lse),
             _stream(dev)))

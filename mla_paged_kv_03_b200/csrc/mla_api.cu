@@ -364,7 +364,7 @@ static int sparse_decode_impl(int row_bytes, const void* q, const uint8_t* kcach
                        const int32_t* indices, int topk, int batch, int s_q, int h_q, int d_v,
                        float softmax_scale, int num_sm_parts, void* workspace,
                        size_t workspace_bytes, void* out, float* lse, void* stream) {
-  const bool v41 = row_bytes == mla::kRow528;
+  const bool v41 = row_bytes != mla::kRow656;  // 512-dim latent: query widened to 576
   MLA_CHECK_ARG(batch >= 0 && s_q >= 1 && h_q >= 1, "bad sizes");
   MLA_CHECK_ARG(topk >= 1, "topk must be >= 1 (got %d)", topk);
   MLA_CHECK_ARG(num_slots >= 1 && num_slots < (1LL << 31), "num_slots must be in [1, 2^31)");
@@ -405,7 +405,11 @@ static int sparse_decode_impl(int row_bytes, const void* q, const uint8_t* kcach
   if (v41) {
     g.q512 = static_cast<const __nv_bfloat16*>(q);
     g.q576 = reinterpret_cast<__nv_bfloat16*>(ws + w.q_off);
+  }
+  if (row_bytes == mla::kRow528) {
     mla::mla_sparse_gather_kernel<mla::kRow528><<<grid, mla::kGatherCtaThreads, 0, st>>>(g);
+  } else if (row_bytes == mla::kRow288) {
+    mla::mla_sparse_gather_kernel<mla::kRow288><<<grid, mla::kGatherCtaThreads, 0, st>>>(g);
   } else {
     mla::mla_sparse_gather_kernel<mla::kRow656><<<grid, mla::kGatherCtaThreads, 0, st>>>(g);
   }
@@ -712,6 +716,15 @@ int mla_sparse_decode(const void* q, const uint8_t* kcache_fp8, int64_t num_slot
                       size_t workspace_bytes, void* out, float* lse, void* stream) {
   return sparse_decode_impl(mla::kRow656, q, kcache_fp8, num_slots, indices, topk, batch, s_q, h_q,
                             d_v, softmax_scale, num_sm_parts, workspace, workspace_bytes, out, lse,
+                            stream);
+}
+
+int mla_sparse_decode_v41_fp4(const void* q, const uint8_t* kcache_288, int64_t num_slots,
+                              const int32_t* indices, int topk, int batch, int s_q, int h_q,
+                              float softmax_scale, int num_sm_parts, void* workspace,
+                              size_t workspace_bytes, void* out, float* lse, void* stream) {
+  return sparse_decode_impl(mla::kRow288, q, kcache_288, num_slots, indices, topk, batch, s_q, h_q,
+                            512, softmax_scale, num_sm_parts, workspace, workspace_bytes, out, lse,
                             stream);
 }
 

@@ -8,9 +8,11 @@
 //    [64 x bf16 RoPE dims]; a nope value is code * scale.
 //  - 528 bytes (V4.1): [512 x E4M3 codes over the whole 512-dim latent]
 //    [16 x E8M0 scale, one per 32 codes]; a value is code * 2^(e - 127).
-//    The buffer row stays 576 wide with dims 512..575 zero, and the 512-wide
-//    query rows are copied into a 576-wide buffer with zero dims 512..575, so
-//    that q . k and the first 512 dims of V are unchanged.
+//  - 288 bytes (V4.1 FP4): [512 x E2M1 codes, two per byte, code 2i in the
+//    low nibble of byte i][32 x E4M3 scale, one per 16 codes].
+//  For both V4.1 rows the buffer row stays 576 wide with dims 512..575 zero,
+//  and the 512-wide query rows are copied into a 576-wide buffer with zero
+//  dims 512..575, so that q . k and the first 512 dims of V are unchanged.
 // Indices (per (sequence, query) pair): physical slots, -1 (or any value
 // outside [0, num_slots)) marks an unused entry; the block table of the cache
 // is not used.  [FlashMLA (AI Wiki), "Interfaces"]
@@ -61,12 +63,29 @@ __device__ __forceinline__ bool gather_valid(int idx, long long num_slots) {
   return idx >= 0 && static_cast<long long>(idx) < num_slots;
 }
 
+// E2M1 code (4 bits: sign, 2 exponent bits with bias 1, 1 mantissa bit) ->
+// fp32, from the format: exponent 0 holds 0 and 0.5.
+__device__ __forceinline__ float e2m1_to_float(uint32_t c) {
+  const uint32_t e = (c >> 1) & 3u, m = c & 1u;
+  const uint32_t mag = e ? (((e + 126u) << 23) | (m << 22)) : (m ? 0x3F000000u : 0u);
+  return __uint_as_float(mag | ((c & 8u) << 28));
+}
+
+// E4M3 byte -> fp32 through the hardware pair conversion (low byte -> low half).
+__device__ __forceinline__ float e4m3_to_float(uint32_t b) {
+  uint32_t h;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(static_cast<uint16_t>(b & 0xFFu)));
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(h & 0xFFFFu)));
+}
+
 // grid (pages_per_pair, pairs): CTA (c, b) handles indices [64c, 64c + 64) of pair b.
 template <int kRowBytes>
 __global__ void __launch_bounds__(kGatherCtaThreads)
     mla_sparse_gather_kernel(const GatherParams G) {
-  static_assert(kRowBytes == kRow656 || kRowBytes == kRow528, "656- or 528-byte rows");
-  constexpr bool kV41 = kRowBytes == kRow528;
+  static_assert(kRowBytes == kRow656 || kRowBytes == kRow528 || kRowBytes == kRow288,
+                "656-, 528- or 288-byte rows");
+  constexpr bool kV41 = kRowBytes != kRow656;  // 512-dim latent, query widened
+  constexpr bool kFp4 = kRowBytes == kRow288;
   __shared__ int s_red[kGatherCtaThreads / 32];
   __shared__ int s_idx[kGatherTokens];
   __shared__ int s_dst[kGatherTokens];  // destination row within the pair, or -1
@@ -146,7 +165,11 @@ __global__ void __launch_bounds__(kGatherCtaThreads)
     eb[k] = 127u;
     if (s_dst[t] >= 0) {
       const uint8_t* row = G.cache + (size_t)s_idx[t] * kRowBytes;
-      if (u < kNope / 16) {
+      if (u < kNope / 16 && kFp4) {
+        const uint2 v = __ldg(reinterpret_cast<const uint2*>(row) + u);  // 16 codes
+        raw[k] = make_uint4(v.x, v.y, 0u, 0u);
+        eb[k] = __ldg(row + kNope / 2 + u);
+      } else if (u < kNope / 16) {
         raw[k] = __ldg(reinterpret_cast<const uint4*>(row) + u);
         if (kV41)
           eb[k] = __ldg(row + kNope + (u >> 1));
@@ -180,7 +203,17 @@ __global__ void __launch_bounds__(kGatherCtaThreads)
     const int dst = s_dst[t];
     if (dst < 0) continue;
     __nv_bfloat16* orow = out_b + (size_t)dst * kD;
-    if (u < kNope / 16) {
+    if (u < kNope / 16 && kFp4) {
+      const float scl = e4m3_to_float(eb[k]);
+      uint32_t r[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const uint32_t byte = ((q < 4 ? raw[k].x : raw[k].y) >> (8 * (q & 3))) & 0xFFu;
+        r[q] = ptx::pack_bf16x2(e2m1_to_float(byte & 0xFu) * scl, e2m1_to_float(byte >> 4) * scl);
+      }
+      *reinterpret_cast<uint4*>(orow + 16 * u) = make_uint4(r[0], r[1], r[2], r[3]);
+      *reinterpret_cast<uint4*>(orow + 16 * u + 8) = make_uint4(r[4], r[5], r[6], r[7]);
+    } else if (u < kNope / 16) {
       const uint32_t words[4] = {raw[k].x, raw[k].y, raw[k].z, raw[k].w};
       const float scl = kV41 ? e8m0_to_float(eb[k]) : sc[k];
       uint32_t r[8];
