@@ -63,19 +63,17 @@ __device__ __forceinline__ bool gather_valid(int idx, long long num_slots) {
   return idx >= 0 && static_cast<long long>(idx) < num_slots;
 }
 
-// E2M1 code (4 bits: sign, 2 exponent bits with bias 1, 1 mantissa bit) ->
-// fp32, from the format: exponent 0 holds 0 and 0.5.
-__device__ __forceinline__ float e2m1_to_float(uint32_t c) {
-  const uint32_t e = (c >> 1) & 3u, m = c & 1u;
-  const uint32_t mag = e ? (((e + 126u) << 23) | (m << 22)) : (m ? 0x3F000000u : 0u);
-  return __uint_as_float(mag | ((c & 8u) << 28));
-}
-
-// E4M3 byte -> fp32 through the hardware pair conversion (low byte -> low half).
-__device__ __forceinline__ float e4m3_to_float(uint32_t b) {
-  uint32_t h;
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(static_cast<uint16_t>(b & 0xFFu)));
-  return __half2float(__ushort_as_half(static_cast<unsigned short>(h & 0xFFFFu)));
+// Eight E2M1 codes (4 bytes, low nibble first) -> four f16x2 pairs through the
+// hardware pair conversion (byte j -> pair j, low nibble -> low half).
+__device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t w, uint32_t (&h)[4]) {
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+      : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+      : "r"(w));
 }
 
 // grid (pages_per_pair, pairs): CTA (c, b) handles indices [64c, 64c + 64) of pair b.
@@ -204,12 +202,21 @@ __global__ void __launch_bounds__(kGatherCtaThreads)
     if (dst < 0) continue;
     __nv_bfloat16* orow = out_b + (size_t)dst * kD;
     if (u < kNope / 16 && kFp4) {
-      const float scl = e4m3_to_float(eb[k]);
+      // code * scale in f16 is exact (at most 6 significant bits, |x| <= 2688),
+      // and so is its bf16 rounding
+      uint32_t s2;
+      asm("cvt.rn.f16x2.e4m3x2 %0, %1;"
+          : "=r"(s2)
+          : "h"(static_cast<uint16_t>((eb[k] & 0xFFu) * 0x0101u)));
+      const __half2 scl2 = *reinterpret_cast<const __half2*>(&s2);
+      uint32_t h[8];
+      e2m1x8_to_f16x2(raw[k].x, *reinterpret_cast<uint32_t(*)[4]>(&h[0]));
+      e2m1x8_to_f16x2(raw[k].y, *reinterpret_cast<uint32_t(*)[4]>(&h[4]));
       uint32_t r[8];
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
-        const uint32_t byte = ((q < 4 ? raw[k].x : raw[k].y) >> (8 * (q & 3))) & 0xFFu;
-        r[q] = ptx::pack_bf16x2(e2m1_to_float(byte & 0xFu) * scl, e2m1_to_float(byte >> 4) * scl);
+        const float2 f = __half22float2(__hmul2(*reinterpret_cast<const __half2*>(&h[q]), scl2));
+        r[q] = ptx::pack_bf16x2(f.x, f.y);
       }
       *reinterpret_cast<uint4*>(orow + 16 * u) = make_uint4(r[0], r[1], r[2], r[3]);
       *reinterpret_cast<uint4*>(orow + 16 * u + 8) = make_uint4(r[4], r[5], r[6], r[7]);
