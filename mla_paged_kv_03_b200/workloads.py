@@ -21,6 +21,9 @@ Workloads (shapes and distributions as specified for this library):
                 q [b, s_q, h_q, 512].
 * ``sparse_v41_fp4`` the same over 288-byte V4.1 FP4 rows: 512 e2m1 codes
                 packed two per byte + 32 e4m3 scales (one per 16 values).
+* ``fused_sparse`` the fused decode in sparse mode: fused-workload queries
+                (h_q=64, gain ~ N(1, 0.1)) over the sparse workload's FP8
+                cache and indices, position L - 1.
 
 The cache of the fused workload is specified as "already rotated at its own
 positions".  A rotation of an isotropic Gaussian pair is again an isotropic
@@ -349,6 +352,57 @@ def sparse_v41_fp4(seed=0, device="cpu", **kw):
     return sparse_v41(seed=seed, device=device, fp4=True, **kw)
 
 
+@dataclass
+class FusedSparseCase:
+    q_raw: torch.Tensor        # [b, 1, h_q, 576] bf16
+    gain: torch.Tensor         # [576] fp32
+    eps: float
+    rope_base: float
+    positions: torch.Tensor    # [b] int32, the query's position (RoPE angle)
+    kcache: torch.Tensor       # [num_blocks, 64, 656] uint8
+    indices: torch.Tensor      # [b, 1, topk] int32, physical slot or -1
+    h_q: int
+    topk: int
+    softmax_scale: float
+    block_table: torch.Tensor = field(default=None)
+    name: str = ""
+    d_v: int = D_QK
+
+    @property
+    def batch(self):
+        return int(self.q_raw.shape[0])
+
+
+def fused_sparse(seed=0, device="cpu", batch=32, h_q=64, seqlen=65536, topk=2048,
+                 invalid_frac=0.05, seqlens=None):
+    """The fused decode in sparse mode: the fused workload's query, gain, eps
+    and RoPE base over the sparse workload's 656-byte FP8 cache and indices
+    (s_q = 1); each query sits at position L - 1 of its sequence."""
+    g = _gen(seed, device)
+    sl = seqlens if seqlens is not None else [seqlen] * batch
+    bt, nb = paged_block_table(sl, g, device=g.device)
+    n_rows = nb * PAGE
+    cache = torch.empty((n_rows, ROW656), dtype=torch.uint8, device=g.device)
+    step = 1 << 16
+    for r0 in range(0, n_rows, step):
+        r1 = min(n_rows, r0 + step)
+        x = torch.randn((r1 - r0, D_NOPE), generator=g, device=g.device, dtype=torch.float32)
+        rope = torch.randn((r1 - r0, D_ROPE), generator=g, device=g.device,
+                           dtype=torch.float32).to(torch.bfloat16)
+        cache[r0:r1] = quantize_rows656(x, rope)
+    q_raw = _randn_bf16((len(sl), 1, h_q, D_QK), g)
+    gain = (1.0 + 0.1 * torch.randn((D_QK,), generator=g, device=g.device,
+                                    dtype=torch.float32))
+    idx = _sparse_indices(sl, bt, 1, topk, invalid_frac, g)
+    pos = torch.tensor([int(L) - 1 for L in sl], dtype=torch.int32)
+    return FusedSparseCase(q_raw=q_raw.to(device), gain=gain.to(device), eps=1e-6,
+                           rope_base=10000.0, positions=pos.to(device),
+                           kcache=cache.view(nb, PAGE, ROW656).to(device),
+                           indices=idx.to(device), h_q=h_q, topk=topk,
+                           softmax_scale=default_scale(), block_table=bt.to(device),
+                           name="fused_sparse")
+
+
 WORKLOADS = {
     "tiny": tiny,
     "compute": compute_bound,
@@ -357,4 +411,5 @@ WORKLOADS = {
     "sparse": sparse,
     "sparse_v41": sparse_v41,
     "sparse_v41_fp4": sparse_v41_fp4,
+    "fused_sparse": fused_sparse,
 }

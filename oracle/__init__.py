@@ -76,6 +76,11 @@ def lib():
         L.oracle_sparse_decode_v41.argtypes = [
             u16p, u8p, ctypes.c_int64, i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
             ctypes.c_int, ctypes.c_double, i64p, ctypes.c_int64, f64p, f64p]
+        L.oracle_fused_sparse_decode.restype = ctypes.c_int
+        L.oracle_fused_sparse_decode.argtypes = [
+            u16p, f64p, ctypes.c_double, ctypes.c_double, i32p, u8p, ctypes.c_int64, i32p,
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double, i64p, ctypes.c_int64,
+            u8p, f64p, f64p]
         _LIB = L
     return _LIB
 
@@ -324,3 +329,33 @@ def sparse_decode_v41(q, kcache, indices, softmax_scale, rows=None):
     if ra is None:
         return out.reshape(b, s_q, h_q, 512), lse.reshape(b, s_q, h_q)
     return out, lse
+
+
+def fused_sparse_decode(q_raw, gain, eps, rope_base, positions, kcache656, indices,
+                        softmax_scale, rows=None):
+    """oracle_fused_sparse_decode: the fused steps over the valid slots of
+    indices [b, 1, topk] in the 656-byte FP8 cache; positions [b] required.
+    Returns (codes uint8, scale fp64, lse fp64)."""
+    b, s_q, h_q, dq = q_raw.shape
+    assert s_q == 1 and dq == _D
+    qa = _np(q_raw, np.uint16)
+    g = np.ascontiguousarray(_np(gain, np.float32), dtype=np.float64)
+    pos = _np(positions, np.int32)
+    ca = _np(kcache656, np.uint8).reshape(-1, 656)
+    ix = _np(indices, np.int32)
+    topk = ix.shape[-1]
+    ra = None if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    n = b * h_q if ra is None else ra.size
+    codes = np.zeros((n, _D), dtype=np.uint8)
+    scale = np.zeros(n, dtype=np.float64)
+    lse = np.zeros(n, dtype=np.float64)
+    rc = lib().oracle_fused_sparse_decode(
+        _ptr(qa, ctypes.c_uint16), _ptr(g, ctypes.c_double), float(eps), float(rope_base),
+        _ptr(pos, ctypes.c_int32), _ptr(ca, ctypes.c_uint8), ca.shape[0], _ptr(ix, ctypes.c_int32),
+        b, h_q, topk, float(softmax_scale), _ptr(ra, ctypes.c_int64), n,
+        _ptr(codes, ctypes.c_uint8), _ptr(scale, ctypes.c_double), _ptr(lse, ctypes.c_double))
+    if rc != 0:
+        raise ValueError("sparse index out of range")
+    if ra is None:
+        return codes.reshape(b, 1, h_q, _D), scale.reshape(b, 1, h_q), lse.reshape(b, 1, h_q)
+    return codes, scale, lse

@@ -371,6 +371,36 @@ void oracle_combine(int n_splits, const double* lse_i, const double* o_i, int d_
  *  o_pre   optional [.., 576]: the fp64 row after conjugate RoPE, before the
  *          cast (lets tests compare the pre-cast values).
  * Step order: [FlashMLA fused norm-RoPE-attention-RoPE-cast kernel card]. */
+/* The fused steps for one query row over n tokens given by `fetch`: RMSNorm
+ * of the raw query, RoPE of its dims 512..575 at `pos`, one bf16 rounding,
+ * attention with d_v = 576, conjugate RoPE of O's dims 512..575, then the
+ * per-row FP8 cast (scale = absmax/448). */
+static void fused_row(const uint16_t* qr, const double* gain, double eps, double rope_base,
+                      double pos, row_fetch_fn fetch, const void* ctx, int n, double scale,
+                      uint8_t* codes, double* out_scale, double* lse, double* o_pre) {
+  double x[ORACLE_D], y[ORACLE_D], o[ORACLE_D], orot[ORACLE_ROPE];
+  double l, amax = 0.0, sc;
+  int d;
+  for (d = 0; d < ORACLE_D; ++d) x[d] = bf16_bits_to_f64(qr[d]);
+  oracle_rmsnorm(x, gain, ORACLE_D, eps, y);
+  oracle_rope64(y + ORACLE_NOPE, pos, rope_base, +1, x + ORACLE_NOPE);
+  for (d = 0; d < ORACLE_NOPE; ++d) x[d] = y[d];
+  for (d = 0; d < ORACLE_D; ++d) x[d] = oracle_round_bf16(x[d]);
+  attend_rows(x, fetch, ctx, n, ORACLE_D, scale, o, &l);
+  oracle_rope64(o + ORACLE_NOPE, pos, rope_base, -1, orot);
+  for (d = 0; d < ORACLE_ROPE; ++d) o[ORACLE_NOPE + d] = orot[d];
+  for (d = 0; d < ORACLE_D; ++d)
+    if (fabs(o[d]) > amax) amax = fabs(o[d]);
+  sc = amax > 0.0 ? amax / 448.0 : 1.0;
+  for (d = 0; d < ORACLE_D; ++d) {
+    float ratio = (float)(o[d] / sc);
+    codes[d] = oracle_e4m3_encode((double)ratio);
+    if (o_pre) o_pre[d] = o[d];
+  }
+  *out_scale = sc;
+  *lse = l;
+}
+
 int oracle_fused_decode(const uint16_t* q_raw, const double* gain, double eps, double rope_base,
                         const int32_t* positions, const uint16_t* kcache,
                         const int32_t* block_table, int max_pages, const int32_t* seqlens,
@@ -386,35 +416,16 @@ int oracle_fused_decode(const uint16_t* q_raw, const double* gain, double eps, d
     int b = (int)(flat / h_q);
     int L = seqlens[b];
     double pos = positions ? (double)positions[b] : (double)(L - 1);
-    const uint16_t* qr = q_raw + (size_t)flat * ORACLE_D;
-    double x[ORACLE_D], y[ORACLE_D], o[ORACLE_D], orot[ORACLE_ROPE];
-    double l, amax = 0.0, sc;
     paged_ctx ctx;
-    int d;
-    for (d = 0; d < ORACLE_D; ++d) x[d] = bf16_bits_to_f64(qr[d]);
-    oracle_rmsnorm(x, gain, ORACLE_D, eps, y);
-    oracle_rope64(y + ORACLE_NOPE, pos, rope_base, +1, x + ORACLE_NOPE);
-    for (d = 0; d < ORACLE_NOPE; ++d) x[d] = y[d];
-    for (d = 0; d < ORACLE_D; ++d) x[d] = oracle_round_bf16(x[d]);
     ctx.kcache = kcache;
     ctx.block_table = block_table;
     ctx.max_pages = max_pages;
     ctx.b = b;
     ctx.lo = 0;
     ctx.page = page;
-    attend_rows(x, fetch_paged_bf16, &ctx, L, ORACLE_D, scale, o, &l);
-    oracle_rope64(o + ORACLE_NOPE, pos, rope_base, -1, orot);
-    for (d = 0; d < ORACLE_ROPE; ++d) o[ORACLE_NOPE + d] = orot[d];
-    for (d = 0; d < ORACLE_D; ++d)
-      if (fabs(o[d]) > amax) amax = fabs(o[d]);
-    sc = amax > 0.0 ? amax / 448.0 : 1.0;
-    for (d = 0; d < ORACLE_D; ++d) {
-      float ratio = (float)(o[d] / sc);
-      codes[(size_t)r * ORACLE_D + d] = oracle_e4m3_encode((double)ratio);
-      if (o_pre) o_pre[(size_t)r * ORACLE_D + d] = o[d];
-    }
-    out_scale[r] = sc;
-    lse[r] = l;
+    fused_row(q_raw + (size_t)flat * ORACLE_D, gain, eps, rope_base, pos, fetch_paged_bf16, &ctx,
+              L, scale, codes + (size_t)r * ORACLE_D, out_scale + r, lse + r,
+              o_pre ? o_pre + (size_t)r * ORACLE_D : 0);
   }
   return 0;
 }
@@ -566,4 +577,44 @@ int oracle_sparse_decode_v41_fp4(const uint16_t* q, const uint8_t* cache, int64_
                                  double* lse) {
   return sparse_decode_512(fetch_row288, q, cache, num_slots, indices, batch, s_q, h_q, topk,
                            scale, rows, n_rows, out, lse);
+}
+
+/* Fused decode in sparse mode: the fused steps of oracle_fused_decode over
+ * the valid slots of indices [b, 1, topk] in the 656-byte FP8 cache (decoded
+ * to 576 dims; V is the whole row, d_v = 576).  positions [b] is required:
+ * the selected tokens say nothing about the query's own position. */
+int oracle_fused_sparse_decode(const uint16_t* q_raw, const double* gain, double eps,
+                               double rope_base, const int32_t* positions, const uint8_t* cache,
+                               int64_t num_slots, const int32_t* indices, int batch, int h_q,
+                               int topk, double scale, const int64_t* rows, int64_t n_rows,
+                               uint8_t* codes, double* out_scale, double* lse) {
+  int64_t total = (int64_t)batch * h_q;
+  int64_t n = rows ? n_rows : total;
+  int64_t r;
+  int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+  for (r = 0; r < n; ++r) {
+    int64_t flat = rows ? rows[r] : r;
+    int b = (int)(flat / h_q);
+    const int32_t* idx = indices + (size_t)b * topk;
+    int32_t* slots = (int32_t*)malloc(sizeof(int32_t) * (size_t)(topk > 0 ? topk : 1));
+    fp8_ctx ctx;
+    int j, cnt = 0;
+    for (j = 0; j < topk; ++j) {
+      int32_t s = idx[j];
+      if (s < 0) continue;
+      if ((int64_t)s >= num_slots) {
+        bad = 1;
+        continue;
+      }
+      slots[cnt++] = s;
+    }
+    ctx.cache = cache;
+    ctx.slots = slots;
+    fused_row(q_raw + (size_t)flat * ORACLE_D, gain, eps, rope_base, (double)positions[b],
+              fetch_fp8, &ctx, cnt, scale, codes + (size_t)r * ORACLE_D, out_scale + r, lse + r,
+              0);
+    free(slots);
+  }
+  return bad ? -1 : 0;
 }
