@@ -48,6 +48,9 @@ WORKLOAD_INFO = {
     "sparse_v41_fp4": ("Token-level sparse decode, V4.1 FP4 288-byte cache (512 e2m1 + 32 e4m3): "
                        "batch 32, s_q 1, h_q 128, d_qk = d_v 512, 65536-token cache per sequence, "
                        "topk 2048, 5% -1 slots", "tensor"),
+    "fused_sparse": ("Fused RMSNorm-RoPE-attn-conjRoPE-FP8 decode in sparse mode over the FP8 "
+                     "656-byte cache: batch 32, s_q 1, h_q 64, d 576, d_v 576, 65536-token cache "
+                     "per sequence, topk 2048, 5% -1 slots, position L - 1", "tensor"),
     "sparse": ("Token-level sparse decode, FP8 656-byte cache: batch 32, s_q 1, h_q 128, d_v 512, "
                "65536-token cache per sequence, topk 2048, 5% -1 slots", "tensor"),
     "tiny": ("Tiny dense decode, bf16: batch 2, s_q 1, h_q 16, lengths {37, 200}", "tensor"),
@@ -133,6 +136,15 @@ def fused_work(case):
     return flops, kv_bytes, kv_bytes + io
 
 
+def fused_sparse_work(case):
+    valid = int((case.indices >= 0).sum())  # sequences x valid slots (s_q = 1)
+    flops = 2 * valid * (576 + 576) * case.h_q
+    kv_bytes = valid * 656
+    io = case.q_raw.numel() * 2 + 576 * 4 + case.indices.numel() * 4 + case.batch * 4 + \
+        case.batch * case.h_q * (576 + 4 + 4)
+    return flops, kv_bytes, kv_bytes + io
+
+
 def sparse_dims(case):
     """(latent width of q . k, bytes per cache row) of a sparse case."""
     row = int(case.kcache.shape[-1])
@@ -170,6 +182,11 @@ class GpuStep:
             self.kind = "fused"
             self.work = fused_work(self.case)
             self.R = self.case.h_q
+        elif name == "fused_sparse":
+            self.case = W.fused_sparse(seed=seed, device=dev)
+            self.kind = "fused_sparse"
+            self.work = fused_sparse_work(self.case)
+            self.R = self.case.h_q
         elif name in ("sparse", "sparse_v41", "sparse_v41_fp4"):
             self.case = W.WORKLOADS[name](seed=seed, device=dev)
             self.kind = "sparse"
@@ -185,12 +202,13 @@ class GpuStep:
             self.lse = torch.empty((b, c.s_q, c.h_q), dtype=torch.float32, device=dev)
             self.ws = torch.empty((B.mla_workspace_size(b, self.R, c.d_v, self.parts),),
                                   dtype=torch.uint8, device=dev)
-        elif self.kind == "fused":
+        elif self.kind in ("fused", "fused_sparse"):
             self.out = torch.empty((b, 1, c.h_q, 576), dtype=torch.uint8, device=dev)
             self.scale = torch.empty((b, 1, c.h_q), dtype=torch.float32, device=dev)
             self.lse = torch.empty((b, 1, c.h_q), dtype=torch.float32, device=dev)
-            self.ws = torch.empty((B.mla_workspace_size(b, self.R, 576, self.parts),),
-                                  dtype=torch.uint8, device=dev)
+            nbytes = (B.mla_workspace_size(b, self.R, 576, self.parts) if self.kind == "fused"
+                      else B.mla_sparse_fused_workspace_size(b, c.h_q, c.topk, self.parts))
+            self.ws = torch.empty((nbytes,), dtype=torch.uint8, device=dev)
         else:
             self.out = torch.empty((b, c.s_q, c.h_q, c.d_v), dtype=torch.bfloat16, device=dev)
             self.lse = torch.empty((b, c.s_q, c.h_q), dtype=torch.float32, device=dev)
@@ -198,13 +216,13 @@ class GpuStep:
                       if name == "sparse" else
                       B.mla_sparse_v41_workspace_size(b, c.s_q, c.h_q, c.topk, self.parts))
             self.ws = torch.empty((nbytes,), dtype=torch.uint8, device=dev)
-        if self.kind != "sparse":
+        if self.kind in ("dense", "fused"):
             self.meta = torch.empty((self.parts, 8), dtype=torch.int32, device=dev)
             self.ns = torch.empty((b + 1,), dtype=torch.int32, device=dev)
 
     def launches_per_step(self):
         # planner + attention kernel + combine (+ the FP8 gather for sparse)
-        return 4 if self.kind == "sparse" else 3
+        return 4 if self.kind in ("sparse", "fused_sparse") else 3
 
     def step(self, q=None):
         B, c = self.B, self.case
@@ -221,16 +239,22 @@ class GpuStep:
                 c.block_table, c.cache_seqlens, m, n, self.parts,
                 softmax_scale=c.softmax_scale, out=self.out, out_scale=self.scale, lse=self.lse,
                 workspace=self.ws)
+        elif self.kind == "fused_sparse":
+            B.mla_sparse_fused_norm_rope_attn_rope_cast(
+                c.q_raw if q is None else q, c.gain, c.eps, c.rope_base, c.positions, c.kcache,
+                c.indices, c.softmax_scale, self.parts, out=self.out, out_scale=self.scale,
+                lse=self.lse, workspace=self.ws)
         else:
             B.mla_sparse_decode(c.q if q is None else q, c.kcache, c.indices, c.d_v,
                                 c.softmax_scale, self.parts, out=self.out, lse=self.lse,
                                 workspace=self.ws)
 
     def query(self):
-        return self.case.q_raw if self.kind == "fused" else self.case.q
+        return self.case.q_raw if self.kind in ("fused", "fused_sparse") else self.case.q
 
     def outputs(self):
-        return [self.out, self.lse] + ([self.scale] if self.kind == "fused" else [])
+        return [self.out, self.lse] + ([self.scale] if self.kind in ("fused", "fused_sparse")
+                                       else [])
 
     def capture(self):
         """One step recorded as a CUDA graph (planner, attention kernel,
@@ -504,7 +528,7 @@ def run_gpu_arm(args, rank, world):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16" if not args.workload.startswith("sparse") else
+        "dtype": "bf16" if "sparse" not in args.workload else
         "bf16 (fp4 cache dequantised)" if args.workload.endswith("fp4") else "bf16 (fp8 cache dequantised)",
         "data": "synthetic",
         "config": {"workload": desc, "name": args.workload,
@@ -545,7 +569,11 @@ def oracle_rows_timed(name, case, rows):
         return time.perf_counter() - t0
     c = case
     t0 = time.perf_counter()
-    if name.startswith("sparse_v41"):
+    if name == "fused_sparse":
+        oracle.fused_sparse_decode(c.q_raw.cpu(), c.gain.cpu(), c.eps, c.rope_base,
+                                   c.positions.cpu(), c.kcache_cpu, c.indices.cpu(),
+                                   c.softmax_scale, rows=rows)
+    elif name.startswith("sparse_v41"):
         oracle.sparse_decode_v41(c.q.cpu(), c.kcache_cpu, c.indices.cpu(), c.softmax_scale,
                                  rows=rows)
     else:
@@ -579,7 +607,7 @@ def row_flops(name, case, rows):
 
 def make_case(name, seed, device="cpu"):
     """The named workload's seeded inputs."""
-    if name.startswith("fused"):
+    if name in ("fused", "fused_b1"):
         return W.fused(seed=seed, device=device, batch=32 if name == "fused" else 1)
     return W.WORKLOADS[name](seed=seed, device=device)
 

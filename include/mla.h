@@ -221,6 +221,32 @@ MLA_API int mla_sparse_decode_v41_fp4(const void* q, const uint8_t* kcache_288, 
                               float softmax_scale, int num_sm_parts, void* workspace,
                               size_t workspace_bytes, void* out, float* lse, void* stream);
 
+/* Workspace bytes for mla_sparse_fused_norm_rope_attn_rope_cast. */
+MLA_API int mla_sparse_fused_workspace_size(int batch, int h_q, int topk, int num_sm_parts,
+                                    size_t* bytes);
+
+/* The fused decode in sparse mode: the steps of
+ * mla_fused_norm_rope_attn_rope_cast (Q RMSNorm, Q-RoPE, attention,
+ * conjugate O-RoPE, FP8 cast; s_q = 1, d_v = 576) over the valid slots of
+ * `indices` in the 656-byte FP8 cache, as mla_sparse_decode selects them
+ * [FlashMLA fused norm-RoPE-attention-RoPE-cast kernel card, "Arithmetic
+ * intensity", "Workarounds"; FlashMLA (AI Wiki), "Interfaces"].
+ *   q_raw, norm_gain, eps, rope_base, out_e4m3, out_scale, lse: as in
+ *                 mla_fused_norm_rope_attn_rope_cast
+ *   positions     int32[batch] query positions, REQUIRED (the selected slots
+ *                 do not give the query's position)
+ *   kcache_fp8, num_slots: as in mla_sparse_decode
+ *   indices       int32[batch, 1, topk] physical slots, -1 = unused
+ *   num_sm_parts  from mla_num_sm_parts(device, h_q, 1)
+ * A row with no valid slot gives O = 0 (codes 0, scale 1) and LSE = -inf.
+ * Ownership, alignment and errors as in mla_sparse_decode. */
+MLA_API int mla_sparse_fused_norm_rope_attn_rope_cast(
+    const void* q_raw, const float* norm_gain, float eps, float rope_base,
+    const int32_t* positions, const uint8_t* kcache_fp8, int64_t num_slots,
+    const int32_t* indices, int topk, int batch, int h_q, float softmax_scale, int num_sm_parts,
+    void* workspace, size_t workspace_bytes, uint8_t* out_e4m3, float* out_scale, float* lse,
+    void* stream);
+
 /* Dense decode without a caller workspace.  This entry point has no
  * counterpart in the method's published interface; it exists for callers
  * that cannot supply scratch memory at decode time (an embedder whose device

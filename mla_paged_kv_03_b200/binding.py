@@ -30,7 +30,8 @@ EXPORTED = [
     "mla_fused_norm_rope_attn_rope_cast", "mla_sparse_workspace_size", "mla_sparse_decode",
     "mla_device_status", "mla_noalloc_scratch_bytes", "mla_decode_fwd_noalloc",
     "mla_set_kernel_events", "mla_sparse_v41_workspace_size", "mla_sparse_decode_v41",
-    "mla_sparse_decode_v41_fp4",
+    "mla_sparse_decode_v41_fp4", "mla_sparse_fused_workspace_size",
+    "mla_sparse_fused_norm_rope_attn_rope_cast",
 ]
 
 
@@ -75,6 +76,9 @@ def lib():
         L.mla_sparse_decode_v41.argtypes = [vp, vp, i64, vp, i32, i32, i32, i32, f32, i32, vp,
                                             sz, vp, vp, vp]
         L.mla_sparse_decode_v41_fp4.argtypes = L.mla_sparse_decode_v41.argtypes
+        L.mla_sparse_fused_workspace_size.argtypes = [i32, i32, i32, i32, szp]
+        L.mla_sparse_fused_norm_rope_attn_rope_cast.argtypes = [
+            vp, vp, f32, f32, vp, vp, i64, vp, i32, i32, i32, f32, i32, vp, sz, vp, vp, vp, vp]
         L.mla_device_status.argtypes = [ip, i32]
         L.mla_noalloc_scratch_bytes.argtypes = []
         L.mla_set_kernel_events.argtypes = [vp, vp]
@@ -161,6 +165,13 @@ def mla_sparse_v41_workspace_size(batch, s_q, h_q, topk, num_sm_parts) -> int:
     out = ctypes.c_size_t(0)
     _check(lib().mla_sparse_v41_workspace_size(int(batch), int(s_q), int(h_q), int(topk),
                                                int(num_sm_parts), ctypes.byref(out)))
+    return int(out.value)
+
+
+def mla_sparse_fused_workspace_size(batch, h_q, topk, num_sm_parts) -> int:
+    out = ctypes.c_size_t(0)
+    _check(lib().mla_sparse_fused_workspace_size(int(batch), int(h_q), int(topk),
+                                                 int(num_sm_parts), ctypes.byref(out)))
     return int(out.value)
 
 
@@ -330,3 +341,42 @@ def device_status(reset: bool = True) -> int:
     if rc not in (MLA_OK, MLA_ERR_TIMEOUT):
         _check(rc)
     return v.value
+
+
+def mla_sparse_fused_norm_rope_attn_rope_cast(q_raw, norm_gain, eps, rope_base, positions,
+                                              kcache_fp8, indices, softmax_scale=None,
+                                              num_sm_parts=None, out=None, out_scale=None,
+                                              lse=None, workspace=None):
+    """The fused decode in sparse mode over the 656-byte FP8 cache.
+    q_raw [b, 1, h_q, 576] bf16; positions [b] int32 (required); indices
+    [b, 1, topk] int32 physical slots (-1 = unused).  Returns (codes uint8
+    [b, 1, h_q, 576], scale fp32 [b, 1, h_q], lse fp32 [b, 1, h_q])."""
+    _require(q_raw.dim() == 4 and q_raw.shape[1] == 1 and q_raw.shape[-1] == D_QK and
+             q_raw.dtype == torch.bfloat16, "q_raw must be [b, 1, h_q, 576] bf16")
+    _require(kcache_fp8.dtype == torch.uint8 and kcache_fp8.shape[-1] == 656,
+             "kcache_fp8 must be uint8 [..., 656]")
+    _require(positions is not None, "positions are required in sparse mode")
+    b, _, h_q, _ = q_raw.shape
+    q_raw = q_raw.contiguous()
+    gain = norm_gain.to(torch.float32).contiguous()
+    pos = positions.to(torch.int32).contiguous()
+    idx = indices.to(torch.int32).contiguous()
+    topk = idx.shape[-1]
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(D_QK)
+    if num_sm_parts is None:
+        num_sm_parts = mla_num_sm_parts(h_q, 1, q_raw.device)
+    dev = q_raw.device
+    if out is None:
+        out = torch.empty((b, 1, h_q, D_QK), dtype=torch.uint8, device=dev)
+    if out_scale is None:
+        out_scale = torch.empty((b, 1, h_q), dtype=torch.float32, device=dev)
+    if lse is None:
+        lse = torch.empty((b, 1, h_q), dtype=torch.float32, device=dev)
+    ws = _workspace(mla_sparse_fused_workspace_size(b, h_q, topk, num_sm_parts), dev, workspace)
+    _check(lib().mla_sparse_fused_norm_rope_attn_rope_cast(
+        _ptr(q_raw), _ptr(gain), float(eps), float(rope_base), _ptr(pos), _ptr(kcache_fp8),
+        kcache_fp8.numel() // 656, _ptr(idx), topk, b, h_q, float(softmax_scale),
+        int(num_sm_parts), _ptr(ws), ws.numel(), _ptr(out), _ptr(out_scale), _ptr(lse),
+        _stream(dev)))
+    return out, out_scale, lse

@@ -360,6 +360,45 @@ int static_scratch_ptr(void** ptr) {
 
 // Both sparse paths: gather + dequantise + compact the valid rows of every
 // (sequence, query) pair, then the dense planner and decode over them.
+// Sparse paths, first half: gather + dequantise + compact the valid tokens of
+// every (sequence, query) pair into the workspace (rows, identity block table,
+// lengths; for the 512-dim V4.1 rows also the query widened to 576 dims,
+// returned in *q_dense), then the planner over those lengths.
+static int sparse_gather_and_plan(int row_bytes, const void* q, const uint8_t* kcache,
+                                  int64_t num_slots, const int32_t* indices, int topk, int pairs,
+                                  int h_q, int num_sm_parts, uint8_t* ws, const SparseWs& w,
+                                  void* stream, const void** q_dense) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  mla::GatherParams g{};
+  g.cache = kcache;
+  g.num_slots = num_slots;
+  g.indices = indices;
+  g.topk = topk;
+  g.pages_per_pair = w.pages_per_pair;
+  g.rows = reinterpret_cast<__nv_bfloat16*>(ws + w.rows_off);
+  g.block_table = reinterpret_cast<int32_t*>(ws + w.bt_off);
+  g.seqlens = reinterpret_cast<int32_t*>(ws + w.len_off);
+  g.h_q = h_q;
+  *q_dense = q;
+  if (row_bytes != mla::kRow656) {
+    g.q512 = static_cast<const __nv_bfloat16*>(q);
+    g.q576 = reinterpret_cast<__nv_bfloat16*>(ws + w.q_off);
+    *q_dense = g.q576;
+  }
+  const dim3 grid(w.pages_per_pair, pairs);
+  if (row_bytes == mla::kRow528) {
+    mla::mla_sparse_gather_kernel<mla::kRow528><<<grid, mla::kGatherCtaThreads, 0, st>>>(g);
+  } else if (row_bytes == mla::kRow288) {
+    mla::mla_sparse_gather_kernel<mla::kRow288><<<grid, mla::kGatherCtaThreads, 0, st>>>(g);
+  } else {
+    mla::mla_sparse_gather_kernel<mla::kRow656><<<grid, mla::kGatherCtaThreads, 0, st>>>(g);
+  }
+  MLA_CUDA(cudaGetLastError());
+  return mla_get_metadata(g.seqlens, pairs, h_q, 1, num_sm_parts,
+                          reinterpret_cast<int32_t*>(ws + w.meta_off),
+                          reinterpret_cast<int32_t*>(ws + w.splits_off), stream);
+}
+
 static int sparse_decode_impl(int row_bytes, const void* q, const uint8_t* kcache, int64_t num_slots,
                        const int32_t* indices, int topk, int batch, int s_q, int h_q, int d_v,
                        float softmax_scale, int num_sm_parts, void* workspace,
@@ -387,43 +426,18 @@ static int sparse_decode_impl(int row_bytes, const void* q, const uint8_t* kcach
   const long long pages = static_cast<long long>(pairs) * w.pages_per_pair;
   MLA_CHECK_ARG(pages * mla::kPage < (1LL << 31), "pairs * topk too large");
   if (batch == 0) return MLA_OK;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-
-  // 1. gather + dequantise + compact the valid tokens of every pair
-  mla::GatherParams g{};
-  g.cache = kcache;
-  g.num_slots = num_slots;
-  g.indices = indices;
-  g.topk = topk;
-  g.pages_per_pair = w.pages_per_pair;
-  g.rows = reinterpret_cast<__nv_bfloat16*>(ws + w.rows_off);
-  g.block_table = reinterpret_cast<int32_t*>(ws + w.bt_off);
-  g.seqlens = reinterpret_cast<int32_t*>(ws + w.len_off);
-  g.h_q = h_q;
-  const dim3 grid(w.pages_per_pair, pairs);
-  if (v41) {
-    g.q512 = static_cast<const __nv_bfloat16*>(q);
-    g.q576 = reinterpret_cast<__nv_bfloat16*>(ws + w.q_off);
-  }
-  if (row_bytes == mla::kRow528) {
-    mla::mla_sparse_gather_kernel<mla::kRow528><<<grid, mla::kGatherCtaThreads, 0, st>>>(g);
-  } else if (row_bytes == mla::kRow288) {
-    mla::mla_sparse_gather_kernel<mla::kRow288><<<grid, mla::kGatherCtaThreads, 0, st>>>(g);
-  } else {
-    mla::mla_sparse_gather_kernel<mla::kRow656><<<grid, mla::kGatherCtaThreads, 0, st>>>(g);
-  }
-  MLA_CUDA(cudaGetLastError());
-
-  // 2. dense decode over the compacted rows: no causal mask, lengths = valid counts
-  int32_t* meta = reinterpret_cast<int32_t*>(ws + w.meta_off);
-  int32_t* splits = reinterpret_cast<int32_t*>(ws + w.splits_off);
-  int rc = mla_get_metadata(g.seqlens, pairs, h_q, 1, num_sm_parts, meta, splits, stream);
+  const void* q_dense = q;
+  int rc = sparse_gather_and_plan(row_bytes, q, kcache, num_slots, indices, topk, pairs, h_q,
+                                  num_sm_parts, ws, w, stream, &q_dense);
   if (rc != MLA_OK) return rc;
-  const void* q_dense = v41 ? static_cast<const void*>(g.q576) : q;
-  return mla_decode_fwd(q_dense, g.rows, g.block_table, w.pages_per_pair, static_cast<int>(pages),
-                        g.seqlens, pairs, 1, h_q, 1, d_v, softmax_scale, 0, meta, splits,
-                        num_sm_parts, ws + w.dense_off, w.dense_bytes, out, lse, stream);
+  // dense decode over the compacted rows: no causal mask, lengths = valid counts
+  return mla_decode_fwd(q_dense, ws + w.rows_off, reinterpret_cast<int32_t*>(ws + w.bt_off),
+                        w.pages_per_pair, static_cast<int>(pages),
+                        reinterpret_cast<int32_t*>(ws + w.len_off), pairs, 1, h_q, 1, d_v,
+                        softmax_scale, 0, reinterpret_cast<int32_t*>(ws + w.meta_off),
+                        reinterpret_cast<int32_t*>(ws + w.splits_off), num_sm_parts,
+                        ws + w.dense_off, w.dense_bytes, out, lse, stream);
 }
 
 extern "C" {
@@ -717,6 +731,55 @@ int mla_sparse_decode(const void* q, const uint8_t* kcache_fp8, int64_t num_slot
   return sparse_decode_impl(mla::kRow656, q, kcache_fp8, num_slots, indices, topk, batch, s_q, h_q,
                             d_v, softmax_scale, num_sm_parts, workspace, workspace_bytes, out, lse,
                             stream);
+}
+
+int mla_sparse_fused_workspace_size(int batch, int h_q, int topk, int num_sm_parts,
+                                    size_t* bytes) {
+  MLA_CHECK_ARG(bytes, "bytes is null");
+  MLA_CHECK_ARG(batch >= 0 && h_q >= 1 && topk >= 1 && num_sm_parts >= 1, "bad sizes");
+  *bytes = sparse_ws_layout(batch, topk, h_q, mla::kD, num_sm_parts).total;
+  return MLA_OK;
+}
+
+int mla_sparse_fused_norm_rope_attn_rope_cast(
+    const void* q_raw, const float* norm_gain, float eps, float rope_base,
+    const int32_t* positions, const uint8_t* kcache_fp8, int64_t num_slots,
+    const int32_t* indices, int topk, int batch, int h_q, float softmax_scale, int num_sm_parts,
+    void* workspace, size_t workspace_bytes, uint8_t* out_e4m3, float* out_scale, float* lse,
+    void* stream) {
+  MLA_CHECK_ARG(batch >= 0 && h_q >= 1, "bad sizes");
+  MLA_CHECK_ARG(topk >= 1, "topk must be >= 1 (got %d)", topk);
+  MLA_CHECK_ARG(num_slots >= 1 && num_slots < (1LL << 31), "num_slots must be in [1, 2^31)");
+  MLA_CHECK_ARG(num_sm_parts >= 1 && num_sm_parts <= mla::kCombineMaxSplits,
+                "num_sm_parts must be in [1, %d]", mla::kCombineMaxSplits);
+  MLA_CHECK_ARG(positions, "positions are required in sparse mode");
+  MLA_CHECK_ARG(q_raw && norm_gain && kcache_fp8 && indices && workspace && out_e4m3 &&
+                    out_scale && lse,
+                "null device pointer");
+  MLA_CHECK_ARG(aligned(q_raw, 16) && aligned(kcache_fp8, 16),
+                "q_raw and the cache must be 16-byte aligned");
+  MLA_CHECK_ARG(aligned(workspace, 256), "workspace must be 256-byte aligned");
+  MLA_CHECK_ARG(aligned(indices, 4) && aligned(positions, 4), "misaligned indices or positions");
+  const SparseWs w = sparse_ws_layout(batch, topk, h_q, mla::kD, num_sm_parts);
+  MLA_CHECK_ARG(workspace_bytes >= w.total, "workspace too small: %zu < %zu", workspace_bytes,
+                w.total);
+  MLA_CHECK_ARG(batch <= mla::kPlanMaxBatch, "at most %d sequences (got %d)", mla::kPlanMaxBatch,
+                batch);
+  const long long pages = static_cast<long long>(batch) * w.pages_per_pair;
+  MLA_CHECK_ARG(pages * mla::kPage < (1LL << 31), "batch * topk too large");
+  if (batch == 0) return MLA_OK;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const void* q_dense = q_raw;
+  int rc = sparse_gather_and_plan(mla::kRow656, q_raw, kcache_fp8, num_slots, indices, topk,
+                                  batch, h_q, num_sm_parts, ws, w, stream, &q_dense);
+  if (rc != MLA_OK) return rc;
+  // the fused steps over the compacted rows; every query sees all its rows
+  return mla_fused_norm_rope_attn_rope_cast(
+      q_raw, norm_gain, eps, rope_base, positions, ws + w.rows_off,
+      reinterpret_cast<int32_t*>(ws + w.bt_off), w.pages_per_pair, static_cast<int>(pages),
+      reinterpret_cast<int32_t*>(ws + w.len_off), batch, h_q, softmax_scale,
+      reinterpret_cast<int32_t*>(ws + w.meta_off), reinterpret_cast<int32_t*>(ws + w.splits_off),
+      num_sm_parts, ws + w.dense_off, w.dense_bytes, out_e4m3, out_scale, lse, stream);
 }
 
 int mla_sparse_decode_v41_fp4(const void* q, const uint8_t* kcache_288, int64_t num_slots,

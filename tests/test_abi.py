@@ -86,6 +86,14 @@ def test_sparse_and_fused_validation():
     rc = L.mla_sparse_decode_v41(16, 16, 100, 16, 2048, 0, 1, 128, 0.04, 74, 256, 1 << 30, 16,
                                  16, None)
     assert rc == B.MLA_OK  # empty batch: nothing launched
+    rc = L.mla_sparse_fused_norm_rope_attn_rope_cast(16, 16, 1e-6, 1e4, None, 16, 100, 16, 2048,
+                                                     2, 64, 0.04, 74, 256, 1 << 30, 16, 16, 16,
+                                                     None)
+    assert rc == B.MLA_ERR_INVALID_ARG  # positions are required
+    assert "positions" in L.mla_last_error().decode()
+    rc = L.mla_sparse_fused_norm_rope_attn_rope_cast(16, 16, 1e-6, 1e4, 16, 16, 100, 16, 2048,
+                                                     2, 64, 0.04, 74, 256, 4096, 16, 16, 16, None)
+    assert rc == B.MLA_ERR_INVALID_ARG  # workspace too small
     rc = L.mla_fused_norm_rope_attn_rope_cast(16, 16, -1.0, 1e4, None, 16, 16, 4, 8, 16, 2, 64,
                                               0.04, 16, 16, 4, 16, 1 << 30, 16, 16, 16, None)
     assert rc == B.MLA_ERR_INVALID_ARG  # eps < 0
@@ -99,6 +107,7 @@ def test_size_queries():
     n = B.mla_workspace_size(64, 128, 512, 74)
     assert n >= (64 + 74) * 128 * 512 * 4
     assert B.mla_sparse_workspace_size(32, 1, 128, 2048, 512, 74) > n // 2
+    assert B.mla_sparse_fused_workspace_size(32, 64, 2048, 148) >= 32 * 2048 * 576 * 2
     # the V4.1 workspace adds the query widened to 576 dims
     assert (B.mla_sparse_v41_workspace_size(32, 1, 128, 2048, 74) >=
             B.mla_sparse_workspace_size(32, 1, 128, 2048, 512, 74) + 32 * 128 * 576 * 2)
