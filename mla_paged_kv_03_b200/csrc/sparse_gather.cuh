@@ -63,6 +63,18 @@ __device__ __forceinline__ bool gather_valid(int idx, long long num_slots) {
   return idx >= 0 && static_cast<long long>(idx) < num_slots;
 }
 
+// a * b rounded to odd in fp32: the truncated product, with its last bit set
+// when the product was inexact.  Rounding that to nearest bf16 (16 bits
+// shorter) gives the correctly rounded bf16 of the exact product, with no
+// double-rounding error (rounding to odd: Boldo and Melquiond, "Emulation of
+// FMA and correctly rounded sums: proved algorithms using rounding to odd",
+// IEEE Transactions on Computers 57(4), 2008).
+__device__ __forceinline__ float mul_round_odd(float a, float b) {
+  const float p = __fmul_rz(a, b);
+  const float e = __fmaf_rz(a, b, -p);  // the exact remainder of the truncation
+  return e != 0.f ? __uint_as_float(__float_as_uint(p) | 1u) : p;
+}
+
 // Eight E2M1 codes (4 bytes, low nibble first) -> four f16x2 pairs through the
 // hardware pair conversion (byte j -> pair j, low nibble -> low half).
 __device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t w, uint32_t (&h)[4]) {
@@ -78,7 +90,7 @@ __device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t w, uint32_t (&h)[4]) {
 
 // grid (pages_per_pair, pairs): CTA (c, b) handles indices [64c, 64c + 64) of pair b.
 template <int kRowBytes>
-__global__ void __launch_bounds__(kGatherCtaThreads)
+__global__ void __launch_bounds__(kGatherCtaThreads, 3)  // 3 CTAs (24 warps) per SM
     mla_sparse_gather_kernel(const GatherParams G) {
   static_assert(kRowBytes == kRow656 || kRowBytes == kRow528 || kRowBytes == kRow288,
                 "656-, 528- or 288-byte rows");
@@ -233,8 +245,9 @@ __global__ void __launch_bounds__(kGatherCtaThreads)
         asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h1) : "h"(hi16));
         const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&h0));
         const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&h1));
-        r[2 * q] = ptx::pack_bf16x2(f0.x * scl, f0.y * scl);
-        r[2 * q + 1] = ptx::pack_bf16x2(f1.x * scl, f1.y * scl);
+        // code * scale rounded once to bf16 (exact for the E8M0 scales)
+        r[2 * q] = ptx::pack_bf16x2(mul_round_odd(f0.x, scl), mul_round_odd(f0.y, scl));
+        r[2 * q + 1] = ptx::pack_bf16x2(mul_round_odd(f1.x, scl), mul_round_odd(f1.y, scl));
       }
       *reinterpret_cast<uint4*>(orow + 16 * u) = make_uint4(r[0], r[1], r[2], r[3]);
       *reinterpret_cast<uint4*>(orow + 16 * u + 8) = make_uint4(r[4], r[5], r[6], r[7]);

@@ -47,6 +47,8 @@
  *  - Fused path: the normalised, rotated query enters the attention in bf16
  *    (the tensor-core operand precision); the pages leave this precision
  *    open, and fixing it makes the FP8 code decisions comparable.
+ *  - Sparse paths: the dequantised rows enter the attention rounded to bf16
+ *    (round to nearest even), as the quantised decoding kernels convert them.
  *  - V4.1 rows: the latent is 512 wide, q . K runs over all 512 dims and V is
  *    the whole latent (d_v = 512).  An E8M0 byte e is the power of two
  *    2^(e - 127); 0xFF is NaN.  In the FP4 row, code 2i sits in the low
@@ -270,9 +272,20 @@ typedef struct {
   const int32_t* slots;
 } fp8_ctx;
 
+/* The attention sees a dequantised row rounded to bf16 (RNE): the quantised
+ * decoding kernels convert their dequantised values with round-to-nearest to
+ * bf16 pairs for the tensor cores [FlashMLA (AI Wiki), "Requirements and
+ * build", NVIDIA toolchain row].  Exact for the V4.1 rows, whose values are
+ * bf16 numbers already. */
+static void round_row_bf16(double* out, int n) {
+  int d;
+  for (d = 0; d < n; ++d) out[d] = oracle_round_bf16(out[d]);
+}
+
 static void fetch_fp8(const void* vctx, int j, double* out) {
   const fp8_ctx* c = (const fp8_ctx*)vctx;
   oracle_decode_row656(c->cache + (size_t)c->slots[j] * ORACLE_ROW656, out);
+  round_row_bf16(out, ORACLE_D);
 }
 
 /* Number of tokens query i (of s_q) of a sequence of length L may see. */
@@ -492,6 +505,7 @@ void oracle_decode_row528(const uint8_t* row, double* out) {
 static void fetch_row528(const void* vctx, int j, double* out) {
   const fp8_ctx* c = (const fp8_ctx*)vctx;
   oracle_decode_row528(c->cache + (size_t)c->slots[j] * ORACLE_ROW528, out);
+  round_row_bf16(out, ORACLE_D41);
 }
 
 /* E2M1 (a 4-bit code): sign, 2 exponent bits with bias 1, 1 mantissa bit;
@@ -516,6 +530,7 @@ void oracle_decode_row288(const uint8_t* row, double* out) {
 static void fetch_row288(const void* vctx, int j, double* out) {
   const fp8_ctx* c = (const fp8_ctx*)vctx;
   oracle_decode_row288(c->cache + (size_t)c->slots[j] * ORACLE_ROW288, out);
+  round_row_bf16(out, ORACLE_D41);
 }
 
 /* Token-level sparse decode over a 512-dim V4.1 cache of `row_bytes`-byte

@@ -421,6 +421,12 @@ def dequant_cache_torch(cache):
     return torch.cat([nope.view(-1, 512), rope], dim=1)
 
 
+def attention_rows(rows):
+    """What the attention sees: the dequantised rows rounded to bf16 by torch
+    (round to nearest even)."""
+    return dequant_cache_torch(rows).to(torch.bfloat16).to(torch.float64)
+
+
 def test_row656_decode_matches_torch_and_encoder_error_bound():
     g = torch.Generator().manual_seed(0)
     x = torch.randn((64, 512), generator=g)
@@ -449,7 +455,7 @@ def sparse_small(seed=0, seqlens=(300, 130), topk=96, h_q=3, invalid_frac=0.05):
 def test_sparse_matches_sdpa_on_dequantised_rows():
     case = sparse_small()
     o, lse = oracle.sparse_decode(case.q, case.kcache, case.indices, 512, case.softmax_scale)
-    K = dequant_cache_torch(case.kcache)
+    K = attention_rows(case.kcache)
     for b in range(case.batch):
         idx = case.indices[b, 0]
         sel = K[idx[idx >= 0].long()]
@@ -470,7 +476,7 @@ def test_sparse_all_tokens_equals_dense_noncausal():
     phys = case.block_table[0].long()[t // 64] * 64 + t % 64
     idx = phys.to(torch.int32).view(1, 1, L)
     o, lse = oracle.sparse_decode(case.q, case.kcache, idx, 512, case.softmax_scale)
-    K = dequant_cache_torch(case.kcache)[phys]
+    K = attention_rows(case.kcache)[phys]
     q = case.q[0, 0].to(torch.float64)
     ro = F.scaled_dot_product_attention(q[None], K[None], K[None, :, :512],
                                         scale=case.softmax_scale)[0]

@@ -1,7 +1,8 @@
 """Pins of the oracle's fused decode in sparse mode (the fused steps over the
 valid slots of a 656-byte FP8 cache) against facts that do not come from the
 oracle: the same step chain built from library routines (torch rms_norm,
-complex rotation, SDPA over torch-dequantised rows, the float8_e4m3fn cast),
+complex rotation, SDPA over torch-dequantised rows rounded to bf16, the
+float8_e4m3fn cast),
 and its reduction to the dense fused oracle when the slots are a sequence's
 tokens in order."""
 import numpy as np
@@ -10,13 +11,13 @@ import torch.nn.functional as F
 
 import oracle
 from mla_paged_kv_03_b200 import workloads as W
-from test_oracle_pins import dequant_cache_torch
+from test_oracle_pins import attention_rows, dequant_cache_torch
 
 
 def library_chain(case):
     b, _, h, _ = case.q_raw.shape
     theta_k = case.rope_base ** (-np.arange(32) * 2.0 / 64.0)
-    K_all = dequant_cache_torch(case.kcache)
+    K_all = attention_rows(case.kcache)
     codes = np.zeros((b, h, 576), dtype=np.uint8)
     scales = np.zeros((b, h))
     lses = np.zeros((b, h))
