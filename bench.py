@@ -335,9 +335,11 @@ class ClockSampler:
 
 
 def sample_clocks_start(dev_index):
-    path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{os.getpid()}.csv")
+    """Fallback when NVML is unavailable: nvidia-smi sampling every 200 ms into
+    a temporary CSV."""
+    import tempfile
+    path = os.path.join(tempfile.gettempdir(), f"mla_bench_clocks_{os.getpid()}.csv")
     try:
-        os.makedirs(os.path.dirname(path), exist_ok=True)
         f = open(path, "w")
         p = subprocess.Popen(
             ["nvidia-smi", f"--id={dev_index}",
