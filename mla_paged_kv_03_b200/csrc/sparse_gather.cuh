@@ -89,8 +89,15 @@ __device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t w, uint32_t (&h)[4]) {
 }
 
 // grid (pages_per_pair, pairs): CTA (c, b) handles indices [64c, 64c + 64) of pair b.
+// Register caps: the FP8 variants would take about 100 registers (2 CTAs per
+// SM) and are held to 3 CTAs; the FP4 variant fits 4.
 template <int kRowBytes>
-__global__ void __launch_bounds__(kGatherCtaThreads, 3)  // 3 CTAs (24 warps) per SM
+constexpr int gather_min_ctas() {
+  return kRowBytes == kRow288 ? 4 : 3;
+}
+
+template <int kRowBytes>
+__global__ void __launch_bounds__(kGatherCtaThreads, gather_min_ctas<kRowBytes>())
     mla_sparse_gather_kernel(const GatherParams G) {
   static_assert(kRowBytes == kRow656 || kRowBytes == kRow528 || kRowBytes == kRow288,
                 "656-, 528- or 288-byte rows");
@@ -245,9 +252,15 @@ __global__ void __launch_bounds__(kGatherCtaThreads, 3)  // 3 CTAs (24 warps) pe
         asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h1) : "h"(hi16));
         const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&h0));
         const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&h1));
-        // code * scale rounded once to bf16 (exact for the E8M0 scales)
-        r[2 * q] = ptx::pack_bf16x2(mul_round_odd(f0.x, scl), mul_round_odd(f0.y, scl));
-        r[2 * q + 1] = ptx::pack_bf16x2(mul_round_odd(f1.x, scl), mul_round_odd(f1.y, scl));
+        // code * scale rounded once to bf16; with the power-of-two E8M0 scales
+        // the product is exact already
+        if (kV41) {
+          r[2 * q] = ptx::pack_bf16x2(f0.x * scl, f0.y * scl);
+          r[2 * q + 1] = ptx::pack_bf16x2(f1.x * scl, f1.y * scl);
+        } else {
+          r[2 * q] = ptx::pack_bf16x2(mul_round_odd(f0.x, scl), mul_round_odd(f0.y, scl));
+          r[2 * q + 1] = ptx::pack_bf16x2(mul_round_odd(f1.x, scl), mul_round_odd(f1.y, scl));
+        }
       }
       *reinterpret_cast<uint4*>(orow + 16 * u) = make_uint4(r[0], r[1], r[2], r[3]);
       *reinterpret_cast<uint4*>(orow + 16 * u + 8) = make_uint4(r[4], r[5], r[6], r[7]);
