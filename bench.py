@@ -252,6 +252,21 @@ class GpuStep:
     def query(self):
         return self.case.q_raw if self.kind in ("fused", "fused_sparse") else self.case.q
 
+    def with_own_buffers(self):
+        """A second handle on the same inputs with its own outputs, workspace
+        and scheduler buffers, so that two steps can be in flight at once."""
+        import copy
+        other = copy.copy(self)
+        other.out = torch.empty_like(self.out)
+        other.lse = torch.empty_like(self.lse)
+        other.ws = torch.empty_like(self.ws)
+        if hasattr(self, "scale"):
+            other.scale = torch.empty_like(self.scale)
+        if hasattr(self, "meta"):
+            other.meta = torch.empty_like(self.meta)
+            other.ns = torch.empty_like(self.ns)
+        return other
+
     def outputs(self):
         return [self.out, self.lse] + ([self.scale] if self.kind in ("fused", "fused_sparse")
                                        else [])
@@ -462,31 +477,52 @@ def run_gpu_arm(args, rank, world):
         torch.distributed.barrier()
     clocks = sampler.stop() if clk is None else sample_clocks_stop(clk)
 
-    # end to end through the same API with host buffers: H2D of the step's
-    # query from pinned memory, the step, D2H of the outputs
+    # end to end through the same API with host buffers: every step copies its
+    # query in from pinned host memory, runs, and copies O and LSE back.  Two
+    # steps are in flight on two streams, each with its own device buffers, so
+    # one step's copies overlap the other's kernels as a serving loop runs
+    # them; the region ends when both streams have drained.
+    ref_out = gs.out.cpu()
     q_dev = gs.query()
     q_host = q_dev.cpu().pin_memory()
-    q_buf = torch.empty_like(q_dev)
-    out_host = torch.empty(gs.out.shape, dtype=gs.out.dtype).pin_memory()
-    lse_host = torch.empty(gs.lse.shape, dtype=gs.lse.dtype).pin_memory()
-    e2e_steps = max(3, min(args.steps, 50))
-    for _ in range(2):
-        q_buf.copy_(q_host, non_blocking=True)
-        gs.step(q_buf)
-        out_host.copy_(gs.out, non_blocking=True)
-        lse_host.copy_(gs.lse, non_blocking=True)
+    slots = [gs, gs.with_own_buffers()]
+    streams = [torch.cuda.Stream(dev) for _ in slots]
+    q_bufs = [torch.empty_like(q_dev) for _ in slots]
+    out_hosts = [torch.empty(gs.out.shape, dtype=gs.out.dtype).pin_memory() for _ in slots]
+    lse_hosts = [torch.empty(gs.lse.shape, dtype=gs.lse.dtype).pin_memory() for _ in slots]
+    has_scale = hasattr(gs, "scale")  # fused outputs: codes, scales and LSE
+    scale_hosts = [torch.empty(gs.scale.shape, dtype=gs.scale.dtype).pin_memory()
+                   for _ in slots] if has_scale else None
+
+    def e2e_step(i):
+        k = i % len(slots)
+        with torch.cuda.stream(streams[k]):
+            q_bufs[k].copy_(q_host, non_blocking=True)
+            slots[k].step(q_bufs[k])
+            out_hosts[k].copy_(slots[k].out, non_blocking=True)
+            lse_hosts[k].copy_(slots[k].lse, non_blocking=True)
+            if has_scale:
+                scale_hosts[k].copy_(slots[k].scale, non_blocking=True)
+
+    e2e_steps = max(4, min(args.steps, 50))
+    torch.cuda.synchronize(dev)
+    for i in range(4):
+        e2e_step(i)
     torch.cuda.synchronize(dev)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(st)
-    for _ in range(e2e_steps):
-        q_buf.copy_(q_host, non_blocking=True)
-        gs.step(q_buf)
-        out_host.copy_(gs.out, non_blocking=True)
-        lse_host.copy_(gs.lse, non_blocking=True)
+    for sk in streams:
+        sk.wait_event(e0)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    for sk in streams:
+        st.wait_stream(sk)
     e1.record(st)
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if not all(torch.equal(h, ref_out) for h in out_hosts):
+        raise RuntimeError("end-to-end outputs differ from the device-timed step's")
     status = gs.B.device_status()
     if status != 0:
         raise RuntimeError(f"device status {status:#x} after timing")
@@ -540,8 +576,9 @@ def run_gpu_arm(args, rank, world):
         "e2e": {"value": round(flops_all / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOPS",
                 "h2d_bytes_per_step": int(q_dev.numel() * q_dev.element_size()),
                 "d2h_bytes_per_step": int(gs.out.numel() * gs.out.element_size() +
-                                          gs.lse.numel() * 4),
-                "ms_per_step": round(e2e_ms, 5)},
+                                          gs.lse.numel() * 4 +
+                                          (gs.scale.numel() * 4 if hasattr(gs, "scale") else 0)),
+                "ms_per_step": round(e2e_ms, 5), "steps_in_flight": 2},
         "gpu_launches": gs.launches_per_step() * args.steps,
         "roofline": roof,
         "clocks": clocks,
