@@ -38,7 +38,7 @@ constexpr int kGatherCtaThreads = 256;
 constexpr int kRowUnits = kD / 8;  // 16-byte bf16 output units per row (72)
 
 struct GatherParams {
-  const uint8_t* cache;     // [num_slots, 656] or [num_slots, 528]
+  const uint8_t* cache;     // [num_slots, 656], [num_slots, 528] or [num_slots, 288]
   long long num_slots;
   const int32_t* indices;   // [pairs, topk]
   int topk;
@@ -46,7 +46,8 @@ struct GatherParams {
   __nv_bfloat16* rows;      // [pairs * pages_per_pair * 64, 576]
   int32_t* block_table;     // [pairs, pages_per_pair]
   int32_t* seqlens;         // [pairs]
-  // 528-byte format only: query rows [pairs * h_q, 512] -> [pairs * h_q, 576]
+  // V4.1 rows (528 / 288 bytes) only: query rows [pairs * h_q, 512] are
+  // widened into [pairs * h_q, 576]
   const __nv_bfloat16* q512;
   __nv_bfloat16* q576;
   int h_q;
