@@ -93,3 +93,23 @@ def test_plan_rejects_bad_arguments():
         B.mla_get_metadata_host([5], 16, 0)
     with pytest.raises(B.MLAError):
         B.mla_get_metadata_host([5], 16, 4, h_kv=2)
+
+
+try:
+    from hypothesis import given, settings, strategies as st
+
+    @settings(max_examples=200, deadline=None)
+    @given(seqlens=st.lists(st.one_of(st.integers(0, 300), st.integers(1000, 70000)),
+                            min_size=1, max_size=120),
+           parts_n=st.integers(1, 600))
+    def test_plan_property_coverage_and_balance(seqlens, parts_n):
+        """Any length mix and partition count: every (sequence, tile) pair is
+        covered exactly once, in order, and no part exceeds the target width
+        by more than one segment overhead."""
+        meta, ns, parts = check_plan(seqlens, parts_n)
+        total = sum(tiles_of(L) + OVERHEAD for L in seqlens)
+        target = -(-total // parts_n)
+        for segs in parts:
+            assert sum(hi - lo + OVERHEAD for (_, lo, hi, _) in segs) <= target + OVERHEAD + 1
+except ImportError:  # pragma: no cover
+    pass
