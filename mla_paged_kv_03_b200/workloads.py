@@ -21,6 +21,9 @@ Workloads (shapes and distributions as specified for this library):
                 q [b, s_q, h_q, 512].
 * ``sparse_v41_fp4`` the same over 288-byte V4.1 FP4 rows: 512 e2m1 codes
                 packed two per byte + 32 e4m3 scales (one per 16 values).
+* ``sparse_prefill`` token-level sparse prefill, no batch dimension: s_q =
+                s_kv = 4096, h_q=128, topk=2048 rows at or before each
+                token's position, per-token top-k length, one sink per head.
 * ``fused_sparse`` the fused decode in sparse mode: fused-workload queries
                 (h_q=64, gain ~ N(1, 0.1)) over the sparse workload's FP8
                 cache and indices, position L - 1.
@@ -403,6 +406,47 @@ def fused_sparse(seed=0, device="cpu", batch=32, h_q=64, seqlen=65536, topk=2048
                            name="fused_sparse")
 
 
+@dataclass
+class PrefillCase:
+    q: torch.Tensor            # [s_q, h_q, 576] bf16
+    kv: torch.Tensor           # [s_kv, 576] bf16, one latent KV head
+    indices: torch.Tensor      # [s_q, topk] int32 rows of kv, -1 = unused
+    topk_length: Optional[torch.Tensor]  # [s_q] int32 or None
+    attn_sink: Optional[torch.Tensor]    # [h_q] fp32 or None
+    h_q: int
+    topk: int
+    softmax_scale: float
+    d_v: int = D_NOPE
+    name: str = ""
+
+    @property
+    def s_q(self):
+        return int(self.q.shape[0])
+
+
+def sparse_prefill(seed=0, device="cpu", s_q=4096, s_kv=4096, h_q=128, topk=2048,
+                   with_length=True, with_sink=True):
+    """Sparse prefill without a batch dimension: query token t sits at
+    position s_kv - s_q + t and draws min(topk, position + 1) distinct rows of
+    kv at or before its position (the rest -1); topk_length[t] is that count;
+    one attention-sink logit per head ~ N(0, 1); q, kv ~ N(0, 1) in bf16."""
+    g = _gen(seed, device)
+    kv = _randn_bf16((s_kv, D_QK), g, chunk_rows=4096)
+    q = _randn_bf16((s_q, h_q, D_QK), g)
+    idx = torch.full((s_q, topk), -1, dtype=torch.int32, device=g.device)
+    lengths = torch.empty((s_q,), dtype=torch.int32)
+    for t in range(s_q):
+        pos = s_kv - s_q + t
+        k = min(topk, pos + 1)
+        idx[t, :k] = torch.randperm(pos + 1, generator=g, device=g.device)[:k].to(torch.int32)
+        lengths[t] = k
+    sink = torch.randn((h_q,), generator=g, device=g.device, dtype=torch.float32)
+    return PrefillCase(q=q.to(device), kv=kv.to(device), indices=idx.to(device),
+                       topk_length=lengths.to(device) if with_length else None,
+                       attn_sink=sink.to(device) if with_sink else None, h_q=h_q, topk=topk,
+                       softmax_scale=default_scale(), name="sparse_prefill")
+
+
 WORKLOADS = {
     "tiny": tiny,
     "compute": compute_bound,
@@ -412,4 +456,5 @@ WORKLOADS = {
     "sparse_v41": sparse_v41,
     "sparse_v41_fp4": sparse_v41_fp4,
     "fused_sparse": fused_sparse,
+    "sparse_prefill": sparse_prefill,
 }

@@ -81,6 +81,10 @@ def lib():
             u16p, f64p, ctypes.c_double, ctypes.c_double, i32p, u8p, ctypes.c_int64, i32p,
             ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double, i64p, ctypes.c_int64,
             u8p, f64p, f64p]
+        L.oracle_sparse_prefill.restype = ctypes.c_int
+        L.oracle_sparse_prefill.argtypes = [
+            u16p, u16p, ctypes.c_int64, i32p, i32p, f64p, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, ctypes.c_int, ctypes.c_double, i64p, ctypes.c_int64, f64p, f64p]
         _LIB = L
     return _LIB
 
@@ -359,3 +363,34 @@ def fused_sparse_decode(q_raw, gain, eps, rope_base, positions, kcache656, indic
     if ra is None:
         return codes.reshape(b, 1, h_q, _D), scale.reshape(b, 1, h_q), lse.reshape(b, 1, h_q)
     return codes, scale, lse
+
+
+def sparse_prefill(q, kv, indices, softmax_scale, d_v=512, topk_length=None, attn_sink=None,
+                   rows=None):
+    """oracle_sparse_prefill.  q [s_q, h_q, 576] bf16; kv [s_kv, 576] bf16;
+    indices [s_q, topk] int32 (-1 = invalid); topk_length [s_q] int32 or None;
+    attn_sink [h_q] or None.  Returns O [s_q, h_q, d_v] and LSE [s_q, h_q]
+    (or the sampled rows)."""
+    s_q, h_q, dq = q.shape
+    assert dq == _D
+    qa = _np(q, np.uint16)
+    ka = _np(kv, np.uint16).reshape(-1, _D)
+    ix = _np(indices, np.int32).reshape(s_q, -1)
+    topk = ix.shape[-1]
+    tl = None if topk_length is None else _np(topk_length, np.int32)
+    sk = None if attn_sink is None else np.ascontiguousarray(_np(attn_sink, np.float32),
+                                                             dtype=np.float64)
+    ra = None if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    n = s_q * h_q if ra is None else ra.size
+    out = np.zeros((n, d_v), dtype=np.float64)
+    lse = np.zeros(n, dtype=np.float64)
+    rc = lib().oracle_sparse_prefill(
+        _ptr(qa, ctypes.c_uint16), _ptr(ka, ctypes.c_uint16), ka.shape[0], _ptr(ix, ctypes.c_int32),
+        _ptr(tl, ctypes.c_int32), _ptr(sk, ctypes.c_double), s_q, h_q, topk, d_v,
+        float(softmax_scale), _ptr(ra, ctypes.c_int64), n, _ptr(out, ctypes.c_double),
+        _ptr(lse, ctypes.c_double))
+    if rc != 0:
+        raise ValueError("sparse index out of range")
+    if ra is None:
+        return out.reshape(s_q, h_q, d_v), lse.reshape(s_q, h_q)
+    return out, lse

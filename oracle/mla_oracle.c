@@ -197,20 +197,23 @@ void oracle_rope64(const double* x, double pos, double base, int sign, double* y
  * j-th attended token into out[576]. */
 typedef void (*row_fetch_fn)(const void* ctx, int j, double* out);
 
-/* Exact attention of one query row q[d_qk] over n tokens:
- *   s_t = scale * q . K_t ;  LSE = m + ln sum exp(s_t - m) ;
+/* Exact attention of one query row q[d_qk] over n tokens, with an optional
+ * attention-sink logit (-inf = none) that joins the normaliser without a
+ * value row:
+ *   s_t = scale * q . K_t ;  m = max(max_t s_t, sink) ;
+ *   LSE = m + ln (sum_t exp(s_t - m) + exp(sink - m)) ;
  *   O   = sum_t exp(s_t - LSE) * K_t[0:d_v]
  * Two passes over the rows (scores, then the weighted sum); n == 0 gives
- * O = 0, LSE = -inf. */
-static void attend_rows_d(const double* q, int d_qk, row_fetch_fn fetch, const void* ctx, int n,
-                          int d_v, double scale, double* o, double* lse) {
+ * O = 0, LSE = sink. */
+static void attend_rows_ds(const double* q, int d_qk, row_fetch_fn fetch, const void* ctx, int n,
+                           int d_v, double scale, double sink, double* o, double* lse) {
   int t, d;
-  double m = -INFINITY, sum = 0.0, l;
+  double m = sink, sum = 0.0, l;
   double k[ORACLE_D];
   double* s;
   for (d = 0; d < d_v; ++d) o[d] = 0.0;
   if (n == 0) {
-    *lse = -INFINITY;
+    *lse = sink;
     return;
   }
   s = (double*)malloc(sizeof(double) * (size_t)n);
@@ -222,6 +225,7 @@ static void attend_rows_d(const double* q, int d_qk, row_fetch_fn fetch, const v
     if (s[t] > m) m = s[t];
   }
   for (t = 0; t < n; ++t) sum += exp(s[t] - m);
+  if (sink != -INFINITY) sum += exp(sink - m);
   l = m + log(sum);
   for (t = 0; t < n; ++t) {
     double p = exp(s[t] - l);
@@ -230,6 +234,11 @@ static void attend_rows_d(const double* q, int d_qk, row_fetch_fn fetch, const v
   }
   *lse = l;
   free(s);
+}
+
+static void attend_rows_d(const double* q, int d_qk, row_fetch_fn fetch, const void* ctx, int n,
+                          int d_v, double scale, double* o, double* lse) {
+  attend_rows_ds(q, d_qk, fetch, ctx, n, d_v, scale, -INFINITY, o, lse);
 }
 
 static void attend_rows(const double* q, row_fetch_fn fetch, const void* ctx, int n, int d_v,
@@ -629,6 +638,69 @@ int oracle_fused_sparse_decode(const uint16_t* q_raw, const double* gain, double
     fused_row(q_raw + (size_t)flat * ORACLE_D, gain, eps, rope_base, (double)positions[b],
               fetch_fp8, &ctx, cnt, scale, codes + (size_t)r * ORACLE_D, out_scale + r, lse + r,
               0);
+    free(slots);
+  }
+  return bad ? -1 : 0;
+}
+
+/* ------------------------------------------------------- sparse prefill */
+
+/* bf16 latent rows [s_kv, 576] addressed by a list of row indices. */
+typedef struct {
+  const uint16_t* kv;
+  const int32_t* slots;
+} kv_rows_ctx;
+
+static void fetch_kv_row(const void* vctx, int j, double* out) {
+  const kv_rows_ctx* c = (const kv_rows_ctx*)vctx;
+  const uint16_t* row = c->kv + (size_t)c->slots[j] * ORACLE_D;
+  int d;
+  for (d = 0; d < ORACLE_D; ++d) out[d] = bf16_bits_to_f64(row[d]);
+}
+
+/* Token-level sparse prefill (no batch dimension).
+ *  q            [s_q, h_q, 576] bf16 bits
+ *  kv           [s_kv, 576] bf16 bits (one latent KV head)
+ *  indices      [s_q, topk] int32 rows of kv, -1 = invalid
+ *  topk_length  [s_q] or NULL: only indices[t][0 .. topk_length[t]) count
+ *  attn_sink    [h_q] or NULL: a per-head logit that joins the softmax
+ *               normaliser without a value row
+ *  out [rows, d_v], lse [rows] (rows of (t, h), or the sampled `rows`). */
+int oracle_sparse_prefill(const uint16_t* q, const uint16_t* kv, int64_t s_kv,
+                          const int32_t* indices, const int32_t* topk_length,
+                          const double* attn_sink, int s_q, int h_q, int topk, int d_v,
+                          double scale, const int64_t* rows, int64_t n_rows, double* out,
+                          double* lse) {
+  int64_t total = (int64_t)s_q * h_q;
+  int64_t n = rows ? n_rows : total;
+  int64_t r;
+  int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+  for (r = 0; r < n; ++r) {
+    int64_t flat = rows ? rows[r] : r;
+    int t = (int)(flat / h_q), h = (int)(flat % h_q);
+    const int32_t* idx = indices + (size_t)t * topk;
+    int len = topk_length ? topk_length[t] : topk;
+    const uint16_t* qr = q + (size_t)flat * ORACLE_D;
+    double qv[ORACLE_D];
+    int32_t* slots = (int32_t*)malloc(sizeof(int32_t) * (size_t)(topk > 0 ? topk : 1));
+    kv_rows_ctx ctx;
+    int j, d, cnt = 0;
+    if (len > topk) len = topk;
+    for (d = 0; d < ORACLE_D; ++d) qv[d] = bf16_bits_to_f64(qr[d]);
+    for (j = 0; j < len; ++j) {
+      int32_t s = idx[j];
+      if (s < 0) continue;
+      if ((int64_t)s >= s_kv) {
+        bad = 1;
+        continue;
+      }
+      slots[cnt++] = s;
+    }
+    ctx.kv = kv;
+    ctx.slots = slots;
+    attend_rows_ds(qv, ORACLE_D, fetch_kv_row, &ctx, cnt, d_v, scale,
+                   attn_sink ? attn_sink[h] : -INFINITY, out + (size_t)r * d_v, lse + r);
     free(slots);
   }
   return bad ? -1 : 0;
