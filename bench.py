@@ -51,6 +51,10 @@ WORKLOAD_INFO = {
     "fused_sparse": ("Fused RMSNorm-RoPE-attn-conjRoPE-FP8 decode in sparse mode over the FP8 "
                      "656-byte cache: batch 32, s_q 1, h_q 64, d 576, d_v 576, 65536-token cache "
                      "per sequence, topk 2048, 5% -1 slots, position L - 1", "tensor"),
+    "sparse_prefill": ("Token-level sparse prefill, bf16 latent KV, no batch dimension: s_q 4096 "
+                       "query tokens x h_q 128 over s_kv 4096 positions, topk 2048 rows at or "
+                       "before each token, per-token top-k length, one sink per head, d_qk 576, "
+                       "d_v 512", "tensor"),
     "sparse": ("Token-level sparse decode, FP8 656-byte cache: batch 32, s_q 1, h_q 128, d_v 512, "
                "65536-token cache per sequence, topk 2048, 5% -1 slots", "tensor"),
     "tiny": ("Tiny dense decode, bf16: batch 2, s_q 1, h_q 16, lengths {37, 200}", "tensor"),
@@ -145,6 +149,32 @@ def fused_sparse_work(case):
     return flops, kv_bytes, kv_bytes + io
 
 
+def prefill_work(case):
+    n = case.topk_length.cpu().clamp(0, case.topk) if case.topk_length is not None else None
+    ix = case.indices.cpu()
+    if n is not None:
+        ix = torch.where(torch.arange(case.topk)[None, :] < n[:, None], ix, torch.full_like(ix, -1))
+    valid = int((ix >= 0).sum())  # (token, row) pairs
+    flops = 2 * valid * (576 + case.d_v) * case.h_q
+    kv_bytes = valid * 1152
+    io = case.q.numel() * 2 + case.indices.numel() * 4 + case.s_q * case.h_q * (case.d_v * 2 + 4)
+    return flops, kv_bytes, kv_bytes + io
+
+
+def prefill_last_pass_work(case, chunk=32):
+    """Work of the prefill's last pass (its last `chunk` query tokens): the
+    attention kernel launch that the kernel events time."""
+    t0 = max(0, case.s_q - chunk)
+    ix = case.indices.cpu()[t0:]
+    if case.topk_length is not None:
+        n = case.topk_length.cpu()[t0:].clamp(0, case.topk)
+        ix = torch.where(torch.arange(case.topk)[None, :] < n[:, None], ix, torch.full_like(ix, -1))
+    valid = int((ix >= 0).sum())
+    flops = 2 * valid * (576 + case.d_v) * case.h_q
+    kv_bytes = valid * 1152
+    return flops, kv_bytes, kv_bytes + (case.s_q - t0) * case.h_q * (576 * 2 + case.d_v * 2 + 4)
+
+
 def sparse_dims(case):
     """(latent width of q . k, bytes per cache row) of a sparse case."""
     row = int(case.kcache.shape[-1])
@@ -187,6 +217,12 @@ class GpuStep:
             self.kind = "fused_sparse"
             self.work = fused_sparse_work(self.case)
             self.R = self.case.h_q
+        elif name == "sparse_prefill":
+            self.case = W.sparse_prefill(seed=seed, device=dev)
+            self.kind = "prefill"
+            self.work = prefill_work(self.case)
+            self.kernel_work = prefill_last_pass_work(self.case)
+            self.R = self.case.h_q
         elif name in ("sparse", "sparse_v41", "sparse_v41_fp4"):
             self.case = W.WORKLOADS[name](seed=seed, device=dev)
             self.kind = "sparse"
@@ -195,7 +231,16 @@ class GpuStep:
         else:
             raise ValueError(name)
         c = self.case
+        if not hasattr(self, "kernel_work"):
+            self.kernel_work = self.work  # one attention launch per step
         self.parts = B.mla_num_sm_parts(self.R, 1, dev)
+        if self.kind == "prefill":
+            self.out = torch.empty((c.s_q, c.h_q, c.d_v), dtype=torch.bfloat16, device=dev)
+            self.lse = torch.empty((c.s_q, c.h_q), dtype=torch.float32, device=dev)
+            self.ws = torch.empty((B.mla_sparse_prefill_workspace_size(c.s_q, c.h_q, c.topk,
+                                                                       self.parts),),
+                                  dtype=torch.uint8, device=dev)
+            return
         b = c.batch
         if self.kind == "dense":
             self.out = torch.empty((b, c.s_q, c.h_q, c.d_v), dtype=torch.bfloat16, device=dev)
@@ -221,7 +266,11 @@ class GpuStep:
             self.ns = torch.empty((b + 1,), dtype=torch.int32, device=dev)
 
     def launches_per_step(self):
-        # planner + attention kernel + combine (+ the FP8 gather for sparse)
+        # planner + attention kernel + combine (+ the FP8 gather for sparse);
+        # the prefill runs that sequence per pass of 32 tokens, then the sinks
+        if self.kind == "prefill":
+            c = self.case
+            return 4 * -(-c.s_q // 32) + (1 if c.attn_sink is not None else 0)
         return 4 if self.kind in ("sparse", "fused_sparse") else 3
 
     def step(self, q=None):
@@ -239,6 +288,11 @@ class GpuStep:
                 c.block_table, c.cache_seqlens, m, n, self.parts,
                 softmax_scale=c.softmax_scale, out=self.out, out_scale=self.scale, lse=self.lse,
                 workspace=self.ws)
+        elif self.kind == "prefill":
+            B.mla_sparse_prefill_fwd(c.q if q is None else q, c.kv, c.indices, c.softmax_scale,
+                                     topk_length=c.topk_length, attn_sink=c.attn_sink,
+                                     num_sm_parts=self.parts, out=self.out, lse=self.lse,
+                                     workspace=self.ws)
         elif self.kind == "fused_sparse":
             B.mla_sparse_fused_norm_rope_attn_rope_cast(
                 c.q_raw if q is None else q, c.gain, c.eps, c.rope_base, c.positions, c.kcache,
@@ -537,7 +591,10 @@ def run_gpu_arm(args, rank, world):
     desc, bound = WORKLOAD_INFO[args.workload]
     tflops = flops_all / (ms_step * 1e-3) / 1e12
     gbs = kv_all / (ms_step * 1e-3) / 1e9
-    # dominant kernel: the attention kernel, one launch per step, timed alone
+    # dominant kernel: the attention kernel, timed alone; for the prefill the
+    # events hold its last launch of the step (the last pass of 32 tokens), so
+    # that launch's own work is the numerator
+    flops, _, total_bytes = gs.kernel_work
     per_launch_s = ms_kernel * 1e-3
     traffic = load_traffic(args.workload)
     if bound == "tensor":
@@ -566,7 +623,7 @@ def run_gpu_arm(args, rank, world):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16" if "sparse" not in args.workload else
+        "dtype": "bf16" if ("sparse" not in args.workload or args.workload == "sparse_prefill") else
         "bf16 (fp4 cache dequantised)" if args.workload.endswith("fp4") else "bf16 (fp8 cache dequantised)",
         "data": "synthetic",
         "config": {"workload": desc, "name": args.workload,
@@ -608,7 +665,12 @@ def oracle_rows_timed(name, case, rows):
         return time.perf_counter() - t0
     c = case
     t0 = time.perf_counter()
-    if name == "fused_sparse":
+    if name == "sparse_prefill":
+        oracle.sparse_prefill(c.q.cpu(), c.kv.cpu(), c.indices.cpu(), c.softmax_scale,
+                              topk_length=None if c.topk_length is None else c.topk_length.cpu(),
+                              attn_sink=None if c.attn_sink is None else c.attn_sink.cpu(),
+                              rows=rows)
+    elif name == "fused_sparse":
         oracle.fused_sparse_decode(c.q_raw.cpu(), c.gain.cpu(), c.eps, c.rope_base,
                                    c.positions.cpu(), c.kcache_cpu, c.indices.cpu(),
                                    c.softmax_scale, rows=rows)
@@ -621,9 +683,26 @@ def oracle_rows_timed(name, case, rows):
     return time.perf_counter() - t0
 
 
+def total_rows_of(case):
+    """Query rows (token, head) of a workload's case."""
+    if isinstance(case, W.PrefillCase):
+        return case.s_q * case.h_q
+    return case.batch * (case.s_q if hasattr(case, "s_q") else 1) * case.h_q
+
+
 def row_flops(name, case, rows):
     """Algorithmic FLOPs of the sampled rows (same counting as the GPU arm)."""
     f = 0
+    if name == "sparse_prefill":
+        ix = case.indices.cpu()
+        if case.topk_length is not None:
+            n = case.topk_length.cpu().clamp(0, case.topk)
+            ix = torch.where(torch.arange(case.topk)[None, :] < n[:, None], ix,
+                             torch.full_like(ix, -1))
+        valid = (ix >= 0).sum(-1).tolist()
+        for r in rows:
+            f += 2 * valid[r // case.h_q] * (576 + case.d_v)
+        return f
     if name in ("compute", "memory", "tiny"):
         sl = case.cache_seqlens.cpu().tolist()
         for r in rows:
@@ -657,8 +736,9 @@ def cpu_baseline(name, seed=0, budget_s=15.0, case=None):
     import oracle
     if case is None:
         case = make_case(name, seed)
-    case.kcache_cpu = case.kcache.cpu()
-    total_rows = case.batch * (case.s_q if hasattr(case, "s_q") else 1) * case.h_q
+    if hasattr(case, "kcache"):
+        case.kcache_cpu = case.kcache.cpu()
+    total_rows = total_rows_of(case)
     rng = np.random.default_rng(seed)
     n = 8
     elapsed = oracle_rows_timed(name, case, np.sort(rng.choice(total_rows, n, replace=False)))
@@ -682,8 +762,9 @@ def run_reference_arm(args, rank, world):
     per_step = max(1.0, args.cpu_budget / max(1, args.steps + args.warmup))
     import numpy as np
     import oracle
-    case.kcache_cpu = case.kcache.cpu()
-    total_rows = case.batch * (case.s_q if hasattr(case, "s_q") else 1) * case.h_q
+    if hasattr(case, "kcache"):
+        case.kcache_cpu = case.kcache.cpu()
+    total_rows = total_rows_of(case)
     rng = np.random.default_rng(args.seed)
     t8 = oracle_rows_timed(name, case, np.sort(rng.choice(total_rows, 8, replace=False))) / 8
     n = int(min(total_rows, max(4, per_step / max(t8, 1e-6))))

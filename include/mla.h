@@ -221,6 +221,36 @@ MLA_API int mla_sparse_decode_v41_fp4(const void* q, const uint8_t* kcache_288, 
                               float softmax_scale, int num_sm_parts, void* workspace,
                               size_t workspace_bytes, void* out, float* lse, void* stream);
 
+/* Workspace bytes for mla_sparse_prefill_fwd (one pass of up to 32 query
+ * tokens: their gathered rows, tables and split partials). */
+MLA_API int mla_sparse_prefill_workspace_size(int s_q, int h_q, int topk, int num_sm_parts,
+                                      size_t* bytes);
+
+/* Token-level sparse prefill, with no batch dimension
+ * [FlashMLA (AI Wiki), "Interfaces": sparse prefill takes optional
+ * attention-sink and per-token top-k-length arguments].
+ *   q             [s_q, h_q, 576] bf16, one row per (query token, head)
+ *   kv            [s_kv, 576] bf16: the latent KV head, one row per position
+ *   indices       int32[s_q, topk]: rows of kv each query token attends to;
+ *                 -1 (or a value outside [0, s_kv)) marks an unused entry
+ *   topk_length   int32[s_q] or NULL: only the first topk_length[t] entries
+ *                 of token t's indices count (clamped to [0, topk])
+ *   attn_sink     fp32[h_q] or NULL: a per-head logit that joins the softmax
+ *                 normaliser without a value row: LSE' = log(e^LSE + e^sink),
+ *                 O' = O e^(LSE - LSE'); a token with no row gets O = 0 and
+ *                 LSE = sink
+ *   d_v           512 (V = kv[:, :512]); softmax_scale usually 1/sqrt(576)
+ *   out, lse      [s_q, h_q, 512] bf16 (16-byte aligned) and [s_q, h_q] fp32
+ *   num_sm_parts  from mla_num_sm_parts(device, h_q, 1)
+ * The tokens are processed in passes of 32 through the sparse decode path
+ * (gather of each token's rows, planner, decode, combine), then the sinks.
+ * Ownership and errors as in mla_sparse_decode. */
+MLA_API int mla_sparse_prefill_fwd(const void* q, const void* kv, int64_t s_kv,
+                           const int32_t* indices, int topk, const int32_t* topk_length,
+                           const float* attn_sink, int s_q, int h_q, int d_v,
+                           float softmax_scale, int num_sm_parts, void* workspace,
+                           size_t workspace_bytes, void* out, float* lse, void* stream);
+
 /* Workspace bytes for mla_sparse_fused_norm_rope_attn_rope_cast. */
 MLA_API int mla_sparse_fused_workspace_size(int batch, int h_q, int topk, int num_sm_parts,
                                     size_t* bytes);

@@ -31,7 +31,8 @@ EXPORTED = [
     "mla_device_status", "mla_noalloc_scratch_bytes", "mla_decode_fwd_noalloc",
     "mla_set_kernel_events", "mla_sparse_v41_workspace_size", "mla_sparse_decode_v41",
     "mla_sparse_decode_v41_fp4", "mla_sparse_fused_workspace_size",
-    "mla_sparse_fused_norm_rope_attn_rope_cast",
+    "mla_sparse_fused_norm_rope_attn_rope_cast", "mla_sparse_prefill_workspace_size",
+    "mla_sparse_prefill_fwd",
 ]
 
 
@@ -77,6 +78,9 @@ def lib():
                                             sz, vp, vp, vp]
         L.mla_sparse_decode_v41_fp4.argtypes = L.mla_sparse_decode_v41.argtypes
         L.mla_sparse_fused_workspace_size.argtypes = [i32, i32, i32, i32, szp]
+        L.mla_sparse_prefill_workspace_size.argtypes = [i32, i32, i32, i32, szp]
+        L.mla_sparse_prefill_fwd.argtypes = [vp, vp, i64, vp, i32, vp, vp, i32, i32, i32, f32,
+                                             i32, vp, sz, vp, vp, vp]
         L.mla_sparse_fused_norm_rope_attn_rope_cast.argtypes = [
             vp, vp, f32, f32, vp, vp, i64, vp, i32, i32, i32, f32, i32, vp, sz, vp, vp, vp, vp]
         L.mla_device_status.argtypes = [ip, i32]
@@ -172,6 +176,13 @@ def mla_sparse_fused_workspace_size(batch, h_q, topk, num_sm_parts) -> int:
     out = ctypes.c_size_t(0)
     _check(lib().mla_sparse_fused_workspace_size(int(batch), int(h_q), int(topk),
                                                  int(num_sm_parts), ctypes.byref(out)))
+    return int(out.value)
+
+
+def mla_sparse_prefill_workspace_size(s_q, h_q, topk, num_sm_parts) -> int:
+    out = ctypes.c_size_t(0)
+    _check(lib().mla_sparse_prefill_workspace_size(int(s_q), int(h_q), int(topk),
+                                                   int(num_sm_parts), ctypes.byref(out)))
     return int(out.value)
 
 
@@ -380,3 +391,39 @@ def mla_sparse_fused_norm_rope_attn_rope_cast(q_raw, norm_gain, eps, rope_base, 
         int(num_sm_parts), _ptr(ws), ws.numel(), _ptr(out), _ptr(out_scale), _ptr(lse),
         _stream(dev)))
     return out, out_scale, lse
+
+
+def mla_sparse_prefill_fwd(q, kv, indices, softmax_scale=None, d_v=512, topk_length=None,
+                           attn_sink=None, num_sm_parts=None, out=None, lse=None,
+                           workspace=None):
+    """Token-level sparse prefill (no batch dimension).  q [s_q, h_q, 576] bf16;
+    kv [s_kv, 576] bf16 (or [s_kv, 1, 576]); indices [s_q, topk] (or
+    [s_q, 1, topk]) int32 rows of kv (-1 = unused); topk_length [s_q] int32 or
+    None; attn_sink [h_q] fp32 or None.  Returns (out [s_q, h_q, d_v] bf16,
+    lse [s_q, h_q] fp32)."""
+    _require(q.dim() == 3 and q.shape[-1] == D_QK and q.dtype == torch.bfloat16,
+             "q must be [s_q, h_q, 576] bf16")
+    _require(kv.dtype == torch.bfloat16 and kv.shape[-1] == D_QK, "kv must be [s_kv, 576] bf16")
+    s_q, h_q, _ = q.shape
+    q = q.contiguous()
+    kv = kv.contiguous()
+    idx = indices.to(torch.int32).contiguous().view(s_q, -1)
+    topk = idx.shape[-1]
+    tl = None if topk_length is None else topk_length.to(torch.int32).contiguous()
+    sk = None if attn_sink is None else attn_sink.to(torch.float32).contiguous()
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(D_QK)
+    if num_sm_parts is None:
+        num_sm_parts = mla_num_sm_parts(h_q, 1, q.device)
+    dev = q.device
+    if out is None:
+        out = torch.empty((s_q, h_q, d_v), dtype=torch.bfloat16, device=dev)
+    if lse is None:
+        lse = torch.empty((s_q, h_q), dtype=torch.float32, device=dev)
+    ws = _workspace(mla_sparse_prefill_workspace_size(s_q, h_q, topk, num_sm_parts), dev,
+                    workspace)
+    _check(lib().mla_sparse_prefill_fwd(
+        _ptr(q), _ptr(kv), kv.numel() // D_QK, _ptr(idx), topk, _ptr(tl), _ptr(sk), s_q, h_q,
+        int(d_v), float(softmax_scale), int(num_sm_parts), _ptr(ws), ws.numel(), _ptr(out),
+        _ptr(lse), _stream(dev)))
+    return out, lse

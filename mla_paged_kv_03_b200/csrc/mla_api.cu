@@ -16,6 +16,7 @@
 #include "decode_kernel.cuh"
 #include "page_kernel.cuh"
 #include "pair_kernel.cuh"
+#include "sink_kernel.cuh"
 #include "sparse_gather.cuh"
 #include "mla_common.h"
 
@@ -367,20 +368,22 @@ int static_scratch_ptr(void** ptr) {
 static int sparse_gather_and_plan(int row_bytes, const void* q, const uint8_t* kcache,
                                   int64_t num_slots, const int32_t* indices, int topk, int pairs,
                                   int h_q, int num_sm_parts, uint8_t* ws, const SparseWs& w,
-                                  void* stream, const void** q_dense) {
+                                  void* stream, const void** q_dense,
+                                  const int32_t* topk_len = nullptr) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   mla::GatherParams g{};
   g.cache = kcache;
   g.num_slots = num_slots;
   g.indices = indices;
   g.topk = topk;
+  g.topk_len = topk_len;
   g.pages_per_pair = w.pages_per_pair;
   g.rows = reinterpret_cast<__nv_bfloat16*>(ws + w.rows_off);
   g.block_table = reinterpret_cast<int32_t*>(ws + w.bt_off);
   g.seqlens = reinterpret_cast<int32_t*>(ws + w.len_off);
   g.h_q = h_q;
   *q_dense = q;
-  if (row_bytes != mla::kRow656) {
+  if (row_bytes == mla::kRow528 || row_bytes == mla::kRow288) {
     g.q512 = static_cast<const __nv_bfloat16*>(q);
     g.q576 = reinterpret_cast<__nv_bfloat16*>(ws + w.q_off);
     *q_dense = g.q576;
@@ -390,6 +393,8 @@ static int sparse_gather_and_plan(int row_bytes, const void* q, const uint8_t* k
     mla::mla_sparse_gather_kernel<mla::kRow528><<<grid, mla::kGatherCtaThreads, 0, st>>>(g);
   } else if (row_bytes == mla::kRow288) {
     mla::mla_sparse_gather_kernel<mla::kRow288><<<grid, mla::kGatherCtaThreads, 0, st>>>(g);
+  } else if (row_bytes == mla::kRowBf16) {
+    mla::mla_sparse_gather_kernel<mla::kRowBf16><<<grid, mla::kGatherCtaThreads, 0, st>>>(g);
   } else {
     mla::mla_sparse_gather_kernel<mla::kRow656><<<grid, mla::kGatherCtaThreads, 0, st>>>(g);
   }
@@ -731,6 +736,77 @@ int mla_sparse_decode(const void* q, const uint8_t* kcache_fp8, int64_t num_slot
   return sparse_decode_impl(mla::kRow656, q, kcache_fp8, num_slots, indices, topk, batch, s_q, h_q,
                             d_v, softmax_scale, num_sm_parts, workspace, workspace_bytes, out, lse,
                             stream);
+}
+
+// Query tokens per pass of the sparse prefill: each pass gathers its tokens'
+// rows into the workspace (pages of 64 bf16 rows per token) and decodes them.
+constexpr int kPrefillChunk = 32;
+
+int mla_sparse_prefill_workspace_size(int s_q, int h_q, int topk, int num_sm_parts,
+                                      size_t* bytes) {
+  MLA_CHECK_ARG(bytes, "bytes is null");
+  MLA_CHECK_ARG(s_q >= 0 && h_q >= 1 && topk >= 1 && num_sm_parts >= 1, "bad sizes");
+  const int chunk = s_q < kPrefillChunk ? (s_q > 0 ? s_q : 1) : kPrefillChunk;
+  *bytes = sparse_ws_layout(chunk, topk, h_q, 512, num_sm_parts).total;
+  return MLA_OK;
+}
+
+int mla_sparse_prefill_fwd(const void* q, const void* kv, int64_t s_kv, const int32_t* indices,
+                           int topk, const int32_t* topk_length, const float* attn_sink, int s_q,
+                           int h_q, int d_v, float softmax_scale, int num_sm_parts,
+                           void* workspace, size_t workspace_bytes, void* out, float* lse,
+                           void* stream) {
+  MLA_CHECK_ARG(s_q >= 0 && h_q >= 1, "bad sizes");
+  MLA_CHECK_ARG(topk >= 1, "topk must be >= 1 (got %d)", topk);
+  MLA_CHECK_ARG(s_kv >= 1 && s_kv < (1LL << 31), "s_kv must be in [1, 2^31)");
+  MLA_CHECK_ARG(d_v == 512, "sparse prefill supports d_v = 512 (got %d)", d_v);
+  MLA_CHECK_ARG(num_sm_parts >= 1 && num_sm_parts <= mla::kCombineMaxSplits,
+                "num_sm_parts must be in [1, %d]", mla::kCombineMaxSplits);
+  MLA_CHECK_ARG(std::isfinite(softmax_scale) && softmax_scale > 0.f,
+                "softmax_scale must be finite and > 0");
+  MLA_CHECK_ARG(q && kv && indices && workspace && out && lse, "null device pointer");
+  MLA_CHECK_ARG(aligned(q, 16) && aligned(kv, 16) && aligned(out, 16),
+                "q, kv and out must be 16-byte aligned");
+  MLA_CHECK_ARG(aligned(workspace, 256), "workspace must be 256-byte aligned");
+  MLA_CHECK_ARG(aligned(lse, 4) && aligned(indices, 4) && aligned(topk_length, 4) &&
+                    aligned(attn_sink, 4),
+                "misaligned lse, indices, topk_length or attn_sink");
+  const int chunk = s_q < kPrefillChunk ? (s_q > 0 ? s_q : 1) : kPrefillChunk;
+  const SparseWs w = sparse_ws_layout(chunk, topk, h_q, d_v, num_sm_parts);
+  MLA_CHECK_ARG(workspace_bytes >= w.total, "workspace too small: %zu < %zu", workspace_bytes,
+                w.total);
+  MLA_CHECK_ARG(static_cast<long long>(chunk) * w.pages_per_pair * mla::kPage < (1LL << 31),
+                "topk too large");
+  if (s_q == 0) return MLA_OK;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const size_t q_row = static_cast<size_t>(h_q) * mla::kD;  // bf16 values per token
+  for (int t0 = 0; t0 < s_q; t0 += chunk) {
+    const int n = s_q - t0 < chunk ? s_q - t0 : chunk;
+    const void* q_t = static_cast<const __nv_bfloat16*>(q) + t0 * q_row;
+    const void* q_dense = q_t;
+    int rc = sparse_gather_and_plan(mla::kRowBf16, q_t, static_cast<const uint8_t*>(kv), s_kv,
+                                    indices + static_cast<size_t>(t0) * topk, topk, n, h_q,
+                                    num_sm_parts, ws, w, stream, &q_dense,
+                                    topk_length ? topk_length + t0 : nullptr);
+    if (rc != MLA_OK) return rc;
+    rc = mla_decode_fwd(q_dense, ws + w.rows_off, reinterpret_cast<int32_t*>(ws + w.bt_off),
+                        w.pages_per_pair, n * w.pages_per_pair,
+                        reinterpret_cast<int32_t*>(ws + w.len_off), n, 1, h_q, 1, d_v,
+                        softmax_scale, 0, reinterpret_cast<int32_t*>(ws + w.meta_off),
+                        reinterpret_cast<int32_t*>(ws + w.splits_off), num_sm_parts,
+                        ws + w.dense_off, w.dense_bytes,
+                        static_cast<__nv_bfloat16*>(out) + static_cast<size_t>(t0) * h_q * d_v,
+                        lse + static_cast<size_t>(t0) * h_q, stream);
+    if (rc != MLA_OK) return rc;
+  }
+  if (attn_sink) {
+    const long long rows = static_cast<long long>(s_q) * h_q;
+    const unsigned grid = static_cast<unsigned>((rows + mla::kSinkWarps - 1) / mla::kSinkWarps);
+    mla::mla_sink_kernel<<<grid, 32 * mla::kSinkWarps, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<__nv_bfloat16*>(out), lse, attn_sink, rows, h_q, d_v);
+    MLA_CUDA(cudaGetLastError());
+  }
+  return MLA_OK;
 }
 
 int mla_sparse_fused_workspace_size(int batch, int h_q, int topk, int num_sm_parts,

@@ -1,0 +1,51 @@
+// sink_kernel.cuh -- attention sinks of the sparse prefill: one logit per
+// head that joins the softmax normaliser without a value row.  For a row with
+// output O and log-sum-exp LSE over its tokens, and the head's sink logit s:
+//   LSE' = log(e^LSE + e^s),   O' = O * e^(LSE - LSE')
+// (a row without tokens keeps O = 0 and gets LSE' = s).  Applied in place
+// after the split combine.  [FlashMLA (AI Wiki), "Interfaces": sparse prefill
+// takes an optional attention-sink argument]
+#pragma once
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "ptx.cuh"
+
+namespace mla {
+
+constexpr int kSinkWarps = 8;
+
+// One warp per (token, head) row of `d_v` bf16 values (d_v a multiple of 8).
+__global__ void __launch_bounds__(32 * kSinkWarps)
+    mla_sink_kernel(__nv_bfloat16* out, float* lse, const float* sink, long long rows, int h_q,
+                    int d_v) {
+  const int lane = threadIdx.x & 31;
+  const long long row = static_cast<long long>(blockIdx.x) * kSinkWarps + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const float s = sink[row % h_q];
+  if (s == -INFINITY) return;
+  const float l = lse[row];
+  float lp, f;
+  if (l == -INFINITY) {
+    lp = s;
+    f = 0.f;
+  } else {
+    const float m = fmaxf(l, s);
+    lp = m + logf(expf(l - m) + expf(s - m));
+    f = expf(l - lp);
+  }
+  uint4* o = reinterpret_cast<uint4*>(out + row * d_v);
+  for (int u = lane; u < d_v / 8; u += 32) {
+    uint4 v = o[u];
+    uint32_t* w = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
+      w[e] = ptx::pack_bf16x2(x.x * f, x.y * f);
+    }
+    o[u] = v;
+  }
+  if (lane == 0) lse[row] = lp;
+}
+
+}  // namespace mla

@@ -10,6 +10,7 @@
 //    [16 x E8M0 scale, one per 32 codes]; a value is code * 2^(e - 127).
 //  - 288 bytes (V4.1 FP4): [512 x E2M1 codes, two per byte, code 2i in the
 //    low nibble of byte i][32 x E4M3 scale, one per 16 codes].
+//  - 1152 bytes: plain bf16 latent rows of 576 dims (sparse prefill), copied.
 //  For both V4.1 rows the buffer row stays 576 wide with dims 512..575 zero,
 //  and the 512-wide query rows are copied into a 576-wide buffer with zero
 //  dims 512..575, so that q . k and the first 512 dims of V are unchanged.
@@ -38,10 +39,11 @@ constexpr int kGatherCtaThreads = 256;
 constexpr int kRowUnits = kD / 8;  // 16-byte bf16 output units per row (72)
 
 struct GatherParams {
-  const uint8_t* cache;     // [num_slots, 656], [num_slots, 528] or [num_slots, 288]
+  const uint8_t* cache;     // [num_slots, row bytes]: 656, 528, 288 or 1152 (bf16)
   long long num_slots;
   const int32_t* indices;   // [pairs, topk]
   int topk;
+  const int32_t* topk_len;  // [pairs] or null: only indices[p][0, topk_len[p]) count
   int pages_per_pair;       // ceil(topk / 64)
   __nv_bfloat16* rows;      // [pairs * pages_per_pair * 64, 576]
   int32_t* block_table;     // [pairs, pages_per_pair]
@@ -91,18 +93,20 @@ __device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t w, uint32_t (&h)[4]) {
 
 // grid (pages_per_pair, pairs): CTA (c, b) handles indices [64c, 64c + 64) of pair b.
 // Register caps: the FP8 variants would take about 100 registers (2 CTAs per
-// SM) and are held to 3 CTAs; the FP4 variant fits 4.
+// SM) and are held to 3 CTAs; the FP4 and bf16 variants fit 4.
 template <int kRowBytes>
 constexpr int gather_min_ctas() {
-  return kRowBytes == kRow288 ? 4 : 3;
+  return (kRowBytes == kRow288 || kRowBytes == kRowBf16) ? 4 : 3;
 }
 
 template <int kRowBytes>
 __global__ void __launch_bounds__(kGatherCtaThreads, gather_min_ctas<kRowBytes>())
     mla_sparse_gather_kernel(const GatherParams G) {
-  static_assert(kRowBytes == kRow656 || kRowBytes == kRow528 || kRowBytes == kRow288,
-                "656-, 528- or 288-byte rows");
-  constexpr bool kV41 = kRowBytes != kRow656;  // 512-dim latent, query widened
+  static_assert(kRowBytes == kRow656 || kRowBytes == kRow528 || kRowBytes == kRow288 ||
+                    kRowBytes == kRowBf16,
+                "656-, 528-, 288- or 1152-byte rows");
+  constexpr bool kBf16 = kRowBytes == kRowBf16;
+  constexpr bool kV41 = kRowBytes == kRow528 || kRowBytes == kRow288;  // 512-dim latent
   constexpr bool kFp4 = kRowBytes == kRow288;
   __shared__ int s_red[kGatherCtaThreads / 32];
   __shared__ int s_idx[kGatherTokens];
@@ -112,10 +116,15 @@ __global__ void __launch_bounds__(kGatherCtaThreads, gather_min_ctas<kRowBytes>(
   const int c = blockIdx.x, b = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int32_t* idx_b = G.indices + (size_t)b * G.topk;
+  int lim = G.topk;  // entries past the pair's top-k length do not count
+  if (G.topk_len) {
+    const int l = __ldg(G.topk_len + b);
+    lim = l < 0 ? 0 : (l < G.topk ? l : G.topk);
+  }
 
   // valid tokens in the pair's earlier chunks: this chunk's first output row
   int cnt = 0;
-  for (int j = tid; j < c * kGatherTokens; j += kGatherCtaThreads)
+  for (int j = tid; j < c * kGatherTokens && j < lim; j += kGatherCtaThreads)
     cnt += gather_valid(__ldg(idx_b + j), G.num_slots) ? 1 : 0;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
@@ -124,9 +133,9 @@ __global__ void __launch_bounds__(kGatherCtaThreads, gather_min_ctas<kRowBytes>(
   // this chunk: validity and rank among the chunk's valid tokens (warps 0, 1)
   if (tid < kGatherTokens) {
     const int j = c * kGatherTokens + tid;
-    const int idx = j < G.topk ? __ldg(idx_b + j) : -1;
+    const int idx = j < lim ? __ldg(idx_b + j) : -1;
     bool v = gather_valid(idx, G.num_slots);
-    if (j < G.topk && idx >= 0 && !v) ptx::set_error(MLA_DEVERR_BAD_INDEX, 0x80);
+    if (j < lim && idx >= 0 && !v) ptx::set_error(MLA_DEVERR_BAD_INDEX, 0x80);
     const unsigned m = __ballot_sync(0xffffffffu, v);
     s_idx[tid] = idx;
     s_dst[tid] = v ? __popc(m & ((1u << lane) - 1)) : -1;  // rank within the warp
@@ -164,109 +173,133 @@ __global__ void __launch_bounds__(kGatherCtaThreads, gather_min_ctas<kRowBytes>(
           make_uint4(0, 0, 0, 0);
   }
 
-  // dequantise: per token 32 units of 16 codes (two 16-byte bf16 outputs
-  // each) and 8 units of the dims 512..575 (bf16 RoPE dims, or zeros for the
-  // 528-byte rows); all loads of a thread are issued before any conversion so
-  // that they overlap
-  constexpr int kUnits = kNope / 16 + kRope / 8;  // 40
-  constexpr int kPer = kGatherTokens * kUnits / kGatherCtaThreads;  // 10
-  static_assert(kGatherTokens * kUnits % kGatherCtaThreads == 0, "even split");
-  uint4 raw[kPer];
-  float sc[kPer];      // 656-byte rows: the fp32 scale
-  uint32_t eb[kPer];   // 528-byte rows: the E8M0 byte, converted after all loads
+  if constexpr (kBf16) {
+    // bf16 rows: each valid token's 72 16-byte units copied as they are, six
+    // units of a thread in flight at a time
+    constexpr int kItems = kGatherTokens * kRowUnits;  // 4608
+    constexpr int kBatch = 6;
+    static_assert(kItems % (kGatherCtaThreads * kBatch) == 0, "even split");
+    for (int i0 = 0; i0 < kItems; i0 += kGatherCtaThreads * kBatch) {
+      uint4 v[kBatch];
+      int dst[kBatch];
 #pragma unroll
-  for (int k = 0; k < kPer; ++k) {
-    const int item = tid + k * kGatherCtaThreads;
-    const int t = item / kUnits, u = item % kUnits;
-    raw[k] = make_uint4(0, 0, 0, 0);
-    sc[k] = 0.f;
-    eb[k] = 127u;
-    if (s_dst[t] >= 0) {
-      const uint8_t* row = G.cache + (size_t)s_idx[t] * kRowBytes;
-      if (u < kNope / 16 && kFp4) {
-        const uint2 v = __ldg(reinterpret_cast<const uint2*>(row) + u);  // 16 codes
-        raw[k] = make_uint4(v.x, v.y, 0u, 0u);
-        eb[k] = __ldg(row + kNope / 2 + u);
-      } else if (u < kNope / 16) {
-        raw[k] = __ldg(reinterpret_cast<const uint4*>(row) + u);
-        if (kV41)
-          eb[k] = __ldg(row + kNope + (u >> 1));
-        else
-          sc[k] = __ldg(reinterpret_cast<const float*>(row + kNope) + (u >> 3));
-      } else if (!kV41) {
-        raw[k] = __ldg(reinterpret_cast<const uint4*>(row + kNope + 16) + (u - kNope / 16));
+      for (int k = 0; k < kBatch; ++k) {
+        const int item = i0 + k * kGatherCtaThreads + tid;
+        const int t = item / kRowUnits, uu = item % kRowUnits;
+        dst[k] = s_dst[t] >= 0 ? s_dst[t] * kRowUnits + uu : -1;
+        v[k] = make_uint4(0, 0, 0, 0);
+        if (dst[k] >= 0)
+          v[k] = __ldg(reinterpret_cast<const uint4*>(G.cache + (size_t)s_idx[t] * kRowBytes) + uu);
       }
+#pragma unroll
+      for (int k = 0; k < kBatch; ++k)
+        if (dst[k] >= 0) reinterpret_cast<uint4*>(out_b)[dst[k]] = v[k];
     }
-  }
-  if (kV41) {
-    // the pair's query rows widened to 576 dims (72 16-byte units a row),
-    // spread over all pages_per_pair CTAs of the pair, while the row loads
-    // above are in flight
-    const int n_items = G.h_q * kRowUnits;
-    for (int item = c * kGatherCtaThreads + tid; item < n_items;
-         item += G.pages_per_pair * kGatherCtaThreads) {
-      const size_t r = (size_t)b * G.h_q + item / kRowUnits;
-      const int uu = item % kRowUnits;
-      const uint4 v = uu < kNope / 8
-                          ? __ldg(reinterpret_cast<const uint4*>(G.q512 + r * kNope) + uu)
-                          : make_uint4(0, 0, 0, 0);
-      *reinterpret_cast<uint4*>(G.q576 + r * kD + 8 * uu) = v;
-    }
-  }
-
+  } else {
+    // dequantise: per token 32 units of 16 codes (two 16-byte bf16 outputs
+    // each) and 8 units of the dims 512..575 (bf16 RoPE dims, or zeros for the
+    // 528-byte rows); all loads of a thread are issued before any conversion so
+    // that they overlap
+    constexpr int kUnits = kNope / 16 + kRope / 8;  // 40
+    constexpr int kPer = kGatherTokens * kUnits / kGatherCtaThreads;  // 10
+    static_assert(kGatherTokens * kUnits % kGatherCtaThreads == 0, "even split");
+    uint4 raw[kPer];
+    float sc[kPer];      // 656-byte rows: the fp32 scale
+    uint32_t eb[kPer];   // 528-byte rows: the E8M0 byte, converted after all loads
 #pragma unroll
-  for (int k = 0; k < kPer; ++k) {
-    const int item = tid + k * kGatherCtaThreads;
-    const int t = item / kUnits, u = item % kUnits;
-    const int dst = s_dst[t];
-    if (dst < 0) continue;
-    __nv_bfloat16* orow = out_b + (size_t)dst * kD;
-    if (u < kNope / 16 && kFp4) {
-      // code * scale in f16 is exact (at most 6 significant bits, |x| <= 2688),
-      // and so is its bf16 rounding
-      uint32_t s2;
-      asm("cvt.rn.f16x2.e4m3x2 %0, %1;"
-          : "=r"(s2)
-          : "h"(static_cast<uint16_t>((eb[k] & 0xFFu) * 0x0101u)));
-      const __half2 scl2 = *reinterpret_cast<const __half2*>(&s2);
-      uint32_t h[8];
-      e2m1x8_to_f16x2(raw[k].x, *reinterpret_cast<uint32_t(*)[4]>(&h[0]));
-      e2m1x8_to_f16x2(raw[k].y, *reinterpret_cast<uint32_t(*)[4]>(&h[4]));
-      uint32_t r[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const float2 f = __half22float2(__hmul2(*reinterpret_cast<const __half2*>(&h[q]), scl2));
-        r[q] = ptx::pack_bf16x2(f.x, f.y);
-      }
-      *reinterpret_cast<uint4*>(orow + 16 * u) = make_uint4(r[0], r[1], r[2], r[3]);
-      *reinterpret_cast<uint4*>(orow + 16 * u + 8) = make_uint4(r[4], r[5], r[6], r[7]);
-    } else if (u < kNope / 16) {
-      const uint32_t words[4] = {raw[k].x, raw[k].y, raw[k].z, raw[k].w};
-      const float scl = kV41 ? e8m0_to_float(eb[k]) : sc[k];
-      uint32_t r[8];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint32_t h0, h1;
-        const uint16_t lo16 = static_cast<uint16_t>(words[q] & 0xFFFF);
-        const uint16_t hi16 = static_cast<uint16_t>(words[q] >> 16);
-        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h0) : "h"(lo16));
-        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h1) : "h"(hi16));
-        const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&h0));
-        const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&h1));
-        // code * scale rounded once to bf16; with the power-of-two E8M0 scales
-        // the product is exact already
-        if (kV41) {
-          r[2 * q] = ptx::pack_bf16x2(f0.x * scl, f0.y * scl);
-          r[2 * q + 1] = ptx::pack_bf16x2(f1.x * scl, f1.y * scl);
-        } else {
-          r[2 * q] = ptx::pack_bf16x2(mul_round_odd(f0.x, scl), mul_round_odd(f0.y, scl));
-          r[2 * q + 1] = ptx::pack_bf16x2(mul_round_odd(f1.x, scl), mul_round_odd(f1.y, scl));
+    for (int k = 0; k < kPer; ++k) {
+      const int item = tid + k * kGatherCtaThreads;
+      const int t = item / kUnits, u = item % kUnits;
+      raw[k] = make_uint4(0, 0, 0, 0);
+      sc[k] = 0.f;
+      eb[k] = 127u;
+      if (s_dst[t] >= 0) {
+        const uint8_t* row = G.cache + (size_t)s_idx[t] * kRowBytes;
+        if (u < kNope / 16 && kFp4) {
+          const uint2 v = __ldg(reinterpret_cast<const uint2*>(row) + u);  // 16 codes
+          raw[k] = make_uint4(v.x, v.y, 0u, 0u);
+          eb[k] = __ldg(row + kNope / 2 + u);
+        } else if (u < kNope / 16) {
+          raw[k] = __ldg(reinterpret_cast<const uint4*>(row) + u);
+          if (kV41)
+            eb[k] = __ldg(row + kNope + (u >> 1));
+          else
+            sc[k] = __ldg(reinterpret_cast<const float*>(row + kNope) + (u >> 3));
+        } else if (!kV41) {
+          raw[k] = __ldg(reinterpret_cast<const uint4*>(row + kNope + 16) + (u - kNope / 16));
         }
       }
-      *reinterpret_cast<uint4*>(orow + 16 * u) = make_uint4(r[0], r[1], r[2], r[3]);
-      *reinterpret_cast<uint4*>(orow + 16 * u + 8) = make_uint4(r[4], r[5], r[6], r[7]);
-    } else {
-      *reinterpret_cast<uint4*>(orow + kNope + 8 * (u - kNope / 16)) = raw[k];
+    }
+    if (kV41) {
+      // the pair's query rows widened to 576 dims (72 16-byte units a row),
+      // spread over all pages_per_pair CTAs of the pair, while the row loads
+      // above are in flight
+      const int n_items = G.h_q * kRowUnits;
+      for (int item = c * kGatherCtaThreads + tid; item < n_items;
+           item += G.pages_per_pair * kGatherCtaThreads) {
+        const size_t r = (size_t)b * G.h_q + item / kRowUnits;
+        const int uu = item % kRowUnits;
+        const uint4 v = uu < kNope / 8
+                            ? __ldg(reinterpret_cast<const uint4*>(G.q512 + r * kNope) + uu)
+                            : make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(G.q576 + r * kD + 8 * uu) = v;
+      }
+    }
+
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+      const int item = tid + k * kGatherCtaThreads;
+      const int t = item / kUnits, u = item % kUnits;
+      const int dst = s_dst[t];
+      if (dst < 0) continue;
+      __nv_bfloat16* orow = out_b + (size_t)dst * kD;
+      if (u < kNope / 16 && kFp4) {
+        // code * scale in f16 is exact (at most 6 significant bits, |x| <= 2688),
+        // and so is its bf16 rounding
+        uint32_t s2;
+        asm("cvt.rn.f16x2.e4m3x2 %0, %1;"
+            : "=r"(s2)
+            : "h"(static_cast<uint16_t>((eb[k] & 0xFFu) * 0x0101u)));
+        const __half2 scl2 = *reinterpret_cast<const __half2*>(&s2);
+        uint32_t h[8];
+        e2m1x8_to_f16x2(raw[k].x, *reinterpret_cast<uint32_t(*)[4]>(&h[0]));
+        e2m1x8_to_f16x2(raw[k].y, *reinterpret_cast<uint32_t(*)[4]>(&h[4]));
+        uint32_t r[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const float2 f = __half22float2(__hmul2(*reinterpret_cast<const __half2*>(&h[q]), scl2));
+          r[q] = ptx::pack_bf16x2(f.x, f.y);
+        }
+        *reinterpret_cast<uint4*>(orow + 16 * u) = make_uint4(r[0], r[1], r[2], r[3]);
+        *reinterpret_cast<uint4*>(orow + 16 * u + 8) = make_uint4(r[4], r[5], r[6], r[7]);
+      } else if (u < kNope / 16) {
+        const uint32_t words[4] = {raw[k].x, raw[k].y, raw[k].z, raw[k].w};
+        const float scl = kV41 ? e8m0_to_float(eb[k]) : sc[k];
+        uint32_t r[8];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t h0, h1;
+          const uint16_t lo16 = static_cast<uint16_t>(words[q] & 0xFFFF);
+          const uint16_t hi16 = static_cast<uint16_t>(words[q] >> 16);
+          asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h0) : "h"(lo16));
+          asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h1) : "h"(hi16));
+          const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&h0));
+          const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&h1));
+          // code * scale rounded once to bf16; with the power-of-two E8M0 scales
+          // the product is exact already
+          if (kV41) {
+            r[2 * q] = ptx::pack_bf16x2(f0.x * scl, f0.y * scl);
+            r[2 * q + 1] = ptx::pack_bf16x2(f1.x * scl, f1.y * scl);
+          } else {
+            r[2 * q] = ptx::pack_bf16x2(mul_round_odd(f0.x, scl), mul_round_odd(f0.y, scl));
+            r[2 * q + 1] = ptx::pack_bf16x2(mul_round_odd(f1.x, scl), mul_round_odd(f1.y, scl));
+          }
+        }
+        *reinterpret_cast<uint4*>(orow + 16 * u) = make_uint4(r[0], r[1], r[2], r[3]);
+        *reinterpret_cast<uint4*>(orow + 16 * u + 8) = make_uint4(r[4], r[5], r[6], r[7]);
+      } else {
+        *reinterpret_cast<uint4*>(orow + kNope + 8 * (u - kNope / 16)) = raw[k];
+      }
     }
   }
 }

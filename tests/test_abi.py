@@ -94,6 +94,15 @@ def test_sparse_and_fused_validation():
     rc = L.mla_sparse_fused_norm_rope_attn_rope_cast(16, 16, 1e-6, 1e4, 16, 16, 100, 16, 2048,
                                                      2, 64, 0.04, 74, 256, 4096, 16, 16, 16, None)
     assert rc == B.MLA_ERR_INVALID_ARG  # workspace too small
+    rc = L.mla_sparse_prefill_fwd(16, 16, 100, 16, 64, None, None, 8, 128, 576, 0.04, 74, 256,
+                                  1 << 30, 16, 16, None)
+    assert rc == B.MLA_ERR_INVALID_ARG  # d_v must be 512
+    rc = L.mla_sparse_prefill_fwd(16, 16, 100, 16, 64, None, None, 8, 128, 512, 0.04, 74, 256,
+                                  1024, 16, 16, None)
+    assert rc == B.MLA_ERR_INVALID_ARG  # workspace too small
+    rc = L.mla_sparse_prefill_fwd(16, 16, 100, 16, 64, None, None, 0, 128, 512, 0.04, 74, 256,
+                                  1 << 30, 16, 16, None)
+    assert rc == B.MLA_OK  # no query token: nothing launched
     rc = L.mla_fused_norm_rope_attn_rope_cast(16, 16, -1.0, 1e4, None, 16, 16, 4, 8, 16, 2, 64,
                                               0.04, 16, 16, 4, 16, 1 << 30, 16, 16, 16, None)
     assert rc == B.MLA_ERR_INVALID_ARG  # eps < 0
@@ -108,6 +117,9 @@ def test_size_queries():
     assert n >= (64 + 74) * 128 * 512 * 4
     assert B.mla_sparse_workspace_size(32, 1, 128, 2048, 512, 74) > n // 2
     assert B.mla_sparse_fused_workspace_size(32, 64, 2048, 148) >= 32 * 2048 * 576 * 2
+    # prefill passes of 32 tokens: the workspace does not grow with s_q
+    assert (B.mla_sparse_prefill_workspace_size(4096, 128, 2048, 74) ==
+            B.mla_sparse_prefill_workspace_size(64, 128, 2048, 74))
     # the V4.1 workspace adds the query widened to 576 dims
     assert (B.mla_sparse_v41_workspace_size(32, 1, 128, 2048, 74) >=
             B.mla_sparse_workspace_size(32, 1, 128, 2048, 512, 74) + 32 * 128 * 576 * 2)
