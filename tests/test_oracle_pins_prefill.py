@@ -87,3 +87,21 @@ def test_prefill_empty_row_gives_zero_and_the_sink():
     o2, l2 = oracle.sparse_prefill(case.q, case.kv, case.indices, case.softmax_scale,
                                    topk_length=lengths)
     assert (o2[1] == 0).all() and np.isneginf(l2[1]).all()
+
+
+def test_prefill_generator_recipe():
+    """Token t sits at position s_kv - s_q + t: its first topk_length[t] =
+    min(topk, position + 1) entries are distinct rows at or before that
+    position and the rest are -1; the draw is fixed by the seed."""
+    case = W.sparse_prefill(seed=5, s_q=80, s_kv=120, h_q=2, topk=64)
+    for t in range(case.s_q):
+        pos = 120 - 80 + t
+        n = int(case.topk_length[t])
+        assert n == min(64, pos + 1)
+        row = case.indices[t]
+        assert (row[n:] == -1).all()
+        valid = row[:n]
+        assert (valid >= 0).all() and (valid <= pos).all()
+        assert len(set(valid.tolist())) == n
+    again = W.sparse_prefill(seed=5, s_q=80, s_kv=120, h_q=2, topk=64)
+    assert torch.equal(case.indices, again.indices) and torch.equal(case.q, again.q)

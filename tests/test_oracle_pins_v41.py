@@ -168,3 +168,21 @@ def test_sparse_v41_fp4_matches_sdpa_on_dequantised_rows():
             rl = torch.logsumexp((q @ sel.T) * case.softmax_scale, dim=-1)
             np.testing.assert_allclose(o[b, i], ro.numpy(), rtol=1e-11, atol=1e-12)
             np.testing.assert_allclose(lse[b, i], rl.numpy(), rtol=1e-12)
+
+
+def test_v41_generators_index_recipe():
+    """Both V4.1 generators draw each query's valid slots without replacement
+    from blocks its own sequence owns, with round(5% * topk) entries -1, and
+    reproduce the same draw from the same seed."""
+    for fp4 in (False, True):
+        seqlens = (300, 130)
+        case = W.sparse_v41(seed=6, batch=2, h_q=2, seqlens=list(seqlens), topk=96, fp4=fp4)
+        for b, L in enumerate(seqlens):
+            own = set(case.block_table[b, :(L + 63) // 64].tolist())
+            row = case.indices[b, 0]
+            idx = row[row >= 0]
+            assert len(set(idx.tolist())) == idx.numel()
+            assert all(s // 64 in own for s in idx.tolist())
+            assert int((row < 0).sum()) == round(0.05 * case.topk)
+        again = W.sparse_v41(seed=6, batch=2, h_q=2, seqlens=list(seqlens), topk=96, fp4=fp4)
+        assert torch.equal(case.kcache, again.kcache) and torch.equal(case.indices, again.indices)
