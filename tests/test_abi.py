@@ -123,3 +123,73 @@ def test_size_queries():
     # the V4.1 workspace adds the query widened to 576 dims
     assert (B.mla_sparse_v41_workspace_size(32, 1, 128, 2048, 74) >=
             B.mla_sparse_workspace_size(32, 1, 128, 2048, 512, 74) + 32 * 128 * 576 * 2)
+
+
+# Every pointer argument of every compute entry point: set to NULL, the call
+# must fail with MLA_ERR_INVALID_ARG before it launches anything.  Fake but
+# aligned addresses fill the other slots (nothing dereferences them).
+def _sparse(L, **o):
+    a = dict(q=16, kc=16, ns=100, idx=16, topk=64, b=2, s_q=1, h_q=128, d_v=512, scale=0.04,
+             parts=74, ws=256, wsb=1 << 30, out=16, lse=16)
+    a.update(o)
+    return L.mla_sparse_decode(a["q"], a["kc"], a["ns"], a["idx"], a["topk"], a["b"], a["s_q"],
+                               a["h_q"], a["d_v"], a["scale"], a["parts"], a["ws"], a["wsb"],
+                               a["out"], a["lse"], None)
+
+
+def _v41(fn, L, **o):
+    a = dict(q=16, kc=16, ns=100, idx=16, topk=64, b=2, s_q=1, h_q=128, scale=0.04, parts=74,
+             ws=256, wsb=1 << 30, out=16, lse=16)
+    a.update(o)
+    return getattr(L, fn)(a["q"], a["kc"], a["ns"], a["idx"], a["topk"], a["b"], a["s_q"],
+                          a["h_q"], a["scale"], a["parts"], a["ws"], a["wsb"], a["out"],
+                          a["lse"], None)
+
+
+def _fused(L, **o):
+    a = dict(q=16, g=16, pos=None, kc=16, bt=16, sl=16, meta=16, ns=16, ws=16, out=16, sc=16,
+             lse=16)
+    a.update(o)
+    return L.mla_fused_norm_rope_attn_rope_cast(a["q"], a["g"], 1e-6, 1e4, a["pos"], a["kc"],
+                                                a["bt"], 4, 8, a["sl"], 2, 64, 0.04, a["meta"],
+                                                a["ns"], 4, a["ws"], 1 << 30, a["out"], a["sc"],
+                                                a["lse"], None)
+
+
+def _fused_sparse(L, **o):
+    a = dict(q=16, g=16, pos=16, kc=16, idx=16, ws=256, out=16, sc=16, lse=16)
+    a.update(o)
+    return L.mla_sparse_fused_norm_rope_attn_rope_cast(a["q"], a["g"], 1e-6, 1e4, a["pos"],
+                                                       a["kc"], 100, a["idx"], 64, 2, 64, 0.04,
+                                                       74, a["ws"], 1 << 30, a["out"], a["sc"],
+                                                       a["lse"], None)
+
+
+def _prefill(L, **o):
+    a = dict(q=16, kv=16, idx=16, ws=256, out=16, lse=16)
+    a.update(o)
+    return L.mla_sparse_prefill_fwd(a["q"], a["kv"], 100, a["idx"], 64, None, None, 8, 128, 512,
+                                    0.04, 74, a["ws"], 1 << 30, a["out"], a["lse"], None)
+
+
+@pytest.mark.parametrize("call,pointer", [
+    (lambda L, **o: _sparse(L, **o), p) for p in ("q", "kc", "idx", "ws", "out", "lse")
+] + [
+    (lambda L, **o: _v41("mla_sparse_decode_v41", L, **o), p)
+    for p in ("q", "kc", "idx", "ws", "out", "lse")
+] + [
+    (lambda L, **o: _v41("mla_sparse_decode_v41_fp4", L, **o), p)
+    for p in ("q", "kc", "idx", "ws", "out", "lse")
+] + [
+    (lambda L, **o: _fused(L, **o), p)
+    for p in ("q", "g", "kc", "bt", "sl", "meta", "ns", "ws", "out", "sc", "lse")
+] + [
+    (lambda L, **o: _fused_sparse(L, **o), p)
+    for p in ("q", "g", "pos", "kc", "idx", "ws", "out", "sc", "lse")
+] + [
+    (lambda L, **o: _prefill(L, **o), p) for p in ("q", "kv", "idx", "ws", "out", "lse")
+])
+def test_null_pointers_are_rejected_before_launch(call, pointer):
+    L = B.lib()
+    assert call(L, **{pointer: None}) == B.MLA_ERR_INVALID_ARG
+    assert L.mla_last_error().decode() != ""
