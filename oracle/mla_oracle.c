@@ -26,7 +26,13 @@
  *       intensity"] and [deepseek-ai/FlashMLA README, "News", 2026.09.10]
  *  - Token-level sparse decode: indices (b, s_q, topk) hold physical slots
  *    (block*64 + offset), -1 marks an invalid slot, block table ignored.
+ *    Sparse prefill has no batch dimension and optional attention-sink and
+ *    per-token top-k-length arguments.
  *      [FlashMLA (AI Wiki), "Interfaces"]
+ *  - The fused kernel is recommended over the standalone sparse kernels, so
+ *    its steps also run over a sparse selection of slots.
+ *      [FlashMLA fused norm-RoPE-attention-RoPE-cast kernel card,
+ *       "Workarounds"]
  *  - The 656-byte FP8 cache row: 512 E4M3 codes, 4 fp32 tile scales (one per
  *    128 values), 64 bf16 RoPE dims.
  *      [FlashMLA (AI Wiki), "The FP8 and FP4 KV cache"]
@@ -47,6 +53,10 @@
  *  - Fused path: the normalised, rotated query enters the attention in bf16
  *    (the tensor-core operand precision); the pages leave this precision
  *    open, and fixing it makes the FP8 code decisions comparable.
+ *  - Sparse prefill: a sink is one logit per head that joins the softmax
+ *    normaliser without a value row (the returned LSE includes it); a
+ *    top-k length counts only the first entries of a token's indices.
+ *  - Fused sparse mode: the query position is an input.
  *  - Sparse paths: the dequantised rows enter the attention rounded to bf16
  *    (round to nearest even), as the quantised decoding kernels convert them.
  *  - V4.1 rows: the latent is 512 wide, q . K runs over all 512 dims and V is
