@@ -47,12 +47,13 @@ def lib():
         L.oracle_combine.argtypes = [ctypes.c_int, f64p, f64p, ctypes.c_int, f64p, f64p]
         L.oracle_dense_decode.restype = ctypes.c_int
         L.oracle_dense_decode.argtypes = [
-            u16p, u16p, i32p, ctypes.c_int, i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            u16p, u16p, ctypes.c_int, i32p, ctypes.c_int, i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
             ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int, i64p, ctypes.c_int64,
             i32p, i32p, f64p, f64p]
         L.oracle_fused_decode.restype = ctypes.c_int
         L.oracle_fused_decode.argtypes = [
-            u16p, f64p, ctypes.c_double, ctypes.c_double, i32p, u16p, i32p, ctypes.c_int, i32p,
+            u16p, f64p, ctypes.c_double, ctypes.c_double, i32p, u16p, ctypes.c_int, i32p,
+            ctypes.c_int, i32p,
             ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double, i64p, ctypes.c_int64,
             u8p, f64p, f64p, f64p]
         L.oracle_sparse_decode.restype = ctypes.c_int
@@ -217,10 +218,13 @@ def combine(lse_i, o_i):
 # -------------------------------------------------------------- decode paths
 
 def dense_decode(q, kcache, block_table, cache_seqlens, d_v, softmax_scale, causal=True,
-                 rows=None, token_lo=None, token_hi=None):
+                 rows=None, token_lo=None, token_hi=None, allow_faults=False):
     """oracle_dense_decode.  q [b, s_q, h_q, 576] bf16; kcache [NB, page, 1, 576]
     bf16; block_table [b, max_pages] int32; cache_seqlens [b] int32.
-    Returns (out fp64 [b, s_q, h_q, d_v] or [n_rows, d_v], lse fp64)."""
+    Returns (out fp64 [b, s_q, h_q, d_v] or [n_rows, d_v], lse fp64).
+    A block id outside [0, NB) reads block 0 and a length above
+    max_pages * page is cut there; such inputs raise ValueError unless
+    allow_faults is set."""
     b, s_q, h_q, dq = q.shape
     assert dq == _D
     page = kcache.shape[1]
@@ -236,20 +240,23 @@ def dense_decode(q, kcache, block_table, cache_seqlens, d_v, softmax_scale, caus
     out = np.zeros((n, d_v), dtype=np.float64)
     lse = np.zeros(n, dtype=np.float64)
     rc = lib().oracle_dense_decode(
-        _ptr(qa, ctypes.c_uint16), _ptr(ka, ctypes.c_uint16), _ptr(bt, ctypes.c_int32), max_pages,
-        _ptr(sl, ctypes.c_int32), b, s_q, h_q, d_v, page, float(softmax_scale), int(bool(causal)),
-        _ptr(ra, ctypes.c_int64), n, _ptr(lo, ctypes.c_int32), _ptr(hi, ctypes.c_int32),
-        _ptr(out, ctypes.c_double), _ptr(lse, ctypes.c_double))
-    assert rc == 0
+        _ptr(qa, ctypes.c_uint16), _ptr(ka, ctypes.c_uint16), kcache.shape[0],
+        _ptr(bt, ctypes.c_int32), max_pages, _ptr(sl, ctypes.c_int32), b, s_q, h_q, d_v, page,
+        float(softmax_scale), int(bool(causal)), _ptr(ra, ctypes.c_int64), n,
+        _ptr(lo, ctypes.c_int32), _ptr(hi, ctypes.c_int32), _ptr(out, ctypes.c_double),
+        _ptr(lse, ctypes.c_double))
+    if rc != 0 and not allow_faults:
+        raise ValueError("block id or sequence length out of range")
     if ra is None:
         return out.reshape(b, s_q, h_q, d_v), lse.reshape(b, s_q, h_q)
     return out, lse
 
 
 def fused_decode(q_raw, gain, eps, rope_base, kcache, block_table, cache_seqlens, softmax_scale,
-                 positions=None, rows=None, want_pre_cast=False):
+                 positions=None, rows=None, want_pre_cast=False, allow_faults=False):
     """oracle_fused_decode (s_q = 1, d_v = 576).
-    Returns (codes uint8, scale fp64, lse fp64[, o_pre fp64])."""
+    Returns (codes uint8, scale fp64, lse fp64[, o_pre fp64]).  Out-of-range
+    block ids and lengths as in dense_decode."""
     b, s_q, h_q, dq = q_raw.shape
     assert s_q == 1 and dq == _D
     page = kcache.shape[1]
@@ -267,11 +274,12 @@ def fused_decode(q_raw, gain, eps, rope_base, kcache, block_table, cache_seqlens
     pre = np.zeros((n, _D), dtype=np.float64) if want_pre_cast else None
     rc = lib().oracle_fused_decode(
         _ptr(qa, ctypes.c_uint16), _ptr(g, ctypes.c_double), float(eps), float(rope_base),
-        _ptr(pos, ctypes.c_int32), _ptr(ka, ctypes.c_uint16), _ptr(bt, ctypes.c_int32),
-        bt.shape[1], _ptr(sl, ctypes.c_int32), b, h_q, page, float(softmax_scale),
-        _ptr(ra, ctypes.c_int64), n, _ptr(codes, ctypes.c_uint8), _ptr(scale, ctypes.c_double),
-        _ptr(lse, ctypes.c_double), _ptr(pre, ctypes.c_double))
-    assert rc == 0
+        _ptr(pos, ctypes.c_int32), _ptr(ka, ctypes.c_uint16), kcache.shape[0],
+        _ptr(bt, ctypes.c_int32), bt.shape[1], _ptr(sl, ctypes.c_int32), b, h_q, page,
+        float(softmax_scale), _ptr(ra, ctypes.c_int64), n, _ptr(codes, ctypes.c_uint8),
+        _ptr(scale, ctypes.c_double), _ptr(lse, ctypes.c_double), _ptr(pre, ctypes.c_double))
+    if rc != 0 and not allow_faults:
+        raise ValueError("block id or sequence length out of range")
     if ra is None:
         codes = codes.reshape(b, 1, h_q, _D)
         scale = scale.reshape(b, 1, h_q)
@@ -281,7 +289,7 @@ def fused_decode(q_raw, gain, eps, rope_base, kcache, block_table, cache_seqlens
     return (codes, scale, lse, pre) if want_pre_cast else (codes, scale, lse)
 
 
-def sparse_decode(q, kcache656, indices, d_v, softmax_scale, rows=None):
+def sparse_decode(q, kcache656, indices, d_v, softmax_scale, rows=None, allow_faults=False):
     """oracle_sparse_decode.  q [b, s_q, h_q, 576] bf16; kcache656 [..., 656] uint8
     (flattened to slots); indices [b, s_q, topk] int32 (-1 = invalid)."""
     b, s_q, h_q, dq = q.shape
@@ -298,14 +306,14 @@ def sparse_decode(q, kcache656, indices, d_v, softmax_scale, rows=None):
         _ptr(qa, ctypes.c_uint16), _ptr(ca, ctypes.c_uint8), ca.shape[0], _ptr(ix, ctypes.c_int32),
         b, s_q, h_q, topk, d_v, float(softmax_scale), _ptr(ra, ctypes.c_int64), n,
         _ptr(out, ctypes.c_double), _ptr(lse, ctypes.c_double))
-    if rc != 0:
+    if rc != 0 and not allow_faults:
         raise ValueError("sparse index out of range")
     if ra is None:
         return out.reshape(b, s_q, h_q, d_v), lse.reshape(b, s_q, h_q)
     return out, lse
 
 
-def sparse_decode_v41(q, kcache, indices, softmax_scale, rows=None):
+def sparse_decode_v41(q, kcache, indices, softmax_scale, rows=None, allow_faults=False):
     """oracle_sparse_decode_v41 (528-byte FP8 rows) or
     oracle_sparse_decode_v41_fp4 (288-byte FP4 rows), told apart by the bytes
     per row.  q [b, s_q, h_q, 512] bf16; kcache [..., 528 | 288] uint8
@@ -328,7 +336,7 @@ def sparse_decode_v41(q, kcache, indices, softmax_scale, rows=None):
         _ptr(qa, ctypes.c_uint16), _ptr(ca, ctypes.c_uint8), ca.shape[0], _ptr(ix, ctypes.c_int32),
         b, s_q, h_q, topk, float(softmax_scale), _ptr(ra, ctypes.c_int64), n,
         _ptr(out, ctypes.c_double), _ptr(lse, ctypes.c_double))
-    if rc != 0:
+    if rc != 0 and not allow_faults:
         raise ValueError("sparse index out of range")
     if ra is None:
         return out.reshape(b, s_q, h_q, 512), lse.reshape(b, s_q, h_q)
@@ -336,7 +344,7 @@ def sparse_decode_v41(q, kcache, indices, softmax_scale, rows=None):
 
 
 def fused_sparse_decode(q_raw, gain, eps, rope_base, positions, kcache656, indices,
-                        softmax_scale, rows=None):
+                        softmax_scale, rows=None, allow_faults=False):
     """oracle_fused_sparse_decode: the fused steps over the valid slots of
     indices [b, 1, topk] in the 656-byte FP8 cache; positions [b] required.
     Returns (codes uint8, scale fp64, lse fp64)."""
@@ -358,7 +366,7 @@ def fused_sparse_decode(q_raw, gain, eps, rope_base, positions, kcache656, indic
         _ptr(pos, ctypes.c_int32), _ptr(ca, ctypes.c_uint8), ca.shape[0], _ptr(ix, ctypes.c_int32),
         b, h_q, topk, float(softmax_scale), _ptr(ra, ctypes.c_int64), n,
         _ptr(codes, ctypes.c_uint8), _ptr(scale, ctypes.c_double), _ptr(lse, ctypes.c_double))
-    if rc != 0:
+    if rc != 0 and not allow_faults:
         raise ValueError("sparse index out of range")
     if ra is None:
         return codes.reshape(b, 1, h_q, _D), scale.reshape(b, 1, h_q), lse.reshape(b, 1, h_q)
@@ -366,7 +374,7 @@ def fused_sparse_decode(q_raw, gain, eps, rope_base, positions, kcache656, indic
 
 
 def sparse_prefill(q, kv, indices, softmax_scale, d_v=512, topk_length=None, attn_sink=None,
-                   rows=None):
+                   rows=None, allow_faults=False):
     """oracle_sparse_prefill.  q [s_q, h_q, 576] bf16; kv [s_kv, 576] bf16;
     indices [s_q, topk] int32 (-1 = invalid); topk_length [s_q] int32 or None;
     attn_sink [h_q] or None.  Returns O [s_q, h_q, d_v] and LSE [s_q, h_q]
@@ -389,7 +397,7 @@ def sparse_prefill(q, kv, indices, softmax_scale, d_v=512, topk_length=None, att
         _ptr(tl, ctypes.c_int32), _ptr(sk, ctypes.c_double), s_q, h_q, topk, d_v,
         float(softmax_scale), _ptr(ra, ctypes.c_int64), n, _ptr(out, ctypes.c_double),
         _ptr(lse, ctypes.c_double))
-    if rc != 0:
+    if rc != 0 and not allow_faults:
         raise ValueError("sparse index out of range")
     if ra is None:
         return out.reshape(s_q, h_q, d_v), lse.reshape(s_q, h_q)

@@ -261,13 +261,41 @@ static void attend_rows(const double* q, row_fetch_fn fetch, const void* ctx, in
 typedef struct {
   const uint16_t* kcache;
   const int32_t* block_table;
-  int max_pages, b, lo, page;
+  int num_blocks, max_pages, b, lo, page;
 } paged_ctx;
+
+/* A block id outside [0, num_blocks) names no page of the cache; it is read
+ * as block 0 (reading: a stand-in that keeps every read inside the cache,
+ * with the fault reported to the caller). */
+static int paged_block(const paged_ctx* c, int page_idx) {
+  int blk = c->block_table[(size_t)c->b * c->max_pages + page_idx];
+  return (blk < 0 || blk >= c->num_blocks) ? 0 : blk;
+}
+
+/* Tokens of sequence b that the block table can reach: a length beyond
+ * max_pages * page is read as that many (reading: the table names no
+ * further page). */
+static int paged_length(int L, int max_pages, int page) {
+  long long cap = (long long)max_pages * page;
+  return (long long)L > cap ? (int)cap : L;
+}
+
+/* 1 when sequence c->b's table has an out-of-range id among its first
+ * ceil(L / page) entries, or its raw length L_raw exceeds the table. */
+static int paged_faults(const paged_ctx* c, int L_raw, int L) {
+  int p, blk;
+  if (L_raw != L) return 1;
+  for (p = 0; p < (L + c->page - 1) / c->page; ++p) {
+    blk = c->block_table[(size_t)c->b * c->max_pages + p];
+    if (blk < 0 || blk >= c->num_blocks) return 1;
+  }
+  return 0;
+}
 
 static void fetch_paged_bf16(const void* vctx, int j, double* out) {
   const paged_ctx* c = (const paged_ctx*)vctx;
   int t = c->lo + j;
-  int blk = c->block_table[(size_t)c->b * c->max_pages + t / c->page];
+  int blk = paged_block(c, t / c->page);
   const uint16_t* row = c->kcache + ((size_t)blk * c->page + (size_t)(t % c->page)) * ORACLE_D;
   int d;
   for (d = 0; d < ORACLE_D; ++d) out[d] = bf16_bits_to_f64(row[d]);
@@ -320,7 +348,9 @@ static int visible_tokens(int L, int s_q, int i, int causal) {
 /* Dense paged MLA decode.
  *  q           [b, s_q, h_q, 576] bf16 bits
  *  kcache      [num_blocks, page, 1, 576] bf16 bits
- *  block_table [b, max_pages] int32
+ *  block_table [b, max_pages] int32; an id outside [0, num_blocks) reads
+ *              block 0, and a length above max_pages * page is read as
+ *              max_pages * page (both are input faults: the return is 1)
  *  seqlens     [b] int32
  *  rows        optional list of n_rows flat row ids (b*s_q + i)*h_q + h;
  *              NULL computes every row.  Outputs are indexed by the flat row
@@ -330,20 +360,21 @@ static int visible_tokens(int L, int s_q, int i, int causal) {
  *              intersected with the visible range (used to form split
  *              partials); NULL = whole range.
  * Returns 0. */
-int oracle_dense_decode(const uint16_t* q, const uint16_t* kcache, const int32_t* block_table,
-                        int max_pages, const int32_t* seqlens, int batch, int s_q, int h_q,
-                        int d_v, int page, double scale, int causal, const int64_t* rows,
-                        int64_t n_rows, const int32_t* token_lo, const int32_t* token_hi,
-                        double* out, double* lse) {
+int oracle_dense_decode(const uint16_t* q, const uint16_t* kcache, int num_blocks,
+                        const int32_t* block_table, int max_pages, const int32_t* seqlens,
+                        int batch, int s_q, int h_q, int d_v, int page, double scale, int causal,
+                        const int64_t* rows, int64_t n_rows, const int32_t* token_lo,
+                        const int32_t* token_hi, double* out, double* lse) {
   int64_t total = (int64_t)batch * s_q * h_q;
   int64_t n = rows ? n_rows : total;
   int64_t r;
-#pragma omp parallel for schedule(dynamic, 1)
+  int fault = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : fault)
   for (r = 0; r < n; ++r) {
     int64_t flat = rows ? rows[r] : r;
     int i = (int)((flat / h_q) % s_q);
     int b = (int)(flat / ((int64_t)h_q * s_q));
-    int L = seqlens[b];
+    int L = paged_length(seqlens[b], max_pages, page);
     int vis = visible_tokens(L, s_q, i, causal);
     int lo = token_lo ? token_lo[b] : 0;
     int hi = token_hi ? token_hi[b] : vis;
@@ -357,13 +388,15 @@ int oracle_dense_decode(const uint16_t* q, const uint16_t* kcache, const int32_t
     for (d = 0; d < ORACLE_D; ++d) qv[d] = bf16_bits_to_f64(qr[d]);
     ctx.kcache = kcache;
     ctx.block_table = block_table;
+    ctx.num_blocks = num_blocks;
     ctx.max_pages = max_pages;
     ctx.b = b;
     ctx.lo = lo;
     ctx.page = page;
+    fault |= paged_faults(&ctx, seqlens[b], L);
     attend_rows(qv, fetch_paged_bf16, &ctx, cnt, d_v, scale, out + (size_t)r * d_v, lse + r);
   }
-  return 0;
+  return fault;
 }
 
 /* LSE-weighted merge of n_splits partial results of one row:
@@ -434,7 +467,7 @@ static void fused_row(const uint16_t* qr, const double* gain, double eps, double
 }
 
 int oracle_fused_decode(const uint16_t* q_raw, const double* gain, double eps, double rope_base,
-                        const int32_t* positions, const uint16_t* kcache,
+                        const int32_t* positions, const uint16_t* kcache, int num_blocks,
                         const int32_t* block_table, int max_pages, const int32_t* seqlens,
                         int batch, int h_q, int page, double scale, const int64_t* rows,
                         int64_t n_rows, uint8_t* codes, double* out_scale, double* lse,
@@ -442,24 +475,29 @@ int oracle_fused_decode(const uint16_t* q_raw, const double* gain, double eps, d
   int64_t total = (int64_t)batch * h_q;
   int64_t n = rows ? n_rows : total;
   int64_t r;
-#pragma omp parallel for schedule(dynamic, 1)
+  int fault = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : fault)
   for (r = 0; r < n; ++r) {
     int64_t flat = rows ? rows[r] : r;
     int b = (int)(flat / h_q);
-    int L = seqlens[b];
-    double pos = positions ? (double)positions[b] : (double)(L - 1);
+    /* the default query position follows the length as given; the tokens
+     * attended stop where the block table does */
+    int L = paged_length(seqlens[b] > 0 ? seqlens[b] : 0, max_pages, page);
+    double pos = positions ? (double)positions[b] : (double)(seqlens[b] - 1);
     paged_ctx ctx;
     ctx.kcache = kcache;
     ctx.block_table = block_table;
+    ctx.num_blocks = num_blocks;
     ctx.max_pages = max_pages;
     ctx.b = b;
     ctx.lo = 0;
     ctx.page = page;
+    fault |= paged_faults(&ctx, seqlens[b], L);
     fused_row(q_raw + (size_t)flat * ORACLE_D, gain, eps, rope_base, pos, fetch_paged_bf16, &ctx,
               L, scale, codes + (size_t)r * ORACLE_D, out_scale + r, lse + r,
               o_pre ? o_pre + (size_t)r * ORACLE_D : 0);
   }
-  return 0;
+  return fault;
 }
 
 /* ----------------------------------------------------------- sparse path */

@@ -301,10 +301,11 @@ def test_sampled_rows_equal_full_rows():
 
 # ------------------------------------------------------------- fused path
 
-def fused_library_reference(case):
+def fused_library_reference(case, positions=None):
     """The fused step chain built from library routines in fp64: torch rms_norm,
     numpy complex rotation, torch SDPA, complex conjugate rotation, and the
-    float8_e4m3fn cast of o/scale (ratio rounded to fp32)."""
+    float8_e4m3fn cast of o/scale (ratio rounded to fp32).  The query of
+    sequence b sits at positions[b] (default L - 1)."""
     b, _, h, _ = case.q_raw.shape
     theta_k = 10000.0 ** (-np.arange(32) * 2.0 / 64.0)
     codes = np.zeros((b, h, 576), dtype=np.uint8)
@@ -313,7 +314,7 @@ def fused_library_reference(case):
     pres = np.zeros((b, h, 576))
     for bi in range(b):
         L = int(case.cache_seqlens[bi])
-        pos = L - 1
+        pos = L - 1 if positions is None else positions[bi]
         x = case.q_raw[bi, 0].to(torch.float64)
         y = F.rms_norm(x, (576,), weight=case.gain.to(torch.float64), eps=case.eps).numpy()
         z = (y[:, 512::2] + 1j * y[:, 513::2]) * np.exp(1j * pos * theta_k)
