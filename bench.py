@@ -161,20 +161,6 @@ def prefill_work(case):
     return flops, kv_bytes, kv_bytes + io
 
 
-def prefill_last_pass_work(case, chunk=32):
-    """Work of the prefill's last pass (its last `chunk` query tokens): the
-    attention kernel launch that the kernel events time."""
-    t0 = max(0, case.s_q - chunk)
-    ix = case.indices.cpu()[t0:]
-    if case.topk_length is not None:
-        n = case.topk_length.cpu()[t0:].clamp(0, case.topk)
-        ix = torch.where(torch.arange(case.topk)[None, :] < n[:, None], ix, torch.full_like(ix, -1))
-    valid = int((ix >= 0).sum())
-    flops = 2 * valid * (576 + case.d_v) * case.h_q
-    kv_bytes = valid * 1152
-    return flops, kv_bytes, kv_bytes + (case.s_q - t0) * case.h_q * (576 * 2 + case.d_v * 2 + 4)
-
-
 def sparse_dims(case):
     """(latent width of q . k, bytes per cache row) of a sparse case."""
     row = int(case.kcache.shape[-1])
@@ -221,7 +207,6 @@ class GpuStep:
             self.case = W.sparse_prefill(seed=seed, device=dev)
             self.kind = "prefill"
             self.work = prefill_work(self.case)
-            self.kernel_work = prefill_last_pass_work(self.case)
             self.R = self.case.h_q
         elif name in ("sparse", "sparse_v41", "sparse_v41_fp4"):
             self.case = W.WORKLOADS[name](seed=seed, device=dev)
@@ -231,8 +216,6 @@ class GpuStep:
         else:
             raise ValueError(name)
         c = self.case
-        if not hasattr(self, "kernel_work"):
-            self.kernel_work = self.work  # one attention launch per step
         self.parts = B.mla_num_sm_parts(self.R, 1, dev)
         if self.kind == "prefill":
             self.out = torch.empty((c.s_q, c.h_q, c.d_v), dtype=torch.bfloat16, device=dev)
@@ -264,6 +247,9 @@ class GpuStep:
         if self.kind in ("dense", "fused"):
             self.meta = torch.empty((self.parts, 8), dtype=torch.int32, device=dev)
             self.ns = torch.empty((b + 1,), dtype=torch.int32, device=dev)
+
+    def attention_launches_per_step(self):
+        return -(-self.case.s_q // 32) if self.kind == "prefill" else 1
 
     def launches_per_step(self):
         # planner + attention kernel + combine (+ the FP8 gather for sparse);
@@ -463,6 +449,80 @@ def reduce_over_ranks(times, work, world, device):
     return [float(x) for x in t], [float(x) for x in w]
 
 
+def roofline_of(bound, flops, total_bytes, ms_kernel, peaks, peak_src, traffic=None):
+    """Roofline entry of one attention launch of `ms_kernel` ms.  The launch is
+    timed alone over a short run (well under a second), so a tensor-bound
+    kernel is held against the burst bf16 peak; its HBM fraction is printed
+    beside it (a kernel at the ridge needs both)."""
+    s = ms_kernel * 1e-3
+    gbs = total_bytes / s / 1e9
+    if bound == "tensor":
+        achieved = flops / s / 1e12
+        peak = peaks["bf16_tflops"]
+        return {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
+                "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                "peak_source": f"{peak_src} bf16 burst (kernel timed alone, short run)",
+                "hbm_achieved_gbs": round(gbs, 1), "hbm_frac": round(gbs / peaks["hbm_gbs"], 4),
+                "traffic": traffic, "kernel_ms": round(ms_kernel, 5)}
+    peak = peaks["hbm_gbs"]
+    return {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(gbs / peak, 4), "peak_source": f"{peak_src} hbm copy",
+            "traffic": traffic, "kernel_ms": round(ms_kernel, 5)}
+
+
+def time_steps(gs, steps, graph, dev):
+    """(ms per step, ms per attention launch) of `steps` steps: the steps as
+    CUDA graph replays (or direct calls) with nothing between them, then the
+    attention kernel alone in a second pass between library-recorded events."""
+    st = torch.cuda.current_stream(dev)
+    run = gs.step
+    if graph:
+        g = gs.capture()
+        for _ in range(3):
+            g.replay()
+        run = g.replay
+    torch.cuda.synchronize(dev)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    ev0.record(st)
+    for _ in range(steps):
+        run()
+    ev1.record(st)
+    torch.cuda.synchronize(dev)
+    ms_step = ev0.elapsed_time(ev1) / steps
+    ks = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ke = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    for i in range(steps):
+        gs.B.mla_set_kernel_events(ks[i], ke[i])
+        gs.step()
+    torch.cuda.synchronize(dev)
+    gs.B.mla_set_kernel_events(None, None)
+    return ms_step, sum(a.elapsed_time(b) for a, b in zip(ks, ke)) / steps
+
+
+def measure_side(name, args, dev, peaks, peak_src):
+    """The HBM-bound workloads measured in the same run as the headline one:
+    step time, attention-kernel time, KV-read GB/s and the HBM roofline
+    fraction of that kernel."""
+    gs = GpuStep(name, seed=args.seed, dev=dev)
+    for _ in range(max(3, args.warmup)):
+        gs.step()
+    torch.cuda.synchronize(dev)
+    if gs.B.device_status() != 0:
+        raise RuntimeError(f"device status set after warm-up of {name}")
+    ms_step, ms_kernel = time_steps(gs, args.steps, args.graph, dev)
+    flops, kv_bytes, total_bytes = gs.work
+    roof = roofline_of(WORKLOAD_INFO[name][1], flops, total_bytes, ms_kernel, peaks, peak_src,
+                       load_traffic(name))
+    out = {"workload": WORKLOAD_INFO[name][0], "ms_per_step": round(ms_step, 5),
+           "tflops": round(flops / (ms_step * 1e-3) / 1e12, 3),
+           "kv_read_gbs": round(kv_bytes / (ms_step * 1e-3) / 1e9, 1),
+           "kernel_ms": round(ms_kernel, 5), "roofline": roof}
+    del gs
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_gpu_arm(args, rank, world):
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
@@ -582,6 +642,7 @@ def run_gpu_arm(args, rank, world):
         raise RuntimeError(f"device status {status:#x} after timing")
 
     ms_step = ms_total / args.steps
+    case_for_cpu = gs.case
     (ms_step, e2e_ms, ms_kernel), (flops_all, kv_all) = reduce_over_ranks(
         [ms_step, e2e_ms, ms_kernel], [flops, kv_bytes], world, dev)
     if rank != 0:
@@ -591,26 +652,16 @@ def run_gpu_arm(args, rank, world):
     desc, bound = WORKLOAD_INFO[args.workload]
     tflops = flops_all / (ms_step * 1e-3) / 1e12
     gbs = kv_all / (ms_step * 1e-3) / 1e9
-    # dominant kernel: the attention kernel, timed alone; for the prefill the
-    # events hold its last launch of the step (the last pass of 32 tokens), so
-    # that launch's own work is the numerator
-    flops, _, total_bytes = gs.kernel_work
-    per_launch_s = ms_kernel * 1e-3
-    traffic = load_traffic(args.workload)
-    if bound == "tensor":
-        achieved = flops / per_launch_s / 1e12
-        peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-        roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
-                "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                "peak_source": f"{peak_src} bf16 sustained (burst {peaks['bf16_tflops']})",
-                "frac_of_burst": round(achieved / peaks["bf16_tflops"], 4), "traffic": traffic,
-                "kernel_ms": round(ms_kernel, 5)}
-    else:
-        achieved = total_bytes / per_launch_s / 1e9
-        peak = peaks["hbm_gbs"]
-        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "peak_source": f"{peak_src} hbm copy",
-                "traffic": traffic, "kernel_ms": round(ms_kernel, 5)}
+    # dominant kernel: the attention kernel, timed alone; a workload with
+    # several attention launches per step (the prefill's passes) is held to
+    # the roofline over the whole step instead
+    flops, _, total_bytes = gs.work
+    multi = gs.attention_launches_per_step() > 1
+    roof = roofline_of(bound, flops, total_bytes, ms_step if multi else ms_kernel, peaks, peak_src,
+                       load_traffic(args.workload))
+    if multi:
+        roof["timed"] = (f"whole step ({gs.attention_launches_per_step()} attention launches "
+                         "and their gathers, planners and combines)")
     line = {
         "metric": METRIC,
         "value": round(tflops, 3),
@@ -640,9 +691,15 @@ def run_gpu_arm(args, rank, world):
         "roofline": roof,
         "clocks": clocks,
     }
+    if args.side and world == 1 and args.workload == "compute":
+        # the memory-bound configurations of the same metric, timed in this run
+        del gs, slots
+        torch.cuda.empty_cache()
+        line["hbm_bound"] = {n: measure_side(n, args, dev, peaks, peak_src)
+                             for n in ("memory", "fused")}
     if args.cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(args.workload, seed=args.seed, budget_s=args.cpu_budget,
-                                            case=gs.case)
+                                            case=case_for_cpu)
     return line
 
 
@@ -802,6 +859,9 @@ def main():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--graph", type=int, default=1,
                     help="time CUDA graph replays of the step (0: direct API calls)")
+    ap.add_argument("--side", type=int, default=1,
+                    help="with the compute workload on one GPU, also time the memory and fused "
+                         "(batch 32) workloads and print them under hbm_bound")
     ap.add_argument("--cpu-baseline", dest="cpu_baseline", type=int, default=1)
     ap.add_argument("--cpu-budget", dest="cpu_budget", type=float, default=15.0)
     args = ap.parse_args()

@@ -37,7 +37,9 @@
  *   - Layouts are dense, row-major, innermost dimension last:
  *       q            [batch, s_q, h_q, 576]        bf16 (16-byte aligned)
  *       kcache       [num_blocks, 64, 1, 576]      bf16 (16-byte aligned)
- *       block_table  [batch, max_pages]            int32
+ *       block_table  [batch, max_pages]            int32 (entries past a
+ *                                                  sequence's last page are
+ *                                                  never read)
  *       cache_seqlens[batch]                       int32
  *       out          [batch, s_q, h_q, d_v]        bf16
  *       lse          [batch, s_q, h_q]             fp32, natural log
@@ -292,7 +294,9 @@ MLA_API int mla_sparse_fused_norm_rope_attn_rope_cast(
  *             MLA_ERR_INVALID_ARG with the bytes it would need.
  *   Device    the current CUDA device; `stream` must belong to it.  The
  *             first call on each device looks up the array's address once;
- *             make that first call outside any stream capture.
+ *             make that first call outside any stream capture.  The address
+ *             is kept for the life of the process, so a cudaDeviceReset
+ *             between calls is not supported.
  *   Sharing   every call on a device uses the same array: calls that may
  *             run at the same time on the GPU (unordered streams) race and
  *             give wrong results.  Order them, e.g. on one stream.
@@ -312,11 +316,42 @@ MLA_API int mla_decode_fwd_noalloc(const void* q, const void* kcache, const int3
  * the calling host thread; pass NULL, NULL to clear it. */
 MLA_API int mla_set_kernel_events(void* start_event, void* stop_event);
 
-/* Reads the device status word that kernels set when a bounded wait expires
- * or an out-of-range block id / index is met: 0 = ok, else (code << 16) |
- * site, code 1 = timeout, 2 = bad index.  Synchronises the device; reset != 0
- * clears the word afterwards.  Returns MLA_ERR_TIMEOUT if the word holds a
- * timeout, else MLA_OK. */
+/* Debug aid, with no counterpart in the method's published interface: while
+ * set, every decode entry point called from this host thread records which
+ * cache rows its kernels read, so that a test can compare the index and
+ * block-table handling with the inputs bit for bit.
+ *   trace     int32 device array (caller-owned) of `capacity` entries, or
+ *             NULL to switch the trace off.  A call writes two planes of N
+ *             entries each (plane 1 starts at trace + N):
+ *               dense and fused decode: N = batch * max_pages * 64; entry
+ *                 b * max_pages * 64 + t holds the physical slot
+ *                 (block * 64 + t % 64) that token t of sequence b was loaded
+ *                 from, plane 0 for the rows read as K and plane 1 for the
+ *                 rows read as V.  Only tokens of pages that hold part of the
+ *                 sequence are written (a partial last page in full); an
+ *                 out-of-range block id shows as block 0.
+ *               sparse decode, fused sparse decode and sparse prefill:
+ *                 N = (batch * s_q | s_q) * topk; entry p * topk + j holds
+ *                 the slot entry j of query p read (-1 if unused or out of
+ *                 range) in plane 0, and the row of the compacted buffer it
+ *                 went to (valid entries numbered in index order) in plane 1.
+ *             Entries the call does not write keep their contents.
+ *   capacity  entries of `trace`; a call needing more than 2 * N returns
+ *             MLA_ERR_INVALID_ARG before any launch.
+ * The setting belongs to the calling host thread. */
+MLA_API int mla_set_slot_trace(int32_t* trace, int64_t capacity);
+
+/* Reads the device status words that kernels set: 0 = ok, else (code << 16)
+ * | site of the first event, code 1 = a bounded wait expired, 2 = an input
+ * named nothing in the cache (a block id outside [0, num_blocks), a length
+ * above max_pages * 64, a sparse index outside [0, num_slots)).  A code-2
+ * fault does not stop any kernel: the block id reads block 0, the length is
+ * cut to max_pages * 64 (the default fused query position still follows the
+ * length as given), and the index is skipped like -1.  A timeout makes every
+ * later bounded wait give up until the words are reset, and it takes
+ * precedence in *status.  Synchronises the device; reset != 0 clears both
+ * words afterwards.  Returns MLA_ERR_TIMEOUT if a wait expired, else
+ * MLA_OK. */
 MLA_API int mla_device_status(int* status, int reset);
 
 #ifdef __cplusplus

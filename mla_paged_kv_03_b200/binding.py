@@ -32,7 +32,7 @@ EXPORTED = [
     "mla_set_kernel_events", "mla_sparse_v41_workspace_size", "mla_sparse_decode_v41",
     "mla_sparse_decode_v41_fp4", "mla_sparse_fused_workspace_size",
     "mla_sparse_fused_norm_rope_attn_rope_cast", "mla_sparse_prefill_workspace_size",
-    "mla_sparse_prefill_fwd",
+    "mla_sparse_prefill_fwd", "mla_set_slot_trace",
 ]
 
 
@@ -86,6 +86,7 @@ def lib():
         L.mla_device_status.argtypes = [ip, i32]
         L.mla_noalloc_scratch_bytes.argtypes = []
         L.mla_set_kernel_events.argtypes = [vp, vp]
+        L.mla_set_slot_trace.argtypes = [vp, i64]
         L.mla_decode_fwd_noalloc.argtypes = [vp, vp, vp, i32, i32, vp, i32, i32, i32, i32, i32,
                                              f32, i32, vp, vp, vp]
         for name in EXPORTED:
@@ -234,6 +235,18 @@ def mla_set_kernel_events(start: Optional[torch.cuda.Event], stop: Optional[torc
         None if stop is None else ctypes.c_void_p(stop.cuda_event)))
 
 
+def mla_set_slot_trace(trace: Optional[torch.Tensor]):
+    """Debug slot trace of the following decode calls of this thread: an
+    int32 device tensor the kernels write the physical slot of every cache row
+    they read into (two planes; layout in include/mla.h), or None to stop."""
+    if trace is None:
+        _check(lib().mla_set_slot_trace(None, 0))
+        return
+    _require(trace.dtype == torch.int32 and trace.is_cuda and trace.is_contiguous(),
+             "trace must be a contiguous int32 CUDA tensor")
+    _check(lib().mla_set_slot_trace(_ptr(trace), trace.numel()))
+
+
 def mla_noalloc_scratch_bytes() -> int:
     return int(lib().mla_noalloc_scratch_bytes())
 
@@ -345,8 +358,14 @@ def mla_sparse_decode(q, kcache_fp8, indices, d_v=512, softmax_scale=None, num_s
     return out, lse
 
 
+MLA_DEVERR_TIMEOUT = 1
+MLA_DEVERR_BAD_INDEX = 2
+
+
 def device_status(reset: bool = True) -> int:
-    """Device status word (0 = ok); synchronises the device."""
+    """Device status word (0 = ok, else code << 16 | site; code 1 = a wait
+    expired, 2 = an out-of-range block id, length or index); synchronises the
+    device."""
     v = ctypes.c_int(0)
     rc = lib().mla_device_status(ctypes.byref(v), int(bool(reset)))
     if rc not in (MLA_OK, MLA_ERR_TIMEOUT):

@@ -219,9 +219,10 @@ __global__ void __launch_bounds__(kCombineThreads) mla_combine_kernel(const Comb
   }
 }
 
-// Device-side planner: the block stages tiles_of(seqlens) in shared memory
-// (or, for very large batches, in the caller's scratch), then one thread runs
-// the same planner the host uses.
+// Device-side planner: one CTA stages the cost prefix sums of at most
+// kPlanMaxBatch sequences in shared memory (larger batches are rejected by
+// the entry points) and evaluates the host planner's closed forms, every
+// sequence and part in parallel.
 constexpr int kPlanThreads = 256;
 constexpr int kPlanMaxBatch = 8192;  // prefix sums live in shared memory
 

@@ -72,6 +72,11 @@ struct DecodeParams {
   float rope_base;
   const int32_t* positions;  // nullable: position = L - 1
   double inv_freq[kRope / 2];  // base^(-2k/64), computed on the host in fp64
+  // debug slot trace (null = off): int32 [2][batch][max_pages * 64], the
+  // physical slot of every token whose cache row a kernel loaded, plane 0 for
+  // the rows read as K, plane 1 for the rows read as V
+  int32_t* trace;
+  long long trace_plane;  // entries per plane
 };
 
 namespace cfg {
@@ -145,7 +150,9 @@ struct __align__(8) Ctrl {
 static_assert(sizeof(Ctrl) <= cfg::kMiscBytes, "control block too large");
 
 struct Unit {
-  int b, lo, hi, split, nsplit, L;
+  int b, lo, hi, split, nsplit;
+  int L;      // tokens attended: cache_seqlens[b], at most max_pages * 64
+  int L_raw;  // cache_seqlens[b] as given (the default query position is L_raw - 1)
 };
 
 // Iterates the (sequence, tile-range) segments of one scheduler part.
@@ -162,16 +169,25 @@ struct UnitIter {
   __device__ bool next(const DecodeParams& P, Unit& u) {
     while (b <= b_end) {
       const int bb = b++;
-      const int L = P.seqlens[bb];
+      const int L_raw = P.seqlens[bb];
       const int lo = (bb == b_first) ? t_begin : 0;
-      const int hi = (bb == b_end) ? t_end : tiles_of(L);
+      const int hi = (bb == b_end) ? t_end : tiles_of(L_raw);  // the planner's tiles
       if (lo >= hi) continue;
       u.b = bb;
       u.lo = lo;
       u.hi = hi;
       u.split = (bb == b_first) ? s_begin : 0;
       u.nsplit = P.num_splits[bb + 1] - P.num_splits[bb];
-      u.L = L;
+      u.L_raw = L_raw;
+      // A length beyond the block table's max_pages * 64 tokens is read as
+      // that many (the block table names no further page) and recorded as an
+      // input fault; tiles past it are fully masked, so every split the
+      // planner counted still writes its (empty) partial.
+      u.L = L_raw;
+      if (L_raw > P.max_pages * kPage) {
+        ptx::set_error(MLA_DEVERR_BAD_INDEX, 0x30);
+        u.L = P.max_pages * kPage;
+      }
       return true;
     }
     return false;
@@ -215,6 +231,18 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Debug slot trace: the calling warp records the physical slot (block * 64 +
+// offset) of the 64 tokens of page `page` of sequence b, in plane 0 (bit 0
+// of `planes`) and / or plane 1 (bit 1).
+__device__ __forceinline__ void trace_page(const DecodeParams& P, int b, int page, int blk,
+                                           int planes) {
+  int32_t* t = P.trace + (size_t)b * P.max_pages * kPage + (size_t)page * kPage;
+  for (int i = threadIdx.x & 31; i < kPage; i += 32) {
+    if (planes & 1) t[i] = blk * kPage + i;
+    if (planes & 2) t[P.trace_plane + i] = blk * kPage + i;
+  }
 }
 
 __device__ __forceinline__ int clamp_block(int blk, int num_blocks) {
@@ -307,7 +335,7 @@ __global__ void __launch_bounds__(Threads<kMode>::value, 1)
     int u_idx = 0;
     Unit u;
     bool ok = true;
-    auto load_pair = [&](const Unit& un, int tile, int pair) -> bool {
+    auto load_pair = [&](const Unit& un, int tile, int pair, int planes) -> bool {
       const uint32_t idx = ring_it++;
       if (static_cast<int>(idx % kL) != role) return true;
       const int slot = idx % kNPair;
@@ -317,16 +345,16 @@ __global__ void __launch_bounds__(Threads<kMode>::value, 1)
       const int c0 = 2 * pair;
       const int nch = (c0 + 1 < kNumChunks) ? 2 : 1;
       const int tok0 = tile * kTileT;
-      int npg = (un.L + kPage - 1) / kPage;
-      if (npg > P.max_pages) {
-        ptx::set_error(MLA_DEVERR_BAD_INDEX, 0x05);
-        npg = P.max_pages;
-      }
+      const int npg = (un.L + kPage - 1) / kPage;  // <= max_pages
       const int p0 = tok0 / kPage;
       int blk0 = p0 < npg ? P.block_table[(size_t)un.b * P.max_pages + p0] : 0;
       int blk1 = (p0 + 1 < npg) ? P.block_table[(size_t)un.b * P.max_pages + p0 + 1] : blk0;
       blk0 = clamp_block(blk0, P.num_blocks);
       blk1 = clamp_block(blk1, P.num_blocks);
+      if (P.trace && pair == 0) {
+        if (p0 < npg) trace_page(P, un.b, p0, blk0, planes);
+        if (p0 + 1 < npg) trace_page(P, un.b, p0 + 1, blk1, planes);
+      }
       if (ptx::elect_one_sync()) {
         ptx::mbar_arrive_expect_tx(&C.slot_full[slot], nch * kSubChunk);
         uint8_t* dst = sRing + slot * kPairBytes;
@@ -346,7 +374,7 @@ __global__ void __launch_bounds__(Threads<kMode>::value, 1)
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         const double pos =
-            P.positions ? static_cast<double>(P.positions[u.b]) : static_cast<double>(u.L - 1);
+            P.positions ? static_cast<double>(P.positions[u.b]) : static_cast<double>(u.L_raw - 1);
         double sn, cs;
         rope_sincos64(pos, P.inv_freq[lane], &sn, &cs);
         C.rope_cs[lane][0] = cs;
@@ -367,11 +395,11 @@ __global__ void __launch_bounds__(Threads<kMode>::value, 1)
       if (ok) {
         const int n = u.hi - u.lo;
         for (int k = 0; k < n && ok; ++k) {
-          for (int pr = 0; pr < 5 && ok; ++pr) ok = load_pair(u, u.lo + k, pr);
+          for (int pr = 0; pr < 5 && ok; ++pr) ok = load_pair(u, u.lo + k, pr, 1);
           if (k >= 1)
-            for (int pr = 0; pr < nv_pairs && ok; ++pr) ok = load_pair(u, u.lo + k - 1, pr);
+            for (int pr = 0; pr < nv_pairs && ok; ++pr) ok = load_pair(u, u.lo + k - 1, pr, 2);
         }
-        for (int pr = 0; pr < nv_pairs && ok; ++pr) ok = load_pair(u, u.hi - 1, pr);
+        for (int pr = 0; pr < nv_pairs && ok; ++pr) ok = load_pair(u, u.hi - 1, pr, 2);
       }
       ++u_idx;
     }

@@ -214,6 +214,26 @@ int launch_combine(const mla::CombineParams& cp, bool fused, cudaStream_t st) {
   return MLA_OK;
 }
 
+// Debug slot trace set by mla_set_slot_trace (per host thread).  The sparse
+// paths trace their gather and switch the trace off (TraceOff) around the
+// dense decode they run over the compacted rows.
+thread_local int32_t* t_trace = nullptr;
+thread_local long long t_trace_cap = 0;
+
+struct TraceOff {
+  int32_t* saved;
+  TraceOff() : saved(t_trace) { t_trace = nullptr; }
+  ~TraceOff() { t_trace = saved; }
+};
+
+int check_trace(long long entries_per_plane) {
+  if (!t_trace) return MLA_OK;
+  MLA_CHECK_ARG(t_trace_cap >= 2 * entries_per_plane,
+                "slot trace holds %lld entries, the call needs %lld", t_trace_cap,
+                2 * entries_per_plane);
+  return MLA_OK;
+}
+
 // Events set by mla_set_kernel_events (per host thread), recorded around the
 // attention kernel of each decode entry point.
 thread_local cudaEvent_t t_kernel_start = nullptr;
@@ -301,7 +321,8 @@ int check_common_dense(const void* q, const void* kcache, const int32_t* block_t
   MLA_CHECK_ARG(h_q >= 1, "h_q must be >= 1 (got %d)", h_q);
   MLA_CHECK_ARG(num_sm_parts >= 1 && num_sm_parts <= mla::kCombineMaxSplits,
                 "num_sm_parts must be in [1, %d] (got %d)", mla::kCombineMaxSplits, num_sm_parts);
-  MLA_CHECK_ARG(max_pages >= 1, "max_pages must be >= 1 (got %d)", max_pages);
+  MLA_CHECK_ARG(max_pages >= 1 && static_cast<long long>(max_pages) * mla::kPage < (1LL << 31),
+                "max_pages must be in [1, 2^31 / 64) (got %d)", max_pages);
   MLA_CHECK_ARG(num_blocks >= 1, "num_blocks must be >= 1 (got %d)", num_blocks);
   MLA_CHECK_ARG(static_cast<long long>(num_blocks) * mla::kPage < (1LL << 31),
                 "num_blocks * 64 must fit in int32");
@@ -315,6 +336,26 @@ int check_common_dense(const void* q, const void* kcache, const int32_t* block_t
                     aligned(num_splits, 4),
                 "int32 arrays must be 4-byte aligned");
   return MLA_OK;
+}
+
+// Every argument check of mla_decode_fwd (nothing is launched).
+int check_dense_decode(const void* q, const void* kcache, const int32_t* block_table,
+                       int max_pages, int num_blocks, const int32_t* cache_seqlens, int batch,
+                       int s_q, int h_q, int h_kv, int d_v, float softmax_scale,
+                       const int32_t* metadata, const int32_t* num_splits, int num_sm_parts,
+                       void* workspace, size_t workspace_bytes, void* out, float* lse) {
+  if (h_kv != 1) return fail(MLA_ERR_UNSUPPORTED, "h_kv must be 1 (got %d)", h_kv);
+  MLA_CHECK_ARG(s_q >= 1, "s_q must be >= 1 (got %d)", s_q);
+  MLA_CHECK_ARG(d_v == 512 || d_v == 576, "d_v must be 512 or 576 (got %d)", d_v);
+  int rc = check_common_dense(q, kcache, block_table, max_pages, num_blocks, cache_seqlens, batch,
+                              h_q, softmax_scale, metadata, num_splits, num_sm_parts, workspace);
+  if (rc != MLA_OK) return rc;
+  MLA_CHECK_ARG(out && lse, "null output pointer");
+  MLA_CHECK_ARG(aligned(out, 16) && aligned(lse, 4), "out must be 16-byte aligned, lse 4-byte");
+  const WsLayout w = dense_ws_layout(batch, s_q * h_q, d_v, num_sm_parts);
+  MLA_CHECK_ARG(workspace_bytes >= w.total, "workspace too small: %zu < %zu", workspace_bytes,
+                w.total);
+  return check_trace(static_cast<long long>(batch) * max_pages * mla::kPage);
 }
 
 // ------------------------------------------------- fixed-scratch decode
@@ -369,9 +410,12 @@ static int sparse_gather_and_plan(int row_bytes, const void* q, const uint8_t* k
                                   int64_t num_slots, const int32_t* indices, int topk, int pairs,
                                   int h_q, int num_sm_parts, uint8_t* ws, const SparseWs& w,
                                   void* stream, const void** q_dense,
-                                  const int32_t* topk_len = nullptr) {
+                                  const int32_t* topk_len = nullptr, int32_t* trace = nullptr,
+                                  long long trace_plane = 0) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   mla::GatherParams g{};
+  g.trace = trace;
+  g.trace_plane = trace_plane;
   g.cache = kcache;
   g.num_slots = num_slots;
   g.indices = indices;
@@ -430,13 +474,17 @@ static int sparse_decode_impl(int row_bytes, const void* q, const uint8_t* kcach
                 mla::kPlanMaxBatch, pairs);
   const long long pages = static_cast<long long>(pairs) * w.pages_per_pair;
   MLA_CHECK_ARG(pages * mla::kPage < (1LL << 31), "pairs * topk too large");
+  int rc = check_trace(static_cast<long long>(pairs) * topk);
+  if (rc != MLA_OK) return rc;
   if (batch == 0) return MLA_OK;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const void* q_dense = q;
-  int rc = sparse_gather_and_plan(row_bytes, q, kcache, num_slots, indices, topk, pairs, h_q,
-                                  num_sm_parts, ws, w, stream, &q_dense);
+  rc = sparse_gather_and_plan(row_bytes, q, kcache, num_slots, indices, topk, pairs, h_q,
+                              num_sm_parts, ws, w, stream, &q_dense, nullptr, t_trace,
+                              static_cast<long long>(pairs) * topk);
   if (rc != MLA_OK) return rc;
   // dense decode over the compacted rows: no causal mask, lengths = valid counts
+  TraceOff off;
   return mla_decode_fwd(q_dense, ws + w.rows_off, reinterpret_cast<int32_t*>(ws + w.bt_off),
                         w.pages_per_pair, static_cast<int>(pages),
                         reinterpret_cast<int32_t*>(ws + w.len_off), pairs, 1, h_q, 1, d_v,
@@ -457,7 +505,15 @@ int mla_decode_fwd_noalloc(const void* q, const void* kcache, const int32_t* blo
   MLA_CHECK_ARG(batch >= 0, "batch must be >= 0 (got %d)", batch);
   MLA_CHECK_ARG(s_q >= 1 && h_q >= 1, "s_q and h_q must be >= 1");
   MLA_CHECK_ARG(d_v == 512 || d_v == 576, "d_v must be 512 or 576 (got %d)", d_v);
-  if (batch == 0) return MLA_OK;
+  MLA_CHECK_ARG(batch <= mla::kPlanMaxBatch, "at most %d sequences (got %d)", mla::kPlanMaxBatch,
+                batch);
+  // the caller's pointers first (the scratch ones are checked with the rest below)
+  MLA_CHECK_ARG(q && kcache && block_table && cache_seqlens && out && lse,
+                "null device pointer argument");
+  MLA_CHECK_ARG(aligned(q, 16) && aligned(kcache, 16) && aligned(out, 16),
+                "q, kcache and out must be 16-byte aligned");
+  MLA_CHECK_ARG(aligned(block_table, 4) && aligned(cache_seqlens, 4) && aligned(lse, 4),
+                "block_table, cache_seqlens and lse must be 4-byte aligned");
   int dev = -1;
   MLA_CUDA(cudaGetDevice(&dev));
   const int R = s_q * h_q;
@@ -480,6 +536,12 @@ int mla_decode_fwd_noalloc(const void* q, const void* kcache, const int32_t* blo
   int32_t* metadata = reinterpret_cast<int32_t*>(b8);
   int32_t* num_splits = reinterpret_cast<int32_t*>(b8 + meta_bytes);
   void* ws = b8 + meta_bytes + splits_bytes;
+  // every check of the decode call, before the planner writes the shared array
+  if ((rc = check_dense_decode(q, kcache, block_table, max_pages, num_blocks, cache_seqlens, batch,
+                               s_q, h_q, h_kv, d_v, softmax_scale, metadata, num_splits, parts, ws,
+                               ws_bytes, out, lse)) != MLA_OK)
+    return rc;
+  if (batch == 0) return MLA_OK;
   if ((rc = mla_get_metadata(cache_seqlens, batch, R, h_kv, parts, metadata, num_splits,
                              stream)) != MLA_OK)
     return rc;
@@ -569,18 +631,12 @@ int mla_decode_fwd(const void* q, const void* kcache, const int32_t* block_table
                    int h_kv, int d_v, float softmax_scale, int causal, const int32_t* metadata,
                    const int32_t* num_splits, int num_sm_parts, void* workspace,
                    size_t workspace_bytes, void* out, float* lse, void* stream) {
-  if (h_kv != 1) return fail(MLA_ERR_UNSUPPORTED, "h_kv must be 1 (got %d)", h_kv);
-  MLA_CHECK_ARG(s_q >= 1, "s_q must be >= 1 (got %d)", s_q);
-  MLA_CHECK_ARG(d_v == 512 || d_v == 576, "d_v must be 512 or 576 (got %d)", d_v);
-  int rc = check_common_dense(q, kcache, block_table, max_pages, num_blocks, cache_seqlens, batch,
-                              h_q, softmax_scale, metadata, num_splits, num_sm_parts, workspace);
+  int rc = check_dense_decode(q, kcache, block_table, max_pages, num_blocks, cache_seqlens, batch,
+                              s_q, h_q, h_kv, d_v, softmax_scale, metadata, num_splits,
+                              num_sm_parts, workspace, workspace_bytes, out, lse);
   if (rc != MLA_OK) return rc;
-  MLA_CHECK_ARG(out && lse, "null output pointer");
-  MLA_CHECK_ARG(aligned(out, 16) && aligned(lse, 4), "out must be 16-byte aligned, lse 4-byte");
   const int R = s_q * h_q;
   const WsLayout w = dense_ws_layout(batch, R, d_v, num_sm_parts);
-  MLA_CHECK_ARG(workspace_bytes >= w.total, "workspace too small: %zu < %zu", workspace_bytes,
-                w.total);
   if (batch == 0) return MLA_OK;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
@@ -612,6 +668,8 @@ int mla_decode_fwd(const void* q, const void* kcache, const int32_t* block_table
   p.lse = lse;
   p.ws_o = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.o_off);
   p.ws_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.lse_off);
+  p.trace = t_trace;
+  p.trace_plane = static_cast<long long>(batch) * max_pages * mla::kPage;
   if (R <= mla::gcfg::kRows && d_v == 512) {
     p.n_groups = 1;
     if ((rc = launch_page_decode(q, kcache, p, st)) != MLA_OK) return rc;
@@ -656,6 +714,8 @@ int mla_fused_norm_rope_attn_rope_cast(
   const WsLayout w = dense_ws_layout(batch, R, d_v, num_sm_parts);
   MLA_CHECK_ARG(workspace_bytes >= w.total, "workspace too small: %zu < %zu", workspace_bytes,
                 w.total);
+  if ((rc = check_trace(static_cast<long long>(batch) * max_pages * mla::kPage)) != MLA_OK)
+    return rc;
   if (batch == 0) return MLA_OK;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
@@ -689,6 +749,8 @@ int mla_fused_norm_rope_attn_rope_cast(
   p.eps = eps;
   p.rope_base = rope_base;
   p.positions = positions;
+  p.trace = t_trace;
+  p.trace_plane = static_cast<long long>(batch) * max_pages * mla::kPage;
   for (int k = 0; k < mla::kRope / 2; ++k)
     p.inv_freq[k] = std::pow(static_cast<double>(rope_base), -2.0 * k / mla::kRope);
   if ((rc = launch_decode<mla::kFused>(tkv, tkv, p, st)) != MLA_OK) return rc;
@@ -777,7 +839,12 @@ int mla_sparse_prefill_fwd(const void* q, const void* kv, int64_t s_kv, const in
                 w.total);
   MLA_CHECK_ARG(static_cast<long long>(chunk) * w.pages_per_pair * mla::kPage < (1LL << 31),
                 "topk too large");
+  const long long trace_plane = static_cast<long long>(s_q) * topk;
+  int rc0 = check_trace(trace_plane);
+  if (rc0 != MLA_OK) return rc0;
   if (s_q == 0) return MLA_OK;
+  int32_t* trace = t_trace;
+  TraceOff off;  // the decode passes over the compacted rows are not traced
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const size_t q_row = static_cast<size_t>(h_q) * mla::kD;  // bf16 values per token
   for (int t0 = 0; t0 < s_q; t0 += chunk) {
@@ -787,7 +854,9 @@ int mla_sparse_prefill_fwd(const void* q, const void* kv, int64_t s_kv, const in
     int rc = sparse_gather_and_plan(mla::kRowBf16, q_t, static_cast<const uint8_t*>(kv), s_kv,
                                     indices + static_cast<size_t>(t0) * topk, topk, n, h_q,
                                     num_sm_parts, ws, w, stream, &q_dense,
-                                    topk_length ? topk_length + t0 : nullptr);
+                                    topk_length ? topk_length + t0 : nullptr,
+                                    trace ? trace + static_cast<size_t>(t0) * topk : nullptr,
+                                    trace_plane);
     if (rc != MLA_OK) return rc;
     rc = mla_decode_fwd(q_dense, ws + w.rows_off, reinterpret_cast<int32_t*>(ws + w.bt_off),
                         w.pages_per_pair, n * w.pages_per_pair,
@@ -843,13 +912,17 @@ int mla_sparse_fused_norm_rope_attn_rope_cast(
                 batch);
   const long long pages = static_cast<long long>(batch) * w.pages_per_pair;
   MLA_CHECK_ARG(pages * mla::kPage < (1LL << 31), "batch * topk too large");
+  int rc = check_trace(static_cast<long long>(batch) * topk);
+  if (rc != MLA_OK) return rc;
   if (batch == 0) return MLA_OK;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const void* q_dense = q_raw;
-  int rc = sparse_gather_and_plan(mla::kRow656, q_raw, kcache_fp8, num_slots, indices, topk,
-                                  batch, h_q, num_sm_parts, ws, w, stream, &q_dense);
+  rc = sparse_gather_and_plan(mla::kRow656, q_raw, kcache_fp8, num_slots, indices, topk, batch,
+                              h_q, num_sm_parts, ws, w, stream, &q_dense, nullptr, t_trace,
+                              static_cast<long long>(batch) * topk);
   if (rc != MLA_OK) return rc;
   // the fused steps over the compacted rows; every query sees all its rows
+  TraceOff off;
   return mla_fused_norm_rope_attn_rope_cast(
       q_raw, norm_gain, eps, rope_base, positions, ws + w.rows_off,
       reinterpret_cast<int32_t*>(ws + w.bt_off), w.pages_per_pair, static_cast<int>(pages),
@@ -877,6 +950,14 @@ int mla_sparse_decode_v41(const void* q, const uint8_t* kcache_528, int64_t num_
 }
 
 
+int mla_set_slot_trace(int32_t* trace, int64_t capacity) {
+  MLA_CHECK_ARG(!trace || capacity >= 0, "capacity must be >= 0");
+  MLA_CHECK_ARG(aligned(trace, 4), "trace must be 4-byte aligned");
+  t_trace = trace;
+  t_trace_cap = trace ? capacity : 0;
+  return MLA_OK;
+}
+
 int mla_set_kernel_events(void* start_event, void* stop_event) {
   t_kernel_start = static_cast<cudaEvent_t>(start_event);
   t_kernel_stop = static_cast<cudaEvent_t>(stop_event);
@@ -886,15 +967,17 @@ int mla_set_kernel_events(void* start_event, void* stop_event) {
 int mla_device_status(int* status, int reset) {
   MLA_CHECK_ARG(status, "status is null");
   MLA_CUDA(cudaDeviceSynchronize());
-  int v = 0;
-  MLA_CUDA(cudaMemcpyFromSymbol(&v, mla::ptx::g_status, sizeof(int)));
-  *status = v;
+  int fault = 0, abort_word = 0;
+  MLA_CUDA(cudaMemcpyFromSymbol(&fault, mla::ptx::g_status, sizeof(int)));
+  MLA_CUDA(cudaMemcpyFromSymbol(&abort_word, mla::ptx::g_abort, sizeof(int)));
+  *status = abort_word != 0 ? abort_word : fault;
   if (reset) {
     const int z = 0;
     MLA_CUDA(cudaMemcpyToSymbol(mla::ptx::g_status, &z, sizeof(int)));
+    MLA_CUDA(cudaMemcpyToSymbol(mla::ptx::g_abort, &z, sizeof(int)));
   }
-  if ((v >> 16) == mla::MLA_DEVERR_TIMEOUT)
-    return fail(MLA_ERR_TIMEOUT, "a kernel wait timed out (site 0x%x)", v & 0xFFFF);
+  if (abort_word != 0)
+    return fail(MLA_ERR_TIMEOUT, "a kernel wait timed out (site 0x%x)", abort_word & 0xFFFF);
   return MLA_OK;
 }
 

@@ -144,7 +144,6 @@ __global__ void __launch_bounds__(gcfg::kThreads, 1)
         ptx::tma_load_3d(sQ, &tm_q, &C.q_full, 0, u.b * P.R, 0);
       }
       __syncwarp();
-      if ((u.L + kPage - 1) / kPage > P.max_pages) ptx::set_error(MLA_DEVERR_BAD_INDEX, 0x85);
       int p0, np;
       page_range(u, p0, np);
       for (int k = 0; k < np && ok; ++k) {
@@ -157,6 +156,7 @@ __global__ void __launch_bounds__(gcfg::kThreads, 1)
         }
         const int blk =
             clamp_block(P.block_table[(size_t)u.b * P.max_pages + p0 + k], P.num_blocks);
+        if (P.trace) trace_page(P, u.b, p0 + k, blk, 3);  // the slot serves K and V
         if (ptx::elect_one_sync()) {
           ptx::mbar_arrive_expect_tx(&C.slot_full[slot], kPageBytes);
           ptx::tma_load_3d(sSlot + slot * kPageBytes, &tm_page, &C.slot_full[slot], 0,

@@ -165,15 +165,17 @@ __global__ void __launch_bounds__(pcfg::kThreads, 1)
   // Physical block of logical page `page`; pages past the sequence or past
   // this split's last tile load `fallback` instead (their tokens are masked).
   auto page_block = [&](const Unit& un, int page, int fallback) -> int {
-    int npg = (un.L + kPage - 1) / kPage;
-    if (npg > P.max_pages) {
-      ptx::set_error(MLA_DEVERR_BAD_INDEX, 0x45);
-      npg = P.max_pages;
-    }
+    const int npg = (un.L + kPage - 1) / kPage;  // <= max_pages
     const int end = min(npg, 2 * un.hi);
     const int pg = page < end ? page : fallback;
     const int blk = pg < npg ? P.block_table[(size_t)un.b * P.max_pages + pg] : 0;
     return clamp_block(blk, P.num_blocks);
+  };
+  // Debug slot trace of the pages a load reads (pages a load only pads with
+  // are not recorded).
+  auto trace_if_real = [&](const Unit& un, int page, int blk, int planes) {
+    const int npg = (un.L + kPage - 1) / kPage;
+    if (page < npg && page < 2 * un.hi) trace_page(P, un.b, page, blk, planes);
   };
 
   if (warp == 0 || warp >= 2 + kSoftmaxWarps) {
@@ -197,6 +199,10 @@ __global__ void __launch_bounds__(pcfg::kThreads, 1)
       const int p0 = 2 * (un.lo + 2 * i);
       const int kb0 = page_block(un, p0 + 2 * static_cast<int>(rank), p0);
       const int kb1 = page_block(un, p0 + 2 * static_cast<int>(rank) + 1, p0);
+      if (P.trace && role == 0) {
+        trace_if_real(un, p0 + 2 * static_cast<int>(rank), kb0, 1);
+        trace_if_real(un, p0 + 2 * static_cast<int>(rank) + 1, kb1, 1);
+      }
       for (int c = 0; c < kNumChunks; ++c) {
         int s;
         bool mine;
@@ -219,6 +225,8 @@ __global__ void __launch_bounds__(pcfg::kThreads, 1)
       int vb[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) vb[q] = page_block(un, p0 + q, p0);
+      if (P.trace && role == 0)
+        for (int q = 0; q < 4; ++q) trace_if_real(un, p0 + q, vb[q], 2);
       for (int j = 0; j < 2; ++j)
         for (int q = 0; q < 4; ++q) {
           int s;

@@ -2,7 +2,7 @@
 // (TMEM allocation, UMMA issue/commit, TMEM loads/stores) and fences.
 //
 // Every wait is bounded: a spin that exceeds the global-timer budget records
-// MLA_DEVERR_TIMEOUT plus a site code in the device status word and returns
+// MLA_DEVERR_TIMEOUT plus a site code in the device abort word and returns
 // false, so callers can unwind instead of hanging the GPU.
 #pragma once
 #include <cstdint>
@@ -26,16 +26,21 @@ __device__ __forceinline__ uint64_t globaltimer() {
 
 // ------------------------------------------------------------------ status
 
-// Device-wide status word: 0 = ok; otherwise (code << 16) | site.  The
-// library is one translation unit, so the definition lives here.
+// Device-wide status words, each 0 = ok, otherwise (code << 16) | site of the
+// first event recorded.  g_status holds the first input fault (a bad block id,
+// index or length), which the kernels replace by a documented stand-in and
+// then carry on; g_abort holds the first bounded wait that expired, and only
+// it makes the other waits give up.  The library is one translation unit, so
+// the definitions live here.
 __device__ int g_status = 0;
+__device__ int g_abort = 0;
 
 __device__ __forceinline__ bool aborted() {
-  return *reinterpret_cast<volatile int*>(&g_status) != 0;
+  return *reinterpret_cast<volatile int*>(&g_abort) != 0;
 }
 
 __device__ __forceinline__ void set_error(int code, int site) {
-  atomicCAS(&g_status, 0, (code << 16) | (site & 0xFFFF));
+  atomicCAS(code == MLA_DEVERR_TIMEOUT ? &g_abort : &g_status, 0, (code << 16) | (site & 0xFFFF));
 }
 
 // ---------------------------------------------------------------- mbarrier

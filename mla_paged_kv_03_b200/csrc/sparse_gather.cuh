@@ -53,6 +53,11 @@ struct GatherParams {
   const __nv_bfloat16* q512;
   __nv_bfloat16* q576;
   int h_q;
+  // debug slot trace (null = off): int32 [2][pairs][topk]; plane 0 holds the
+  // slot each entry read (-1 for an unused entry), plane 1 the row of the
+  // compacted buffer it went to (-1 likewise)
+  int32_t* trace;
+  long long trace_plane;  // entries per plane
 };
 
 // E8M0 byte -> fp32: 2^(e - 127) (e = 0 is the fp32 subnormal 2^-127),
@@ -152,6 +157,11 @@ __global__ void __launch_bounds__(kGatherCtaThreads, gather_min_ctas<kRowBytes>(
   if (tid < kGatherTokens && s_dst[tid] >= 0)
     s_dst[tid] += before + (tid >= 32 ? s_base : 0);
   __syncthreads();
+  if (G.trace && tid < kGatherTokens && c * kGatherTokens + tid < G.topk) {
+    int32_t* t = G.trace + (size_t)b * G.topk + c * kGatherTokens + tid;
+    t[0] = s_dst[tid] >= 0 ? s_idx[tid] : -1;
+    t[G.trace_plane] = s_dst[tid];
+  }
 
   __nv_bfloat16* out_b = G.rows + (size_t)b * G.pages_per_pair * kGatherTokens * kD;
   if (tid == 0) G.block_table[(size_t)b * G.pages_per_pair + c] = b * G.pages_per_pair + c;

@@ -172,8 +172,17 @@ def _prefill(L, **o):
                                     0.04, 74, a["ws"], 1 << 30, a["out"], a["lse"], None)
 
 
+def _noalloc(L, **o):
+    a = dict(q=16, kc=16, bt=16, sl=16, out=16, lse=16)
+    a.update(o)
+    return L.mla_decode_fwd_noalloc(a["q"], a["kc"], a["bt"], 4, 100, a["sl"], 2, 1, 16, 1, 512,
+                                    0.04, 1, a["out"], a["lse"], None)
+
+
 @pytest.mark.parametrize("call,pointer", [
     (lambda L, **o: _sparse(L, **o), p) for p in ("q", "kc", "idx", "ws", "out", "lse")
+] + [
+    (lambda L, **o: _noalloc(L, **o), p) for p in ("q", "kc", "bt", "sl", "out", "lse")
 ] + [
     (lambda L, **o: _v41("mla_sparse_decode_v41", L, **o), p)
     for p in ("q", "kc", "idx", "ws", "out", "lse")
@@ -193,3 +202,20 @@ def test_null_pointers_are_rejected_before_launch(call, pointer):
     L = B.lib()
     assert call(L, **{pointer: None}) == B.MLA_ERR_INVALID_ARG
     assert L.mla_last_error().decode() != ""
+
+
+def test_slot_trace_too_small_is_rejected_before_launch():
+    L = B.lib()
+    assert L.mla_set_slot_trace(16, 200) == B.MLA_OK  # each call below needs >= 256
+    try:
+        assert call_decode() == B.MLA_ERR_INVALID_ARG
+        assert "slot trace" in L.mla_last_error().decode()
+        assert _sparse(L) == B.MLA_ERR_INVALID_ARG
+        assert _prefill(L) == B.MLA_ERR_INVALID_ARG
+    finally:
+        assert L.mla_set_slot_trace(None, 0) == B.MLA_OK
+    assert L.mla_set_slot_trace(18, 100) == B.MLA_ERR_INVALID_ARG  # misaligned
+
+
+def test_max_pages_beyond_int32_tokens_is_rejected():
+    assert call_decode(max_pages=1 << 25) == B.MLA_ERR_INVALID_ARG

@@ -30,12 +30,15 @@ def _noalloc(case, q, kc, bt, sl):
 
 
 def test_noalloc_matches_workspace_path_on_consecutive_calls():
-    # 32 rows per sequence (1-CTA kernel), then 128 rows (CTA-pair kernel),
-    # then the first case again: each call reuses the same scratch array.
+    # 32 rows per sequence (page kernel), 128 rows (CTA-pair kernel), d_v 576
+    # (1-CTA kernel, whose partials are 576 wide), then the first case again:
+    # each call reuses the same scratch array.
     cases = [
         W.make_dense(W.lengths_loguniform(24, 64, 6000, seed=5), 2, 16, seed=5, name="mem"),
         W.make_dense(W.lengths_uniform(3, 500, 3000, seed=6), 1, 128, seed=6, q_std=0.5,
                      k_std=0.5, name="h128"),
+        W.make_dense(W.lengths_uniform(5, 100, 4000, seed=8), 1, 64, seed=8, d_v=576,
+                     name="dv576"),
     ]
     cases.append(cases[0])
     for case in cases:
