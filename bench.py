@@ -492,6 +492,9 @@ def time_steps(gs, steps, graph, dev):
     ms_step = ev0.elapsed_time(ev1) / steps
     ks = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     ke = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    for e in ks + ke:
+        e.record(st)  # creates the CUDA event behind the handle
+    torch.cuda.synchronize(dev)
     for i in range(steps):
         gs.B.mla_set_kernel_events(ks[i], ke[i])
         gs.step()
