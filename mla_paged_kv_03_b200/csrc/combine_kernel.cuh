@@ -253,15 +253,16 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* total) {
 
 // Split-KV planner of one CTA: the closed forms of mla_common.h evaluated in
 // parallel (prefix sums by block scans, one metadata row per thread).
-__device__ void plan_block(const int32_t* seqlens, int batch, int num_parts,
+__device__ void plan_block(const int32_t* seqlens, int batch, int num_parts, int o, int g,
                            int32_t* metadata, int32_t* num_splits) {
+  const int u = g * kPlanTileCost;
   __shared__ int32_t C[kPlanMaxBatch + 1];
   const int tid = threadIdx.x;
   int carry = 0;
   for (int base = 0; base < batch; base += kPlanThreads) {
     const int b = base + tid;
     const int L = b < batch ? seqlens[b] : 0;
-    const int v = b < batch ? tiles_of(L) + kSegmentOverheadTiles : 0;
+    const int v = b < batch ? o + u * granules_of(L, g) : 0;
     int chunk_total;
     const int ex = block_exclusive_scan(v, &chunk_total);
     if (b < batch) C[b] = carry + ex;
@@ -269,14 +270,14 @@ __device__ void plan_block(const int32_t* seqlens, int batch, int num_parts,
   }
   if (tid == 0) C[batch] = carry;
   __syncthreads();
-  const int w = plan_width(carry, num_parts);
+  const int w = plan_width(carry, num_parts, u);
   for (int p = tid; p < num_parts; p += kPlanThreads)
-    plan_part_row(C, batch, w, p, metadata + p * kMetaInts);
+    plan_part_row(C, batch, w, o, g, p, metadata + p * kMetaInts);
   int nsum = 0;
   if (tid == 0) num_splits[0] = 0;
   for (int base = 0; base < batch; base += kPlanThreads) {
     const int b = base + tid;
-    const int v = b < batch ? plan_last_part(C, b, w) - plan_first_part(C, b, w) + 1 : 0;
+    const int v = b < batch ? plan_last_part(C, b, w, u) - plan_first_part(C, b, w, o) + 1 : 0;
     int chunk_total;
     const int ex = block_exclusive_scan(v, &chunk_total);
     if (b < batch) num_splits[b + 1] = nsum + ex + v;
@@ -285,11 +286,12 @@ __device__ void plan_block(const int32_t* seqlens, int batch, int num_parts,
 }
 
 __global__ void __launch_bounds__(kPlanThreads) mla_plan_kernel(const int32_t* seqlens, int batch,
-                                                               int num_parts, int32_t* metadata,
+                                                               int num_parts, int overhead,
+                                                               int granule, int32_t* metadata,
                                                                int32_t* num_splits) {
   ptx::grid_dep_wait();
   ptx::grid_dep_launch();  // the decode grid waits for this one at its start
-  plan_block(seqlens, batch, num_parts, metadata, num_splits);
+  plan_block(seqlens, batch, num_parts, overhead, granule, metadata, num_splits);
 }
 
 }  // namespace mla

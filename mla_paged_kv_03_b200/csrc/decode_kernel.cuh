@@ -171,7 +171,8 @@ struct UnitIter {
       const int bb = b++;
       const int L_raw = P.seqlens[bb];
       const int lo = (bb == b_first) ? t_begin : 0;
-      const int hi = (bb == b_end) ? t_end : tiles_of(L_raw);  // the planner's tiles
+      const int tiles = tiles_of(L_raw);  // the planner's tiles
+      const int hi = (bb == b_end) ? min(t_end, tiles) : tiles;
       if (lo >= hi) continue;
       u.b = bb;
       u.lo = lo;

@@ -106,23 +106,6 @@ int make_latent_map3(CUtensorMap* map, const void* base, long long rows, int box
   return MLA_OK;
 }
 
-template <int kMode>
-int prepare_kernel() {
-  static int done = 0;
-  static int rc = MLA_OK;
-  static std::mutex mu;
-  std::lock_guard<std::mutex> lk(mu);
-  if (!done) {
-    cudaError_t e = cudaFuncSetAttribute(mla::mla_decode_kernel<kMode>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         mla::cfg::kSmemBytes);
-    rc = (e == cudaSuccess) ? MLA_OK
-                            : fail(MLA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-    done = 1;
-  }
-  return rc;
-}
-
 struct WsLayout {
   size_t o_off, lse_off, total;
 };
@@ -249,11 +232,21 @@ int record_stop(cudaStream_t st) {
   return MLA_OK;
 }
 
+// 1-CTA kernel (tokens on M = 128, V re-read for PV) for 33..64 query rows per
+// CTA, d_v 576 and the fused variant.
 template <int kMode>
 int launch_decode(const CUtensorMap& tq, const CUtensorMap& tkv, const mla::DecodeParams& p,
                   cudaStream_t st) {
-  int rc = prepare_kernel<kMode>();
-  if (rc != MLA_OK) return rc;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(mla::mla_decode_kernel<kMode>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    mla::cfg::kSmemBytes);
+  });
+  if (attr_err != cudaSuccess)
+    return fail(MLA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(attr_err));
+  int rc = MLA_OK;
   const unsigned grid = static_cast<unsigned>(p.num_parts * p.n_groups);
   if ((rc = record_start(st)) != MLA_OK) return rc;
   PdlLaunch L(dim3(grid), dim3(mla::Threads<kMode>::value), mla::cfg::kSmemBytes, st);
@@ -262,28 +255,25 @@ int launch_decode(const CUtensorMap& tq, const CUtensorMap& tkv, const mla::Deco
 }
 
 // Page-resident kernel for up to 32 query rows per KV head (d_v 512).
-int launch_page_decode(const void* q, const void* kcache, const mla::DecodeParams& p,
+int launch_page_decode(const void* q, const CUtensorMap& tkv, const mla::DecodeParams& p,
                        cudaStream_t st) {
-  CUtensorMap tq3, tpage;
+  using Cfg = mla::PageCfg;
+  CUtensorMap tq3;
   int rc = make_latent_map3(&tq3, q, static_cast<long long>(p.batch) * p.R, mla::kNumChunks,
-                            mla::gcfg::kRows);
+                            Cfg::kRows);
   if (rc != MLA_OK) return rc;
-  if ((rc = make_latent_map3(&tpage, kcache, static_cast<long long>(p.num_blocks) * mla::kPage,
-                             mla::kNumChunks)) != MLA_OK)
-    return rc;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
     attr_err = cudaFuncSetAttribute(mla::mla_page_decode_kernel,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    mla::gcfg::kSmemBytes);
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
   });
   if (attr_err != cudaSuccess)
     return fail(MLA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(attr_err));
-  PdlLaunch L(dim3(static_cast<unsigned>(p.num_parts)), dim3(mla::gcfg::kThreads),
-              mla::gcfg::kSmemBytes, st);
+  PdlLaunch L(dim3(static_cast<unsigned>(p.num_parts * p.n_groups)), dim3(Cfg::kThreads),
+              Cfg::kSmemBytes, st);
   if ((rc = record_start(st)) != MLA_OK) return rc;
-  MLA_CUDA(cudaLaunchKernelEx(&L.cfg, mla::mla_page_decode_kernel, tq3, tpage, p));
+  MLA_CUDA(cudaLaunchKernelEx(&L.cfg, mla::mla_page_decode_kernel, tq3, tkv, p));
   return record_stop(st);
 }
 
@@ -592,7 +582,8 @@ int mla_get_metadata(const int32_t* cache_seqlens, int batch, int heads_per_kv, 
   MLA_CHECK_ARG(batch <= mla::kPlanMaxBatch, "the device planner takes at most %d sequences (got %d)",
                 mla::kPlanMaxBatch, batch);
   mla::mla_plan_kernel<<<1, mla::kPlanThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-      cache_seqlens, batch, num_sm_parts, metadata, num_splits);
+      cache_seqlens, batch, num_sm_parts, mla::plan_overhead(heads_per_kv),
+      mla::plan_granule(heads_per_kv), metadata, num_splits);
   MLA_CUDA(cudaGetLastError());
   return MLA_OK;
 }
@@ -605,16 +596,19 @@ int mla_get_metadata_host(const int32_t* cache_seqlens, int batch, int heads_per
   MLA_CHECK_ARG(metadata && num_splits && (cache_seqlens || batch == 0), "null host pointer");
   for (int b = 0; b < batch; ++b)
     MLA_CHECK_ARG(cache_seqlens[b] >= 0, "cache_seqlens[%d] = %d is negative", b, cache_seqlens[b]);
-  std::vector<int32_t> tiles(static_cast<size_t>(batch));
+  const int o = mla::plan_overhead(heads_per_kv);
+  const int g = mla::plan_granule(heads_per_kv);
+  std::vector<int32_t> granules(static_cast<size_t>(batch));
   long long total = 0;
   for (int b = 0; b < batch; ++b) {
-    tiles[b] = mla::tiles_of(cache_seqlens[b]);
-    total += tiles[b] + mla::kSegmentOverheadTiles;
+    granules[b] = mla::granules_of(cache_seqlens[b], g);
+    total += o + static_cast<long long>(mla::kPlanTileCost) * g * granules[b];
   }
   MLA_CHECK_ARG(total <= mla::kPlanMaxTotal, "total planner cost %lld above %lld", total,
                 mla::kPlanMaxTotal);
   std::vector<int32_t> prefix(static_cast<size_t>(batch) + 1);
-  mla::plan_splits_host(tiles.data(), batch, num_sm_parts, metadata, num_splits, prefix.data());
+  mla::plan_splits_host(granules.data(), batch, num_sm_parts, o, g, metadata, num_splits,
+                        prefix.data());
   return MLA_OK;
 }
 
@@ -640,8 +634,7 @@ int mla_decode_fwd(const void* q, const void* kcache, const int32_t* block_table
   if (batch == 0) return MLA_OK;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
-  CUtensorMap tq, tkv;
-  if ((rc = make_latent_map(&tq, q, static_cast<long long>(batch) * R)) != MLA_OK) return rc;
+  CUtensorMap tkv;
   if ((rc = make_latent_map(&tkv, kcache, static_cast<long long>(num_blocks) * mla::kPage)) !=
       MLA_OK)
     return rc;
@@ -670,15 +663,18 @@ int mla_decode_fwd(const void* q, const void* kcache, const int32_t* block_table
   p.ws_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.lse_off);
   p.trace = t_trace;
   p.trace_plane = static_cast<long long>(batch) * max_pages * mla::kPage;
-  if (R <= mla::gcfg::kRows && d_v == 512) {
+  if (R <= 32 && d_v == 512) {
     p.n_groups = 1;
-    if ((rc = launch_page_decode(q, kcache, p, st)) != MLA_OK) return rc;
+    rc = launch_page_decode(q, tkv, p, st);
   } else if (R > mla::kRowsPerCta && d_v == 512) {
     p.n_groups = mla::ceil_div(R, 2 * mla::kRowsPerCta);
-    if ((rc = launch_pair_decode(q, kcache, tkv, p, st)) != MLA_OK) return rc;
-  } else if ((rc = launch_decode<mla::kDense>(tq, tkv, p, st)) != MLA_OK) {
-    return rc;
+    rc = launch_pair_decode(q, kcache, tkv, p, st);
+  } else {
+    CUtensorMap tq;
+    if ((rc = make_latent_map(&tq, q, static_cast<long long>(batch) * R)) != MLA_OK) return rc;
+    rc = launch_decode<mla::kDense>(tq, tkv, p, st);
   }
+  if (rc != MLA_OK) return rc;
 
   mla::CombineParams cp{};
   cp.batch = batch;
@@ -753,7 +749,8 @@ int mla_fused_norm_rope_attn_rope_cast(
   p.trace_plane = static_cast<long long>(batch) * max_pages * mla::kPage;
   for (int k = 0; k < mla::kRope / 2; ++k)
     p.inv_freq[k] = std::pow(static_cast<double>(rope_base), -2.0 * k / mla::kRope);
-  if ((rc = launch_decode<mla::kFused>(tkv, tkv, p, st)) != MLA_OK) return rc;
+  rc = launch_decode<mla::kFused>(tkv, tkv, p, st);
+  if (rc != MLA_OK) return rc;
 
   mla::CombineParams cp{};
   cp.batch = batch;

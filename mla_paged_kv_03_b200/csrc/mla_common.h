@@ -30,12 +30,39 @@ constexpr int kRowsPerCta = 64;
 constexpr int kChunkD = 64;
 constexpr int kNumChunks = kD / kChunkD;  // 9
 
-// Planner cost of one work segment beyond its tiles (Q load, pipeline fill,
-// epilogue), in tile units.
-constexpr int kSegmentOverheadTiles = 2;
+// Planner costs, in units of a quarter tile (32 tokens): a tile costs
+// kPlanTileCost; one work segment (a sequence, or the part of one, that a CTA
+// takes) costs a further overhead for its Q load, pipeline fill and epilogue.
+// Work is dealt in granules of whole tiles: two for the CTA-pair kernel, which
+// steps over 256 tokens at a time (a split of an odd tile count would leave
+// half a step idle), one tile for the others.  The overhead and the granule
+// depend on the kernel that will run, which the planner knows from the rows
+// per KV head; the overheads are the fastest values of sweeps over the
+// benchmark workloads on B200.
+constexpr int kPlanTileCost = 4;
+#ifndef MLA_PLAN_OVH_PAGE
+#define MLA_PLAN_OVH_PAGE 4
+#endif
+#ifndef MLA_PLAN_OVH_CTA
+#define MLA_PLAN_OVH_CTA 16
+#endif
+#ifndef MLA_PLAN_OVH_PAIR
+#define MLA_PLAN_OVH_PAIR 8
+#endif
+constexpr int kPlanOverheadPage = MLA_PLAN_OVH_PAGE;  // <= 32 rows per KV head (page kernel)
+constexpr int kPlanOverheadCta = MLA_PLAN_OVH_CTA;    // 33..64 rows (1-CTA kernel)
+constexpr int kPlanOverheadPair = MLA_PLAN_OVH_PAIR;  // > 64 rows (CTA-pair kernel)
+
+MLA_HD inline int plan_overhead(int heads_per_kv) {
+  return heads_per_kv <= 32 ? kPlanOverheadPage
+                            : (heads_per_kv <= 64 ? kPlanOverheadCta : kPlanOverheadPair);
+}
+
+MLA_HD inline int plan_granule(int heads_per_kv) { return heads_per_kv > 64 ? 2 : 1; }
 
 // Metadata row per SM part: {begin_b, begin_tile, end_b, end_tile,
-// first_split, 0, 0, 0}; end_tile is exclusive within batch end_b.
+// first_split, 0, 0, 0}; end_tile is exclusive within batch end_b (it may pass
+// that sequence's last tile, see the planner below).
 constexpr int kMetaInts = 8;
 
 // Device status codes (upper 16 bits of the status word).
@@ -51,26 +78,34 @@ MLA_HD inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
 // O = 0, LSE = -inf result.
 MLA_HD inline int tiles_of(int L) { return L > 0 ? ceil_div(L, kTileT) : 1; }
 
+// Planner granules (of g tiles) a sequence of length L contributes.
+MLA_HD inline int granules_of(int L, int g) { return (tiles_of(L) + g - 1) / g; }
+
 // The planner counts in int32: the total cost sum(tiles + overhead) of a
 // call must stay below this (checked by the entry points).
 constexpr long long kPlanMaxTotal = (1LL << 30);
 
 // ------------------------------------------------------- split-KV planner
 //
-// The sequences' work is laid out on one cost line: sequence b occupies
-// [C[b], C[b+1]) with C[b+1] = C[b] + kSegmentOverheadTiles + tiles_of(L_b);
-// its overhead positions come first and tile t sits at C[b] + overhead + t.
-// The line is cut into num_parts intervals of width W = ceil(total /
-// num_parts); part p takes the tiles whose positions fall in [pW, (p+1)W).
-// Each part therefore covers one contiguous run of (sequence, tile) pairs and
-// costs at most W plus one segment overhead (that of a sequence continued
-// from the previous part).  Every quantity below is a closed form of C, so
-// the device planner computes all parts and sequences in parallel and the
-// host planner reaches the identical result with plain loops.
+// The sequences' work is laid out on one cost line: with granules of g tiles,
+// each costing u = g * kPlanTileCost, sequence b occupies [C[b], C[b+1]) with
+// C[b+1] = C[b] + o + u * granules_of(L_b, g) (o the segment overhead); its
+// overhead comes first and granule t starts at C[b] + o + u t.  The line is
+// cut into num_parts intervals of width W = ceil(total / num_parts); part p
+// takes the granules whose start falls in [pW, (p+1)W).  Each part therefore
+// covers one contiguous run of (sequence, tile) pairs and costs at most W plus
+// one granule and one segment overhead (that of a sequence continued from the
+// previous part).  Tile indices in the metadata are granule indices times g;
+// a part's end tile may pass its last sequence's tiles by less than g (the
+// kernels clamp it).  Every quantity below is a closed form of C, so the
+// device planner computes all parts and sequences in parallel and the host
+// planner reaches the identical result with plain loops.
 
-MLA_HD inline int plan_width(int total, int num_parts) {
+// At least one granule (u) wide, so that every interval lying within a
+// sequence's granules holds a granule start (the split counts rely on that).
+MLA_HD inline int plan_width(int total, int num_parts, int u) {
   const int w = (total + num_parts - 1) / num_parts;
-  return w < 1 ? 1 : w;
+  return w < u ? u : w;
 }
 
 // Sequence b with C[b] <= x < C[b+1] (C holds batch + 1 prefix sums).
@@ -86,11 +121,14 @@ MLA_HD inline int plan_seq_at(const int32_t* C, int batch, int x) {
   return lo;
 }
 
-// Parts holding tiles of sequence b: [plan_first_part(b), plan_last_part(b)].
-MLA_HD inline int plan_first_part(const int32_t* C, int b, int w) {
-  return (C[b] + kSegmentOverheadTiles) / w;
+// Parts holding tiles of sequence b: [plan_first_part(b), plan_last_part(b)]
+// (the parts of its first and last granule starts; u = granule cost).
+MLA_HD inline int plan_first_part(const int32_t* C, int b, int w, int o) {
+  return (C[b] + o) / w;
 }
-MLA_HD inline int plan_last_part(const int32_t* C, int b, int w) { return (C[b + 1] - 1) / w; }
+MLA_HD inline int plan_last_part(const int32_t* C, int b, int w, int u) {
+  return (C[b + 1] - u) / w;
+}
 
 MLA_HD inline void plan_mark_empty(int32_t* m, int batch) {
   m[0] = batch;  // empty part: begins after every sequence
@@ -102,8 +140,9 @@ MLA_HD inline void plan_mark_empty(int32_t* m, int batch) {
 
 // Metadata row of part p: {begin_b, begin_tile, end_b, end_tile (exclusive),
 // first_split, 0, 0, 0}, or an empty row.
-MLA_HD inline void plan_part_row(const int32_t* C, int batch, int w, int p, int32_t* m) {
-  const int o = kSegmentOverheadTiles;
+MLA_HD inline void plan_part_row(const int32_t* C, int batch, int w, int o, int g, int p,
+                                 int32_t* m) {
+  const int u = g * kPlanTileCost;
   const int total = C[batch];
   const long long s64 = static_cast<long long>(p) * w;
   if (batch == 0 || s64 >= total) {
@@ -112,38 +151,50 @@ MLA_HD inline void plan_part_row(const int32_t* C, int batch, int w, int p, int3
   }
   const int s = static_cast<int>(s64);
   const int e = (total - s > w) ? s + w : total;  // interval [s, e)
-  const int b0 = plan_seq_at(C, batch, s);
-  int t0 = s - C[b0] - o;
-  if (t0 < 0) t0 = 0;  // s inside b0's overhead: its first tile
-  int b1 = plan_seq_at(C, batch, e - 1);
-  int t1 = e - 1 - C[b1] - o;  // last tile in the interval
-  if (t1 < 0) {                // e - 1 inside b1's overhead: the previous sequence's last tile
-    --b1;
-    if (b1 >= 0) t1 = C[b1 + 1] - C[b1] - o - 1;
+  // first granule starting at or after s
+  int b0 = plan_seq_at(C, batch, s);
+  const int r0 = s - C[b0] - o;
+  int t0 = r0 <= 0 ? 0 : (r0 + u - 1) / u;
+  if (C[b0] + o + u * t0 >= C[b0 + 1]) {  // past b0's last granule start
+    ++b0;
+    t0 = 0;
   }
-  if (b1 < b0 || (b1 == b0 && t1 < t0)) {  // only overhead positions
+  // last granule starting before e
+  int b1 = plan_seq_at(C, batch, e - 1);
+  const int r1 = e - 1 - C[b1] - o;
+  int t1 = r1 < 0 ? -1 : r1 / u;
+  if (t1 < 0) {  // e - 1 inside b1's overhead: the previous sequence's last granule
+    --b1;
+    if (b1 >= 0) t1 = (C[b1 + 1] - C[b1] - o) / u - 1;
+  }
+  if (b0 >= batch || b1 < b0 || (b1 == b0 && t1 < t0)) {  // no tile starts in [s, e)
     plan_mark_empty(m, batch);
     return;
   }
   m[0] = b0;
-  m[1] = t0;
+  m[1] = t0 * g;
   m[2] = b1;
-  m[3] = t1 + 1;
-  m[4] = p - plan_first_part(C, b0, w);
+  m[3] = (t1 + 1) * g;
+  m[4] = p - plan_first_part(C, b0, w, o);
   m[5] = m[6] = m[7] = 0;
 }
 
 // Host planner: metadata[num_parts][8] and num_splits[batch + 1] from the
-// per-sequence tile counts (same result as the device planner).
-inline void plan_splits_host(const int32_t* tiles, int batch, int num_parts, int32_t* metadata,
-                             int32_t* num_splits, int32_t* C /* batch + 1 scratch */) {
+// per-sequence tile counts and the segment overhead o (same result as the
+// device planner).
+inline void plan_splits_host(const int32_t* granules, int batch, int num_parts, int o, int g,
+                             int32_t* metadata, int32_t* num_splits,
+                             int32_t* C /* batch + 1 scratch */) {
+  const int u = g * kPlanTileCost;
   C[0] = 0;
-  for (int b = 0; b < batch; ++b) C[b + 1] = C[b] + tiles[b] + kSegmentOverheadTiles;
-  const int w = plan_width(C[batch], num_parts);
-  for (int p = 0; p < num_parts; ++p) plan_part_row(C, batch, w, p, metadata + p * kMetaInts);
+  for (int b = 0; b < batch; ++b) C[b + 1] = C[b] + o + u * granules[b];
+  const int w = plan_width(C[batch], num_parts, u);
+  for (int p = 0; p < num_parts; ++p)
+    plan_part_row(C, batch, w, o, g, p, metadata + p * kMetaInts);
   num_splits[0] = 0;
   for (int b = 0; b < batch; ++b)
-    num_splits[b + 1] = num_splits[b] + plan_last_part(C, b, w) - plan_first_part(C, b, w) + 1;
+    num_splits[b + 1] =
+        num_splits[b] + plan_last_part(C, b, w, u) - plan_first_part(C, b, w, o) + 1;
 }
 
 }  // namespace mla

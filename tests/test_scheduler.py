@@ -8,7 +8,29 @@ import torch
 from mla_paged_kv_03_b200 import binding as B
 
 TILE = 128
-OVERHEAD = 2
+
+
+def _planner_constants():
+    """The planner's cost of a tile and the segment overheads, read from the
+    library's shared header (kPlanTileCost, MLA_PLAN_OVH_* defaults)."""
+    import os
+    import re
+    src = open(os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                            "mla_paged_kv_03_b200", "csrc", "mla_common.h")).read()
+    tile = int(re.search(r"kPlanTileCost = (\d+);", src).group(1))
+    ovh = {k: int(v) for k, v in re.findall(r"#define MLA_PLAN_OVH_(\w+) (\d+)", src)}
+    return tile, ovh
+
+
+TILE_COST, OVH = _planner_constants()
+
+
+def overhead_for(heads_per_kv):
+    return OVH["PAGE"] if heads_per_kv <= 32 else (OVH["CTA"] if heads_per_kv <= 64 else OVH["PAIR"])
+
+
+def granule_for(heads_per_kv):
+    return 2 if heads_per_kv > 64 else 1
 
 
 def tiles_of(L):
@@ -23,16 +45,34 @@ def expand(meta, ns, seqlens):
         segs = []
         for b in range(b0, b1 + 1):
             lo = t0 if b == b0 else 0
-            hi = t1 if b == b1 else tiles_of(seqlens[b])
+            hi = min(t1, tiles_of(seqlens[b])) if b == b1 else tiles_of(seqlens[b])
             if lo < hi:
                 segs.append((b, lo, hi, s0 if b == b0 else 0))
         parts.append(segs)
     return parts
 
 
-def check_plan(seqlens, parts_n):
-    meta, ns = B.mla_get_metadata_host(seqlens, 16, parts_n)
+def seg_cost(lo, hi, heads_per_kv):
+    """Planner cost of a segment of tiles [lo, hi): its granules and one overhead."""
+    g = granule_for(heads_per_kv)
+    return g * TILE_COST * (-(-(hi - lo) // g)) + overhead_for(heads_per_kv)
+
+
+def plan_total(seqlens, heads_per_kv):
+    g = granule_for(heads_per_kv)
+    return sum(g * TILE_COST * (-(-tiles_of(L) // g)) + overhead_for(heads_per_kv)
+               for L in seqlens)
+
+
+def check_plan(seqlens, parts_n, heads_per_kv=16):
+    meta, ns = B.mla_get_metadata_host(seqlens, heads_per_kv, parts_n)
     parts = expand(meta, ns, seqlens)
+    g = granule_for(heads_per_kv)
+    for segs in parts:
+        for (b, lo, hi, s) in segs:
+            # splits start on a granule; only a sequence's last split may be ragged
+            assert lo % g == 0
+            assert (hi - lo) % g == 0 or hi == tiles_of(seqlens[b])
     seen = {b: [] for b in range(len(seqlens))}
     for segs in parts:
         for (b, lo, hi, s) in segs:
@@ -60,30 +100,43 @@ def check_plan(seqlens, parts_n):
 ])
 @pytest.mark.parametrize("parts_n", [1, 2, 7, 74, 148, 500])
 def test_plan_covers_every_tile_once(seqlens, parts_n):
-    check_plan(seqlens, parts_n)
+    for heads_per_kv in (16, 64, 128):
+        check_plan(seqlens, parts_n, heads_per_kv)
 
 
-def test_plan_random_mixes_and_balance():
-    rng = random.Random(0)
+@pytest.mark.parametrize("heads_per_kv", [16, 64, 128])
+def test_plan_random_mixes_and_balance(heads_per_kv):
+    rng = random.Random(heads_per_kv)
+    o = overhead_for(heads_per_kv)
     for trial in range(40):
         b = rng.randint(1, 200)
         seqlens = [int(rng.choice([rng.randint(0, 300), rng.randint(1000, 20000)])) for _ in range(b)]
         parts_n = rng.choice([1, 3, 74, 148])
-        meta, ns, parts = check_plan(seqlens, parts_n)
-        total = sum(tiles_of(L) + OVERHEAD for L in seqlens)
-        target = -(-total // parts_n)
-        costs = [sum(hi - lo + OVERHEAD for (_, lo, hi, _) in segs) for segs in parts]
-        # every part but the last stays within one segment overhead of the target
-        for c in costs[:-1]:
-            assert c <= target + OVERHEAD + 1
+        meta, ns, parts = check_plan(seqlens, parts_n, heads_per_kv)
+        u = granule_for(heads_per_kv) * TILE_COST
+        total = plan_total(seqlens, heads_per_kv)
+        target = max(-(-total // parts_n), u)
+        costs = [sum(seg_cost(lo, hi, heads_per_kv) for (_, lo, hi, _) in segs) for segs in parts]
+        # every part stays within one granule and one segment overhead of the target
+        for c in costs:
+            assert c <= target + u + o
         assert sum(costs) >= total
 
 
 def test_plan_uniform_lengths_split_evenly():
-    meta, ns, parts = check_plan([65536 // 32] * 32, 74)
-    costs = [sum(hi - lo + OVERHEAD for (_, lo, hi, _) in segs) for segs in parts]
+    o, u = overhead_for(128), 2 * TILE_COST
+    meta, ns, parts = check_plan([65536 // 32] * 32, 74, heads_per_kv=128)
+    costs = [sum(seg_cost(lo, hi, 128) for (_, lo, hi, _) in segs) for segs in parts]
     nonempty = [c for c in costs if c]
-    assert max(nonempty) - min(nonempty) <= 2 * OVERHEAD + 2
+    assert max(nonempty) - min(nonempty) <= 2 * o + 2 * u
+
+
+def test_plan_parts_narrower_than_a_tile():
+    """More parts than quarter-tile units: the width stays one tile, so no
+    split count includes a part that holds none of the sequence's tiles."""
+    for seqlens in ([1], [1, 1], [130, 0, 5], [64] * 10):
+        check_plan(seqlens, 500)
+        check_plan(seqlens, 500, heads_per_kv=128)
 
 
 def test_plan_rejects_bad_arguments():
@@ -101,15 +154,17 @@ try:
     @settings(max_examples=200, deadline=None)
     @given(seqlens=st.lists(st.one_of(st.integers(0, 300), st.integers(1000, 70000)),
                             min_size=1, max_size=120),
-           parts_n=st.integers(1, 600))
-    def test_plan_property_coverage_and_balance(seqlens, parts_n):
+           parts_n=st.integers(1, 600), heads_per_kv=st.sampled_from([16, 64, 128]))
+    def test_plan_property_coverage_and_balance(seqlens, parts_n, heads_per_kv):
         """Any length mix and partition count: every (sequence, tile) pair is
         covered exactly once, in order, and no part exceeds the target width
-        by more than one segment overhead."""
-        meta, ns, parts = check_plan(seqlens, parts_n)
-        total = sum(tiles_of(L) + OVERHEAD for L in seqlens)
-        target = -(-total // parts_n)
+        by more than one tile and one segment overhead."""
+        o = overhead_for(heads_per_kv)
+        u = granule_for(heads_per_kv) * TILE_COST
+        meta, ns, parts = check_plan(seqlens, parts_n, heads_per_kv)
+        target = max(-(-plan_total(seqlens, heads_per_kv) // parts_n), u)
         for segs in parts:
-            assert sum(hi - lo + OVERHEAD for (_, lo, hi, _) in segs) <= target + OVERHEAD + 1
+            cost = sum(seg_cost(lo, hi, heads_per_kv) for (_, lo, hi, _) in segs)
+            assert cost <= target + u + o
 except ImportError:  # pragma: no cover
     pass
