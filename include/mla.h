@@ -312,8 +312,10 @@ MLA_API int mla_decode_fwd_noalloc(const void* q, const void* kcache, const int3
  * right before it launches its attention kernel and `stop_event` right after,
  * so that a caller can time that kernel alone (cudaEventElapsedTime) next to
  * the planner and combine launches of the same call.  Both are cudaEvent_t
- * handles owned by the caller (NULL = do not record).  The setting belongs to
- * the calling host thread; pass NULL, NULL to clear it. */
+ * handles owned by the caller (NULL = do not record).  Inside a stream
+ * capture they become event-record nodes of the graph, timed at each replay.
+ * The setting belongs to the calling host thread; pass NULL, NULL to clear
+ * it. */
 MLA_API int mla_set_kernel_events(void* start_event, void* stop_event);
 
 /* Debug aid, with no counterpart in the method's published interface: while

@@ -222,15 +222,22 @@ int check_trace(long long entries_per_plane) {
 thread_local cudaEvent_t t_kernel_start = nullptr;
 thread_local cudaEvent_t t_kernel_stop = nullptr;
 
-int record_start(cudaStream_t st) {
-  if (t_kernel_start) MLA_CUDA(cudaEventRecord(t_kernel_start, st));
+// Inside a stream capture an event is recorded as an event-record node of the
+// graph (cudaEventRecordExternal), so that its replay can be timed.
+int record_event(cudaEvent_t ev, cudaStream_t st) {
+  if (!ev) return MLA_OK;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  MLA_CUDA(cudaStreamIsCapturing(st, &cs));
+  if (cs == cudaStreamCaptureStatusActive)
+    MLA_CUDA(cudaEventRecordWithFlags(ev, st, cudaEventRecordExternal));
+  else
+    MLA_CUDA(cudaEventRecord(ev, st));
   return MLA_OK;
 }
 
-int record_stop(cudaStream_t st) {
-  if (t_kernel_stop) MLA_CUDA(cudaEventRecord(t_kernel_stop, st));
-  return MLA_OK;
-}
+int record_start(cudaStream_t st) { return record_event(t_kernel_start, st); }
+
+int record_stop(cudaStream_t st) { return record_event(t_kernel_stop, st); }
 
 // 1-CTA kernel (tokens on M = 128, V re-read for PV) for 33..64 query rows per
 // CTA, d_v 576 and the fused variant.
