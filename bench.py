@@ -248,6 +248,26 @@ class GpuStep:
             self.meta = torch.empty((self.parts, 8), dtype=torch.int32, device=dev)
             self.ns = torch.empty((b + 1,), dtype=torch.int32, device=dev)
 
+    def plan_summary(self):
+        """The split plan of a step: partitions, splits and sequences split
+        (from the host planner, bit-identical to the device planner the step
+        runs), for the lengths the attention kernel sees."""
+        c = self.case
+        if self.kind in ("dense", "fused"):
+            lengths = c.cache_seqlens.cpu()
+        elif self.kind == "prefill":
+            lengths = (c.topk_length.cpu() if c.topk_length is not None
+                       else (c.indices.cpu() >= 0).sum(-1).to(torch.int32))
+        else:
+            lengths = (c.indices.cpu() >= 0).sum(-1).reshape(-1).to(torch.int32)
+        lengths = lengths.to(torch.int32)
+        if self.kind == "prefill":
+            lengths = lengths[:32]  # one pass of 32 query tokens
+        _, ns = self.B.mla_get_metadata_host(lengths, self.R, self.parts)
+        per = (ns[1:] - ns[:-1]).tolist()
+        return {"num_sm_parts": self.parts, "splits": int(ns[-1]),
+                "sequences_split": int(sum(1 for n in per if n > 1)), "max_splits": int(max(per))}
+
     def attention_launches_per_step(self):
         return -(-self.case.s_q // 32) if self.kind == "prefill" else 1
 
@@ -695,7 +715,8 @@ def run_gpu_arm(args, rank, world):
         "config": {"workload": desc, "name": args.workload,
                    "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas x{world}",
                    "launch": "CUDA graph replay of one API step" if args.graph
-                   else "direct API calls"},
+                   else "direct API calls",
+                   "plan": gs.plan_summary()},
         "e2e": {"value": round(flops_all / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOPS",
                 "h2d_bytes_per_step": int(q_dev.numel() * q_dev.element_size()),
                 "d2h_bytes_per_step": int(gs.out.numel() * gs.out.element_size() +

@@ -58,3 +58,18 @@ def assert_fp8_close(codes, scale, ref_codes, ref_scale, min_equal=0.999):
                              f"(index, gpu, oracle) {det}")
     rel = np.abs(s - ref_scale) / np.maximum(np.abs(ref_scale), 1e-30)
     assert (rel <= 1e-3).all(), f"scale rel err {rel.max():.3e}"
+
+
+def full_size_rows(rows_per_unit, unit_sizes, n_random, seed):
+    """Rows checked in a full-size parity test: n_random rows drawn at random,
+    plus every row of the first unit (sequence, query pair or token), of the
+    largest one and of the last one, so that every head, every split of a
+    long sequence and every role a CTA takes is covered at least once."""
+    unit_sizes = np.asarray(unit_sizes)
+    n_units = unit_sizes.size
+    total = n_units * rows_per_unit
+    rng = np.random.default_rng(seed)
+    rows = set(rng.choice(total, size=min(n_random, total), replace=False).tolist())
+    for u in {0, int(np.argmax(unit_sizes)), n_units - 1}:
+        rows.update(range(u * rows_per_unit, (u + 1) * rows_per_unit))
+    return np.array(sorted(rows), dtype=np.int64)

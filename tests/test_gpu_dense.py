@@ -7,7 +7,7 @@ import torch
 import oracle
 from mla_paged_kv_03_b200 import binding as B
 from mla_paged_kv_03_b200 import workloads as W
-from parity_util import assert_lse_close, assert_out_close
+from parity_util import assert_lse_close, assert_out_close, full_size_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -97,13 +97,6 @@ def test_large_scores_trigger_rescale():
     check_full(c)
 
 
-def sampled_rows(case, n, seed):
-    rng = np.random.default_rng(seed)
-    total = case.batch * case.s_q * case.h_q
-    rows = rng.choice(total, size=min(n, total), replace=False)
-    return np.sort(rows)
-
-
 @pytest.mark.parametrize("name", ["compute", "memory"])
 def test_full_size_sampled(name):
     """Full-size workloads in the benchmark's launch configuration, checked on
@@ -114,7 +107,7 @@ def test_full_size_sampled(name):
     cpu = W.DenseCase(q=case.q.cpu(), kcache=case.kcache.cpu(), block_table=case.block_table.cpu(),
                       cache_seqlens=case.cache_seqlens.cpu(), s_q=case.s_q, h_q=case.h_q,
                       d_v=case.d_v, causal=case.causal, softmax_scale=case.softmax_scale)
-    rows = sampled_rows(case, 48, 0)
+    rows = full_size_rows(case.s_q * case.h_q, cpu.cache_seqlens.numpy(), 48, 0)
     ro, rl = oracle.dense_decode(cpu.q, cpu.kcache, cpu.block_table, cpu.cache_seqlens, cpu.d_v,
                                  cpu.softmax_scale, causal=cpu.causal, rows=rows)
     assert_out_close(out.reshape(-1, case.d_v)[torch.as_tensor(rows)], ro)

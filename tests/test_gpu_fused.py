@@ -8,7 +8,7 @@ import torch
 import oracle
 from mla_paged_kv_03_b200 import binding as B
 from mla_paged_kv_03_b200 import workloads as W
-from parity_util import assert_fp8_close, assert_lse_close
+from parity_util import assert_fp8_close, assert_lse_close, full_size_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -66,7 +66,5 @@ def test_fused_full_size_sampled(batch):
     dev = torch.device("cuda")
     case = W.fused(seed=0, device=dev, batch=batch)
     gpu = run_gpu(case)
-    rng = np.random.default_rng(batch)
-    total = case.batch * case.h_q
-    rows = np.sort(rng.choice(total, size=min(48, total), replace=False))
+    rows = full_size_rows(case.h_q, case.cache_seqlens.cpu().numpy(), 48, batch)
     check(case, rows=rows, gpu=gpu)

@@ -7,7 +7,7 @@ import torch
 import oracle
 from mla_paged_kv_03_b200 import binding as B
 from mla_paged_kv_03_b200 import workloads as W
-from parity_util import assert_fp8_close, assert_lse_close
+from parity_util import assert_fp8_close, assert_lse_close, full_size_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -75,6 +75,6 @@ def test_fused_sparse_full_size_sampled():
     dev = torch.device("cuda")
     case = W.fused_sparse(seed=0, device=dev)
     gpu = run_gpu(case)
-    rng = np.random.default_rng(8)
-    rows = np.sort(rng.choice(case.batch * case.h_q, size=48, replace=False))
+    valid = (case.indices.cpu() >= 0).sum(-1).reshape(-1).numpy()
+    rows = full_size_rows(case.h_q, valid, 48, 8)
     check(case, rows=rows, gpu=gpu)

@@ -8,7 +8,7 @@ import torch
 import oracle
 from mla_paged_kv_03_b200 import binding as B
 from mla_paged_kv_03_b200 import workloads as W
-from parity_util import assert_lse_close, assert_out_close
+from parity_util import assert_lse_close, assert_out_close, full_size_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -81,6 +81,5 @@ def test_prefill_full_size_sampled():
     dev = torch.device("cuda")
     case = W.sparse_prefill(seed=0, device=dev)
     gpu = run_gpu(case)
-    rng = np.random.default_rng(9)
-    rows = np.sort(rng.choice(case.s_q * case.h_q, size=64, replace=False))
+    rows = full_size_rows(case.h_q, case.topk_length.cpu().numpy(), 64, 9)
     check(case, rows=rows, gpu=gpu)

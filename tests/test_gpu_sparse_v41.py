@@ -8,7 +8,7 @@ import torch
 import oracle
 from mla_paged_kv_03_b200 import binding as B
 from mla_paged_kv_03_b200 import workloads as W
-from parity_util import assert_lse_close, assert_out_close
+from parity_util import assert_lse_close, assert_out_close, full_size_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -66,7 +66,6 @@ def test_sparse_v41_full_size_sampled():
     dev = torch.device("cuda")
     case = W.sparse_v41(seed=0, device=dev)
     gpu = run_gpu(case)
-    rng = np.random.default_rng(6)
-    total = case.batch * case.s_q * case.h_q
-    rows = np.sort(rng.choice(total, size=48, replace=False))
+    valid = (case.indices.cpu() >= 0).sum(-1).reshape(-1).numpy()
+    rows = full_size_rows(case.h_q, valid, 48, 6)
     check(case, rows=rows, gpu=gpu)

@@ -6,6 +6,7 @@ import pytest
 import torch
 
 from mla_paged_kv_03_b200 import workloads as W
+from parity_util import full_size_rows
 from test_gpu_sparse_v41 import check, run_gpu
 
 pytestmark = pytest.mark.gpu
@@ -41,7 +42,6 @@ def test_sparse_v41_fp4_full_size_sampled():
     dev = torch.device("cuda")
     case = W.sparse_v41_fp4(seed=0, device=dev)
     gpu = run_gpu(case)
-    rng = np.random.default_rng(7)
-    total = case.batch * case.s_q * case.h_q
-    rows = np.sort(rng.choice(total, size=48, replace=False))
+    valid = (case.indices.cpu() >= 0).sum(-1).reshape(-1).numpy()
+    rows = full_size_rows(case.h_q, valid, 48, 7)
     check(case, rows=rows, gpu=gpu)
