@@ -261,22 +261,25 @@ class GpuStep:
         else:
             lengths = (c.indices.cpu() >= 0).sum(-1).reshape(-1).to(torch.int32)
         lengths = lengths.to(torch.int32)
+        parts = self.parts
         if self.kind == "prefill":
-            lengths = lengths[:32]  # one pass of 32 query tokens
-        _, ns = self.B.mla_get_metadata_host(lengths, self.R, self.parts)
+            lengths = lengths[:8192].clamp(0, c.topk)  # one launch
+            parts = min(parts, self.B.mla_num_sms(self.dev) // (2 * -(-c.h_q // 128)))
+        _, ns = self.B.mla_get_metadata_host(lengths, self.R, parts)
         per = (ns[1:] - ns[:-1]).tolist()
-        return {"num_sm_parts": self.parts, "splits": int(ns[-1]),
+        return {"num_sm_parts": parts, "splits": int(ns[-1]),
                 "sequences_split": int(sum(1 for n in per if n > 1)), "max_splits": int(max(per))}
 
     def attention_launches_per_step(self):
-        return -(-self.case.s_q // 32) if self.kind == "prefill" else 1
+        return -(-self.case.s_q // 8192) if self.kind == "prefill" else 1
 
     def launches_per_step(self):
         # planner + attention kernel + combine (+ the FP8 gather for sparse);
-        # the prefill runs that sequence per pass of 32 tokens, then the sinks
+        # the prefill runs lengths, planner, attention and combine per launch of
+        # up to 8192 query tokens, then the sinks
         if self.kind == "prefill":
             c = self.case
-            return 4 * -(-c.s_q // 32) + (1 if c.attn_sink is not None else 0)
+            return 4 * -(-c.s_q // 8192) + (1 if c.attn_sink is not None else 0)
         return 4 if self.kind in ("sparse", "fused_sparse") else 3
 
     def step(self, q=None):

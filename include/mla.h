@@ -223,8 +223,9 @@ MLA_API int mla_sparse_decode_v41_fp4(const void* q, const uint8_t* kcache_288, 
                               float softmax_scale, int num_sm_parts, void* workspace,
                               size_t workspace_bytes, void* out, float* lse, void* stream);
 
-/* Workspace bytes for mla_sparse_prefill_fwd (one pass of up to 32 query
- * tokens: their gathered rows, tables and split partials). */
+/* Workspace bytes for mla_sparse_prefill_fwd: the clamped lengths and split
+ * plan of up to 8192 query tokens and the partials of the tokens split over
+ * several parts (2 * num_sm_parts * h_q rows of 512 fp32). */
 MLA_API int mla_sparse_prefill_workspace_size(int s_q, int h_q, int topk, int num_sm_parts,
                                       size_t* bytes);
 
@@ -244,8 +245,10 @@ MLA_API int mla_sparse_prefill_workspace_size(int s_q, int h_q, int topk, int nu
  *   d_v           512 (V = kv[:, :512]); softmax_scale usually 1/sqrt(576)
  *   out, lse      [s_q, h_q, 512] bf16 (16-byte aligned) and [s_q, h_q] fp32
  *   num_sm_parts  from mla_num_sm_parts(device, h_q, 1)
- * The tokens are processed in passes of 32 through the sparse decode path
- * (gather of each token's rows, planner, decode, combine), then the sinks.
+ * Each query token is one unit of the CTA-pair attention kernel, whose loads
+ * fetch the token's rows straight from kv (four named rows per TMA copy); a
+ * launch covers up to 8192 tokens, then the sinks are applied.  num_sm_parts
+ * is capped at the device's SMs / (2 ceil(h_q / 128)) CTA pairs.
  * Ownership and errors as in mla_sparse_decode. */
 MLA_API int mla_sparse_prefill_fwd(const void* q, const void* kv, int64_t s_kv,
                            const int32_t* indices, int topk, const int32_t* topk_length,
@@ -332,11 +335,15 @@ MLA_API int mla_set_kernel_events(void* start_event, void* stop_event);
  *                 rows read as V.  Only tokens of pages that hold part of the
  *                 sequence are written (a partial last page in full); an
  *                 out-of-range block id shows as block 0.
- *               sparse decode, fused sparse decode and sparse prefill:
- *                 N = (batch * s_q | s_q) * topk; entry p * topk + j holds
- *                 the slot entry j of query p read (-1 if unused or out of
- *                 range) in plane 0, and the row of the compacted buffer it
- *                 went to (valid entries numbered in index order) in plane 1.
+ *               sparse decode and fused sparse decode: N = batch * s_q *
+ *                 topk; entry p * topk + j holds the slot entry j of query p
+ *                 read (-1 if unused or out of range) in plane 0, and the row
+ *                 of the compacted buffer it went to (valid entries numbered
+ *                 in index order) in plane 1.
+ *               sparse prefill: N = s_q * topk; entry t * topk + j holds the
+ *                 kv row entry j of token t read in plane 0 and j itself in
+ *                 plane 1 (the rows are read in place), both -1 for an entry
+ *                 that is unused, out of range or past the token's length.
  *             Entries the call does not write keep their contents.
  *   capacity  entries of `trace`; a call needing more than 2 * N returns
  *             MLA_ERR_INVALID_ARG before any launch.

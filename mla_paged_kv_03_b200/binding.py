@@ -117,6 +117,15 @@ def _require(cond, msg):
 
 # ---------------------------------------------------------------- scheduler
 
+def mla_num_sms(device=None) -> int:
+    """Streaming multiprocessors of `device` (default: the current device)."""
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    out = ctypes.c_int(0)
+    _check(lib().mla_num_sms(dev.index if dev.index is not None else torch.cuda.current_device(),
+                             ctypes.byref(out)))
+    return int(out.value)
+
+
 def mla_num_sm_parts(heads_per_kv: int, h_kv: int = 1, device=None) -> int:
     dev = torch.cuda.current_device() if device is None else torch.device(device).index or 0
     out = ctypes.c_int(0)

@@ -22,6 +22,8 @@ namespace mla {
 struct CombineParams {
   int batch, R, d_v, h_q;
   const int32_t* num_splits;  // [batch + 1]
+  const int32_t* ws_base;     // [batch] first partial row of each split sequence, or null
+                              // (then num_splits[b])
   const float* ws_o;          // [total_splits, R, d_v]
   const float* ws_lse;        // [total_splits, R]
   __nv_bfloat16* out;         // dense: [batch*R, d_v]
@@ -73,8 +75,8 @@ __global__ void __launch_bounds__(kCombineThreads) mla_combine_kernel(const Comb
   if (row_id >= static_cast<long long>(P.batch) * P.R) return;
   const int b = static_cast<int>(row_id / P.R);
   const int r = static_cast<int>(row_id % P.R);
-  const int base = P.num_splits[b];
-  const int n = P.num_splits[b + 1] - base;
+  const int n = P.num_splits[b + 1] - P.num_splits[b];
+  const int base = P.ws_base ? P.ws_base[b] : P.num_splits[b];
   if (!kFusedOut && n <= 1) return;  // written directly by the decode kernel
 
   // LSE of the merged row: max-subtracted log-sum-exp of the split LSEs
@@ -254,7 +256,7 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* total) {
 // Split-KV planner of one CTA: the closed forms of mla_common.h evaluated in
 // parallel (prefix sums by block scans, one metadata row per thread).
 __device__ void plan_block(const int32_t* seqlens, int batch, int num_parts, int o, int g,
-                           int32_t* metadata, int32_t* num_splits) {
+                           int32_t* metadata, int32_t* num_splits, int32_t* ws_base) {
   const int u = g * kPlanTileCost;
   __shared__ int32_t C[kPlanMaxBatch + 1];
   const int tid = threadIdx.x;
@@ -283,15 +285,29 @@ __device__ void plan_block(const int32_t* seqlens, int batch, int num_parts, int
     if (b < batch) num_splits[b + 1] = nsum + ex + v;
     nsum += chunk_total;
   }
+  if (ws_base) {
+    // compact partial rows: only sequences split over several parts own rows
+    // (at most 2 num_parts in all: a part holds at most two split segments)
+    int wsum = 0;
+    for (int base = 0; base < batch; base += kPlanThreads) {
+      const int b = base + tid;
+      const int v = b < batch ? plan_last_part(C, b, w, u) - plan_first_part(C, b, w, o) + 1 : 0;
+      int chunk_total;
+      const int ex = block_exclusive_scan(v > 1 ? v : 0, &chunk_total);
+      if (b < batch) ws_base[b] = wsum + ex;
+      wsum += chunk_total;
+    }
+  }
 }
 
 __global__ void __launch_bounds__(kPlanThreads) mla_plan_kernel(const int32_t* seqlens, int batch,
                                                                int num_parts, int overhead,
                                                                int granule, int32_t* metadata,
-                                                               int32_t* num_splits) {
+                                                               int32_t* num_splits,
+                                                               int32_t* ws_base) {
   ptx::grid_dep_wait();
   ptx::grid_dep_launch();  // the decode grid waits for this one at its start
-  plan_block(seqlens, batch, num_parts, overhead, granule, metadata, num_splits);
+  plan_block(seqlens, batch, num_parts, overhead, granule, metadata, num_splits, ws_base);
 }
 
 }  // namespace mla

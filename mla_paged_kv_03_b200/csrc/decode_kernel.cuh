@@ -77,6 +77,15 @@ struct DecodeParams {
   // the rows read as K, plane 1 for the rows read as V
   int32_t* trace;
   long long trace_plane;  // entries per plane
+  // gather mode (CTA-pair kernel): the cache is a bf16 row array
+  // [gather_rows, 576] and token t of unit b is row gather_idx[b *
+  // gather_stride + t] (an entry outside [0, gather_rows) is masked)
+  const int32_t* gather_idx;
+  int gather_stride;
+  int gather_rows;
+  // split partials of sequence b start at ws row ws_base[b] (only split
+  // sequences own rows), or at num_splits[b] when ws_base is null
+  const int32_t* ws_base;
 };
 
 namespace cfg {
@@ -778,7 +787,7 @@ __global__ void __launch_bounds__(Threads<kMode>::value, 1)
       }
       ptx::named_bar_sync(bar_sync, 128);
       const bool partial = P.always_partial || u.nsplit > 1;
-      const int ws_row0 = (P.num_splits[u.b] + u.split) * P.R;
+      const int ws_row0 = ((P.ws_base ? P.ws_base[u.b] : P.num_splits[u.b]) + u.split) * P.R;
       const int rows_here = min(kRowsPerCta, P.R - grp * kRowsPerCta);
       if (wt < 32) {
         const float l = (C.red[4 * sg][wt] + C.red[4 * sg + 1][wt]) +

@@ -86,6 +86,22 @@ int make_latent_map(CUtensorMap* map, const void* base, long long rows) {
   return MLA_OK;
 }
 
+// 2-D bf16 view [rows, 576] with a box one row high and 64 wide, 128-byte
+// swizzle: the map of the TMA gather4 loads (four named rows per copy).
+int make_gather_map(CUtensorMap* map, const void* base, long long rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(mla::kD), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(mla::kD) * 2};
+  cuuint32_t box[2] = {64, 1};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled (gather) failed (%d)", (int)r);
+  return MLA_OK;
+}
+
 // 3-D bf16 view of the same rows: {64 dims, rows, 9 chunks of 64 dims}
 // (strides 1152 B and 128 B) with a {64, box_rows, box_chunks} box, 128-byte
 // swizzle; one copy lands [box_chunks][box_rows][64 dims] in shared memory.
@@ -286,18 +302,22 @@ int launch_page_decode(const void* q, const CUtensorMap& tkv, const mla::DecodeP
 
 // 2-CTA kernel for more than 64 query rows per KV head: clusters of two CTAs,
 // one pair per scheduler part and 128-row group.
+// In gather mode tkv is the gather map of the row array and no V map is used.
+template <bool kGather>
 int launch_pair_decode(const void* q, const void* kcache, const CUtensorMap& tkv,
                        const mla::DecodeParams& p, cudaStream_t st) {
   CUtensorMap tq3, tv3;
   int rc = make_latent_map3(&tq3, q, static_cast<long long>(p.batch) * p.R, mla::kNumChunks);
   if (rc != MLA_OK) return rc;
-  if ((rc = make_latent_map3(&tv3, kcache, static_cast<long long>(p.num_blocks) * mla::kPage, 2)) !=
-      MLA_OK)
+  if (kGather)
+    tv3 = tkv;
+  else if ((rc = make_latent_map3(&tv3, kcache, static_cast<long long>(p.num_blocks) * mla::kPage,
+                                  2)) != MLA_OK)
     return rc;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(mla::mla_pair_decode_kernel,
+    attr_err = cudaFuncSetAttribute(mla::mla_pair_decode_kernel<kGather>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     mla::pcfg::kSmemBytes);
   });
@@ -306,7 +326,7 @@ int launch_pair_decode(const void* q, const void* kcache, const CUtensorMap& tkv
   PdlLaunch L(dim3(static_cast<unsigned>(2 * p.num_parts * p.n_groups)), dim3(mla::pcfg::kThreads),
               mla::pcfg::kSmemBytes, st, 2);
   if ((rc = record_start(st)) != MLA_OK) return rc;
-  MLA_CUDA(cudaLaunchKernelEx(&L.cfg, mla::mla_pair_decode_kernel, tq3, tkv, tv3, p));
+  MLA_CUDA(cudaLaunchKernelEx(&L.cfg, mla::mla_pair_decode_kernel<kGather>, tq3, tkv, tv3, p));
   return record_stop(st);
 }
 
@@ -407,7 +427,7 @@ static int sparse_gather_and_plan(int row_bytes, const void* q, const uint8_t* k
                                   int64_t num_slots, const int32_t* indices, int topk, int pairs,
                                   int h_q, int num_sm_parts, uint8_t* ws, const SparseWs& w,
                                   void* stream, const void** q_dense,
-                                  const int32_t* topk_len = nullptr, int32_t* trace = nullptr,
+                                  int32_t* trace = nullptr,
                                   long long trace_plane = 0) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   mla::GatherParams g{};
@@ -417,7 +437,6 @@ static int sparse_gather_and_plan(int row_bytes, const void* q, const uint8_t* k
   g.num_slots = num_slots;
   g.indices = indices;
   g.topk = topk;
-  g.topk_len = topk_len;
   g.pages_per_pair = w.pages_per_pair;
   g.rows = reinterpret_cast<__nv_bfloat16*>(ws + w.rows_off);
   g.block_table = reinterpret_cast<int32_t*>(ws + w.bt_off);
@@ -434,8 +453,6 @@ static int sparse_gather_and_plan(int row_bytes, const void* q, const uint8_t* k
     mla::mla_sparse_gather_kernel<mla::kRow528><<<grid, mla::kGatherCtaThreads, 0, st>>>(g);
   } else if (row_bytes == mla::kRow288) {
     mla::mla_sparse_gather_kernel<mla::kRow288><<<grid, mla::kGatherCtaThreads, 0, st>>>(g);
-  } else if (row_bytes == mla::kRowBf16) {
-    mla::mla_sparse_gather_kernel<mla::kRowBf16><<<grid, mla::kGatherCtaThreads, 0, st>>>(g);
   } else {
     mla::mla_sparse_gather_kernel<mla::kRow656><<<grid, mla::kGatherCtaThreads, 0, st>>>(g);
   }
@@ -477,7 +494,7 @@ static int sparse_decode_impl(int row_bytes, const void* q, const uint8_t* kcach
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const void* q_dense = q;
   rc = sparse_gather_and_plan(row_bytes, q, kcache, num_slots, indices, topk, pairs, h_q,
-                              num_sm_parts, ws, w, stream, &q_dense, nullptr, t_trace,
+                              num_sm_parts, ws, w, stream, &q_dense, t_trace,
                               static_cast<long long>(pairs) * topk);
   if (rc != MLA_OK) return rc;
   // dense decode over the compacted rows: no causal mask, lengths = valid counts
@@ -489,6 +506,47 @@ static int sparse_decode_impl(int row_bytes, const void* q, const uint8_t* kcach
                         reinterpret_cast<int32_t*>(ws + w.splits_off), num_sm_parts,
                         ws + w.dense_off, w.dense_bytes, out, lse, stream);
 }
+
+namespace {
+
+// Query tokens per launch of the sparse prefill (the device planner's limit).
+constexpr int kPrefillPass = mla::kPlanMaxBatch;
+
+// Workspace of the sparse prefill, for one pass of up to kPrefillPass tokens:
+// the clamped top-k lengths, the split plan (metadata, num_splits, compact
+// partial bases) and the partials of the query tokens split over several
+// parts (at most 2 * parts of them).
+struct PrefillWs {
+  size_t len_off, meta_off, splits_off, base_off, o_off, lse_off, total;
+};
+
+PrefillWs prefill_ws_layout(int tokens, int h_q, int parts) {
+  PrefillWs w{};
+  const size_t rows = 2 * static_cast<size_t>(parts) * h_q;
+  w.len_off = 0;
+  w.meta_off = align_up(static_cast<size_t>(tokens) * 4, 256);
+  w.splits_off = w.meta_off + align_up(static_cast<size_t>(parts) * mla::kMetaInts * 4, 256);
+  w.base_off = w.splits_off + align_up((static_cast<size_t>(tokens) + 1) * 4, 256);
+  w.o_off = w.base_off + align_up(static_cast<size_t>(tokens) * 4, 256);
+  w.lse_off = w.o_off + align_up(rows * 512 * 4, 256);
+  w.total = w.lse_off + align_up(rows * 4, 256);
+  return w;
+}
+
+// CTA-pair parts of the prefill launch: at most the caller's count, and no
+// more pairs than the device has SMs for.
+int prefill_parts(int num_sm_parts, int h_q, int* parts) {
+  int dev = 0, sms = 0;
+  MLA_CUDA(cudaGetDevice(&dev));
+  MLA_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  const int groups = mla::ceil_div(h_q, 2 * mla::kRowsPerCta);
+  const int cap = sms / (2 * groups);
+  *parts = num_sm_parts < cap ? num_sm_parts : cap;
+  if (*parts < 1) *parts = 1;
+  return MLA_OK;
+}
+
+}  // namespace
 
 extern "C" {
 
@@ -590,7 +648,7 @@ int mla_get_metadata(const int32_t* cache_seqlens, int batch, int heads_per_kv, 
                 mla::kPlanMaxBatch, batch);
   mla::mla_plan_kernel<<<1, mla::kPlanThreads, 0, static_cast<cudaStream_t>(stream)>>>(
       cache_seqlens, batch, num_sm_parts, mla::plan_overhead(heads_per_kv),
-      mla::plan_granule(heads_per_kv), metadata, num_splits);
+      mla::plan_granule(heads_per_kv), metadata, num_splits, nullptr);
   MLA_CUDA(cudaGetLastError());
   return MLA_OK;
 }
@@ -675,7 +733,7 @@ int mla_decode_fwd(const void* q, const void* kcache, const int32_t* block_table
     rc = launch_page_decode(q, tkv, p, st);
   } else if (R > mla::kRowsPerCta && d_v == 512) {
     p.n_groups = mla::ceil_div(R, 2 * mla::kRowsPerCta);
-    rc = launch_pair_decode(q, kcache, tkv, p, st);
+    rc = launch_pair_decode<false>(q, kcache, tkv, p, st);
   } else {
     CUtensorMap tq;
     if ((rc = make_latent_map(&tq, q, static_cast<long long>(batch) * R)) != MLA_OK) return rc;
@@ -804,16 +862,12 @@ int mla_sparse_decode(const void* q, const uint8_t* kcache_fp8, int64_t num_slot
                             stream);
 }
 
-// Query tokens per pass of the sparse prefill: each pass gathers its tokens'
-// rows into the workspace (pages of 64 bf16 rows per token) and decodes them.
-constexpr int kPrefillChunk = 32;
-
 int mla_sparse_prefill_workspace_size(int s_q, int h_q, int topk, int num_sm_parts,
                                       size_t* bytes) {
   MLA_CHECK_ARG(bytes, "bytes is null");
   MLA_CHECK_ARG(s_q >= 0 && h_q >= 1 && topk >= 1 && num_sm_parts >= 1, "bad sizes");
-  const int chunk = s_q < kPrefillChunk ? (s_q > 0 ? s_q : 1) : kPrefillChunk;
-  *bytes = sparse_ws_layout(chunk, topk, h_q, 512, num_sm_parts).total;
+  const int tokens = s_q < kPrefillPass ? (s_q > 0 ? s_q : 1) : kPrefillPass;
+  *bytes = prefill_ws_layout(tokens, h_q, num_sm_parts).total;
   return MLA_OK;
 }
 
@@ -837,45 +891,81 @@ int mla_sparse_prefill_fwd(const void* q, const void* kv, int64_t s_kv, const in
   MLA_CHECK_ARG(aligned(lse, 4) && aligned(indices, 4) && aligned(topk_length, 4) &&
                     aligned(attn_sink, 4),
                 "misaligned lse, indices, topk_length or attn_sink");
-  const int chunk = s_q < kPrefillChunk ? (s_q > 0 ? s_q : 1) : kPrefillChunk;
-  const SparseWs w = sparse_ws_layout(chunk, topk, h_q, d_v, num_sm_parts);
+  const int tokens = s_q < kPrefillPass ? (s_q > 0 ? s_q : 1) : kPrefillPass;
+  const PrefillWs w = prefill_ws_layout(tokens, h_q, num_sm_parts);
   MLA_CHECK_ARG(workspace_bytes >= w.total, "workspace too small: %zu < %zu", workspace_bytes,
                 w.total);
-  MLA_CHECK_ARG(static_cast<long long>(chunk) * w.pages_per_pair * mla::kPage < (1LL << 31),
-                "topk too large");
   const long long trace_plane = static_cast<long long>(s_q) * topk;
-  int rc0 = check_trace(trace_plane);
-  if (rc0 != MLA_OK) return rc0;
+  int rc = check_trace(trace_plane);
+  if (rc != MLA_OK) return rc;
   if (s_q == 0) return MLA_OK;
-  int32_t* trace = t_trace;
-  TraceOff off;  // the decode passes over the compacted rows are not traced
+  int parts = 0;
+  if ((rc = prefill_parts(num_sm_parts, h_q, &parts)) != MLA_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int32_t* lengths = reinterpret_cast<int32_t*>(ws + w.len_off);
+  int32_t* meta = reinterpret_cast<int32_t*>(ws + w.meta_off);
+  int32_t* splits = reinterpret_cast<int32_t*>(ws + w.splits_off);
+  int32_t* base = reinterpret_cast<int32_t*>(ws + w.base_off);
+  if (t_trace) {  // entries no load reaches stay -1
+    MLA_CUDA(cudaMemsetAsync(t_trace, 0xFF, 2 * static_cast<size_t>(trace_plane) * 4, st));
+  }
+  CUtensorMap tkv;
+  if ((rc = make_gather_map(&tkv, kv, s_kv)) != MLA_OK) return rc;
   const size_t q_row = static_cast<size_t>(h_q) * mla::kD;  // bf16 values per token
-  for (int t0 = 0; t0 < s_q; t0 += chunk) {
-    const int n = s_q - t0 < chunk ? s_q - t0 : chunk;
+  for (int t0 = 0; t0 < s_q; t0 += kPrefillPass) {
+    const int n = s_q - t0 < kPrefillPass ? s_q - t0 : kPrefillPass;
+    mla::mla_prefill_lengths_kernel<<<mla::ceil_div(n, 256), 256, 0, st>>>(
+        topk_length ? topk_length + t0 : nullptr, topk, n, lengths);
+    MLA_CUDA(cudaGetLastError());
+    mla::mla_plan_kernel<<<1, mla::kPlanThreads, 0, st>>>(
+        lengths, n, parts, mla::plan_overhead(h_q), mla::plan_granule(h_q), meta, splits, base);
+    MLA_CUDA(cudaGetLastError());
+    mla::DecodeParams p{};
+    p.batch = n;
+    p.s_q = 1;
+    p.h_q = h_q;
+    p.R = h_q;
+    p.d_v = d_v;
+    p.n_groups = mla::ceil_div(h_q, 2 * mla::kRowsPerCta);
+    p.num_parts = parts;
+    p.num_blocks = 1;
+    p.max_pages = mla::ceil_div(topk, mla::kPage);
+    p.causal = 0;
+    p.always_partial = 0;
+    p.scale_log2 = softmax_scale * 1.4426950408889634f;
+    p.seqlens = lengths;
+    p.metadata = meta;
+    p.num_splits = splits;
+    p.ws_base = base;
+    p.out = static_cast<__nv_bfloat16*>(out) + static_cast<size_t>(t0) * h_q * d_v;
+    p.lse = lse + static_cast<size_t>(t0) * h_q;
+    p.ws_o = reinterpret_cast<float*>(ws + w.o_off);
+    p.ws_lse = reinterpret_cast<float*>(ws + w.lse_off);
+    p.gather_idx = indices + static_cast<size_t>(t0) * topk;
+    p.gather_stride = topk;
+    p.gather_rows = static_cast<int>(s_kv);
+    p.trace = t_trace ? t_trace + static_cast<size_t>(t0) * topk : nullptr;
+    p.trace_plane = trace_plane;
     const void* q_t = static_cast<const __nv_bfloat16*>(q) + t0 * q_row;
-    const void* q_dense = q_t;
-    int rc = sparse_gather_and_plan(mla::kRowBf16, q_t, static_cast<const uint8_t*>(kv), s_kv,
-                                    indices + static_cast<size_t>(t0) * topk, topk, n, h_q,
-                                    num_sm_parts, ws, w, stream, &q_dense,
-                                    topk_length ? topk_length + t0 : nullptr,
-                                    trace ? trace + static_cast<size_t>(t0) * topk : nullptr,
-                                    trace_plane);
-    if (rc != MLA_OK) return rc;
-    rc = mla_decode_fwd(q_dense, ws + w.rows_off, reinterpret_cast<int32_t*>(ws + w.bt_off),
-                        w.pages_per_pair, n * w.pages_per_pair,
-                        reinterpret_cast<int32_t*>(ws + w.len_off), n, 1, h_q, 1, d_v,
-                        softmax_scale, 0, reinterpret_cast<int32_t*>(ws + w.meta_off),
-                        reinterpret_cast<int32_t*>(ws + w.splits_off), num_sm_parts,
-                        ws + w.dense_off, w.dense_bytes,
-                        static_cast<__nv_bfloat16*>(out) + static_cast<size_t>(t0) * h_q * d_v,
-                        lse + static_cast<size_t>(t0) * h_q, stream);
-    if (rc != MLA_OK) return rc;
+    if ((rc = launch_pair_decode<true>(q_t, kv, tkv, p, st)) != MLA_OK) return rc;
+    mla::CombineParams cp{};
+    cp.batch = n;
+    cp.R = h_q;
+    cp.d_v = d_v;
+    cp.h_q = h_q;
+    cp.num_splits = splits;
+    cp.ws_base = base;
+    cp.ws_o = p.ws_o;
+    cp.ws_lse = p.ws_lse;
+    cp.out = p.out;
+    cp.lse = p.lse;
+    if ((rc = launch_combine(cp, false, st)) != MLA_OK) return rc;
   }
   if (attn_sink) {
     const long long rows = static_cast<long long>(s_q) * h_q;
     const unsigned grid = static_cast<unsigned>((rows + mla::kSinkWarps - 1) / mla::kSinkWarps);
-    mla::mla_sink_kernel<<<grid, 32 * mla::kSinkWarps, 0, static_cast<cudaStream_t>(stream)>>>(
+    mla::mla_sink_kernel<<<grid, 32 * mla::kSinkWarps, 0, st>>>(
         static_cast<__nv_bfloat16*>(out), lse, attn_sink, rows, h_q, d_v);
     MLA_CUDA(cudaGetLastError());
   }
@@ -922,7 +1012,7 @@ int mla_sparse_fused_norm_rope_attn_rope_cast(
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const void* q_dense = q_raw;
   rc = sparse_gather_and_plan(mla::kRow656, q_raw, kcache_fp8, num_slots, indices, topk, batch,
-                              h_q, num_sm_parts, ws, w, stream, &q_dense, nullptr, t_trace,
+                              h_q, num_sm_parts, ws, w, stream, &q_dense, t_trace,
                               static_cast<long long>(batch) * topk);
   if (rc != MLA_OK) return rc;
   // the fused steps over the compacted rows; every query sees all its rows

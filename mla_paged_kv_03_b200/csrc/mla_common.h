@@ -21,7 +21,6 @@ constexpr int kPage = 64;        // paged cache block size [FlashMLA (AI Wiki), 
 constexpr int kRow656 = 656;     // FP8 cache row [FlashMLA (AI Wiki), "The FP8 and FP4 KV cache"]
 constexpr int kRow528 = 528;     // V4.1 FP8 cache row (512 e4m3 + 16 e8m0), same section
 constexpr int kRow288 = 288;     // V4.1 FP4 cache row (512 e2m1 + 32 e4m3), same section
-constexpr int kRowBf16 = 1152;   // plain bf16 latent row of 576 dims (sparse prefill)
 
 // Kernel tiling: 128-token tiles (two pages), at most 64 query rows per CTA,
 // 64-dim (128-byte) column chunks in the SW128 layout.

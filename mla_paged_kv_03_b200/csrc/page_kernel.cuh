@@ -562,7 +562,8 @@ __global__ void __launch_bounds__(PageCfg::kThreads, 1)
       }
       ptx::named_bar_sync(1, kSm);
       const bool partial = P.always_partial || u.nsplit > 1;
-      const int ws_row0 = (P.num_splits[u.b] + u.split) * P.R + grp * kRows;
+      const int ws_row0 =
+          ((P.ws_base ? P.ws_base[u.b] : P.num_splits[u.b]) + u.split) * P.R + grp * kRows;
       const int rows_here = min(kRows, P.R - grp * kRows);
       if (wt < kRows) {
         const float l = (C.red[0][wt] + C.red[1][wt]) + (C.red[2][wt] + C.red[3][wt]);

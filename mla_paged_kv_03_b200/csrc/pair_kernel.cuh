@@ -98,6 +98,11 @@ __device__ __forceinline__ bool warp_wait_cluster(uint64_t* bar, uint32_t parity
   return __all_sync(0xffffffffu, mine);
 }
 
+// kGather: the tokens of a unit are rows of a bf16 array named by per-unit
+// index lists (sparse prefill): K and V come in by TMA gather4 loads of four
+// rows at a time (tm_kv is then a map with a box one row high), and entries
+// that name no row are masked.
+template <bool kGather>
 __global__ void __launch_bounds__(pcfg::kThreads, 1)
     mla_pair_decode_kernel(const __grid_constant__ CUtensorMap tm_q3,
                            const __grid_constant__ CUtensorMap tm_kv,
@@ -171,6 +176,13 @@ __global__ void __launch_bounds__(pcfg::kThreads, 1)
     const int blk = pg < npg ? P.block_table[(size_t)un.b * P.max_pages + pg] : 0;
     return clamp_block(blk, P.num_blocks);
   };
+  // Gather mode: the row of index entry e of unit `un` (row 0, masked, for an
+  // entry past the unit's length or naming no row).
+  auto gather_row = [&](const Unit& un, int e) -> int {
+    if (e >= un.L) return 0;
+    const int r = P.gather_idx[(size_t)un.b * P.gather_stride + e];
+    return (r >= 0 && r < P.gather_rows) ? r : 0;
+  };
   // Debug slot trace of the pages a load reads (pages a load only pads with
   // are not recorded).
   auto trace_if_real = [&](const Unit& un, int page, int blk, int planes) {
@@ -196,6 +208,45 @@ __global__ void __launch_bounds__(pcfg::kThreads, 1)
     };
     // K of step i: chunk c = [this CTA's 128 tokens (two pages)][64 dims]
     auto load_k = [&](const Unit& un, int i) -> bool {
+      if constexpr (kGather) {
+        // this CTA's 128 entries of the step: lane l loads rows 4l .. 4l + 3
+        const int e0 = un.lo * kTileT + kStepT * i + 128 * static_cast<int>(rank) + 4 * lane;
+        int r[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) r[k] = gather_row(un, e0 + k);
+        if (role == 0) {
+          // an entry past the rows is an input fault (negative ones mark unused entries)
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            if (e0 + k < un.L && P.gather_idx[(size_t)un.b * P.gather_stride + e0 + k] >= P.gather_rows)
+              ptx::set_error(MLA_DEVERR_BAD_INDEX, 0x46);
+        }
+        if (P.trace && role == 0) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int e = e0 + k;
+            if (e < un.L) {
+              const int raw = P.gather_idx[(size_t)un.b * P.gather_stride + e];
+              const bool ok_row = raw >= 0 && raw < P.gather_rows;
+              P.trace[(size_t)un.b * P.gather_stride + e] = ok_row ? raw : -1;
+              P.trace[P.trace_plane + (size_t)un.b * P.gather_stride + e] = ok_row ? e : -1;
+            }
+          }
+        }
+        for (int c = 0; c < kNumChunks; ++c) {
+          int s;
+          bool mine;
+          if (!acquire(s, mine)) return false;
+          if (!mine) continue;
+          const uint32_t bar = leader_addr(&C.full[s]);
+          if (leader && ptx::elect_one_sync()) ptx::mbar_arrive_expect_tx(&C.full[s], 2u * kStage);
+          __syncwarp();
+          ptx::tma_gather4_pair(sRing + s * kStage + lane * 512, &tm_kv, bar, c * kChunkD, r[0],
+                                r[1], r[2], r[3]);
+          __syncwarp();
+        }
+        return true;
+      }
       const int p0 = 2 * (un.lo + 2 * i);
       const int kb0 = page_block(un, p0 + 2 * static_cast<int>(rank), p0);
       const int kb1 = page_block(un, p0 + 2 * static_cast<int>(rank) + 1, p0);
@@ -221,6 +272,34 @@ __global__ void __launch_bounds__(pcfg::kThreads, 1)
     };
     // V of step i: stage (j, q) = [page q][this CTA's 128 dims of slice j], one 3-D box
     auto load_v = [&](const Unit& un, int i) -> bool {
+      if constexpr (kGather) {
+        // stage (j, q): entries [64 q, 64 q + 64) of the step, this CTA's 128
+        // dims of slice j; lane l loads rows 4 (l % 16) .. + 3 of chunk l / 16
+        const int h = lane >> 4;
+        int r[4][4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            r[q][k] = gather_row(un, un.lo * kTileT + kStepT * i + 64 * q + 4 * (lane & 15) + k);
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            int s;
+            bool mine;
+            if (!acquire(s, mine)) return false;
+            if (!mine) continue;
+            const uint32_t bar = leader_addr(&C.full[s]);
+            if (leader && ptx::elect_one_sync())
+              ptx::mbar_arrive_expect_tx(&C.full[s], 2u * kStage);
+            __syncwarp();
+            ptx::tma_gather4_pair(sRing + s * kStage + h * kBox + (lane & 15) * 512, &tm_kv, bar,
+                                  kChunkD * (4 * j + 2 * static_cast<int>(rank) + h), r[q][0],
+                                  r[q][1], r[q][2], r[q][3]);
+            __syncwarp();
+          }
+        return true;
+      }
       const int p0 = 2 * (un.lo + 2 * i);
       int vb[4];
 #pragma unroll
@@ -427,6 +506,16 @@ __global__ void __launch_bounds__(pcfg::kThreads, 1)
       for (int i = 0; i < n && ok; ++i) {
         const uint32_t g = gt + i;
         const int sb = g & 1;
+        // gather mode: which of this quarter's 64 entries name a row
+        uint32_t vmask[2] = {0xffffffffu, 0xffffffffu};
+        if constexpr (kGather) {
+          const int e = u.lo * kTileT + kStepT * i + 64 * quarter + lane;
+          int r0 = 0, r1 = 0;
+          if (e < u.L) r0 = P.gather_idx[(size_t)u.b * P.gather_stride + e];
+          if (e + 32 < u.L) r1 = P.gather_idx[(size_t)u.b * P.gather_stride + e + 32];
+          vmask[0] = __ballot_sync(0xffffffffu, r0 >= 0 && r0 < P.gather_rows);
+          vmask[1] = __ballot_sync(0xffffffffu, r1 >= 0 && r1 < P.gather_rows);
+        }
         ok = sm_wait_cluster(&C.s_full[sb], (g >> 1) & 1, 0x61);
         if (!ok) break;
         ptx::tc_fence_after();
@@ -453,7 +542,8 @@ __global__ void __launch_bounds__(pcfg::kThreads, 1)
             if (cc) ptx::tmem_ld_wait_regs(xb);
 #pragma unroll
             for (int j = 0; j < 32; j += 2) {
-              const bool v0 = 32 * cc + j < nvalid, v1 = 32 * cc + j + 1 < nvalid;
+              const bool v0 = 32 * cc + j < nvalid && ((vmask[cc] >> j) & 1u);
+              const bool v1 = 32 * cc + j + 1 < nvalid && ((vmask[cc] >> (j + 1)) & 1u);
               mx = v0 ? fmaxf(mx, x[j]) : mx;
               mx = v1 ? fmaxf(mx, x[j + 1]) : mx;
               const float p0 = v0 ? ex2(fmaf(x[j], P.scale_log2, -m)) : 0.f;
@@ -530,7 +620,7 @@ __global__ void __launch_bounds__(pcfg::kThreads, 1)
       if (!ok) break;
       ptx::tc_fence_after();
       const bool partial = P.always_partial || u.nsplit > 1;
-      const int ws_row = (P.num_splits[u.b] + u.split) * P.R + rg;
+      const int ws_row = ((P.ws_base ? P.ws_base[u.b] : P.num_splits[u.b]) + u.split) * P.R + rg;
       const float inv = l > 0.f ? 1.0f / l : 0.f;
       float o[2][32];
       ptx::tmem_ld32(lane_addr + kOCol + 128 * wg, o[0]);

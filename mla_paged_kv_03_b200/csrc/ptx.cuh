@@ -391,6 +391,20 @@ __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m
       : "memory");
 }
 
+// TMA load of four rows (y0..y3) of a 2-D tensor whose map has a box one row
+// high, CTA-pair form: the four box rows land one after the other at dst (in
+// the map's swizzle) and their bytes count on the mbarrier at `bar_cluster`.
+__device__ __forceinline__ void tma_gather4_pair(void* dst, const CUtensorMap* map,
+                                                 uint32_t bar_cluster, int x, int y0, int y1,
+                                                 int y2, int y3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4"
+      ".mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(x), "r"(y0), "r"(y1), "r"(y2),
+      "r"(y3)
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                    smem_u32(dst_smem)),

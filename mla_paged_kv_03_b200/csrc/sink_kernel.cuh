@@ -15,6 +15,17 @@ namespace mla {
 
 constexpr int kSinkWarps = 8;
 
+// The sparse prefill's per-token lengths: topk_length[t] clamped to [0, topk],
+// or topk for every token when no lengths are given.
+__global__ void __launch_bounds__(256)
+    mla_prefill_lengths_kernel(const int32_t* topk_len, int topk, int s_q, int32_t* out) {
+  ptx::grid_dep_wait();
+  const int t = blockIdx.x * 256 + threadIdx.x;
+  if (t >= s_q) return;
+  const int l = topk_len ? topk_len[t] : topk;
+  out[t] = l < 0 ? 0 : (l < topk ? l : topk);
+}
+
 // One warp per (token, head) row of `d_v` bf16 values (d_v a multiple of 8).
 __global__ void __launch_bounds__(32 * kSinkWarps)
     mla_sink_kernel(__nv_bfloat16* out, float* lse, const float* sink, long long rows, int h_q,

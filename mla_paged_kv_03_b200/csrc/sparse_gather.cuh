@@ -10,7 +10,6 @@
 //    [16 x E8M0 scale, one per 32 codes]; a value is code * 2^(e - 127).
 //  - 288 bytes (V4.1 FP4): [512 x E2M1 codes, two per byte, code 2i in the
 //    low nibble of byte i][32 x E4M3 scale, one per 16 codes].
-//  - 1152 bytes: plain bf16 latent rows of 576 dims (sparse prefill), copied.
 //  For both V4.1 rows the buffer row stays 576 wide with dims 512..575 zero,
 //  and the 512-wide query rows are copied into a 576-wide buffer with zero
 //  dims 512..575, so that q . k and the first 512 dims of V are unchanged.
@@ -39,11 +38,10 @@ constexpr int kGatherCtaThreads = 256;
 constexpr int kRowUnits = kD / 8;  // 16-byte bf16 output units per row (72)
 
 struct GatherParams {
-  const uint8_t* cache;     // [num_slots, row bytes]: 656, 528, 288 or 1152 (bf16)
+  const uint8_t* cache;     // [num_slots, row bytes]: 656, 528 or 288
   long long num_slots;
   const int32_t* indices;   // [pairs, topk]
   int topk;
-  const int32_t* topk_len;  // [pairs] or null: only indices[p][0, topk_len[p]) count
   int pages_per_pair;       // ceil(topk / 64)
   __nv_bfloat16* rows;      // [pairs * pages_per_pair * 64, 576]
   int32_t* block_table;     // [pairs, pages_per_pair]
@@ -101,16 +99,14 @@ __device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t w, uint32_t (&h)[4]) {
 // SM) and are held to 3 CTAs; the FP4 and bf16 variants fit 4.
 template <int kRowBytes>
 constexpr int gather_min_ctas() {
-  return (kRowBytes == kRow288 || kRowBytes == kRowBf16) ? 4 : 3;
+  return kRowBytes == kRow288 ? 4 : 3;
 }
 
 template <int kRowBytes>
 __global__ void __launch_bounds__(kGatherCtaThreads, gather_min_ctas<kRowBytes>())
     mla_sparse_gather_kernel(const GatherParams G) {
-  static_assert(kRowBytes == kRow656 || kRowBytes == kRow528 || kRowBytes == kRow288 ||
-                    kRowBytes == kRowBf16,
-                "656-, 528-, 288- or 1152-byte rows");
-  constexpr bool kBf16 = kRowBytes == kRowBf16;
+  static_assert(kRowBytes == kRow656 || kRowBytes == kRow528 || kRowBytes == kRow288,
+                "656-, 528- or 288-byte rows");
   constexpr bool kV41 = kRowBytes == kRow528 || kRowBytes == kRow288;  // 512-dim latent
   constexpr bool kFp4 = kRowBytes == kRow288;
   __shared__ int s_red[kGatherCtaThreads / 32];
@@ -121,11 +117,7 @@ __global__ void __launch_bounds__(kGatherCtaThreads, gather_min_ctas<kRowBytes>(
   const int c = blockIdx.x, b = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int32_t* idx_b = G.indices + (size_t)b * G.topk;
-  int lim = G.topk;  // entries past the pair's top-k length do not count
-  if (G.topk_len) {
-    const int l = __ldg(G.topk_len + b);
-    lim = l < 0 ? 0 : (l < G.topk ? l : G.topk);
-  }
+  const int lim = G.topk;
 
   // valid tokens in the pair's earlier chunks: this chunk's first output row
   int cnt = 0;
@@ -177,35 +169,14 @@ __global__ void __launch_bounds__(kGatherCtaThreads, gather_min_ctas<kRowBytes>(
     }
     __syncthreads();
     const int n = s_n;
-    const int end = (n + kGatherTokens - 1) / kGatherTokens * kGatherTokens;
+    // a pair without valid tokens still has its first page read (fully masked)
+    const int end = n > 0 ? (n + kGatherTokens - 1) / kGatherTokens * kGatherTokens : kGatherTokens;
     for (int item = tid; item < (end - n) * kRowUnits; item += kGatherCtaThreads)
       *reinterpret_cast<uint4*>(out_b + (size_t)(n + item / kRowUnits) * kD + 8 * (item % kRowUnits)) =
           make_uint4(0, 0, 0, 0);
   }
 
-  if constexpr (kBf16) {
-    // bf16 rows: each valid token's 72 16-byte units copied as they are, six
-    // units of a thread in flight at a time
-    constexpr int kItems = kGatherTokens * kRowUnits;  // 4608
-    constexpr int kBatch = 6;
-    static_assert(kItems % (kGatherCtaThreads * kBatch) == 0, "even split");
-    for (int i0 = 0; i0 < kItems; i0 += kGatherCtaThreads * kBatch) {
-      uint4 v[kBatch];
-      int dst[kBatch];
-#pragma unroll
-      for (int k = 0; k < kBatch; ++k) {
-        const int item = i0 + k * kGatherCtaThreads + tid;
-        const int t = item / kRowUnits, uu = item % kRowUnits;
-        dst[k] = s_dst[t] >= 0 ? s_dst[t] * kRowUnits + uu : -1;
-        v[k] = make_uint4(0, 0, 0, 0);
-        if (dst[k] >= 0)
-          v[k] = __ldg(reinterpret_cast<const uint4*>(G.cache + (size_t)s_idx[t] * kRowBytes) + uu);
-      }
-#pragma unroll
-      for (int k = 0; k < kBatch; ++k)
-        if (dst[k] >= 0) reinterpret_cast<uint4*>(out_b)[dst[k]] = v[k];
-    }
-  } else {
+  {
     // dequantise: per token 32 units of 16 codes (two 16-byte bf16 outputs
     // each) and 8 units of the dims 512..575 (bf16 RoPE dims, or zeros for the
     // 528-byte rows); all loads of a thread are issued before any conversion so

@@ -285,8 +285,12 @@ def test_sparse_slot_trace_matches_indices(kind):
     if kind == "prefill":
         valid &= torch.arange(idx.shape[1])[None, :] < case.topk_length[:, None]
     exp0 = torch.where(valid, idx, torch.full_like(idx, -1))
-    exp1 = torch.where(valid, valid.to(torch.int32).cumsum(1, dtype=torch.int32) - 1,
-                       torch.full_like(idx, -1))
+    if kind == "prefill":  # rows are read in place: plane 1 holds the entry's own position
+        pos = torch.arange(idx.shape[1], dtype=torch.int32).expand_as(idx)
+        exp1 = torch.where(valid, pos, torch.full_like(idx, -1))
+    else:  # compacted in index order
+        exp1 = torch.where(valid, valid.to(torch.int32).cumsum(1, dtype=torch.int32) - 1,
+                           torch.full_like(idx, -1))
     assert torch.equal(tr[0].view_as(idx), exp0), "slot of each entry"
     assert torch.equal(tr[1].view_as(idx), exp1), "compacted row of each entry"
     assert status_code(reset=True) == BAD
