@@ -234,7 +234,7 @@ class GpuStep:
             self.out = torch.empty((b, 1, c.h_q, 576), dtype=torch.uint8, device=dev)
             self.scale = torch.empty((b, 1, c.h_q), dtype=torch.float32, device=dev)
             self.lse = torch.empty((b, 1, c.h_q), dtype=torch.float32, device=dev)
-            nbytes = (B.mla_workspace_size(b, self.R, 576, self.parts) if self.kind == "fused"
+            nbytes = (B.mla_fused_workspace_size(b, self.R, self.parts) if self.kind == "fused"
                       else B.mla_sparse_fused_workspace_size(b, c.h_q, c.topk, self.parts))
             self.ws = torch.empty((nbytes,), dtype=torch.uint8, device=dev)
         else:

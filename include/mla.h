@@ -113,10 +113,15 @@ MLA_API int mla_get_metadata(const int32_t* cache_seqlens, int batch, int heads_
 MLA_API int mla_get_metadata_host(const int32_t* cache_seqlens, int batch, int heads_per_kv, int h_kv,
                           int num_sm_parts, int32_t* metadata, int32_t* num_splits);
 
-/* Workspace bytes for mla_decode_fwd / mla_fused_norm_rope_attn_rope_cast:
- * fp32 partial outputs and LSEs of up to batch + num_sm_parts splits of
- * `rows_per_kv` (= s_q*h_q) rows of d_v values. */
+/* Workspace bytes for mla_decode_fwd: fp32 partial outputs and LSEs of up
+ * to batch + num_sm_parts splits of `rows_per_kv` (= s_q*h_q) rows of d_v
+ * values. */
 MLA_API int mla_workspace_size(int batch, int rows_per_kv, int d_v, int num_sm_parts, size_t* bytes);
+
+/* Workspace bytes for mla_fused_norm_rope_attn_rope_cast: the split partials
+ * of mla_workspace_size(batch, h_q, 576, num_sm_parts), then the normalised,
+ * rotated query rows (batch * h_q rows of 576 bf16). */
+MLA_API int mla_fused_workspace_size(int batch, int h_q, int num_sm_parts, size_t* bytes);
 
 /* Dense paged MLA decode, bf16 in, bf16 out + fp32 LSE
  * (flash_mla_with_kvcache of the port README's "Usage").
@@ -140,7 +145,9 @@ MLA_API int mla_decode_fwd(const void* q, const void* kcache, const int32_t* blo
                    size_t workspace_bytes, void* out, float* lse, void* stream);
 
 /* Fused Q RMSNorm -> Q-RoPE -> attention -> conjugate O-RoPE -> FP8 cast,
- * s_q = 1, d_v = 576 (V is the whole latent row).
+ * s_q = 1, d_v = 576 (V is the whole latent row).  Three launches on
+ * `stream`: the query prologue (once per row, into the workspace), the
+ * attention kernel, and the split combine with the output RoPE and the cast.
  *   q_raw           [batch, 1, h_q, 576] bf16, before normalisation
  *   norm_gain       fp32[576], shared by all heads; eps added to mean(x^2)
  *   rope_base       RoPE base (e.g. 10000); pairs (2k, 2k+1) of dims
@@ -152,7 +159,8 @@ MLA_API int mla_decode_fwd(const void* q, const void* kcache, const int32_t* blo
  *   out_scale       fp32[batch, 1, h_q]: absmax(O_row) / 448 (1 for a zero row);
  *                   O ~= code * scale
  *   lse             fp32[batch, 1, h_q]
- *   metadata, num_splits from mla_get_metadata with heads_per_kv = h_q. */
+ *   metadata, num_splits from mla_get_metadata with heads_per_kv = h_q
+ *   workspace       >= mla_fused_workspace_size() bytes, 16-byte aligned. */
 MLA_API int mla_fused_norm_rope_attn_rope_cast(
     const void* q_raw, const float* norm_gain, float eps, float rope_base,
     const int32_t* positions, const void* kcache, const int32_t* block_table, int max_pages,

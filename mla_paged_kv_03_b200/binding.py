@@ -26,7 +26,8 @@ MLA_ERR_TIMEOUT = -4
 D_QK = 576
 EXPORTED = [
     "mla_last_error", "mla_num_sms", "mla_num_sm_parts", "mla_metadata_size",
-    "mla_get_metadata", "mla_get_metadata_host", "mla_workspace_size", "mla_decode_fwd",
+    "mla_get_metadata", "mla_get_metadata_host", "mla_workspace_size", "mla_fused_workspace_size",
+    "mla_decode_fwd",
     "mla_fused_norm_rope_attn_rope_cast", "mla_sparse_workspace_size", "mla_sparse_decode",
     "mla_device_status", "mla_noalloc_scratch_bytes", "mla_decode_fwd_noalloc",
     "mla_set_kernel_events", "mla_sparse_v41_workspace_size", "mla_sparse_decode_v41",
@@ -65,6 +66,7 @@ def lib():
         L.mla_get_metadata.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp]
         L.mla_get_metadata_host.argtypes = [vp, i32, i32, i32, i32, vp, vp]
         L.mla_workspace_size.argtypes = [i32, i32, i32, i32, szp]
+        L.mla_fused_workspace_size.argtypes = [i32, i32, i32, szp]
         L.mla_decode_fwd.argtypes = [vp, vp, vp, i32, i32, vp, i32, i32, i32, i32, i32, f32, i32,
                                      vp, vp, i32, vp, sz, vp, vp, vp]
         L.mla_fused_norm_rope_attn_rope_cast.argtypes = [
@@ -165,6 +167,13 @@ def mla_workspace_size(batch, rows_per_kv, d_v, num_sm_parts) -> int:
     out = ctypes.c_size_t(0)
     _check(lib().mla_workspace_size(int(batch), int(rows_per_kv), int(d_v), int(num_sm_parts),
                                     ctypes.byref(out)))
+    return out.value
+
+
+def mla_fused_workspace_size(batch, h_q, num_sm_parts) -> int:
+    out = ctypes.c_size_t(0)
+    _check(lib().mla_fused_workspace_size(int(batch), int(h_q), int(num_sm_parts),
+                                          ctypes.byref(out)))
     return out.value
 
 
@@ -308,7 +317,7 @@ def mla_fused_norm_rope_attn_rope_cast(q_raw, norm_gain, eps, rope_base, kcache,
         out_scale = torch.empty((b, 1, h_q), dtype=torch.float32, device=dev)
     if lse is None:
         lse = torch.empty((b, 1, h_q), dtype=torch.float32, device=dev)
-    ws = _workspace(mla_workspace_size(b, h_q, D_QK, num_sm_parts), dev, workspace)
+    ws = _workspace(mla_fused_workspace_size(b, h_q, num_sm_parts), dev, workspace)
     bt = block_table.contiguous()
     pos = None if positions is None else positions.to(torch.int32).contiguous()
     _check(lib().mla_fused_norm_rope_attn_rope_cast(

@@ -23,8 +23,12 @@
 //
 // Roles (warps):  0, 10, 11 = TMA loaders (0 also loads Q),  1 = MMA issuer +
 //   TMEM owner,  2..9 = two softmax warpgroups (one thread per token lane of
-//   the tile and 32 query-row columns each; also the epilogue and, for the
-//   fused variant, the Q RMSNorm + RoPE prologue).
+//   the tile and 32 query-row columns each; also the epilogue).
+//
+// The fused variant differs only in P: it keeps P to about 16 bits as a bf16
+// hi/lo pair (two PV UMMAs per k-step), so that O is accurate enough for its
+// E4M3 output codes.  Its query arrives already normalised and rotated (the
+// prologue kernel), and its epilogue always goes through the combine kernel.
 //
 // Softmax uses a lazily updated per-row reference max m: scores are
 // exponentiated against m until some score exceeds m by more than 8 (log2
@@ -65,13 +69,6 @@ struct DecodeParams {
   float* lse;                 // [batch*R]
   float* ws_o;                // [total_splits, R, d_v] fp32 partial O (normalised)
   float* ws_lse;              // [total_splits, R]
-  // fused prologue
-  const __nv_bfloat16* q_raw;  // [batch, 1, h_q, 576]
-  const float* gain;           // [576]
-  float eps;
-  float rope_base;
-  const int32_t* positions;  // nullable: position = L - 1
-  double inv_freq[kRope / 2];  // base^(-2k/64), computed on the host in fp64
   // debug slot trace (null = off): int32 [2][batch][max_pages * 64], the
   // physical slot of every token whose cache row a kernel loaded, plane 0 for
   // the rows read as K, plane 1 for the rows read as V
@@ -147,21 +144,19 @@ struct __align__(8) Ctrl {
   uint64_t p_full[cfg::kNP], p_empty[cfg::kNP];
   uint64_t o_free;
   uint64_t drain;
-  uint64_t rope_full;
   uint32_t tmem_base;
   uint32_t pad;
   float red[8][32];     // cross-warp reduction scratch [group*4 + warp][column]
   float m[64];          // per-column reference max (log2 domain)
   float alpha[64];      // per-column rescale factor, then 1/l in the epilogue
   int lim[64];          // per-column visible-token limit of the current unit
-  double rope_cs[32][2];  // cos/sin of the current unit's query position (fp64)
 };
 static_assert(sizeof(Ctrl) <= cfg::kMiscBytes, "control block too large");
 
 struct Unit {
   int b, lo, hi, split, nsplit;
   int L;      // tokens attended: cache_seqlens[b], at most max_pages * 64
-  int L_raw;  // cache_seqlens[b] as given (the default query position is L_raw - 1)
+  int L_raw;  // cache_seqlens[b] as given (the planner counted its tiles)
 };
 
 // Iterates the (sequence, tile-range) segments of one scheduler part.
@@ -299,7 +294,7 @@ __global__ void __launch_bounds__(Threads<kMode>::value, 1)
       ptx::mbar_init(&C.slot_full[i], 1);
       ptx::mbar_init(&C.slot_empty[i], 1);
     }
-    ptx::mbar_init(&C.q_full, kMode == kFused ? 128 * kSoftmaxGroups : 1);
+    ptx::mbar_init(&C.q_full, 1);
     ptx::mbar_init(&C.q_empty, 1);
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(&C.s_full[i], 1);
@@ -311,7 +306,7 @@ __global__ void __launch_bounds__(Threads<kMode>::value, 1)
     }
     ptx::mbar_init(&C.o_free, 128 * kSoftmaxGroups);
     ptx::mbar_init(&C.drain, 1);
-    ptx::mbar_init(&C.rope_full, 32);
+
     ptx::fence_mbar_init();
   }
   if (warp == 1) {
@@ -319,7 +314,7 @@ __global__ void __launch_bounds__(Threads<kMode>::value, 1)
     ptx::tmem_relinquish();
   }
   if (warp == 0 && lane == 0) {
-    if (kMode != kFused) ptx::prefetch_tmap(&tm_q);
+    ptx::prefetch_tmap(&tm_q);
     ptx::prefetch_tmap(&tm_kv);
   }
   ptx::tc_fence_before();
@@ -335,11 +330,7 @@ __global__ void __launch_bounds__(Threads<kMode>::value, 1)
   if (warp == 0 || warp >= kFirstExtraLoader) {
     // ============================== loaders ==============================
     // Pair slot j of the ring is filled by loader warp j % kL (whole warp,
-    // one elected lane issues the copies).  Warp 0 also loads Q; for the fused
-    // variant it computes, per unit, the cos/sin table of the query
-    // position: theta_k = pos * base^(-2k/64), pos = positions[b] or L - 1.
-    // A unit's table may be overwritten once the previous unit's QK finished
-    // (q_empty), which implies the prologue that read it is done.
+    // one elected lane issues the copies).  Warp 0 also loads Q.
     const int role = warp == 0 ? 0 : warp - kFirstExtraLoader + 1;
     uint32_t ring_it = 0;
     int u_idx = 0;
@@ -379,20 +370,9 @@ __global__ void __launch_bounds__(Threads<kMode>::value, 1)
       return true;
     };
     while (ok && it.template next<kMode>(P, u)) {
-      if (kMode == kFused && role == 0) {
-        ok = ptx::mbar_wait(&C.q_empty, (u_idx & 1) ^ 1, 0x06);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        const double pos =
-            P.positions ? static_cast<double>(P.positions[u.b]) : static_cast<double>(u.L_raw - 1);
-        double sn, cs;
-        rope_sincos64(pos, P.inv_freq[lane], &sn, &cs);
-        C.rope_cs[lane][0] = cs;
-        C.rope_cs[lane][1] = sn;
-        ptx::mbar_arrive(&C.rope_full);
-      }
-      if (kMode != kFused && role == 0) {
-        // Q rows [64*grp, 64*grp+64) of this sequence (or query pair)
+      if (role == 0) {
+        // Q rows [64*grp, 64*grp+64) of this sequence (or query pair); for the
+        // fused variant the normalised, rotated rows of the prologue kernel
         ok = __all_sync(0xffffffffu, ptx::mbar_wait(&C.q_empty, (u_idx & 1) ^ 1, 0x02));
         if (ok && ptx::elect_one_sync()) {
           ptx::mbar_arrive_expect_tx(&C.q_full, kQBytes);
@@ -422,7 +402,7 @@ __global__ void __launch_bounds__(Threads<kMode>::value, 1)
       if (static_cast<int>(last % kL) != role) continue;
       ptx::mbar_wait(&C.slot_full[last % kNPair], (last / kNPair) & 1, 0x03);
     }
-    if (kMode != kFused && role == 0 && u_idx > 0) ptx::mbar_wait(&C.q_full, (u_idx - 1) & 1, 0x04);
+    if (role == 0 && u_idx > 0) ptx::mbar_wait(&C.q_full, (u_idx - 1) & 1, 0x04);
     __syncwarp();
   } else if (warp == 1) {
     // ============================== MMA issuer ==============================
@@ -576,90 +556,6 @@ __global__ void __launch_bounds__(Threads<kMode>::value, 1)
         }
         C.lim[cb + wt] = lim;
         C.m[cb + wt] = -INFINITY;
-      }
-      // ---- fused prologue: RMSNorm + Q-RoPE into the swizzled Q tile
-      if (kMode == kFused) {
-        // Q buffer free (previous unit's QK done) and this unit's RoPE table
-        // written by the loader warp.
-        if (!wg_wait(&C.q_empty, (u_idx & 1) ^ 1, 0x21, kBarAllSoftmax, 128 * kSoftmaxGroups) ||
-            !wg_wait(&C.rope_full, u_idx & 1, 0x26, kBarAllSoftmax, 128 * kSoftmaxGroups)) {
-          ok = false;
-          break;
-        }
-        // RMSNorm and RoPE in fp64; one bf16 rounding at the end.  Each warp
-        // takes every 8th row; a row's 72 16-byte units are loaded once (3 per
-        // lane) and the next row's units are in flight while this one is
-        // transformed.
-        const int wl = (threadIdx.x - 64) >> 5;  // warp within both groups (0..7)
-        constexpr int kRowStep = 4 * kSoftmaxGroups;
-        auto load_row = [&](int r, uint4* w) {
-          const int rg = grp * kRowsPerCta + r;
-          const __nv_bfloat16* src = P.q_raw + ((size_t)u.b * P.R + (rg < P.R ? rg : 0)) * kD;
-#pragma unroll
-          for (int j = 0; j < 3; ++j) {
-            const int uu = lane + 32 * j;
-            w[j] = uu < kD / 8 ? *reinterpret_cast<const uint4*>(src + uu * 8) : make_uint4(0, 0, 0, 0);
-          }
-        };
-        uint4 wcur[3], wnext[3];
-        load_row(wl, wcur);
-        for (int r = wl; r < kRowsPerCta; r += kRowStep) {
-          if (r + kRowStep < kRowsPerCta) load_row(r + kRowStep, wnext);
-          const bool valid = grp * kRowsPerCta + r < P.R;
-          double ss = 0.0;
-#pragma unroll
-          for (int j = 0; j < 3; ++j) {
-            const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&wcur[j]);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 f = __bfloat1622float2(h[e]);
-              ss = fma(static_cast<double>(f.x), static_cast<double>(f.x), ss);
-              ss = fma(static_cast<double>(f.y), static_cast<double>(f.y), ss);
-            }
-          }
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-          const double inv = valid ? 1.0 / sqrt(ss / static_cast<double>(kD) + P.eps) : 0.0;
-#pragma unroll
-          for (int j = 0; j < 3; ++j) {
-            const int uu = lane + 32 * j;
-            if (uu < kD / 8) {
-              const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&wcur[j]);
-              const float4 g0 = __ldg(reinterpret_cast<const float4*>(P.gain + uu * 8));
-              const float4 g1 = __ldg(reinterpret_cast<const float4*>(P.gain + uu * 8 + 4));
-              const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-              double y[8];
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const float2 f = __bfloat1622float2(h[e]);
-                y[2 * e] = static_cast<double>(f.x) * inv * static_cast<double>(gv[2 * e]);
-                y[2 * e + 1] = static_cast<double>(f.y) * inv * static_cast<double>(gv[2 * e + 1]);
-              }
-              if (uu >= kNope / 8) {
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  const int k = (uu * 8 - kNope) / 2 + e;
-                  const double c = C.rope_cs[k][0], sn = C.rope_cs[k][1];
-                  const double a = y[2 * e], bq = y[2 * e + 1];
-                  y[2 * e] = a * c - bq * sn;
-                  y[2 * e + 1] = a * sn + bq * c;
-                }
-              }
-              uint4 o;
-              o.x = ptx::pack_bf16x2_f64(y[0], y[1]);
-              o.y = ptx::pack_bf16x2_f64(y[2], y[3]);
-              o.z = ptx::pack_bf16x2_f64(y[4], y[5]);
-              o.w = ptx::pack_bf16x2_f64(y[6], y[7]);
-              const int c = uu >> 3, unit = uu & 7;
-              *reinterpret_cast<uint4*>(sQ + c * (kRowsPerCta * 128) + r * 128 +
-                                        ((unit ^ (r & 7)) << 4)) = o;
-            }
-          }
-#pragma unroll
-          for (int j = 0; j < 3; ++j) wcur[j] = wnext[j];
-        }
-        ptx::fence_proxy_async_smem();
-        ptx::mbar_arrive(&C.q_full);
       }
       ptx::named_bar_sync(bar_sync, 128);  // C.lim, C.m of this group visible
 

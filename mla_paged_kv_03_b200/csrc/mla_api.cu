@@ -16,6 +16,7 @@
 #include "decode_kernel.cuh"
 #include "page_kernel.cuh"
 #include "pair_kernel.cuh"
+#include "prologue_kernel.cuh"
 #include "sink_kernel.cuh"
 #include "sparse_gather.cuh"
 #include "mla_common.h"
@@ -123,7 +124,7 @@ int make_latent_map3(CUtensorMap* map, const void* base, long long rows, int box
 }
 
 struct WsLayout {
-  size_t o_off, lse_off, total;
+  size_t o_off, lse_off, q_off, total;
 };
 
 WsLayout dense_ws_layout(int batch, int R, int d_v, int parts) {
@@ -132,6 +133,15 @@ WsLayout dense_ws_layout(int batch, int R, int d_v, int parts) {
   w.o_off = 0;
   w.lse_off = align_up(splits * R * d_v * sizeof(float), 256);
   w.total = w.lse_off + align_up(splits * R * sizeof(float), 256);
+  return w;
+}
+
+// Fused decode workspace: the dense layout (d_v 576), then the normalised,
+// rotated query rows [batch * R, 576] bf16 that the prologue kernel writes.
+WsLayout fused_ws_layout(int batch, int R, int parts) {
+  WsLayout w = dense_ws_layout(batch, R, mla::kD, parts);
+  w.q_off = align_up(w.total, 256);
+  w.total = w.q_off + align_up(static_cast<size_t>(batch) * R * mla::kD * 2, 256);
   return w;
 }
 
@@ -146,7 +156,8 @@ struct SparseWs {
 // Workspace of the sparse paths: the compacted bf16 rows, their identity
 // block table and lengths, the planner's output, the dense path's own
 // workspace and, for the 528-byte rows, the query widened to 576 dims.
-SparseWs sparse_ws_layout(int pairs, int topk, int R, int d_v, int parts, bool v41 = false) {
+SparseWs sparse_ws_layout(int pairs, int topk, int R, int d_v, int parts, bool v41 = false,
+                          bool fused = false) {
   SparseWs w{};
   w.pages_per_pair = mla::ceil_div(topk, mla::kPage);
   const size_t pages = static_cast<size_t>(pairs) * w.pages_per_pair;
@@ -156,7 +167,8 @@ SparseWs sparse_ws_layout(int pairs, int topk, int R, int d_v, int parts, bool v
   w.meta_off = w.len_off + align_up(static_cast<size_t>(pairs) * 4, 256);
   w.splits_off = w.meta_off + align_up(static_cast<size_t>(parts) * mla::kMetaInts * 4, 256);
   w.dense_off = w.splits_off + align_up((static_cast<size_t>(pairs) + 1) * 4, 256);
-  w.dense_bytes = dense_ws_layout(pairs, R, d_v, parts).total;
+  w.dense_bytes = fused ? fused_ws_layout(pairs, R, parts).total
+                        : dense_ws_layout(pairs, R, d_v, parts).total;
   w.q_off = w.dense_off + align_up(w.dense_bytes, 256);
   w.total = v41 ? w.q_off + align_up(static_cast<size_t>(pairs) * R * mla::kD * 2, 256)
                 : w.dense_off + w.dense_bytes;
@@ -685,6 +697,13 @@ int mla_workspace_size(int batch, int rows_per_kv, int d_v, int num_sm_parts, si
   return MLA_OK;
 }
 
+int mla_fused_workspace_size(int batch, int h_q, int num_sm_parts, size_t* bytes) {
+  MLA_CHECK_ARG(bytes, "bytes is null");
+  MLA_CHECK_ARG(batch >= 0 && h_q >= 1 && num_sm_parts >= 1, "bad sizes");
+  *bytes = fused_ws_layout(batch, h_q, num_sm_parts).total;
+  return MLA_OK;
+}
+
 int mla_decode_fwd(const void* q, const void* kcache, const int32_t* block_table, int max_pages,
                    int num_blocks, const int32_t* cache_seqlens, int batch, int s_q, int h_q,
                    int h_kv, int d_v, float softmax_scale, int causal, const int32_t* metadata,
@@ -772,7 +791,7 @@ int mla_fused_norm_rope_attn_rope_cast(
   MLA_CHECK_ARG(std::isfinite(rope_base) && rope_base > 0.f, "rope_base must be > 0");
   const int R = h_q;
   const int d_v = mla::kD;
-  const WsLayout w = dense_ws_layout(batch, R, d_v, num_sm_parts);
+  const WsLayout w = fused_ws_layout(batch, R, num_sm_parts);
   MLA_CHECK_ARG(workspace_bytes >= w.total, "workspace too small: %zu < %zu", workspace_bytes,
                 w.total);
   if ((rc = check_trace(static_cast<long long>(batch) * max_pages * mla::kPage)) != MLA_OK)
@@ -805,16 +824,30 @@ int mla_fused_norm_rope_attn_rope_cast(
   p.num_splits = num_splits;
   p.ws_o = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.o_off);
   p.ws_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.lse_off);
-  p.q_raw = static_cast<const __nv_bfloat16*>(q_raw);
-  p.gain = norm_gain;
-  p.eps = eps;
-  p.rope_base = rope_base;
-  p.positions = positions;
   p.trace = t_trace;
   p.trace_plane = static_cast<long long>(batch) * max_pages * mla::kPage;
+
+  // prologue: Q RMSNorm + RoPE, once per row, into the workspace
+  mla::FusedQParams fq{};
+  fq.q_raw = static_cast<const __nv_bfloat16*>(q_raw);
+  fq.gain = norm_gain;
+  fq.eps = eps;
+  fq.positions = positions;
+  fq.seqlens = cache_seqlens;
+  fq.rows = batch * R;
+  fq.R = R;
   for (int k = 0; k < mla::kRope / 2; ++k)
-    p.inv_freq[k] = std::pow(static_cast<double>(rope_base), -2.0 * k / mla::kRope);
-  rc = launch_decode<mla::kFused>(tkv, tkv, p, st);
+    fq.inv_freq[k] = std::pow(static_cast<double>(rope_base), -2.0 * k / mla::kRope);
+  fq.q_out = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(workspace) + w.q_off);
+  {
+    PdlLaunch L(dim3(static_cast<unsigned>(mla::ceil_div(fq.rows, mla::kPrologueWarps))),
+                dim3(32 * mla::kPrologueWarps), 0, st);
+    MLA_CUDA(cudaLaunchKernelEx(&L.cfg, mla::mla_fused_q_kernel, fq));
+  }
+  CUtensorMap tq;
+  if ((rc = make_latent_map(&tq, fq.q_out, static_cast<long long>(batch) * R)) != MLA_OK)
+    return rc;
+  rc = launch_decode<mla::kFused>(tq, tkv, p, st);
   if (rc != MLA_OK) return rc;
 
   mla::CombineParams cp{};
@@ -830,7 +863,7 @@ int mla_fused_norm_rope_attn_rope_cast(
   cp.out_scale = out_scale;
   cp.seqlens = cache_seqlens;
   cp.positions = positions;
-  for (int k = 0; k < mla::kRope / 2; ++k) cp.inv_freq[k] = p.inv_freq[k];
+  for (int k = 0; k < mla::kRope / 2; ++k) cp.inv_freq[k] = fq.inv_freq[k];
   return launch_combine(cp, true, st);
 }
 
@@ -976,7 +1009,7 @@ int mla_sparse_fused_workspace_size(int batch, int h_q, int topk, int num_sm_par
                                     size_t* bytes) {
   MLA_CHECK_ARG(bytes, "bytes is null");
   MLA_CHECK_ARG(batch >= 0 && h_q >= 1 && topk >= 1 && num_sm_parts >= 1, "bad sizes");
-  *bytes = sparse_ws_layout(batch, topk, h_q, mla::kD, num_sm_parts).total;
+  *bytes = sparse_ws_layout(batch, topk, h_q, mla::kD, num_sm_parts, false, true).total;
   return MLA_OK;
 }
 
@@ -999,7 +1032,7 @@ int mla_sparse_fused_norm_rope_attn_rope_cast(
                 "q_raw and the cache must be 16-byte aligned");
   MLA_CHECK_ARG(aligned(workspace, 256), "workspace must be 256-byte aligned");
   MLA_CHECK_ARG(aligned(indices, 4) && aligned(positions, 4), "misaligned indices or positions");
-  const SparseWs w = sparse_ws_layout(batch, topk, h_q, mla::kD, num_sm_parts);
+  const SparseWs w = sparse_ws_layout(batch, topk, h_q, mla::kD, num_sm_parts, false, true);
   MLA_CHECK_ARG(workspace_bytes >= w.total, "workspace too small: %zu < %zu", workspace_bytes,
                 w.total);
   MLA_CHECK_ARG(batch <= mla::kPlanMaxBatch, "at most %d sequences (got %d)", mla::kPlanMaxBatch,

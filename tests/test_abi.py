@@ -117,6 +117,11 @@ def test_size_queries():
     assert n >= (64 + 74) * 128 * 512 * 4
     assert B.mla_sparse_workspace_size(32, 1, 128, 2048, 512, 74) > n // 2
     assert B.mla_sparse_fused_workspace_size(32, 64, 2048, 148) >= 32 * 2048 * 576 * 2
+    # the fused decode adds the prologue's query rows to the dense workspace
+    assert (B.mla_fused_workspace_size(32, 64, 148) >=
+            B.mla_workspace_size(32, 64, 576, 148) + 32 * 64 * 576 * 2)
+    assert (B.mla_sparse_fused_workspace_size(32, 64, 2048, 148) >=
+            B.mla_fused_workspace_size(32, 64, 148) + 32 * 2048 * 576 * 2)
     # prefill: partials only for tokens split over several parts (at most
     # 2 * parts of them), plus per-token tables of one pass of <= 8192 tokens
     n_pf = B.mla_sparse_prefill_workspace_size(4096, 128, 2048, 74)

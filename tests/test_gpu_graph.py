@@ -80,7 +80,7 @@ def test_graph_fused():
     codes = torch.empty((b, 1, case.h_q, 576), dtype=torch.uint8, device=dev)
     scale = torch.empty((b, 1, case.h_q), dtype=torch.float32, device=dev)
     lse = torch.empty((b, 1, case.h_q), dtype=torch.float32, device=dev)
-    ws = torch.empty((B.mla_workspace_size(b, case.h_q, 576, parts),), dtype=torch.uint8, device=dev)
+    ws = torch.empty((B.mla_fused_workspace_size(b, case.h_q, parts),), dtype=torch.uint8, device=dev)
 
     def step():
         m, n, _ = B.mla_get_metadata(sl, case.h_q, 1, parts)
