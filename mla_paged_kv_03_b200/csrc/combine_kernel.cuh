@@ -255,8 +255,9 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* total) {
 
 // Split-KV planner of one CTA: the closed forms of mla_common.h evaluated in
 // parallel (prefix sums by block scans, one metadata row per thread).
-__device__ void plan_block(const int32_t* seqlens, int batch, int num_parts, int o, int g,
+__device__ void plan_block(const int32_t* seqlens, int batch, int num_parts, const PlanParams pp,
                            int32_t* metadata, int32_t* num_splits, int32_t* ws_base) {
+  const int o = pp.o, g = pp.g;
   const int u = g * kPlanTileCost;
   __shared__ int32_t C[kPlanMaxBatch + 1];
   const int tid = threadIdx.x;
@@ -272,7 +273,7 @@ __device__ void plan_block(const int32_t* seqlens, int batch, int num_parts, int
   }
   if (tid == 0) C[batch] = carry;
   __syncthreads();
-  const int w = plan_width(carry, num_parts, u);
+  const int w = plan_width(carry, num_parts, pp);
   for (int p = tid; p < num_parts; p += kPlanThreads)
     plan_part_row(C, batch, w, o, g, p, metadata + p * kMetaInts);
   int nsum = 0;
@@ -301,13 +302,13 @@ __device__ void plan_block(const int32_t* seqlens, int batch, int num_parts, int
 }
 
 __global__ void __launch_bounds__(kPlanThreads) mla_plan_kernel(const int32_t* seqlens, int batch,
-                                                               int num_parts, int overhead,
-                                                               int granule, int32_t* metadata,
+                                                               int num_parts, const PlanParams pp,
+                                                               int32_t* metadata,
                                                                int32_t* num_splits,
                                                                int32_t* ws_base) {
   ptx::grid_dep_wait();
   ptx::grid_dep_launch();  // the decode grid waits for this one at its start
-  plan_block(seqlens, batch, num_parts, overhead, granule, metadata, num_splits, ws_base);
+  plan_block(seqlens, batch, num_parts, pp, metadata, num_splits, ws_base);
 }
 
 }  // namespace mla

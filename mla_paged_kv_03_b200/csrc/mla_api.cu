@@ -659,8 +659,8 @@ int mla_get_metadata(const int32_t* cache_seqlens, int batch, int heads_per_kv, 
   MLA_CHECK_ARG(batch <= mla::kPlanMaxBatch, "the device planner takes at most %d sequences (got %d)",
                 mla::kPlanMaxBatch, batch);
   mla::mla_plan_kernel<<<1, mla::kPlanThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-      cache_seqlens, batch, num_sm_parts, mla::plan_overhead(heads_per_kv),
-      mla::plan_granule(heads_per_kv), metadata, num_splits, nullptr);
+      cache_seqlens, batch, num_sm_parts, mla::plan_params(heads_per_kv), metadata, num_splits,
+      nullptr);
   MLA_CUDA(cudaGetLastError());
   return MLA_OK;
 }
@@ -673,18 +673,17 @@ int mla_get_metadata_host(const int32_t* cache_seqlens, int batch, int heads_per
   MLA_CHECK_ARG(metadata && num_splits && (cache_seqlens || batch == 0), "null host pointer");
   for (int b = 0; b < batch; ++b)
     MLA_CHECK_ARG(cache_seqlens[b] >= 0, "cache_seqlens[%d] = %d is negative", b, cache_seqlens[b]);
-  const int o = mla::plan_overhead(heads_per_kv);
-  const int g = mla::plan_granule(heads_per_kv);
+  const mla::PlanParams pp = mla::plan_params(heads_per_kv);
   std::vector<int32_t> granules(static_cast<size_t>(batch));
   long long total = 0;
   for (int b = 0; b < batch; ++b) {
-    granules[b] = mla::granules_of(cache_seqlens[b], g);
-    total += o + static_cast<long long>(mla::kPlanTileCost) * g * granules[b];
+    granules[b] = mla::granules_of(cache_seqlens[b], pp.g);
+    total += pp.o + static_cast<long long>(mla::kPlanTileCost) * pp.g * granules[b];
   }
   MLA_CHECK_ARG(total <= mla::kPlanMaxTotal, "total planner cost %lld above %lld", total,
                 mla::kPlanMaxTotal);
   std::vector<int32_t> prefix(static_cast<size_t>(batch) + 1);
-  mla::plan_splits_host(granules.data(), batch, num_sm_parts, o, g, metadata, num_splits,
+  mla::plan_splits_host(granules.data(), batch, num_sm_parts, pp, metadata, num_splits,
                         prefix.data());
   return MLA_OK;
 }
@@ -952,7 +951,7 @@ int mla_sparse_prefill_fwd(const void* q, const void* kv, int64_t s_kv, const in
         topk_length ? topk_length + t0 : nullptr, topk, n, lengths);
     MLA_CUDA(cudaGetLastError());
     mla::mla_plan_kernel<<<1, mla::kPlanThreads, 0, st>>>(
-        lengths, n, parts, mla::plan_overhead(h_q), mla::plan_granule(h_q), meta, splits, base);
+        lengths, n, parts, mla::plan_params(h_q), meta, splits, base);
     MLA_CUDA(cudaGetLastError());
     mla::DecodeParams p{};
     p.batch = n;

@@ -37,7 +37,10 @@ constexpr int kNumChunks = kD / kChunkD;  // 9
 // half a step idle), one tile for the others.  The overhead and the granule
 // depend on the kernel that will run, which the planner knows from the rows
 // per KV head; the overheads are the fastest values of sweeps over the
-// benchmark workloads on B200.
+// benchmark workloads on B200.  A part of the 1-CTA kernel is also at least
+// two tiles wide: at batch 1 (the fused decode) one-tile parts leave the
+// attention kernel latency-bound and make the combine read 148 partials per
+// row, and two-tile parts were the fastest step of a sweep over 1..8 tiles.
 constexpr int kPlanTileCost = 4;
 #ifndef MLA_PLAN_OVH_PAGE
 #define MLA_PLAN_OVH_PAGE 4
@@ -52,12 +55,18 @@ constexpr int kPlanOverheadPage = MLA_PLAN_OVH_PAGE;  // <= 32 rows per KV head 
 constexpr int kPlanOverheadCta = MLA_PLAN_OVH_CTA;    // 33..64 rows (1-CTA kernel)
 constexpr int kPlanOverheadPair = MLA_PLAN_OVH_PAIR;  // > 64 rows (CTA-pair kernel)
 
-MLA_HD inline int plan_overhead(int heads_per_kv) {
-  return heads_per_kv <= 32 ? kPlanOverheadPage
-                            : (heads_per_kv <= 64 ? kPlanOverheadCta : kPlanOverheadPair);
-}
+constexpr int kPlanMinWidthCta = 2 * kPlanTileCost;
 
-MLA_HD inline int plan_granule(int heads_per_kv) { return heads_per_kv > 64 ? 2 : 1; }
+// The planner's constants for the kernel that serves `heads_per_kv` rows:
+// segment overhead o, granule g (tiles) and minimum part width (cost units).
+struct PlanParams {
+  int o, g, wmin;
+};
+MLA_HD inline PlanParams plan_params(int heads_per_kv) {
+  if (heads_per_kv <= 32) return {kPlanOverheadPage, 1, 0};
+  if (heads_per_kv <= 64) return {kPlanOverheadCta, 1, kPlanMinWidthCta};
+  return {kPlanOverheadPair, 2, 0};
+}
 
 // Metadata row per SM part: {begin_b, begin_tile, end_b, end_tile,
 // first_split, 0, 0, 0}; end_tile is exclusive within batch end_b (it may pass
@@ -90,7 +99,8 @@ constexpr long long kPlanMaxTotal = (1LL << 30);
 // each costing u = g * kPlanTileCost, sequence b occupies [C[b], C[b+1]) with
 // C[b+1] = C[b] + o + u * granules_of(L_b, g) (o the segment overhead); its
 // overhead comes first and granule t starts at C[b] + o + u t.  The line is
-// cut into num_parts intervals of width W = ceil(total / num_parts); part p
+// cut into num_parts intervals of width W = ceil(total / num_parts) (or the
+// kernel's minimum width, when larger; the parts past the end stay empty); part p
 // takes the granules whose start falls in [pW, (p+1)W).  Each part therefore
 // covers one contiguous run of (sequence, tile) pairs and costs at most W plus
 // one granule and one segment overhead (that of a sequence continued from the
@@ -101,10 +111,13 @@ constexpr long long kPlanMaxTotal = (1LL << 30);
 // planner reaches the identical result with plain loops.
 
 // At least one granule (u) wide, so that every interval lying within a
-// sequence's granules holds a granule start (the split counts rely on that).
-MLA_HD inline int plan_width(int total, int num_parts, int u) {
+// sequence's granules holds a granule start (the split counts rely on that),
+// and at least the kernel's minimum width.
+MLA_HD inline int plan_width(int total, int num_parts, const PlanParams& pp) {
   const int w = (total + num_parts - 1) / num_parts;
-  return w < u ? u : w;
+  const int u = pp.g * kPlanTileCost;
+  const int m = u > pp.wmin ? u : pp.wmin;
+  return w < m ? m : w;
 }
 
 // Sequence b with C[b] <= x < C[b+1] (C holds batch + 1 prefix sums).
@@ -179,15 +192,16 @@ MLA_HD inline void plan_part_row(const int32_t* C, int batch, int w, int o, int 
 }
 
 // Host planner: metadata[num_parts][8] and num_splits[batch + 1] from the
-// per-sequence tile counts and the segment overhead o (same result as the
-// device planner).
-inline void plan_splits_host(const int32_t* granules, int batch, int num_parts, int o, int g,
-                             int32_t* metadata, int32_t* num_splits,
+// per-sequence granule counts and the kernel's planner constants (same
+// result as the device planner).
+inline void plan_splits_host(const int32_t* granules, int batch, int num_parts,
+                             const PlanParams& pp, int32_t* metadata, int32_t* num_splits,
                              int32_t* C /* batch + 1 scratch */) {
+  const int o = pp.o, g = pp.g;
   const int u = g * kPlanTileCost;
   C[0] = 0;
   for (int b = 0; b < batch; ++b) C[b + 1] = C[b] + o + u * granules[b];
-  const int w = plan_width(C[batch], num_parts, u);
+  const int w = plan_width(C[batch], num_parts, pp);
   for (int p = 0; p < num_parts; ++p)
     plan_part_row(C, batch, w, o, g, p, metadata + p * kMetaInts);
   num_splits[0] = 0;

@@ -68,3 +68,37 @@ def test_fused_full_size_sampled(batch):
     gpu = run_gpu(case)
     rows = full_size_rows(case.h_q, case.cache_seqlens.cpu().numpy(), 48, batch)
     check(case, rows=rows, gpu=gpu)
+
+
+@pytest.mark.parametrize("explicit_positions", [False, True])
+def test_fused_prologue_rows_bit_exact(explicit_positions):
+    """The prologue's normalised, rotated bf16 query rows, read back from the
+    workspace (they follow the mla_workspace_size(batch, h_q, 576, parts)
+    bytes of split partials), equal the oracle's RMSNorm -> RoPE -> bf16
+    rounding bit for bit on every element of 512 rows."""
+    dev = torch.device("cuda")
+    batch = 8
+    case = W.fused(seed=5, batch=batch)
+    sl = case.cache_seqlens.to(dev)
+    pos = (torch.randint(0, 1 << 20, (batch,), generator=torch.Generator().manual_seed(11),
+                         dtype=torch.int32) if explicit_positions else None)
+    meta, ns, parts = B.mla_get_metadata(sl, case.h_q, 1)
+    ws = torch.zeros((B.mla_fused_workspace_size(batch, case.h_q, parts),), dtype=torch.uint8,
+                     device=dev)
+    B.mla_fused_norm_rope_attn_rope_cast(
+        case.q_raw.to(dev), case.gain.to(dev), case.eps, case.rope_base, case.kcache.to(dev),
+        case.block_table.to(dev), sl, meta, ns, parts, softmax_scale=case.softmax_scale,
+        positions=None if pos is None else pos.to(dev), workspace=ws)
+    torch.cuda.synchronize()
+    assert B.device_status() == 0
+    rows = batch * case.h_q
+    off = B.mla_workspace_size(batch, case.h_q, 576, parts)
+    q_gpu = ws[off:off + rows * 576 * 2].view(torch.bfloat16).view(rows, 576).cpu().double().numpy()
+    raw = case.q_raw.cpu().double().numpy().reshape(rows, 576)
+    gain = case.gain.cpu().double().numpy()
+    for r in range(rows):
+        b = r // case.h_q
+        p = int(pos[b]) if pos is not None else int(case.cache_seqlens[b]) - 1
+        y = oracle.rmsnorm(raw[r], gain, case.eps)
+        y[512:] = oracle.rope64(y[512:], p, case.rope_base, +1)
+        np.testing.assert_array_equal(q_gpu[r], oracle.round_bf16(y), err_msg=f"row {r}")
