@@ -274,13 +274,14 @@ class GpuStep:
         return -(-self.case.s_q // 8192) if self.kind == "prefill" else 1
 
     def launches_per_step(self):
-        # planner + attention kernel + combine (+ the FP8 gather for sparse);
-        # the prefill runs lengths, planner, attention and combine per launch of
-        # up to 8192 query tokens, then the sinks
+        # planner + attention kernel + combine (+ the FP8 gather for sparse, +
+        # the query prologue for fused); the prefill runs lengths, planner,
+        # attention and combine per launch of up to 8192 query tokens, then the
+        # sinks
         if self.kind == "prefill":
             c = self.case
             return 4 * -(-c.s_q // 8192) + (1 if c.attn_sink is not None else 0)
-        return 4 if self.kind in ("sparse", "fused_sparse") else 3
+        return 3 + (self.kind in ("sparse", "fused_sparse")) + (self.kind in ("fused", "fused_sparse"))
 
     def step(self, q=None):
         B, c = self.B, self.case
