@@ -21,8 +21,14 @@
 // address arithmetic then stays warp-uniform, and a group of eight N = 256
 // UMMAs covers the cost of the barrier waits between groups.
 //
-// Roles (warps): 0 loader (both CTAs), 1 MMA issuer (leader CTA) and TMEM
-// owner (both), 2..5 softmax / epilogue (both).
+// Roles (warps): 0, 10, 11 loaders (both CTAs), 1 MMA issuer (leader CTA)
+// and TMEM owner (both), 2..9 two softmax / epilogue warpgroups (both).
+//
+// Gather mode (sparse prefill): a unit is one query token, and its "cache" is
+// the rows of a bf16 [s_kv, 576] array that the token's index list names.
+// The loaders fetch them with TMA gather4 copies (four named rows, one 64-dim
+// chunk each), so neighbouring tokens that select the same rows share them
+// through L2; the softmax masks the entries that name no row.
 #pragma once
 #include "decode_kernel.cuh"
 

@@ -1,6 +1,6 @@
 """GPU parity of the token-level sparse prefill (C ABI mla_sparse_prefill_fwd:
-per-token top-k length, per-head attention sinks, passes of 32 tokens)
-against the fp64 oracle."""
+per-token top-k length, per-head attention sinks, one attention launch per
+8192 query tokens) against the fp64 oracle."""
 import numpy as np
 import pytest
 import torch
@@ -45,10 +45,21 @@ def small(seed=0, s_q=100, s_kv=100, h_q=128, topk=64, **kw):
     return W.sparse_prefill(seed=seed, s_q=s_q, s_kv=s_kv, h_q=h_q, topk=topk, **kw)
 
 
-def test_prefill_lengths_and_sinks_several_passes():
-    case = small()                      # 100 tokens: passes of 32, 32, 32 and 4
+def test_prefill_lengths_and_sinks():
+    case = small()
     assert int(case.topk_length.min()) < case.topk
     check(case)
+
+
+def test_prefill_more_tokens_than_one_launch():
+    """8200 tokens: two launches of the attention kernel (8192 and 8 tokens),
+    checked on every head of the first tokens and of those around the seam."""
+    dev = torch.device("cuda")
+    case = W.sparse_prefill(seed=5, s_q=8200, s_kv=8200, h_q=16, topk=8, device=dev)
+    gpu = run_gpu(case)
+    toks = list(range(4)) + list(range(8186, 8200))
+    rows = [t * case.h_q + h for t in toks for h in range(case.h_q)]
+    check(case, rows=rows, gpu=gpu)
 
 
 def test_prefill_without_lengths_or_sinks():
