@@ -628,6 +628,8 @@ __global__ void __launch_bounds__(pcfg::kThreads, 1)
       const bool partial = P.always_partial || u.nsplit > 1;
       const int ws_row = ((P.ws_base ? P.ws_base[u.b] : P.num_splits[u.b]) + u.split) * P.R + rg;
       const float inv = l > 0.f ? 1.0f / l : 0.f;
+      const bool ws32 = (reinterpret_cast<uintptr_t>(P.ws_o) & 31) == 0;
+      const bool out32 = (reinterpret_cast<uintptr_t>(P.out) & 31) == 0;
       float o[2][32];
       ptx::tmem_ld32(lane_addr + kOCol + 128 * wg, o[0]);
 #pragma unroll
@@ -637,12 +639,38 @@ __global__ void __launch_bounds__(pcfg::kThreads, 1)
         const float* v = o[c & 1];
         if (row_valid) {
           const int d0 = 256 * wg + 128 * h + 32 * c;
-          if (partial) {
+          // A thread holds 32 consecutive dims of its row: whole 32-byte sectors
+          // per store where the buffer's base is 32-byte aligned (rows are
+          // multiples of 32 bytes), 16-byte stores otherwise.  (Staging O
+          // through shared memory so that eight lanes write one 128-byte line
+          // was measured slower: more store instructions.)
+          if (partial && ws32) {
+            float* dst = P.ws_o + (size_t)ws_row * P.d_v + d0;
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              ptx::st_global_v8(dst + 8 * q, v[8 * q] * inv, v[8 * q + 1] * inv,
+                                v[8 * q + 2] * inv, v[8 * q + 3] * inv, v[8 * q + 4] * inv,
+                                v[8 * q + 5] * inv, v[8 * q + 6] * inv, v[8 * q + 7] * inv);
+          } else if (partial) {
             float4* dst = reinterpret_cast<float4*>(P.ws_o + (size_t)ws_row * P.d_v + d0);
 #pragma unroll
             for (int q = 0; q < 8; ++q)
               dst[q] = make_float4(v[4 * q] * inv, v[4 * q + 1] * inv, v[4 * q + 2] * inv,
                                    v[4 * q + 3] * inv);
+          } else if (out32) {
+            __nv_bfloat16* dst = P.out + ((size_t)u.b * P.R + rg) * P.d_v + d0;
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+              const float* w = v + 16 * q;
+              ptx::st_global_v8(dst + 16 * q, ptx::pack_bf16x2(w[0] * inv, w[1] * inv),
+                                ptx::pack_bf16x2(w[2] * inv, w[3] * inv),
+                                ptx::pack_bf16x2(w[4] * inv, w[5] * inv),
+                                ptx::pack_bf16x2(w[6] * inv, w[7] * inv),
+                                ptx::pack_bf16x2(w[8] * inv, w[9] * inv),
+                                ptx::pack_bf16x2(w[10] * inv, w[11] * inv),
+                                ptx::pack_bf16x2(w[12] * inv, w[13] * inv),
+                                ptx::pack_bf16x2(w[14] * inv, w[15] * inv));
+            }
           } else {
             uint4* dst = reinterpret_cast<uint4*>(P.out + ((size_t)u.b * P.R + rg) * P.d_v + d0);
 #pragma unroll
