@@ -232,8 +232,8 @@ MLA_API int mla_sparse_decode_v41_fp4(const void* q, const uint8_t* kcache_288, 
                               size_t workspace_bytes, void* out, float* lse, void* stream);
 
 /* Workspace bytes for mla_sparse_prefill_fwd: the clamped lengths and split
- * plan of up to 8192 query tokens and the partials of the tokens split over
- * several parts (2 * num_sm_parts * h_q rows of 512 fp32). */
+ * plan of up to 8192 query tokens, the list of the tokens split over several
+ * parts, and their partials (2 * num_sm_parts * h_q rows of 512 fp32). */
 MLA_API int mla_sparse_prefill_workspace_size(int s_q, int h_q, int topk, int num_sm_parts,
                                       size_t* bytes);
 
@@ -255,8 +255,10 @@ MLA_API int mla_sparse_prefill_workspace_size(int s_q, int h_q, int topk, int nu
  *   num_sm_parts  from mla_num_sm_parts(device, h_q, 1)
  * Each query token is one unit of the CTA-pair attention kernel, whose loads
  * fetch the token's rows straight from kv (four named rows per TMA copy); a
- * launch covers up to 8192 tokens, then the sinks are applied.  num_sm_parts
- * is capped at the device's SMs / (2 ceil(h_q / 128)) CTA pairs.
+ * launch covers up to 8192 tokens.  The sinks join each row's normaliser
+ * where the row is finished (the attention kernel, or the combine of the
+ * tokens split over several parts).  num_sm_parts is capped at the device's
+ * SMs / (2 ceil(h_q / 128)) CTA pairs.
  * Ownership and errors as in mla_sparse_decode. */
 MLA_API int mla_sparse_prefill_fwd(const void* q, const void* kv, int64_t s_kv,
                            const int32_t* indices, int topk, const int32_t* topk_length,

@@ -35,6 +35,11 @@ struct CombineParams {
   const int32_t* positions;   // nullable: L - 1
   double inv_freq[kRope / 2]; // base^(-2k/64), computed on the host in fp64
   int row_per_cta;            // 1: a CTA's warps share one row's splits (few rows)
+  // optional: the rows are those of the sequences seq_list[0 .. list_len)
+  // (-1 entries are skipped) instead of all batch sequences
+  const int32_t* seq_list;
+  int list_len;
+  const float* sink;          // nullable: per-head sink logits joining the normaliser
 };
 
 __device__ __forceinline__ uint32_t cvt_e4m3x4(float a, float b, float c, float d) {
@@ -72,8 +77,10 @@ __global__ void __launch_bounds__(kCombineThreads) mla_combine_kernel(const Comb
   const bool shared_row = P.row_per_cta != 0;
   const long long row_id =
       shared_row ? blockIdx.x : static_cast<long long>(blockIdx.x) * kCombineWarps + warp;
-  if (row_id >= static_cast<long long>(P.batch) * P.R) return;
-  const int b = static_cast<int>(row_id / P.R);
+  const int nseq = P.seq_list ? P.list_len : P.batch;
+  if (row_id >= static_cast<long long>(nseq) * P.R) return;
+  const int b = P.seq_list ? P.seq_list[row_id / P.R] : static_cast<int>(row_id / P.R);
+  if (b < 0) return;
   const int r = static_cast<int>(row_id % P.R);
   const int n = P.num_splits[b + 1] - P.num_splits[b];
   const int base = P.ws_base ? P.ws_base[b] : P.num_splits[b];
@@ -90,7 +97,19 @@ __global__ void __launch_bounds__(kCombineThreads) mla_combine_kernel(const Comb
     for (int i = lane; i < n; i += 32) sum += expf(lse_i[(size_t)i * P.R] - m);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-  const float lse = (m == -INFINITY) ? -INFINITY : m + logf(sum);
+  float lse = (m == -INFINITY) ? -INFINITY : m + logf(sum);
+  if (P.sink) {
+    // the head's sink logit joins the normaliser (no value row)
+    const float sk = P.sink[r % P.h_q];
+    if (sk != -INFINITY) {
+      if (lse == -INFINITY) {
+        lse = sk;
+      } else {
+        const float mp = fmaxf(lse, sk);
+        lse = mp + logf(expf(lse - mp) + expf(sk - mp));
+      }
+    }
+  }
 
   // O = sum_i exp(LSE_i - LSE) O_i
   const int ngroups = P.d_v / 4;
@@ -256,7 +275,8 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* total) {
 // Split-KV planner of one CTA: the closed forms of mla_common.h evaluated in
 // parallel (prefix sums by block scans, one metadata row per thread).
 __device__ void plan_block(const int32_t* seqlens, int batch, int num_parts, const PlanParams pp,
-                           int32_t* metadata, int32_t* num_splits, int32_t* ws_base) {
+                           int32_t* metadata, int32_t* num_splits, int32_t* ws_base,
+                           int32_t* split_list, int list_cap) {
   const int o = pp.o, g = pp.g;
   const int u = g * kPlanTileCost;
   __shared__ int32_t C[kPlanMaxBatch + 1];
@@ -299,16 +319,32 @@ __device__ void plan_block(const int32_t* seqlens, int batch, int num_parts, con
       wsum += chunk_total;
     }
   }
+  if (split_list) {
+    // the split sequences in order (at most num_parts - 1: each lies across
+    // a part boundary), then -1 up to list_cap
+    for (int i = tid; i < list_cap; i += kPlanThreads) split_list[i] = -1;
+    __syncthreads();
+    int ksum = 0;
+    for (int base = 0; base < batch; base += kPlanThreads) {
+      const int b = base + tid;
+      const int v = b < batch ? plan_last_part(C, b, w, u) - plan_first_part(C, b, w, o) + 1 : 0;
+      int chunk_total;
+      const int ex = block_exclusive_scan(v > 1 ? 1 : 0, &chunk_total);
+      if (b < batch && v > 1 && ksum + ex < list_cap) split_list[ksum + ex] = b;
+      ksum += chunk_total;
+    }
+  }
 }
 
 __global__ void __launch_bounds__(kPlanThreads) mla_plan_kernel(const int32_t* seqlens, int batch,
                                                                int num_parts, const PlanParams pp,
                                                                int32_t* metadata,
                                                                int32_t* num_splits,
-                                                               int32_t* ws_base) {
+                                                               int32_t* ws_base,
+                                                               int32_t* split_list, int list_cap) {
   ptx::grid_dep_wait();
   ptx::grid_dep_launch();  // the decode grid waits for this one at its start
-  plan_block(seqlens, batch, num_parts, pp, metadata, num_splits, ws_base);
+  plan_block(seqlens, batch, num_parts, pp, metadata, num_splits, ws_base, split_list, list_cap);
 }
 
 }  // namespace mla

@@ -83,6 +83,9 @@ struct DecodeParams {
   // split partials of sequence b start at ws row ws_base[b] (only split
   // sequences own rows), or at num_splits[b] when ws_base is null
   const int32_t* ws_base;
+  // sparse prefill: per-head attention sink logits (natural-log units) or
+  // null; folded into the rows the kernel finishes (unsplit ones)
+  const float* sink;
 };
 
 namespace cfg {

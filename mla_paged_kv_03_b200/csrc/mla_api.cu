@@ -17,7 +17,7 @@
 #include "page_kernel.cuh"
 #include "pair_kernel.cuh"
 #include "prologue_kernel.cuh"
-#include "sink_kernel.cuh"
+#include "prefill_kernel.cuh"
 #include "sparse_gather.cuh"
 #include "mla_common.h"
 
@@ -201,7 +201,7 @@ struct PdlLaunch {
 };
 
 int launch_combine(const mla::CombineParams& cp, bool fused, cudaStream_t st) {
-  const long long rows = static_cast<long long>(cp.batch) * cp.R;
+  const long long rows = static_cast<long long>(cp.seq_list ? cp.list_len : cp.batch) * cp.R;
   if (rows == 0) return MLA_OK;
   // few rows (fewer warps than a few per SM): a CTA per row, warps share its splits
   mla::CombineParams c = cp;
@@ -529,7 +529,7 @@ constexpr int kPrefillPass = mla::kPlanMaxBatch;
 // partial bases) and the partials of the query tokens split over several
 // parts (at most 2 * parts of them).
 struct PrefillWs {
-  size_t len_off, meta_off, splits_off, base_off, o_off, lse_off, total;
+  size_t len_off, meta_off, splits_off, base_off, list_off, o_off, lse_off, total;
 };
 
 PrefillWs prefill_ws_layout(int tokens, int h_q, int parts) {
@@ -539,7 +539,8 @@ PrefillWs prefill_ws_layout(int tokens, int h_q, int parts) {
   w.meta_off = align_up(static_cast<size_t>(tokens) * 4, 256);
   w.splits_off = w.meta_off + align_up(static_cast<size_t>(parts) * mla::kMetaInts * 4, 256);
   w.base_off = w.splits_off + align_up((static_cast<size_t>(tokens) + 1) * 4, 256);
-  w.o_off = w.base_off + align_up(static_cast<size_t>(tokens) * 4, 256);
+  w.list_off = w.base_off + align_up(static_cast<size_t>(tokens) * 4, 256);
+  w.o_off = w.list_off + align_up(static_cast<size_t>(parts) * 4, 256);
   w.lse_off = w.o_off + align_up(rows * 512 * 4, 256);
   w.total = w.lse_off + align_up(rows * 4, 256);
   return w;
@@ -660,7 +661,7 @@ int mla_get_metadata(const int32_t* cache_seqlens, int batch, int heads_per_kv, 
                 mla::kPlanMaxBatch, batch);
   mla::mla_plan_kernel<<<1, mla::kPlanThreads, 0, static_cast<cudaStream_t>(stream)>>>(
       cache_seqlens, batch, num_sm_parts, mla::plan_params(heads_per_kv), metadata, num_splits,
-      nullptr);
+      nullptr, nullptr, 0);
   MLA_CUDA(cudaGetLastError());
   return MLA_OK;
 }
@@ -939,6 +940,7 @@ int mla_sparse_prefill_fwd(const void* q, const void* kv, int64_t s_kv, const in
   int32_t* meta = reinterpret_cast<int32_t*>(ws + w.meta_off);
   int32_t* splits = reinterpret_cast<int32_t*>(ws + w.splits_off);
   int32_t* base = reinterpret_cast<int32_t*>(ws + w.base_off);
+  int32_t* split_list = reinterpret_cast<int32_t*>(ws + w.list_off);
   if (t_trace) {  // entries no load reaches stay -1
     MLA_CUDA(cudaMemsetAsync(t_trace, 0xFF, 2 * static_cast<size_t>(trace_plane) * 4, st));
   }
@@ -951,7 +953,7 @@ int mla_sparse_prefill_fwd(const void* q, const void* kv, int64_t s_kv, const in
         topk_length ? topk_length + t0 : nullptr, topk, n, lengths);
     MLA_CUDA(cudaGetLastError());
     mla::mla_plan_kernel<<<1, mla::kPlanThreads, 0, st>>>(
-        lengths, n, parts, mla::plan_params(h_q), meta, splits, base);
+        lengths, n, parts, mla::plan_params(h_q), meta, splits, base, split_list, parts);
     MLA_CUDA(cudaGetLastError());
     mla::DecodeParams p{};
     p.batch = n;
@@ -979,6 +981,7 @@ int mla_sparse_prefill_fwd(const void* q, const void* kv, int64_t s_kv, const in
     p.gather_rows = static_cast<int>(s_kv);
     p.trace = t_trace ? t_trace + static_cast<size_t>(t0) * topk : nullptr;
     p.trace_plane = trace_plane;
+    p.sink = attn_sink;
     const void* q_t = static_cast<const __nv_bfloat16*>(q) + t0 * q_row;
     if ((rc = launch_pair_decode<true>(q_t, kv, tkv, p, st)) != MLA_OK) return rc;
     mla::CombineParams cp{};
@@ -992,14 +995,10 @@ int mla_sparse_prefill_fwd(const void* q, const void* kv, int64_t s_kv, const in
     cp.ws_lse = p.ws_lse;
     cp.out = p.out;
     cp.lse = p.lse;
+    cp.seq_list = split_list;  // only the tokens split over several parts
+    cp.list_len = parts;
+    cp.sink = attn_sink;
     if ((rc = launch_combine(cp, false, st)) != MLA_OK) return rc;
-  }
-  if (attn_sink) {
-    const long long rows = static_cast<long long>(s_q) * h_q;
-    const unsigned grid = static_cast<unsigned>((rows + mla::kSinkWarps - 1) / mla::kSinkWarps);
-    mla::mla_sink_kernel<<<grid, 32 * mla::kSinkWarps, 0, st>>>(
-        static_cast<__nv_bfloat16*>(out), lse, attn_sink, rows, h_q, d_v);
-    MLA_CUDA(cudaGetLastError());
   }
   return MLA_OK;
 }

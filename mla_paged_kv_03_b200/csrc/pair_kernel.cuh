@@ -627,7 +627,26 @@ __global__ void __launch_bounds__(pcfg::kThreads, 1)
       ptx::tc_fence_after();
       const bool partial = P.always_partial || u.nsplit > 1;
       const int ws_row = ((P.ws_base ? P.ws_base[u.b] : P.num_splits[u.b]) + u.split) * P.R + rg;
-      const float inv = l > 0.f ? 1.0f / l : 0.f;
+      float inv = l > 0.f ? 1.0f / l : 0.f;
+      float lv = l > 0.f ? (m_used + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+      if (!partial && P.sink) {
+        // attention sink of the row's head (a logit without a value row): it
+        // joins the normaliser, l' = l + 2^(sink - m) (max-shifted); a row
+        // split over several parts gets it in the combine instead
+        const float sk = P.sink[rg % P.h_q];
+        if (sk != -INFINITY) {
+          if (l > 0.f) {
+            const float s2 = sk * 1.4426950408889634f;
+            const float mp = fmaxf(m_used, s2);
+            const float f = ex2(m_used - mp);
+            const float l2 = l * f + ex2(s2 - mp);
+            inv = f / l2;
+            lv = (mp + __log2f(l2)) * 0.69314718055994531f;
+          } else {
+            lv = sk;  // no row: O stays 0
+          }
+        }
+      }
       const bool ws32 = (reinterpret_cast<uintptr_t>(P.ws_o) & 31) == 0;
       const bool out32 = (reinterpret_cast<uintptr_t>(P.out) & 31) == 0;
       float o[2][32];
@@ -683,7 +702,6 @@ __global__ void __launch_bounds__(pcfg::kThreads, 1)
         }
       }
       if (row_valid && quarter == 0) {
-        const float lv = l > 0.f ? (m_used + __log2f(l)) * 0.69314718055994531f : -INFINITY;
         if (partial)
           P.ws_lse[ws_row] = lv;
         else

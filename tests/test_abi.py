@@ -123,10 +123,11 @@ def test_size_queries():
     assert (B.mla_sparse_fused_workspace_size(32, 64, 2048, 148) >=
             B.mla_fused_workspace_size(32, 64, 148) + 32 * 2048 * 576 * 2)
     # prefill: partials only for tokens split over several parts (at most
-    # 2 * parts of them), plus per-token tables of one pass of <= 8192 tokens
+    # 2 * parts of them), plus per-token tables of one pass of <= 8192 tokens and
+    # the list of split tokens (one entry per part)
     n_pf = B.mla_sparse_prefill_workspace_size(4096, 128, 2048, 74)
     partials = 2 * 74 * 128 * (512 + 1) * 4
-    assert partials <= n_pf < partials + 4096 * 12 + 74 * 32 + 5 * 256
+    assert partials <= n_pf < partials + 4096 * 12 + 74 * 36 + 6 * 256
     assert (B.mla_sparse_prefill_workspace_size(20000, 128, 2048, 74) ==
             B.mla_sparse_prefill_workspace_size(8192, 128, 2048, 74))
     # the V4.1 workspace adds the query widened to 576 dims
