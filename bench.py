@@ -276,11 +276,10 @@ class GpuStep:
     def launches_per_step(self):
         # planner + attention kernel + combine (+ the FP8 gather for sparse, +
         # the query prologue for fused); the prefill runs lengths, planner,
-        # attention and combine per launch of up to 8192 query tokens, then the
-        # sinks
+        # attention and combine per launch of up to 8192 query tokens
         if self.kind == "prefill":
             c = self.case
-            return 4 * -(-c.s_q // 8192) + (1 if c.attn_sink is not None else 0)
+            return 4 * -(-c.s_q // 8192)
         return 3 + (self.kind in ("sparse", "fused_sparse")) + (self.kind in ("fused", "fused_sparse"))
 
     def step(self, q=None):
