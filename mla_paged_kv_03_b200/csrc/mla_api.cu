@@ -839,11 +839,11 @@ int mla_fused_norm_rope_attn_rope_cast(
   for (int k = 0; k < mla::kRope / 2; ++k)
     fq.inv_freq[k] = std::pow(static_cast<double>(rope_base), -2.0 * k / mla::kRope);
   fq.q_out = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(workspace) + w.q_off);
-  {
-    PdlLaunch L(dim3(static_cast<unsigned>(mla::ceil_div(fq.rows, mla::kPrologueWarps))),
-                dim3(32 * mla::kPrologueWarps), 0, st);
-    MLA_CUDA(cudaLaunchKernelEx(&L.cfg, mla::mla_fused_q_kernel, fq));
-  }
+  // an ordinary launch: the prologue reads the caller's inputs, which the
+  // preceding work of the stream may still be writing
+  mla::mla_fused_q_kernel<<<static_cast<unsigned>(mla::ceil_div(fq.rows, mla::kPrologueWarps)),
+                            32 * mla::kPrologueWarps, 0, st>>>(fq);
+  MLA_CUDA(cudaGetLastError());
   CUtensorMap tq;
   if ((rc = make_latent_map(&tq, fq.q_out, static_cast<long long>(batch) * R)) != MLA_OK)
     return rc;

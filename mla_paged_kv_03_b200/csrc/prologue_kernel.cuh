@@ -39,8 +39,9 @@ constexpr int kPrologueWarps = 8;
 __global__ void __launch_bounds__(32 * kPrologueWarps)
     mla_fused_q_kernel(const FusedQParams P) {
   __shared__ double cs[kPrologueWarps][kRope / 2][2];
-  // the attention grid may start its setup now; it waits for this grid's
-  // completion before it reads the rows
+  // Launched in stream order (after all earlier work of the stream), so the
+  // inputs are complete; the attention grid may start its setup now and
+  // waits for this grid's completion before it reads the rows.
   ptx::grid_dep_launch();
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -110,9 +111,6 @@ __global__ void __launch_bounds__(32 * kPrologueWarps)
       }
     }
   }
-  // this grid completes only after the kernels before it (the planner), so
-  // that the attention grid's wait on it also covers them
-  ptx::grid_dep_wait();
 }
 
 }  // namespace mla
