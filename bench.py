@@ -317,7 +317,7 @@ class GpuStep:
 
     def with_own_buffers(self):
         """A second handle on the same inputs with its own outputs, workspace
-        and scheduler buffers, so that two steps can be in flight at once."""
+        and scheduler buffers, so that several steps can be in flight at once."""
         import copy
         other = copy.copy(self)
         other.out = torch.empty_like(self.out)
@@ -574,6 +574,9 @@ def measure_side(name, args, dev, peaks, peak_src):
     return out
 
 
+E2E_IN_FLIGHT = 3  # end-to-end steps in flight (streams with their own buffers)
+
+
 def run_gpu_arm(args, rank, world):
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
@@ -630,14 +633,16 @@ def run_gpu_arm(args, rank, world):
     clocks = sampler.stop() if clk is None else sample_clocks_stop(clk)
 
     # end to end through the same API with host buffers: every step copies its
-    # query in from pinned host memory, runs, and copies O and LSE back.  Two
-    # steps are in flight on two streams, each with its own device buffers, so
-    # one step's copies overlap the other's kernels as a serving loop runs
-    # them; the region ends when both streams have drained.
+    # query in from pinned host memory, runs, and copies O and LSE back.  Three
+    # steps are in flight on three streams, each with its own device buffers,
+    # so that the host-to-device copies, the kernels and the device-to-host
+    # copies of consecutive steps overlap as a serving loop runs them (with two,
+    # a stream's next upload waits for its previous download and the copy
+    # engine idles); the region ends when every stream has drained.
     ref_out = gs.out.cpu()
     q_dev = gs.query()
     q_host = q_dev.cpu().pin_memory()
-    slots = [gs, gs.with_own_buffers()]
+    slots = [gs] + [gs.with_own_buffers() for _ in range(E2E_IN_FLIGHT - 1)]
     streams = [torch.cuda.Stream(dev) for _ in slots]
     q_bufs = [torch.empty_like(q_dev) for _ in slots]
     out_hosts = [torch.empty(gs.out.shape, dtype=gs.out.dtype).pin_memory() for _ in slots]
@@ -725,7 +730,7 @@ def run_gpu_arm(args, rank, world):
                 "d2h_bytes_per_step": int(gs.out.numel() * gs.out.element_size() +
                                           gs.lse.numel() * 4 +
                                           (gs.scale.numel() * 4 if hasattr(gs, "scale") else 0)),
-                "ms_per_step": round(e2e_ms, 5), "steps_in_flight": 2},
+                "ms_per_step": round(e2e_ms, 5), "steps_in_flight": E2E_IN_FLIGHT},
         "gpu_launches": gs.launches_per_step() * args.steps,
         "roofline": roof,
         "clocks": clocks,
