@@ -86,6 +86,10 @@ struct DecodeParams {
   // sparse prefill: per-head attention sink logits (natural-log units) or
   // null; folded into the rows the kernel finishes (unsplit ones)
   const float* sink;
+  // CTA-pair kernel: 64-dim chunks of q . k, 9 (the 576-dim latent; 0 reads
+  // as 9) or 8 (a 512-dim latent: q is [rows, 512], and the cache's dims
+  // 512..575 are not read)
+  int qk_chunks;
 };
 
 namespace cfg {

@@ -107,12 +107,12 @@ int make_gather_map(CUtensorMap* map, const void* base, long long rows) {
 // (strides 1152 B and 128 B) with a {64, box_rows, box_chunks} box, 128-byte
 // swizzle; one copy lands [box_chunks][box_rows][64 dims] in shared memory.
 int make_latent_map3(CUtensorMap* map, const void* base, long long rows, int box_chunks,
-                     int box_rows = 64) {
+                     int box_rows = 64, int row_elems = mla::kD) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(mla::kChunkD), static_cast<cuuint64_t>(rows),
-                        static_cast<cuuint64_t>(mla::kNumChunks)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(mla::kD) * 2,
+                        static_cast<cuuint64_t>(row_elems / mla::kChunkD)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(row_elems) * 2,
                            static_cast<cuuint64_t>(mla::kChunkD) * 2};
   cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), static_cast<cuuint32_t>(box_chunks)};
   cuuint32_t estr[3] = {1, 1, 1};
@@ -237,6 +237,17 @@ struct TraceOff {
   ~TraceOff() { t_trace = saved; }
 };
 
+// q . k chunks of the CTA-pair kernel for the dense decode a sparse path runs
+// internally (0: the 576-dim latent); the V4.1 paths set 8 around that call,
+// passing their 512-wide query as it is.
+thread_local int t_qk_chunks = 0;
+
+struct QkChunks {
+  int saved;
+  explicit QkChunks(int n) : saved(t_qk_chunks) { t_qk_chunks = n; }
+  ~QkChunks() { t_qk_chunks = saved; }
+};
+
 int check_trace(long long entries_per_plane) {
   if (!t_trace) return MLA_OK;
   MLA_CHECK_ARG(t_trace_cap >= 2 * entries_per_plane,
@@ -319,7 +330,10 @@ template <bool kGather>
 int launch_pair_decode(const void* q, const void* kcache, const CUtensorMap& tkv,
                        const mla::DecodeParams& p, cudaStream_t st) {
   CUtensorMap tq3, tv3;
-  int rc = make_latent_map3(&tq3, q, static_cast<long long>(p.batch) * p.R, mla::kNumChunks);
+  // q is [rows, 64 * qk_chunks] (576 wide, or 512 for a 512-dim latent)
+  const int qk = p.qk_chunks ? p.qk_chunks : mla::kNumChunks;
+  int rc = make_latent_map3(&tq3, q, static_cast<long long>(p.batch) * p.R, qk, 64,
+                            qk * mla::kChunkD);
   if (rc != MLA_OK) return rc;
   if (kGather)
     tv3 = tkv;
@@ -440,7 +454,7 @@ static int sparse_gather_and_plan(int row_bytes, const void* q, const uint8_t* k
                                   int h_q, int num_sm_parts, uint8_t* ws, const SparseWs& w,
                                   void* stream, const void** q_dense,
                                   int32_t* trace = nullptr,
-                                  long long trace_plane = 0) {
+                                  long long trace_plane = 0, bool widen_q = true) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   mla::GatherParams g{};
   g.trace = trace;
@@ -455,7 +469,7 @@ static int sparse_gather_and_plan(int row_bytes, const void* q, const uint8_t* k
   g.seqlens = reinterpret_cast<int32_t*>(ws + w.len_off);
   g.h_q = h_q;
   *q_dense = q;
-  if (row_bytes == mla::kRow528 || row_bytes == mla::kRow288) {
+  if ((row_bytes == mla::kRow528 || row_bytes == mla::kRow288) && widen_q) {
     g.q512 = static_cast<const __nv_bfloat16*>(q);
     g.q576 = reinterpret_cast<__nv_bfloat16*>(ws + w.q_off);
     *q_dense = g.q576;
@@ -505,12 +519,17 @@ static int sparse_decode_impl(int row_bytes, const void* q, const uint8_t* kcach
   if (batch == 0) return MLA_OK;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const void* q_dense = q;
+  // V4.1 rows with more than 64 query rows per KV head: the CTA-pair kernel
+  // takes the 512-wide query as it is and reads 8 chunks of each row; the
+  // other kernels see the query widened to 576 dims with zeros
+  const bool native512 = v41 && h_q > mla::kRowsPerCta && d_v == 512;
   rc = sparse_gather_and_plan(row_bytes, q, kcache, num_slots, indices, topk, pairs, h_q,
                               num_sm_parts, ws, w, stream, &q_dense, t_trace,
-                              static_cast<long long>(pairs) * topk);
+                              static_cast<long long>(pairs) * topk, !native512);
   if (rc != MLA_OK) return rc;
   // dense decode over the compacted rows: no causal mask, lengths = valid counts
   TraceOff off;
+  QkChunks qk(native512 ? mla::kNumChunks - 1 : 0);
   return mla_decode_fwd(q_dense, ws + w.rows_off, reinterpret_cast<int32_t*>(ws + w.bt_off),
                         w.pages_per_pair, static_cast<int>(pages),
                         reinterpret_cast<int32_t*>(ws + w.len_off), pairs, 1, h_q, 1, d_v,
@@ -747,6 +766,9 @@ int mla_decode_fwd(const void* q, const void* kcache, const int32_t* block_table
   p.ws_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.lse_off);
   p.trace = t_trace;
   p.trace_plane = static_cast<long long>(batch) * max_pages * mla::kPage;
+  p.qk_chunks = t_qk_chunks;
+  if (t_qk_chunks && !(R > mla::kRowsPerCta && d_v == 512))
+    return fail(MLA_ERR_UNSUPPORTED, "a 512-wide query needs the CTA-pair kernel");
   if (R <= 32 && d_v == 512) {
     p.n_groups = 1;
     rc = launch_page_decode(q, tkv, p, st);

@@ -130,6 +130,7 @@ __global__ void __launch_bounds__(pcfg::kThreads, 1)
   const int part = pair / P.n_groups;
   const int grp = pair % P.n_groups;  // 128-row group
 
+  const int nqk = P.qk_chunks ? P.qk_chunks : kNumChunks;  // 64-dim chunks of q . k
   ptx::grid_dep_wait();    // the planner's metadata is complete
   ptx::grid_dep_launch();  // the combine grid may be scheduled as CTAs retire
   const int32_t* meta = P.metadata + part * kMetaInts;
@@ -239,7 +240,7 @@ __global__ void __launch_bounds__(pcfg::kThreads, 1)
             }
           }
         }
-        for (int c = 0; c < kNumChunks; ++c) {
+        for (int c = 0; c < nqk; ++c) {
           int s;
           bool mine;
           if (!acquire(s, mine)) return false;
@@ -260,7 +261,7 @@ __global__ void __launch_bounds__(pcfg::kThreads, 1)
         trace_if_real(un, p0 + 2 * static_cast<int>(rank), kb0, 1);
         trace_if_real(un, p0 + 2 * static_cast<int>(rank) + 1, kb1, 1);
       }
-      for (int c = 0; c < kNumChunks; ++c) {
+      for (int c = 0; c < nqk; ++c) {
         int s;
         bool mine;
         if (!acquire(s, mine)) return false;
@@ -336,7 +337,7 @@ __global__ void __launch_bounds__(pcfg::kThreads, 1)
         }
         const int row0 = u.b * P.R + grp * 128 + static_cast<int>(rank) * kRows;
         if (ptx::elect_one_sync()) {
-          if (leader) ptx::mbar_arrive_expect_tx(&C.q_full, 2u * kQBytes);
+          if (leader) ptx::mbar_arrive_expect_tx(&C.q_full, 2u * nqk * kBox);
           ptx::tma_load_3d_pair(sQ, &tm_q3, leader_addr(&C.q_full), 0, row0, 0);
         }
         __syncwarp();
@@ -397,9 +398,8 @@ __global__ void __launch_bounds__(pcfg::kThreads, 1)
         const int sb = g & 1;
         if (!warp_wait_cluster(&C.s_empty[sb], ((g >> 1) & 1) ^ 1, 0x52)) return false;
         const uint32_t d_tmem = tmem + kSCol + sb * 128;
-#pragma unroll
-        for (int c0 = 0; c0 < kNumChunks; c0 += 2) {
-          const bool two = c0 + 1 < kNumChunks;
+        for (int c0 = 0; c0 < nqk; c0 += 2) {
+          const bool two = c0 + 1 < nqk;
           int s0 = 0, s1 = 0;
           if (!next_stage(s0)) return false;
           if (two && !next_stage(s1)) return false;
@@ -410,9 +410,8 @@ __global__ void __launch_bounds__(pcfg::kThreads, 1)
             if (two) {
               qk_chunk(d_tmem, s1, c0 + 1);
               ptx::umma_commit_pair_mc(&C.empty[s1], 0x3);
-            } else {
-              ptx::umma_commit_pair_mc(&C.s_full[sb], 0x3);
             }
+            if (c0 + 2 >= nqk) ptx::umma_commit_pair_mc(&C.s_full[sb], 0x3);
           }
           __syncwarp();
         }

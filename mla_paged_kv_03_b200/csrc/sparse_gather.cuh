@@ -211,7 +211,7 @@ __global__ void __launch_bounds__(kGatherCtaThreads, gather_min_ctas<kRowBytes>(
         }
       }
     }
-    if (kV41) {
+    if (kV41 && G.q576) {
       // the pair's query rows widened to 576 dims (72 16-byte units a row),
       // spread over all pages_per_pair CTAs of the pair, while the row loads
       // above are in flight
