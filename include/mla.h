@@ -189,8 +189,8 @@ MLA_API int mla_sparse_decode(const void* q, const uint8_t* kcache_fp8, int64_t 
                       size_t workspace_bytes, void* out, float* lse, void* stream);
 
 /* Workspace bytes for mla_sparse_decode_v41 and mla_sparse_decode_v41_fp4:
- * those of mla_sparse_decode with d_v = 512, plus the query widened to 576
- * dims. */
+ * those of mla_sparse_decode with d_v = 512, plus room for the query widened
+ * to 576 dims (used when h_q <= 64). */
 MLA_API int mla_sparse_v41_workspace_size(int batch, int s_q, int h_q, int topk, int num_sm_parts,
                                   size_t* bytes);
 
@@ -208,10 +208,12 @@ MLA_API int mla_sparse_v41_workspace_size(int batch, int s_q, int h_q, int topk,
  *                 [batch, s_q, h_q] fp32
  *   softmax_scale usually 1/sqrt(512)
  *   num_sm_parts  from mla_num_sm_parts(device, h_q, 1)
- * The dequantised rows (and the query) are widened to the 576-dim layout of
- * the dense kernels with zero dims 512..575, which leaves q . k and the
- * output unchanged.  Ownership, alignment (q, the cache and out 16-byte
- * aligned, workspace 256-byte aligned) and errors as in mla_sparse_decode. */
+ * The dequantised rows are written in the 576-dim layout of the dense kernels
+ * with zero dims 512..575.  With h_q > 64 the CTA-pair kernel reads the
+ * 512-wide query as it is and multiplies 512 dims of each row; otherwise the
+ * query is widened with zero dims too, which leaves q . k unchanged.
+ * Ownership, alignment (q, the cache and out 16-byte aligned, workspace
+ * 256-byte aligned) and errors as in mla_sparse_decode. */
 MLA_API int mla_sparse_decode_v41(const void* q, const uint8_t* kcache_528, int64_t num_slots,
                           const int32_t* indices, int topk, int batch, int s_q, int h_q,
                           float softmax_scale, int num_sm_parts, void* workspace,
