@@ -19,10 +19,11 @@ def _planner_constants():
                             "mla_paged_kv_03_b200", "csrc", "mla_common.h")).read()
     tile = int(re.search(r"kPlanTileCost = (\d+);", src).group(1))
     ovh = {k: int(v) for k, v in re.findall(r"#define MLA_PLAN_OVH_(\w+) (\d+)", src)}
-    return tile, ovh
+    min_cta = int(re.search(r"kPlanMinWidthCta = (\d+) \* kPlanTileCost;", src).group(1)) * tile
+    return tile, ovh, min_cta
 
 
-TILE_COST, OVH = _planner_constants()
+TILE_COST, OVH, MIN_WIDTH_CTA = _planner_constants()
 
 
 def overhead_for(heads_per_kv):
@@ -31,6 +32,16 @@ def overhead_for(heads_per_kv):
 
 def granule_for(heads_per_kv):
     return 2 if heads_per_kv > 64 else 1
+
+
+def min_width_for(heads_per_kv):
+    """The 1-CTA kernel's parts are at least two tiles wide."""
+    return MIN_WIDTH_CTA if 32 < heads_per_kv <= 64 else 0
+
+
+def target_width(seqlens, parts_n, heads_per_kv):
+    u = granule_for(heads_per_kv) * TILE_COST
+    return max(-(-plan_total(seqlens, heads_per_kv) // parts_n), u, min_width_for(heads_per_kv))
 
 
 def tiles_of(L):
@@ -115,7 +126,7 @@ def test_plan_random_mixes_and_balance(heads_per_kv):
         meta, ns, parts = check_plan(seqlens, parts_n, heads_per_kv)
         u = granule_for(heads_per_kv) * TILE_COST
         total = plan_total(seqlens, heads_per_kv)
-        target = max(-(-total // parts_n), u)
+        target = target_width(seqlens, parts_n, heads_per_kv)
         costs = [sum(seg_cost(lo, hi, heads_per_kv) for (_, lo, hi, _) in segs) for segs in parts]
         # every part stays within one granule and one segment overhead of the target
         for c in costs:
@@ -137,6 +148,23 @@ def test_plan_parts_narrower_than_a_tile():
     for seqlens in ([1], [1, 1], [130, 0, 5], [64] * 10):
         check_plan(seqlens, 500)
         check_plan(seqlens, 500, heads_per_kv=128)
+
+
+def test_plan_minimum_width_of_the_one_cta_kernel():
+    """Batch 1 on the 1-CTA kernel (64 rows per KV head): parts are at least
+    two tiles wide, so fewer parts than SMs hold work and the rest are empty;
+    the page and CTA-pair plans of the same sequence use every part."""
+    L = 17000  # 133 tiles
+    meta, ns, parts = check_plan([L], 148, heads_per_kv=64)
+    tiles = [sum(hi - lo for (_, lo, hi, _) in segs) for segs in parts]
+    used = [t for t in tiles if t]
+    assert all(t >= 2 for t in used[:-1])
+    # (the first parts lie inside the sequence's overhead and stay empty too)
+    assert len(used) <= -(-plan_total([L], 64) // target_width([L], 148, 64)) < 148
+    assert int(ns[1]) == len(used)
+    for h in (16, 128):
+        _, ns_h, parts_h = check_plan([L], 148, heads_per_kv=h)
+        assert int(ns_h[1]) > len(used)
 
 
 def test_plan_rejects_bad_arguments():
@@ -162,7 +190,7 @@ try:
         o = overhead_for(heads_per_kv)
         u = granule_for(heads_per_kv) * TILE_COST
         meta, ns, parts = check_plan(seqlens, parts_n, heads_per_kv)
-        target = max(-(-plan_total(seqlens, heads_per_kv) // parts_n), u)
+        target = target_width(seqlens, parts_n, heads_per_kv)
         for segs in parts:
             cost = sum(seg_cost(lo, hi, heads_per_kv) for (_, lo, hi, _) in segs)
             assert cost <= target + u + o
