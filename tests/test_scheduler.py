@@ -153,7 +153,7 @@ def test_plan_parts_narrower_than_a_tile():
 def test_plan_minimum_width_of_the_one_cta_kernel():
     """Batch 1 on the 1-CTA kernel (64 rows per KV head): parts are at least
     two tiles wide, so fewer parts than SMs hold work and the rest are empty;
-    the page and CTA-pair plans of the same sequence use every part."""
+    the page kernel's plan of the same sequence splits it more finely."""
     L = 17000  # 133 tiles
     meta, ns, parts = check_plan([L], 148, heads_per_kv=64)
     tiles = [sum(hi - lo for (_, lo, hi, _) in segs) for segs in parts]
@@ -162,9 +162,9 @@ def test_plan_minimum_width_of_the_one_cta_kernel():
     # (the first parts lie inside the sequence's overhead and stay empty too)
     assert len(used) <= -(-plan_total([L], 64) // target_width([L], 148, 64)) < 148
     assert int(ns[1]) == len(used)
-    for h in (16, 128):
-        _, ns_h, parts_h = check_plan([L], 148, heads_per_kv=h)
-        assert int(ns_h[1]) > len(used)
+    # the page kernel's plan of the same sequence (no minimum) uses ~all parts
+    _, ns16, _ = check_plan([L], 148, heads_per_kv=16)
+    assert int(ns16[1]) > len(used)
 
 
 def test_plan_rejects_bad_arguments():
